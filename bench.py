@@ -1,0 +1,358 @@
+"""Benchmark of the MoE layer forward on B200 (one process per GPU).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload prefill]
+    python bench.py --impl reference ...        # the CPU oracle, timed on host cores
+
+One step = one full layer forward (routing, permutation, routed and shared
+expert GEMMs, combine) over one batch of T tokens already resident in HBM.
+Under torchrun every rank runs its own batch with a full weight replica
+(token-parallel, no collective on the data path): weak scaling, value = all
+ranks' tokens / max-over-ranks time.  Prints one JSON line on rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from sparse_mixture_experts_03_b200 import accounting, moe  # noqa: E402
+from sparse_mixture_experts_03_b200.inputs import WORKLOADS, _randn, make_inputs  # noqa: E402
+
+METRIC = "MoE layer tokens/sec and TFLOP/s at 1 B200; % of roofline (TC or HBM)"
+L2_FLUSH_BYTES = 512 << 20  # > 126 MB L2
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": p["hbm_gbs"], "bf16_tflops": p["bf16_tflops"],
+                "bf16_tflops_sustained": p.get("bf16_tflops_sustained"), "source": "measured"}
+    except (OSError, KeyError, ValueError):
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                "source": "fallback"}
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons of one GPU through NVML (read only)."""
+
+    def __init__(self, device_index: int, period_s: float = 0.02):
+        self.samples, self.reasons = [], set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._period = period_s
+        self._ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            bus = torch.cuda.get_device_properties(device_index)
+            handle = None
+            try:
+                pci = "%08X:%02X:%02X.0" % (bus.pci_domain_id, bus.pci_bus_id, bus.pci_device_id)
+                handle = pynvml.nvmlDeviceGetHandleByPciBusId(pci.encode())
+            except Exception:
+                handle = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self._nv, self._h = pynvml, handle
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(handle, pynvml.NVML_CLOCK_SM)
+            self._ok = True
+        except Exception as e:  # no NVML: report it, do not guess
+            self.error = str(e)
+
+    def _run(self):
+        nv = self._nv
+        names = {
+            "hw_slowdown": getattr(nv, "nvmlClocksEventReasonHwSlowdown", 0x8),
+            "hw_thermal_slowdown": getattr(nv, "nvmlClocksEventReasonHwThermalSlowdown", 0x40),
+            "sw_thermal_slowdown": getattr(nv, "nvmlClocksEventReasonSwThermalSlowdown", 0x20),
+            "sw_power_cap": getattr(nv, "nvmlClocksEventReasonSwPowerCap", 0x4),
+        }
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for n, bit in names.items():
+                    if r & bit:
+                        self.reasons.add(n)
+            except Exception:
+                pass
+            self._stop.wait(self._period)
+
+    def __enter__(self):
+        if self._ok:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self._ok:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self):
+        if not self._ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [],
+                    "note": getattr(self, "error", "no samples")}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def max_over_ranks(v: float, world: int) -> float:
+    if world == 1:
+        return v
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+
+
+def cpu_baseline(w, inp, budget_s: float = 15.0):
+    """Time the CPU oracle (as it stands) on a bounded sample of the workload's tokens."""
+    import oracle
+    nthreads = os.cpu_count() or 1
+    probe = np.arange(min(w.T, max(8, nthreads)), dtype=np.int32)
+    t0 = time.perf_counter()
+    oracle.forward(inp.x, inp.W_router, inp.W_gate_up, inp.W_down, inp.W_shared, w.k,
+                   w.n_group, w.topk_group, w.inter, w.n_shared, tokens=probe, nthreads=nthreads)
+    per_tok = (time.perf_counter() - t0) / len(probe)
+    n = int(min(w.T, max(len(probe), budget_s / max(per_tok, 1e-9))))
+    n = max(nthreads, n // nthreads * nthreads) if n >= nthreads else n
+    toks = np.linspace(0, w.T - 1, n).astype(np.int32)
+    t0 = time.perf_counter()
+    oracle.forward(inp.x, inp.W_router, inp.W_gate_up, inp.W_down, inp.W_shared, w.k,
+                   w.n_group, w.topk_group, w.inter, w.n_shared, tokens=toks, nthreads=nthreads)
+    dt = time.perf_counter() - t0
+    return {"value": n / dt, "unit": "tokens/s", "cores": nthreads, "kind": "oracle",
+            "sample": f"{n} of {w.T} tokens of the {w.name} workload (full layer per token, "
+                      f"fp64), {dt:.1f} s wall"}
+
+
+def run_reference(args, w):
+    """--impl reference: the CPU oracle timed on the host cores, same metric/config."""
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle
+    inp = make_inputs(w)
+    nthreads = os.cpu_count() or 1
+    # bounded sample per step, sized so warmup+steps finish in a few minutes
+    probe = np.arange(min(w.T, max(4, nthreads)), dtype=np.int32)
+    t0 = time.perf_counter()
+    oracle.forward(inp.x, inp.W_router, inp.W_gate_up, inp.W_down, inp.W_shared, w.k,
+                   w.n_group, w.topk_group, w.inter, w.n_shared, tokens=probe, nthreads=nthreads)
+    per_tok = (time.perf_counter() - t0) / len(probe)
+    total_steps = args.steps + args.warmup
+    per_step_budget = 150.0 / max(total_steps, 1)
+    n = int(max(1, min(w.T, per_step_budget / max(per_tok, 1e-9))))
+    rng = np.random.default_rng(0)
+    times = []
+    for s in range(total_steps):
+        toks = np.sort(rng.choice(w.T, size=n, replace=False)).astype(np.int32)
+        t0 = time.perf_counter()
+        oracle.forward(inp.x, inp.W_router, inp.W_gate_up, inp.W_down, inp.W_shared, w.k,
+                       w.n_group, w.topk_group, w.inter, w.n_shared, tokens=toks,
+                       nthreads=nthreads)
+        if s >= args.warmup:
+            times.append(time.perf_counter() - t0)
+    sec = sum(times) / len(times)
+    value = n / sec
+    flops = accounting.flops_per_token(w.d, w.E, w.k, w.inter, w.n_shared) * n
+    out = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": sec * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": f"{w.name}: {w.describe()}", "tokens_per_step": n,
+                   "l2": "host CPU run"},
+        "tflops": flops / sec / 1e12,
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": nthreads, "kind": "oracle",
+                         "sample": f"{n} random tokens of {w.T} per step"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(out), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="prefill", choices=sorted(WORKLOADS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    w = WORKLOADS[args.workload]
+    if args.impl == "reference":
+        run_reference(args, w)
+        return
+
+    world, rank, local = dist_setup()
+    dev = torch.device("cuda", local)
+    inp = make_inputs(w)
+    if rank > 0:  # each rank its own batch of tokens, same weights
+        x = _randn((w.T, w.d), w.seed + rank, 0)
+        inp.x = x.to(inp.x.dtype)
+    x = inp.x.to(dev)
+    Wr, Wgu, Wd = inp.W_router.to(dev), inp.W_gate_up.to(dev), inp.W_down.to(dev)
+    Wsh = inp.W_shared.to(dev) if inp.W_shared is not None else None
+    y = torch.empty(w.T, w.d, dtype=torch.float32, device=dev)
+    idx = torch.empty(w.T, w.k, dtype=torch.int32, device=dev)
+    wt = torch.empty(w.T, w.k, dtype=torch.float32, device=dev)
+    ws = moe.alloc_workspace(w.T, w.d, w.E, w.k, w.inter, w.n_shared, x.dtype, dev)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step(xin=x, yout=y):
+        moe.forward(xin, Wr, Wgu, Wd, Wsh, w.k, w.n_group, w.topk_group, w.inter, w.n_shared,
+                    y=yout, topk_idx=idx, topk_w=wt, workspace=ws)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    st, site = moe.device_status(ws)
+    if st != moe.MOE_OK:
+        raise SystemExit(f"device status after warm-up: {moe.status_string(st)} (site {site})")
+
+    # ---- timed region: per-step events around the forward, L2 flushed between steps
+    n_ev = moe.N_STAGE_EVENTS
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    stage_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)]
+                for _ in range(args.steps)]
+    for evs in stage_ev:  # create the CUDA handles
+        for e in evs:
+            e.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    with ClockSampler(local) as clocks:
+        for i in range(args.steps):
+            flush.fill_(float(i))
+            moe.set_stage_events(stage_ev[i])
+            starts[i].record(stream)
+            step()
+            ends[i].record(stream)
+        moe.set_stage_events(None)
+        torch.cuda.synchronize()
+    barrier(world)
+    step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    ms = sum(step_ms) / len(step_ms)
+    ms = max_over_ranks(ms, world)
+    stage_ms = np.zeros(n_ev - 1)
+    for evs in stage_ev:
+        stage_ms += np.array([evs[j].elapsed_time(evs[j + 1]) for j in range(n_ev - 1)])
+    stage_ms /= args.steps
+    st, site = moe.device_status(ws)
+    if st != moe.MOE_OK:
+        raise SystemExit(f"device status after timing: {moe.status_string(st)} (site {site})")
+
+    # ---- end to end through the public call: pinned host x in, y out, every step
+    x_host = inp.x.pin_memory()
+    y_host = torch.empty(w.T, w.d, dtype=torch.float32).pin_memory()
+    x_dev2 = torch.empty_like(x)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for _ in range(3):
+        x_dev2.copy_(x_host, non_blocking=True)
+        step(x_dev2, y)
+        y_host.copy_(y, non_blocking=True)
+    barrier(world)
+    e2e_steps = max(10, args.steps // 4)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        x_dev2.copy_(x_host, non_blocking=True)
+        step(x_dev2, y)
+        y_host.copy_(y, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, world)
+
+    # ---- accounting
+    gi = idx.cpu().numpy()
+    rows = w.T * w.k
+    flops = accounting.layer_flops(w.T, w.d, w.E, w.k, w.inter, w.n_shared)
+    n_touched = accounting.touched_experts(gi, w.E)
+    bytes_alg = accounting.layer_bytes(w.T, w.d, w.E, w.inter, w.n_shared, n_touched)
+    pk = peaks()
+    tflops = flops / (ms * 1e-3) / 1e12
+    roof_ms = max(flops / (pk["bf16_tflops"] * 1e12), bytes_alg / (pk["hbm_gbs"] * 1e9)) * 1e3
+    names = moe.STAGES
+    stage = {n: float(v) for n, v in zip(names, stage_ms)}
+    # dominant kernel: the routed gate/up grouped GEMM (largest FLOP share)
+    g1_flops = accounting.gate_up_flops(rows, w.d, w.inter)
+    dom_ms = stage["gate_up_routed"]
+    dom_ach = g1_flops / (dom_ms * 1e-3) / 1e12
+    launches_per_step = 9 if w.n_shared > 0 else 8
+    value = world * w.T / (ms * 1e-3)
+    out = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) activations, N(0,1/fan_in) weights; no dataset)",
+        "config": {"workload": f"{w.name}: {w.describe()}", "global_batch": world * w.T,
+                   "tokens_per_gpu": w.T, "parallelism": f"token-parallel x{world} (replicas)",
+                   "l2": "flushed between timed steps (512 MB write); weights 1.28 GB > L2",
+                   "out_dtype": "f32"},
+        "tflops": tflops,
+        "roofline_layer": {"bound": "tensor", "roofline_ms": roof_ms,
+                           "frac": roof_ms / ms, "peak_tflops": pk["bf16_tflops"],
+                           "hbm_gbs": pk["hbm_gbs"], "alg_bytes": bytes_alg,
+                           "touched_experts": n_touched, "peak_source": pk["source"]},
+        "roofline": {"bound": "tensor", "kernel": "grouped_gemm_tc<SWIGLU> (routed gate/up)",
+                     "achieved": dom_ach, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                     "frac": dom_ach / pk["bf16_tflops"], "traffic": None,
+                     "flops_per_launch": g1_flops, "avg_launch_ms": dom_ms,
+                     "peak_kind": f"bf16 burst ({pk['source']})"},
+        "stage_ms": stage,
+        "gpu_launches": launches_per_step * args.steps,
+        "e2e": {"value": world * w.T / (e2e_ms * 1e-3), "unit": "tokens/s",
+                "h2d_bytes_per_step": x.numel() * x.element_size(),
+                "d2h_bytes_per_step": y.numel() * y.element_size(), "ms_per_step": e2e_ms},
+        "clocks": clocks.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(w, inp)
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,191 @@
+/*
+ * moe.h -- C ABI of the B200 (sm_100a) fine-grained Mixture-of-Experts layer
+ * forward.
+ *
+ * The layer (per token x of length d) is the one described on the FusionLLM
+ * page "FusionLLM：融合 MLA、GDN 与 MoE 的高效混合架构大模型训练框架", section
+ * "混合专家（MoE）" (fine-grained DeepSeekMoE layer, group-limited routing,
+ * bias-free sigmoid gating) with the sizes of its section "模型配置与规模"
+ * (64 routed experts, 6 active, 4 shared, moe_inter_dim 1536, dim 2048):
+ *
+ *   s_e  = sigmoid(W_router[e] . x)                       gate scores
+ *   keep the topk_group of n_group expert groups with the largest max score,
+ *   idx  = the k largest s_e inside the kept groups (descending, ties to the
+ *          lower index), w_j = s_idx[j] / sum_j s_idx[j]
+ *   y    = sum_j w_j * SwiGLU_{idx[j]}(x) + sum_s SwiGLU_shared_s(x)
+ *   SwiGLU_e(x) = W_down[e] (silu(W_gate[e] x) * (W_up[e] x))
+ *
+ * (router g(x) = W_g x and fixed-k top-k: "大模型工程（一）：Transformer 到
+ * MoE", section "MoE 数学：路由、容量与平衡详解"; weighted sum over the chosen
+ * experts: its MoEBlock listing, section "混合专家：更多参数，相同 FLOPs", and
+ * the moe_layer pseudocode of "开源混合架构大模型技术解析", section 四.)
+ *
+ * Conventions for every entry point:
+ *   - Pointers named as device pointers must point to memory of the current
+ *     CUDA device; the library reads or writes them only from kernels queued
+ *     on `stream` (a cudaStream_t passed as void*, NULL = legacy default
+ *     stream).  Calls are asynchronous unless stated otherwise: they return
+ *     after queueing work and never synchronise the stream.
+ *   - The caller owns every buffer.  The library allocates no device memory;
+ *     it keeps only per-process caches (kernel attributes).
+ *   - All matrices are row-major and contiguous.  Device pointers must be
+ *     16-byte aligned; `workspace` must be 256-byte aligned.
+ *   - Errors: invalid arguments are reported synchronously, before anything
+ *     is queued, as a negative moe_status.  A failed launch returns
+ *     MOE_ERR_CUDA.  Faults found on the device (a wait that ran out of time,
+ *     a bounds check) do not trap: the kernel records a code in the status
+ *     word at the start of the workspace, returns early, and the host reads
+ *     it with moe_get_device_status().
+ *   - T = 0 is valid and queues nothing.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+#define MOE_EXTERN extern "C"
+#else
+#define MOE_EXTERN extern
+#endif
+#define MOE_API MOE_EXTERN __attribute__((visibility("default")))
+
+typedef enum {
+    MOE_OK = 0,
+    MOE_ERR_INVALID_ARG = -1, /* a size, pointer or alignment check failed          */
+    MOE_ERR_UNSUPPORTED = -2, /* valid, but outside what the kernels implement      */
+    MOE_ERR_CUDA = -3,        /* a CUDA runtime call or kernel launch failed        */
+    MOE_ERR_WORKSPACE = -4,   /* workspace NULL or smaller than moe_workspace_bytes */
+    MOE_ERR_TIMEOUT = -5,     /* device: a bounded wait gave up                     */
+    MOE_ERR_DEVICE = -6       /* device: a bounds check failed                      */
+} moe_status;
+
+typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype;
+
+/*
+ * Shape limits checked by every entry point (else MOE_ERR_INVALID_ARG or
+ * MOE_ERR_UNSUPPORTED):
+ *   T >= 0, T * k < 2^31;  1 <= E <= 256;  1 <= n_group <= 32;
+ *   E % n_group == 0;  1 <= topk_group <= n_group;  1 <= k <= 8;
+ *   k <= topk_group * (E / n_group);
+ *   d % 64 == 0;  inter % 128 == 0;  0 <= n_shared;
+ *   bf16 path (moe_forward): d % 256 == 0 (output tiles of 256 columns).
+ */
+
+/*
+ * moe_workspace_bytes -- bytes of device workspace moe_forward needs for
+ * these sizes.  Host only, no CUDA calls.  Returns 0 for invalid sizes.
+ */
+MOE_API size_t moe_workspace_bytes(int T, int d, int E, int k, int inter, int n_shared,
+                                   int in_dt);
+
+/* Regions of the workspace (byte offsets from its start). */
+enum {
+    MOE_WS_STATUS = 0,       /* int32[64]: [0] status code, [1] where, [2..3] info     */
+    MOE_WS_COUNTS = 1,       /* int32[E]   tokens routed to each expert                */
+    MOE_WS_OFFSETS = 2,      /* int32[E+1] first row of each expert in the permuted
+                                layout; segments are padded to 128 rows              */
+    MOE_WS_BLOCK_COUNTS = 3, /* int32[ceil(T/256) * E] per-block histogram / bases     */
+    MOE_WS_TOPK_IDX = 4,     /* int32[T*k] chosen experts (used when no output given)  */
+    MOE_WS_TOPK_W = 5,       /* f32[T*k]   gate weights                               */
+    MOE_WS_ROW_SRC = 6,      /* int32[rows_cap] permuted row -> t*k + j, or -1 (pad)    */
+    MOE_WS_X_PERM = 7,       /* in_dt[rows_cap, d] x rows in expert-contiguous order    */
+    MOE_WS_H = 8,            /* in_dt[rows_cap, inter] silu(gate) * up, routed rows    */
+    MOE_WS_H_SHARED = 9,     /* in_dt[T, n_shared*inter] the same for shared experts   */
+    MOE_WS_SLOTS = 10,       /* f32[T*k, d] w_j * expert output, token order            */
+    MOE_WS_TOTAL = 11        /* total size                                            */
+};
+/* rows_cap = T*k + 128*E (the padded permuted layout never needs more). */
+
+/*
+ * moe_workspace_layout -- fill offsets[0..n-1] (n <= MOE_WS_TOTAL + 1) with
+ * the byte offsets of the regions above, offsets[MOE_WS_TOTAL] with the
+ * total.  Host only.  Returns MOE_OK or MOE_ERR_INVALID_ARG.
+ */
+MOE_API int moe_workspace_layout(int T, int d, int E, int k, int inter, int n_shared,
+                                 int in_dt, size_t *offsets, int n);
+
+/*
+ * moe_route -- routing only: router GEMM, sigmoid, group limit, top-k,
+ * normalisation.
+ *   x         device, in_dt[T, d]
+ *   W_router  device, in_dt[E, d]
+ *   topk_idx  device, int32[T, k] out: chosen experts, descending score,
+ *             ties to the lower index
+ *   topk_w    device, f32[T, k]   out: normalised gate weights (sum to 1)
+ * Logits accumulate in fp32; selection compares fp32 logits (sigmoid is
+ * monotone, so this is the same choice as comparing scores), weights are
+ * fp32 sigmoid values normalised over the chosen k.
+ */
+MOE_API int moe_route(const void *x, const void *W_router, int T, int d, int E, int k,
+                      int n_group, int topk_group, int in_dt, int32_t *topk_idx,
+                      float *topk_w, void *stream);
+
+/*
+ * moe_forward -- the whole layer.
+ *   x          device, in_dt[T, d]
+ *   W_router   device, in_dt[E, d]
+ *   W_gate_up  device, in_dt[E, 2*inter, d]: rows [0, inter) gate, [inter, 2*inter) up
+ *   W_down     device, in_dt[E, d, inter]
+ *   W_shared   device, in_dt: gate_up [2*S*inter, d] (the S gate blocks, then
+ *              the S up blocks) followed by down [d, S*inter]; NULL iff
+ *              n_shared == 0
+ *   y          device, out_dt[T, d] out
+ *   topk_idx_out, topk_w_out  device, optional (NULL = keep in workspace)
+ *   workspace  device, >= moe_workspace_bytes(...) bytes, 256-byte aligned;
+ *              its contents need no initialisation and are overwritten
+ * Arithmetic: in_dt inputs, fp32 accumulation everywhere; the SwiGLU hidden
+ * h is stored as in_dt between the two expert GEMMs; each routed expert's
+ * output is scaled by its gate weight in fp32 and the final sum is
+ * y = shared + slot_0 + ... + slot_{k-1} in that fixed order, so y is bitwise
+ * reproducible from run to run.  bf16 uses tcgen05 tensor cores; f32 uses
+ * CUDA cores.
+ */
+MOE_API int moe_forward(const void *x, const void *W_router, const void *W_gate_up,
+                        const void *W_down, const void *W_shared, int T, int d, int E, int k,
+                        int n_group, int topk_group, int inter, int n_shared, int in_dt,
+                        int out_dt, void *y, int32_t *topk_idx_out, float *topk_w_out,
+                        void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * moe_get_device_status -- synchronise `stream`, then copy the status word
+ * of `workspace` to *status (MOE_OK or a negative code) and, if `where` is
+ * not NULL, the code of the kernel site that set it.  Returns MOE_OK or
+ * MOE_ERR_CUDA.
+ */
+MOE_API int moe_get_device_status(const void *workspace, int *status, int *where,
+                                  void *stream);
+
+/* moe_clear_device_status -- queue a reset of the status word to MOE_OK. */
+MOE_API int moe_clear_device_status(void *workspace, void *stream);
+
+/*
+ * moe_selftest_timeout -- queue one kernel that waits on a barrier nothing
+ * will ever signal, with a limit of `limit_us` microseconds (1..1000000); when
+ * the limit runs out the kernel writes MOE_ERR_TIMEOUT into the status word of
+ * `workspace` and returns.  Exercises the bounded-wait path of the GEMM
+ * kernels without hanging the GPU.
+ */
+MOE_API int moe_selftest_timeout(void *workspace, int limit_us, void *stream);
+
+/*
+ * moe_set_stage_events -- optional instrumentation for benchmarks.  With
+ * events != NULL (n == MOE_N_STAGE_EVENTS handles of type cudaEvent_t, created
+ * by the caller), every following moe_forward in this process records
+ * events[i] on its stream: [0] start, [1] after routing, [2] after the
+ * permutation, [3] after the routed gate/up GEMM, [4] after the shared gate/up
+ * GEMM, [5] after the routed down GEMM, [6] at the end.  events == NULL turns
+ * it off.  Process-wide setting, not thread-safe.  Returns MOE_OK or
+ * MOE_ERR_INVALID_ARG.
+ */
+#define MOE_N_STAGE_EVENTS 7
+MOE_API int moe_set_stage_events(void *const *events, int n);
+
+/* moe_status_string -- static text for a status code. */
+MOE_API const char *moe_status_string(int status);
+
+/* moe_version -- ABI version of this header (1). */
+MOE_API int moe_version(void);
+
+#endif /* MOE_B200_H */

@@ -1,0 +1,374 @@
+// Grouped GEMM on the 5th-generation tensor cores (tcgen05, sm_100a), fed by
+// TMA, accumulating in tensor memory, with the MoE epilogues fused:
+//   EPI_SWIGLU   gate/up projection: one tile holds 128 gate rows and the 128
+//                matching up rows of B, so the epilogue sees both halves of
+//                SwiGLU for the same 128 output columns and writes
+//                h = silu(gate) * up as bf16 (SwiGLU: "大模型工程（一）：
+//                Transformer 到 MoE", section "变了什么，为什么变", item 3).
+//   EPI_SCATTER  down projection of the routed experts: each output row is
+//                scaled by its gate weight and written to the token-order
+//                slot (t, j) it came from (the weighted combine of the
+//                MoEBlock listing, section "混合专家：更多参数，相同 FLOPs").
+//   EPI_COMBINE  down projection of the shared experts, with the final sum
+//                y = shared + slot_0 + ... + slot_{k-1} in fixed order (the
+//                always-on shared experts: "FusionLLM：融合 MLA、GDN 与 MoE 的
+//                高效混合架构大模型训练框架", section "模型配置与规模").
+//
+// The grouped GEMM after routing is named as a fused kernel target on the
+// FusionLLM page (section "融合内核"); this is a fresh design for B200:
+//   - persistent CTAs (one per SM) walk a tile list built on the device from
+//     the per-expert row offsets: tile = (128-row block, N tile); the group
+//     (expert) of a row block is found by binary search in the offsets;
+//   - warp 0 issues TMA loads (128B swizzle, K-major boxes of 64 x 128) into a
+//     4-stage ring; warp 1 issues tcgen05.mma M=128 N=256 K=16 from one
+//     thread and commits to mbarriers; warps 2..5 drain the accumulator from
+//     TMEM (tcgen05.ld) and run the epilogue;
+//   - two 256-column fp32 accumulators (all 512 TMEM columns) let the
+//     epilogue of one tile overlap the main loop of the next;
+//   - every wait is bounded; a CTA that gives up records MOE_ERR_TIMEOUT in
+//     the status word, lets its other roles stop, drains its tensor-core work
+//     and frees TMEM before returning.
+// No cluster launch and no multicast loads.
+#include "moe_device.cuh"
+#include "moe_internal.h"
+
+namespace moe {
+
+namespace {
+
+constexpr int BM = 128;           // rows per tile (MMA M, TMEM lanes)
+constexpr int BK = 64;            // K per stage: one 128-byte swizzle atom of bf16
+constexpr int BNB = 256;          // B rows per tile (MMA N)
+constexpr int kStages = 4;
+constexpr int kABytes = BM * BK * 2;        // 16 KiB
+constexpr int kBBytes = BNB * BK * 2;       // 32 KiB
+constexpr int kStageBytes = kABytes + kBBytes;
+constexpr int kTmemCols = 512;              // 2 accumulators x 256 fp32 columns
+constexpr int kThreads = 192;               // 6 warps
+constexpr int kEpiThreads = 128;
+constexpr uint32_t kIdesc = idesc_bf16_f32(BM, BNB);
+constexpr int kMaxOffsets = kMaxE + 1;
+
+struct __align__(8) SmemTail {
+    uint64_t full[kStages];
+    uint64_t empty[kStages];
+    uint64_t tfull[2];
+    uint64_t tempty[2];
+    uint64_t drain;
+    uint32_t tmem_base;
+    int abort;
+    int offsets[kMaxOffsets];
+};
+
+constexpr size_t kSmemBytes = 1024 /*alignment slack*/ + (size_t)kStages * kStageBytes +
+                              sizeof(SmemTail);
+
+__device__ __forceinline__ int find_group(const int* off, int n_groups, int row) {
+    int lo = 0, hi = n_groups - 1;
+    while (lo < hi) {
+        int mid = (lo + hi + 1) >> 1;
+        if (off[mid] <= row)
+            lo = mid;
+        else
+            hi = mid - 1;
+    }
+    return lo;
+}
+
+__device__ __forceinline__ float silu_mul(float g, float u) {
+    return __fdividef(g, 1.0f + __expf(-g)) * u;
+}
+
+template <int EPI>
+__global__ void __launch_bounds__(kThreads, 1)
+    grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
+                           const __grid_constant__ CUtensorMap tmB, const GemmArgs args) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    SmemTail* tail = reinterpret_cast<SmemTail*>(smem + (size_t)kStages * kStageBytes);
+    volatile int* abort_flag = &tail->abort;
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int n_groups = args.offsets != nullptr ? args.n_groups : 1;
+
+    if (tid == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&tail->full[s], 1);
+            mbar_init(&tail->empty[s], 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(&tail->tfull[a], 1);
+            mbar_init(&tail->tempty[a], kEpiThreads);
+        }
+        mbar_init(&tail->drain, 1);
+        tail->abort = 0;
+        fence_barrier_init();
+    }
+    if (args.offsets != nullptr) {
+        for (int i = tid; i <= n_groups; i += kThreads) tail->offsets[i] = args.offsets[i];
+    } else if (tid == 0) {
+        tail->offsets[0] = 0;
+        tail->offsets[1] = (args.static_rows + BM - 1) / BM * BM;
+    }
+    if (warp == 1) {
+        tmem_alloc(&tail->tmem_base, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+
+    const uint32_t tmem_base = tail->tmem_base;
+    const int total_rows = tail->offsets[n_groups];
+    const int total_tiles = (total_rows / BM) * args.n_tiles;
+    const int kb_count = args.K / BK;
+    const uint64_t limit = args.wait_limit_ns;
+
+    if (warp == 0) {
+        // ------------------------------------------------ TMA producer
+        if (lane == 0) {
+            tma_prefetch_desc(&tmA);
+            tma_prefetch_desc(&tmB);
+            int s = 0;
+            uint32_t ph = 0;
+            bool ok = true;
+            uint32_t issued = 0, issued_ph = 0;  // per stage: loaded at least once / parity
+            for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x) {
+                const int mblk = tile / args.n_tiles, nt = tile % args.n_tiles;
+                const int row0 = mblk * BM;
+                const int g = find_group(tail->offsets, n_groups, row0);
+                const int b0 = (int)(g * args.b_group_stride) + nt * args.b_tile_step;
+                const int b1 = b0 + args.b_half_off;
+                for (int kb = 0; kb < kb_count; ++kb) {
+                    if (!mbar_wait_bounded(&tail->empty[s], ph ^ 1u, abort_flag, args.status,
+                                           SITE_GEMM_PRODUCER, limit)) {
+                        ok = false;
+                        break;
+                    }
+                    uint8_t* sa = smem + (size_t)s * kStageBytes;
+                    uint8_t* sb = sa + kABytes;
+                    mbar_arrive_expect_tx(&tail->full[s], kStageBytes);
+                    tma_load_2d(sa, &tmA, &tail->full[s], kb * BK, row0);
+                    tma_load_2d(sb, &tmB, &tail->full[s], kb * BK, b0);
+                    tma_load_2d(sb + kBBytes / 2, &tmB, &tail->full[s], kb * BK, b1);
+                    issued |= 1u << s;
+                    issued_ph = (issued_ph & ~(1u << s)) | (ph << s);
+                    if (++s == kStages) {
+                        s = 0;
+                        ph ^= 1u;
+                    }
+                }
+            }
+            if (!ok) {
+                // let copies already in flight land before the CTA goes away
+                for (int i = 0; i < kStages; ++i)
+                    if ((issued >> i) & 1u)
+                        mbar_wait_bounded(&tail->full[i], (issued_ph >> i) & 1u, nullptr,
+                                          nullptr, 0, limit);
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            int s = 0;
+            uint32_t ph = 0;
+            int it = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x, ++it) {
+                const int acc = it & 1;
+                const uint32_t aph = (it >> 1) & 1;
+                if (!mbar_wait_bounded(&tail->tempty[acc], aph ^ 1u, abort_flag, args.status,
+                                       SITE_GEMM_MMA, limit)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BNB);
+                for (int kb = 0; kb < kb_count; ++kb) {
+                    if (!mbar_wait_bounded(&tail->full[s], ph, abort_flag, args.status,
+                                           SITE_GEMM_MMA, limit)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t a_addr = smem_u32(smem + (size_t)s * kStageBytes);
+                    const uint32_t b_addr = a_addr + kABytes;
+#pragma unroll
+                    for (int kk = 0; kk < BK / 16; ++kk) {
+                        const uint64_t ad = sw128_kmajor_desc(a_addr + kk * 32);
+                        const uint64_t bd = sw128_kmajor_desc(b_addr + kk * 32);
+                        tc_mma_f16(d_tmem, ad, bd, kIdesc, (kb | kk) != 0 ? 1u : 0u);
+                    }
+                    tc_commit(&tail->empty[s]);
+                    if (++s == kStages) {
+                        s = 0;
+                        ph ^= 1u;
+                    }
+                }
+                if (!ok) break;
+                tc_commit(&tail->tfull[acc]);
+            }
+            // all tensor-core work of this CTA is complete once `drain` fires
+            tc_commit(&tail->drain);
+            mbar_wait_bounded(&tail->drain, 0u, nullptr, args.status, SITE_GEMM_DRAIN, limit);
+        }
+    } else {
+        // ------------------------------------------------ epilogue (warps 2..5)
+        const int wq = warp & 3;  // TMEM lane quarter this warp may access
+        const int r_local = wq * 32 + lane;
+        int it = 0;
+        for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x, ++it) {
+            const int acc = it & 1;
+            const uint32_t aph = (it >> 1) & 1;
+            const bool got = mbar_wait_bounded(&tail->tfull[acc], aph, abort_flag, args.status,
+                                               SITE_GEMM_EPILOGUE, limit);
+            // tcgen05.ld below is warp-collective: leave together or not at all
+            if (!__all_sync(0xffffffffu, got)) break;
+            tc_fence_after();
+            const int mblk = tile / args.n_tiles, nt = tile % args.n_tiles;
+            const int grow = mblk * BM + r_local;
+            const uint32_t taddr =
+                tmem_base + (uint32_t)(acc * BNB) + ((uint32_t)(wq * 32) << 16);
+            const int col0 = nt * args.out_col_step;
+
+            if constexpr (EPI == EPI_SWIGLU) {
+                const bool valid = grow < args.valid_rows;
+                __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(args.out) +
+                                      (size_t)grow * args.out_ld + col0;
+#pragma unroll 1
+                for (int c = 0; c < BNB / 2; c += 32) {
+                    uint32_t g[32], u[32];
+                    tmem_ld32(taddr + c, g);
+                    tmem_ld32(taddr + BNB / 2 + c, u);
+                    tmem_ld_wait();
+                    uint32_t p[16];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i)
+                        p[i] = pack_bf16x2(
+                            silu_mul(__uint_as_float(g[2 * i]), __uint_as_float(u[2 * i])),
+                            silu_mul(__uint_as_float(g[2 * i + 1]),
+                                     __uint_as_float(u[2 * i + 1])));
+                    if (valid) {
+                        uint4* dst = reinterpret_cast<uint4*>(orow + c);
+#pragma unroll
+                        for (int q = 0; q < 4; ++q)
+                            dst[q] = make_uint4(p[4 * q], p[4 * q + 1], p[4 * q + 2], p[4 * q + 3]);
+                    }
+                }
+            } else if constexpr (EPI == EPI_SCATTER) {
+                const int src = grow < args.valid_rows ? args.row_src[grow] : -1;
+                const float wv = src >= 0 ? args.topk_w[src] : 0.f;
+                float* orow = static_cast<float*>(args.out) + (size_t)(src >= 0 ? src : 0) *
+                                                                  args.out_ld + col0;
+#pragma unroll 1
+                for (int c = 0; c < BNB; c += 32) {
+                    uint32_t v[32];
+                    tmem_ld32(taddr + c, v);
+                    tmem_ld_wait();
+                    if (src >= 0) {
+                        float4* dst = reinterpret_cast<float4*>(orow + c);
+#pragma unroll
+                        for (int q = 0; q < 8; ++q)
+                            dst[q] = make_float4(wv * __uint_as_float(v[4 * q]),
+                                                 wv * __uint_as_float(v[4 * q + 1]),
+                                                 wv * __uint_as_float(v[4 * q + 2]),
+                                                 wv * __uint_as_float(v[4 * q + 3]));
+                    }
+                }
+            } else {  // EPI_COMBINE
+                const bool valid = grow < args.valid_rows;
+                const size_t t = valid ? (size_t)grow : 0;
+#pragma unroll 1
+                for (int c = 0; c < BNB; c += 32) {
+                    uint32_t v[32];
+                    tmem_ld32(taddr + c, v);
+                    tmem_ld_wait();
+                    if (valid) {
+                        float a[32];
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) a[i] = __uint_as_float(v[i]);
+                        for (int j = 0; j < args.k; ++j) {
+                            const float4* sp = reinterpret_cast<const float4*>(
+                                args.slots + (t * args.k + j) * args.out_ld + col0 + c);
+#pragma unroll
+                            for (int q = 0; q < 8; ++q) {
+                                float4 b = __ldg(sp + q);
+                                a[4 * q] += b.x;
+                                a[4 * q + 1] += b.y;
+                                a[4 * q + 2] += b.z;
+                                a[4 * q + 3] += b.w;
+                            }
+                        }
+                        if (args.out_f32) {
+                            float4* dst = reinterpret_cast<float4*>(
+                                static_cast<float*>(args.out) + t * args.out_ld + col0 + c);
+#pragma unroll
+                            for (int q = 0; q < 8; ++q)
+                                dst[q] = make_float4(a[4 * q], a[4 * q + 1], a[4 * q + 2],
+                                                     a[4 * q + 3]);
+                        } else {
+                            uint4* dst = reinterpret_cast<uint4*>(
+                                static_cast<__nv_bfloat16*>(args.out) + t * args.out_ld + col0 + c);
+#pragma unroll
+                            for (int q = 0; q < 4; ++q)
+                                dst[q] = make_uint4(pack_bf16x2(a[8 * q], a[8 * q + 1]),
+                                                    pack_bf16x2(a[8 * q + 2], a[8 * q + 3]),
+                                                    pack_bf16x2(a[8 * q + 4], a[8 * q + 5]),
+                                                    pack_bf16x2(a[8 * q + 6], a[8 * q + 7]));
+                        }
+                    }
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(&tail->tempty[acc]);
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem_base, kTmemCols);
+}
+
+// A kernel that waits on a barrier nothing signals, to exercise the bounded
+// wait and the status report without hanging anything.
+__global__ void selftest_timeout_kernel(int* status, unsigned long long limit_ns) {
+    __shared__ uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        abort_flag = 0;
+        fence_barrier_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0)
+        mbar_wait_bounded(&bar, 0u, &abort_flag, status, SITE_SELFTEST, limit_ns);
+}
+
+}  // namespace
+
+size_t gemm_tc_smem_bytes() { return kSmemBytes; }
+
+cudaError_t launch_gemm_tc(int epi, const CUtensorMap& tmA, const CUtensorMap& tmB,
+                           const GemmArgs& a, int grid, cudaStream_t s) {
+    void (*kern)(const CUtensorMap, const CUtensorMap, const GemmArgs) = nullptr;
+    switch (epi) {
+        case EPI_SWIGLU: kern = grouped_gemm_tc_kernel<EPI_SWIGLU>; break;
+        case EPI_SCATTER: kern = grouped_gemm_tc_kernel<EPI_SCATTER>; break;
+        case EPI_COMBINE: kern = grouped_gemm_tc_kernel<EPI_COMBINE>; break;
+        default: return cudaErrorInvalidValue;
+    }
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)kSmemBytes);
+    if (e != cudaSuccess) return e;
+    kern<<<grid, kThreads, kSmemBytes, s>>>(tmA, tmB, a);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_selftest_timeout(int* status, unsigned long long limit_ns, cudaStream_t s) {
+    selftest_timeout_kernel<<<1, 32, 0, s>>>(status, limit_ns);
+    return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,456 @@
+// C ABI of the MoE layer forward: argument checks, workspace layout, TMA
+// descriptors and the launch sequence
+//   route -> permute (histogram, scan, rank) -> gather rows
+//   -> gate/up grouped GEMM + SwiGLU (routed; shared)
+//   -> down grouped GEMM with weighted scatter to token-order slots (routed)
+//   -> down GEMM of the shared experts with the fixed-order final sum.
+// Everything runs on the caller's stream; nothing here synchronises it except
+// moe_get_device_status, and nothing here allocates device memory.
+#include <cudaTypedefs.h>
+#include <limits.h>
+#include <string.h>
+
+#include "../../include/moe.h"
+#include "moe_internal.h"
+
+namespace {
+
+using namespace moe;
+
+constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s per wait
+constexpr size_t kRegionAlign = 1024;
+
+struct Layout {
+    size_t off[MOE_WS_TOTAL + 1];
+    int rows_cap;
+    int nb;
+};
+
+size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+int check_sizes(int T, int d, int E, int k, int inter, int n_shared, int in_dt) {
+    if (T < 0 || d <= 0 || E < 1 || E > kMaxE || k < 1 || k > kMaxK || inter <= 0 ||
+        n_shared < 0)
+        return MOE_ERR_INVALID_ARG;
+    if (in_dt != MOE_F32 && in_dt != MOE_BF16) return MOE_ERR_INVALID_ARG;
+    if (k > E) return MOE_ERR_INVALID_ARG;
+    if ((long long)T * k + 128LL * E >= (long long)INT_MAX) return MOE_ERR_INVALID_ARG;
+    if (d % 64 != 0 || inter % 128 != 0) return MOE_ERR_UNSUPPORTED;
+    return MOE_OK;
+}
+
+int check_routing(int E, int k, int n_group, int topk_group) {
+    if (n_group < 1 || n_group > kMaxGroups || E % n_group != 0) return MOE_ERR_INVALID_ARG;
+    if (topk_group < 1 || topk_group > n_group) return MOE_ERR_INVALID_ARG;
+    if (k > topk_group * (E / n_group)) return MOE_ERR_INVALID_ARG;
+    return MOE_OK;
+}
+
+bool make_layout(int T, int d, int E, int k, int inter, int n_shared, int in_dt, Layout& L) {
+    if (check_sizes(T, d, E, k, inter, n_shared, in_dt) != MOE_OK) return false;
+    const size_t esz = in_dt == MOE_BF16 ? 2 : 4;
+    const size_t Tk = (size_t)T * k;
+    L.rows_cap = (int)(Tk + (size_t)kRowAlign * E);
+    L.nb = (T + kPermBlockTokens - 1) / kPermBlockTokens;
+    const size_t sizes[MOE_WS_TOTAL] = {
+        sizeof(int) * kStatusWords,                     // STATUS
+        sizeof(int) * E,                                // COUNTS
+        sizeof(int) * (E + 1),                          // OFFSETS
+        sizeof(int) * (size_t)(L.nb > 0 ? L.nb : 1) * E,  // BLOCK_COUNTS
+        sizeof(int) * Tk,                               // TOPK_IDX
+        sizeof(float) * Tk,                             // TOPK_W
+        sizeof(int) * (size_t)L.rows_cap,               // ROW_SRC
+        esz * (size_t)L.rows_cap * d,                   // X_PERM
+        esz * (size_t)L.rows_cap * inter,               // H
+        esz * (size_t)T * n_shared * inter,             // H_SHARED
+        sizeof(float) * Tk * d,                         // SLOTS
+    };
+    size_t o = 0;
+    for (int i = 0; i < MOE_WS_TOTAL; ++i) {
+        L.off[i] = o;
+        o = align_up(o + sizes[i], kRegionAlign);
+    }
+    L.off[MOE_WS_TOTAL] = o;
+    return true;
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// Host-side check that p is memory the device can address (device or managed
+// allocation).  Catches host pointers before any kernel could dereference them.
+bool is_device_ptr(const void* p) {
+    if (p == nullptr) return false;
+    cudaPointerAttributes at;
+    if (cudaPointerGetAttributes(&at, p) != cudaSuccess) {
+        cudaGetLastError();
+        return false;
+    }
+    return at.type == cudaMemoryTypeDevice || at.type == cudaMemoryTypeManaged;
+}
+
+int num_sms() {
+    static int cached[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+    if (dev < 0 || dev >= 64) return 148;
+    if (cached[dev] == 0) {
+        int n = 0;
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        cached[dev] = n > 0 ? n : 148;
+    }
+    return cached[dev];
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static bool tried = false;
+    if (!tried) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+        tried = true;
+    }
+    return fn;
+}
+
+// bf16 matrix [rows, cols] row-major, TMA box of 64 columns x 128 rows, 128B swizzle.
+bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols) {
+    auto fn = encode_fn();
+    if (fn == nullptr || rows == 0) return false;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {cols * 2};
+    cuuint32_t box[2] = {64, 128};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+int ret(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+template <typename T>
+T* at(void* ws, const Layout& L, int region) {
+    return reinterpret_cast<T*>(static_cast<char*>(ws) + L.off[region]);
+}
+
+cudaEvent_t g_stage_events[MOE_N_STAGE_EVENTS];
+bool g_stage_events_on = false;
+
+void stage_mark(int i, cudaStream_t s) {
+    if (g_stage_events_on) cudaEventRecord(g_stage_events[i], s);
+}
+
+int grid_for(long long tiles) {
+    const int n = num_sms();
+    return (int)(tiles < n ? (tiles > 0 ? tiles : 1) : n);
+}
+
+}  // namespace
+
+extern "C" {
+
+MOE_API int moe_version(void) { return 1; }
+
+MOE_API const char* moe_status_string(int status) {
+    switch (status) {
+        case MOE_OK: return "ok";
+        case MOE_ERR_INVALID_ARG: return "invalid argument";
+        case MOE_ERR_UNSUPPORTED: return "unsupported shape or dtype";
+        case MOE_ERR_CUDA: return "CUDA error";
+        case MOE_ERR_WORKSPACE: return "workspace missing or too small";
+        case MOE_ERR_TIMEOUT: return "device wait timed out";
+        case MOE_ERR_DEVICE: return "device bounds check failed";
+        default: return "unknown status";
+    }
+}
+
+MOE_API size_t moe_workspace_bytes(int T, int d, int E, int k, int inter, int n_shared,
+                                   int in_dt) {
+    Layout L;
+    if (!make_layout(T, d, E, k, inter, n_shared, in_dt, L)) return 0;
+    return L.off[MOE_WS_TOTAL];
+}
+
+MOE_API int moe_workspace_layout(int T, int d, int E, int k, int inter, int n_shared, int in_dt,
+                                 size_t* offsets, int n) {
+    Layout L;
+    if (offsets == nullptr || n < 1 || n > MOE_WS_TOTAL + 1) return MOE_ERR_INVALID_ARG;
+    if (!make_layout(T, d, E, k, inter, n_shared, in_dt, L)) return MOE_ERR_INVALID_ARG;
+    for (int i = 0; i < n; ++i) offsets[i] = L.off[i];
+    return MOE_OK;
+}
+
+MOE_API int moe_route(const void* x, const void* W_router, int T, int d, int E, int k,
+                      int n_group, int topk_group, int in_dt, int32_t* topk_idx, float* topk_w,
+                      void* stream) {
+    int st = check_sizes(T, d, E, k, 128, 0, in_dt);
+    if (st != MOE_OK) return st;
+    st = check_routing(E, k, n_group, topk_group);
+    if (st != MOE_OK) return st;
+    if (T == 0) return MOE_OK;
+    if (!is_device_ptr(x) || !is_device_ptr(W_router) || !is_device_ptr(topk_idx) ||
+        !is_device_ptr(topk_w))
+        return MOE_ERR_INVALID_ARG;
+    if (!aligned(x, 16) || !aligned(W_router, 16) || !aligned(topk_idx, 4) ||
+        !aligned(topk_w, 4))
+        return MOE_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (in_dt == MOE_BF16)
+        return ret(launch_route_bf16(x, W_router, T, d, E, k, n_group, topk_group, topk_idx,
+                                     topk_w, nullptr, s));
+    return ret(launch_route_f32(x, W_router, T, d, E, k, n_group, topk_group, topk_idx, topk_w,
+                                nullptr, s));
+}
+
+MOE_API int moe_forward(const void* x, const void* W_router, const void* W_gate_up,
+                        const void* W_down, const void* W_shared, int T, int d, int E, int k,
+                        int n_group, int topk_group, int inter, int n_shared, int in_dt,
+                        int out_dt, void* y, int32_t* topk_idx_out, float* topk_w_out,
+                        void* workspace, size_t workspace_bytes, void* stream) {
+    int st = check_sizes(T, d, E, k, inter, n_shared, in_dt);
+    if (st != MOE_OK) return st;
+    st = check_routing(E, k, n_group, topk_group);
+    if (st != MOE_OK) return st;
+    if (out_dt != MOE_F32 && out_dt != MOE_BF16) return MOE_ERR_INVALID_ARG;
+    if (in_dt == MOE_BF16 && d % 256 != 0) return MOE_ERR_UNSUPPORTED;
+    if ((n_shared > 0) != (W_shared != nullptr)) return MOE_ERR_INVALID_ARG;
+    Layout L;
+    make_layout(T, d, E, k, inter, n_shared, in_dt, L);
+    if (workspace == nullptr || workspace_bytes < L.off[MOE_WS_TOTAL]) return MOE_ERR_WORKSPACE;
+    if (T == 0) return MOE_OK;
+    const void* dev_ptrs[] = {x, W_router, W_gate_up, W_down, y, workspace};
+    for (const void* p : dev_ptrs)
+        if (!is_device_ptr(p) || !aligned(p, 16)) return MOE_ERR_INVALID_ARG;
+    if (n_shared > 0 && (!is_device_ptr(W_shared) || !aligned(W_shared, 16)))
+        return MOE_ERR_INVALID_ARG;
+    if (!aligned(workspace, 256)) return MOE_ERR_INVALID_ARG;
+    if ((topk_idx_out != nullptr && (!is_device_ptr(topk_idx_out) || !aligned(topk_idx_out, 4))) ||
+        (topk_w_out != nullptr && (!is_device_ptr(topk_w_out) || !aligned(topk_w_out, 4))))
+        return MOE_ERR_INVALID_ARG;
+
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    int* status = at<int>(workspace, L, MOE_WS_STATUS);
+    int32_t* idx = topk_idx_out != nullptr ? topk_idx_out : at<int32_t>(workspace, L, MOE_WS_TOPK_IDX);
+    float* w = topk_w_out != nullptr ? topk_w_out : at<float>(workspace, L, MOE_WS_TOPK_W);
+    int32_t* counts = at<int32_t>(workspace, L, MOE_WS_COUNTS);
+    int32_t* offsets = at<int32_t>(workspace, L, MOE_WS_OFFSETS);
+    int32_t* block_counts = at<int32_t>(workspace, L, MOE_WS_BLOCK_COUNTS);
+    int32_t* row_src = at<int32_t>(workspace, L, MOE_WS_ROW_SRC);
+    void* x_perm = at<char>(workspace, L, MOE_WS_X_PERM);
+    void* h = at<char>(workspace, L, MOE_WS_H);
+    void* h_sh = at<char>(workspace, L, MOE_WS_H_SHARED);
+    float* slots = at<float>(workspace, L, MOE_WS_SLOTS);
+    const int SI = n_shared * inter;
+    const bool bf16 = in_dt == MOE_BF16;
+    const int out_f32 = out_dt == MOE_F32 ? 1 : 0;
+
+    stage_mark(0, s);
+    // 1. routing (also resets the status word)
+    cudaError_t e = bf16 ? launch_route_bf16(x, W_router, T, d, E, k, n_group, topk_group, idx, w,
+                                             status, s)
+                         : launch_route_f32(x, W_router, T, d, E, k, n_group, topk_group, idx, w,
+                                            status, s);
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
+    stage_mark(1, s);
+    // 2. permutation: histogram, scan, stable ranks, row gather
+    e = launch_permute(idx, T, k, E, block_counts, counts, offsets, row_src, status, s);
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
+    e = launch_gather_rows(x, d, bf16 ? 2 : 4, k, offsets + E, row_src, L.rows_cap, x_perm,
+                           num_sms(), s);
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
+    stage_mark(2, s);
+
+    GemmArgs g1{};
+    g1.K = d;
+    g1.n_groups = E;
+    g1.offsets = offsets;
+    g1.b_group_stride = 2LL * inter;
+    g1.b_half_off = inter;
+    g1.valid_rows = INT_MAX;
+    g1.out = h;
+    g1.out_ld = inter;
+    g1.out_f32 = bf16 ? 0 : 1;
+    g1.status = status;
+    g1.wait_limit_ns = kWaitLimitNs;
+
+    GemmArgs g1s = g1;
+    g1s.offsets = nullptr;
+    g1s.n_groups = 1;
+    g1s.static_rows = T;
+    g1s.b_group_stride = 0;
+    g1s.b_half_off = SI;
+    g1s.valid_rows = T;
+    g1s.out = h_sh;
+    g1s.out_ld = SI;
+
+    GemmArgs g2{};
+    g2.K = inter;
+    g2.n_groups = E;
+    g2.offsets = offsets;
+    g2.b_group_stride = d;
+    g2.valid_rows = INT_MAX;
+    g2.out = slots;
+    g2.out_ld = d;
+    g2.row_src = row_src;
+    g2.topk_w = w;
+    g2.k = k;
+    g2.status = status;
+    g2.wait_limit_ns = kWaitLimitNs;
+
+    GemmArgs g2s = g2;
+    g2s.K = SI;
+    g2s.offsets = nullptr;
+    g2s.n_groups = 1;
+    g2s.static_rows = T;
+    g2s.b_group_stride = 0;
+    g2s.valid_rows = T;
+    g2s.out = y;
+    g2s.slots = slots;
+    g2s.out_f32 = out_f32;
+
+    const char* Wsh_gu = static_cast<const char*>(W_shared);
+    const char* Wsh_dn = Wsh_gu == nullptr ? nullptr
+                                           : Wsh_gu + (size_t)2 * SI * d * (bf16 ? 2 : 4);
+
+    if (bf16) {
+        const int rows_tiles = L.rows_cap / 128;
+        // 3. gate/up + SwiGLU, routed experts
+        g1.n_tiles = inter / 128;
+        g1.b_tile_step = 128;
+        g1.out_col_step = 128;
+        CUtensorMap tA, tB;
+        if (!make_map(&tA, x_perm, (uint64_t)L.rows_cap, d) ||
+            !make_map(&tB, W_gate_up, (uint64_t)E * 2 * inter, d))
+            return MOE_ERR_CUDA;
+        e = launch_gemm_tc(EPI_SWIGLU, tA, tB, g1, grid_for((long long)rows_tiles * g1.n_tiles), s);
+        if (e != cudaSuccess) return MOE_ERR_CUDA;
+        stage_mark(3, s);
+        // 4. gate/up + SwiGLU, shared experts (all tokens)
+        if (n_shared > 0) {
+            g1s.n_tiles = SI / 128;
+            g1s.b_tile_step = 128;
+            g1s.out_col_step = 128;
+            if (!make_map(&tA, x, (uint64_t)T, d) || !make_map(&tB, Wsh_gu, (uint64_t)2 * SI, d))
+                return MOE_ERR_CUDA;
+            e = launch_gemm_tc(EPI_SWIGLU, tA, tB, g1s,
+                               grid_for((long long)((T + 127) / 128) * g1s.n_tiles), s);
+            if (e != cudaSuccess) return MOE_ERR_CUDA;
+        }
+        stage_mark(4, s);
+        // 5. down projection, routed: weighted scatter into token-order slots
+        g2.n_tiles = d / 256;
+        g2.b_tile_step = 256;
+        g2.b_half_off = 128;
+        g2.out_col_step = 256;
+        if (!make_map(&tA, h, (uint64_t)L.rows_cap, inter) ||
+            !make_map(&tB, W_down, (uint64_t)E * d, inter))
+            return MOE_ERR_CUDA;
+        e = launch_gemm_tc(EPI_SCATTER, tA, tB, g2, grid_for((long long)rows_tiles * g2.n_tiles), s);
+        if (e != cudaSuccess) return MOE_ERR_CUDA;
+        stage_mark(5, s);
+        // 6. down projection, shared, with the final fixed-order sum
+        if (n_shared > 0) {
+            g2s.n_tiles = d / 256;
+            g2s.b_tile_step = 256;
+            g2s.b_half_off = 128;
+            g2s.out_col_step = 256;
+            if (!make_map(&tA, h_sh, (uint64_t)T, SI) || !make_map(&tB, Wsh_dn, (uint64_t)d, SI))
+                return MOE_ERR_CUDA;
+            e = launch_gemm_tc(EPI_COMBINE, tA, tB, g2s,
+                               grid_for((long long)((T + 127) / 128) * g2s.n_tiles), s);
+            if (e != cudaSuccess) return MOE_ERR_CUDA;
+        } else {
+            e = launch_combine_slots(slots, T, d, k, y, out_f32, s);
+            if (e != cudaSuccess) return MOE_ERR_CUDA;
+        }
+        stage_mark(6, s);
+        return MOE_OK;
+    }
+
+    // fp32: CUDA-core grouped GEMMs, 64-column output tiles
+    const float* Wgu = static_cast<const float*>(W_gate_up);
+    const float* Wdn = static_cast<const float*>(W_down);
+    g1.n_tiles = inter / 64;
+    g1.b_tile_step = 64;
+    g1.out_col_step = 64;
+    e = launch_gemm_simt(EPI_SWIGLU, static_cast<const float*>(x_perm), Wgu, g1, L.rows_cap, s);
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
+    stage_mark(3, s);
+    if (n_shared > 0) {
+        g1s.n_tiles = SI / 64;
+        g1s.b_tile_step = 64;
+        g1s.out_col_step = 64;
+        e = launch_gemm_simt(EPI_SWIGLU, static_cast<const float*>(x),
+                             reinterpret_cast<const float*>(Wsh_gu), g1s,
+                             (T + 127) / 128 * 128, s);
+        if (e != cudaSuccess) return MOE_ERR_CUDA;
+    }
+    stage_mark(4, s);
+    g2.n_tiles = d / 64;
+    g2.b_tile_step = 64;
+    g2.b_half_off = 0;
+    g2.out_col_step = 64;
+    e = launch_gemm_simt(EPI_SCATTER, static_cast<const float*>(h), Wdn, g2, L.rows_cap, s);
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
+    stage_mark(5, s);
+    if (n_shared > 0) {
+        g2s.n_tiles = d / 64;
+        g2s.b_tile_step = 64;
+        g2s.b_half_off = 0;
+        g2s.out_col_step = 64;
+        e = launch_gemm_simt(EPI_COMBINE, static_cast<const float*>(h_sh),
+                             reinterpret_cast<const float*>(Wsh_dn), g2s,
+                             (T + 127) / 128 * 128, s);
+    } else {
+        e = launch_combine_slots(slots, T, d, k, y, out_f32, s);
+    }
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
+    stage_mark(6, s);
+    return MOE_OK;
+}
+
+MOE_API int moe_set_stage_events(void* const* events, int n) {
+    if (events == nullptr) {
+        g_stage_events_on = false;
+        return MOE_OK;
+    }
+    if (n != MOE_N_STAGE_EVENTS) return MOE_ERR_INVALID_ARG;
+    for (int i = 0; i < n; ++i) {
+        if (events[i] == nullptr) return MOE_ERR_INVALID_ARG;
+        g_stage_events[i] = static_cast<cudaEvent_t>(events[i]);
+    }
+    g_stage_events_on = true;
+    return MOE_OK;
+}
+
+MOE_API int moe_get_device_status(const void* workspace, int* status, int* where, void* stream) {
+    if (workspace == nullptr || status == nullptr) return MOE_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    int buf[2] = {0, 0};
+    if (cudaMemcpyAsync(buf, workspace, sizeof(buf), cudaMemcpyDeviceToHost, s) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return MOE_ERR_CUDA;
+    *status = buf[0];
+    if (where != nullptr) *where = buf[1];
+    return MOE_OK;
+}
+
+MOE_API int moe_clear_device_status(void* workspace, void* stream) {
+    if (workspace == nullptr) return MOE_ERR_INVALID_ARG;
+    return ret(cudaMemsetAsync(workspace, 0, sizeof(int) * kStatusWords,
+                               static_cast<cudaStream_t>(stream)));
+}
+
+MOE_API int moe_selftest_timeout(void* workspace, int limit_us, void* stream) {
+    if (workspace == nullptr || limit_us < 1 || limit_us > 1000000) return MOE_ERR_INVALID_ARG;
+    if (!is_device_ptr(workspace)) return MOE_ERR_INVALID_ARG;
+    return ret(launch_selftest_timeout(static_cast<int*>(workspace),
+                                       (unsigned long long)limit_us * 1000ull,
+                                       static_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"

@@ -1,0 +1,76 @@
+// Host-side declarations shared by the .cu files of the library (launchers
+// and argument structs).  Not part of the public ABI.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace moe {
+
+constexpr int kMaxE = 256;
+constexpr int kMaxGroups = 32;
+constexpr int kMaxK = 8;
+constexpr int kRowAlign = 128;         // expert segments of the permuted layout are padded to this
+constexpr int kPermBlockTokens = 256;  // tokens per block of the permutation kernels
+constexpr int kStatusWords = 64;       // int32 words of the status region of the workspace
+
+// Epilogue variants of the grouped GEMMs.
+enum Epi : int {
+    EPI_SWIGLU = 0,   // out = bf16/f32 silu(gate) * up, columns [nt*cols, ...)
+    EPI_SCATTER = 1,  // slots[row_src[r]] = topk_w[row_src[r]] * acc  (rows with row_src < 0 skipped)
+    EPI_COMBINE = 2,  // y[t] = acc + slots[t*k + 0] + ... + slots[t*k + k-1]
+};
+
+// One grouped GEMM  out[r, n] = sum_c A[r, c] * B[b_row(r, n), c]  over row
+// groups.  Rows of group g are [off[g], off[g+1]) of A (a multiple of 128
+// rows each); with offsets == nullptr there is one group of static_rows rows.
+struct GemmArgs {
+    int K;                 // reduction length
+    int n_tiles;           // output tiles along N per group
+    int n_groups;          // groups (experts); ignored when offsets == nullptr
+    const int32_t* offsets;
+    int static_rows;
+    long long b_group_stride;  // B rows between consecutive groups
+    int b_tile_step;           // B rows between consecutive N tiles
+    int b_half_off;            // B row offset of the second half of a tile's B rows
+    int valid_rows;            // SWIGLU/COMBINE: rows >= valid_rows are not stored
+    void* out;
+    int out_ld;                // elements per output row
+    int out_col_step;          // output columns per N tile
+    const int32_t* row_src;    // SCATTER
+    const float* topk_w;       // SCATTER
+    const float* slots;        // COMBINE
+    int k;                     // SCATTER/COMBINE
+    int out_f32;               // COMBINE: y dtype (1 f32, 0 bf16); SWIGLU f32 path: 1
+    int* status;
+    unsigned long long wait_limit_ns;
+};
+
+// ---- launchers (return a cudaError_t from the launch)
+cudaError_t launch_route_bf16(const void* x, const void* Wr, int T, int d, int E, int k, int G,
+                              int TG, int32_t* idx, float* w, int* status, cudaStream_t s);
+cudaError_t launch_route_f32(const void* x, const void* Wr, int T, int d, int E, int k, int G,
+                             int TG, int32_t* idx, float* w, int* status, cudaStream_t s);
+
+cudaError_t launch_permute(const int32_t* idx, int T, int k, int E, int32_t* block_counts,
+                           int32_t* counts, int32_t* offsets, int32_t* row_src, int* status,
+                           cudaStream_t s);
+cudaError_t launch_gather_rows(const void* x, int d, int elem_bytes, int k,
+                               const int32_t* offsets_total, const int32_t* row_src,
+                               int rows_cap, void* x_perm, int num_sms, cudaStream_t s);
+cudaError_t launch_combine_slots(const float* slots, int T, int d, int k, void* y, int out_f32,
+                                 cudaStream_t s);
+
+cudaError_t launch_gemm_simt(int epi, const float* A, const float* B, const GemmArgs& a,
+                             int rows_cap, cudaStream_t s);
+
+// tcgen05 path.  tmA: A rows [*, K] bf16, box {64, 128}; tmB: B rows [*, K] bf16, box {64, 128}.
+size_t gemm_tc_smem_bytes();
+cudaError_t launch_gemm_tc(int epi, const CUtensorMap& tmA, const CUtensorMap& tmB,
+                           const GemmArgs& a, int grid, cudaStream_t s);
+
+cudaError_t launch_selftest_timeout(int* status, unsigned long long limit_ns, cudaStream_t s);
+
+}  // namespace moe

@@ -1,0 +1,237 @@
+// Permutation stage: per-expert histogram, prefix-sum scan, and a coalesced,
+// vectorised scatter of token rows into an expert-contiguous layout, so the
+// grouped GEMMs see each expert's tokens as one block of rows (the dispatch
+// step between routing and the experts: tokens go only to their chosen
+// experts, "开源混合架构大模型技术解析", section 四, and 七 item 3 on scheduling
+// tokens that route to different experts).
+//
+// Layout produced: expert e owns rows [offsets[e], offsets[e+1]) of x_perm,
+// a segment padded to a multiple of 128 rows.  Inside a segment the real rows
+// come first, in increasing token order (stable), then padding rows whose
+// row_src is -1.  row_src[r] = t*k + j for the row holding slot j of token t.
+#include "moe_device.cuh"
+#include "moe_internal.h"
+
+namespace moe {
+
+namespace {
+
+constexpr int kWarps = kPermBlockTokens / 32;
+
+// Load the k expert ids of token t (or -1s past T); out-of-range ids are
+// recorded as a device error and treated as absent.
+__device__ __forceinline__ void load_slots(const int32_t* __restrict__ idx, int t, int T, int k,
+                                           int E, int (&my)[kMaxK], int* status) {
+#pragma unroll
+    for (int j = 0; j < kMaxK; ++j) {
+        int e = -1;
+        if (j < k && t < T) {
+            e = idx[(size_t)t * k + j];
+            if (e < 0 || e >= E) {
+                set_status(status, MOE_ERR_DEVICE, SITE_PERMUTE, e);
+                e = -1;
+            }
+        }
+        my[j] = e;
+    }
+}
+
+__device__ __forceinline__ bool holds(const int (&my)[kMaxK], int e) {
+    bool h = false;
+#pragma unroll
+    for (int j = 0; j < kMaxK; ++j) h |= (my[j] == e);
+    return h;
+}
+
+// Histogram of each block of 256 tokens: block_counts[b][e].
+__global__ void __launch_bounds__(kPermBlockTokens) perm_count_kernel(
+    const int32_t* __restrict__ idx, int T, int k, int E, int32_t* __restrict__ block_counts,
+    int* status) {
+    __shared__ int wcnt[kWarps][kMaxE];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int t = blockIdx.x * kPermBlockTokens + tid;
+    int my[kMaxK];
+    load_slots(idx, t, T, k, E, my, status);
+    for (int e = 0; e < E; ++e) {
+        unsigned b = __ballot_sync(0xffffffffu, holds(my, e));
+        if (lane == 0) wcnt[warp][e] = __popc(b);
+    }
+    __syncthreads();
+    for (int e = tid; e < E; e += kPermBlockTokens) {
+        int s = 0;
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) s += wcnt[w][e];
+        block_counts[(size_t)blockIdx.x * E + e] = s;
+    }
+}
+
+// One CTA: per expert, exclusive scan of the block histogram over blocks
+// (in place), total counts, 128-padded segment offsets, and row_src = -1 on
+// the padding rows.
+__global__ void __launch_bounds__(1024) perm_scan_kernel(int32_t* __restrict__ block_counts,
+                                                         int nb, int E,
+                                                         int32_t* __restrict__ counts,
+                                                         int32_t* __restrict__ offsets,
+                                                         int32_t* __restrict__ row_src) {
+    __shared__ int s_cnt[kMaxE];
+    __shared__ int s_off[kMaxE + 1];
+    const int tid = threadIdx.x;
+    for (int e = tid; e < E; e += blockDim.x) {
+        int run = 0;
+        for (int b = 0; b < nb; ++b) {
+            int c = block_counts[(size_t)b * E + e];
+            block_counts[(size_t)b * E + e] = run;
+            run += c;
+        }
+        counts[e] = run;
+        s_cnt[e] = run;
+    }
+    __syncthreads();
+    if (tid == 0) {
+        int run = 0;
+        for (int e = 0; e < E; ++e) {
+            s_off[e] = run;
+            run += (s_cnt[e] + kRowAlign - 1) / kRowAlign * kRowAlign;
+        }
+        s_off[E] = run;
+    }
+    __syncthreads();
+    for (int e = tid; e <= E; e += blockDim.x) offsets[e] = s_off[e];
+    for (int i = tid; i < E * kRowAlign; i += blockDim.x) {
+        int e = i / kRowAlign, r = i % kRowAlign;
+        int row = s_off[e] + s_cnt[e] + r;
+        if (row < s_off[e + 1]) row_src[row] = -1;
+    }
+}
+
+// Stable rank of every (token, slot) inside its expert, and row_src of the
+// destination row.
+__global__ void __launch_bounds__(kPermBlockTokens) perm_rank_kernel(
+    const int32_t* __restrict__ idx, int T, int k, int E,
+    const int32_t* __restrict__ block_base, const int32_t* __restrict__ offsets,
+    int32_t* __restrict__ row_src, int* status) {
+    __shared__ int wbase[kWarps][kMaxE];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int t = blockIdx.x * kPermBlockTokens + tid;
+    int my[kMaxK], rank[kMaxK];
+    load_slots(idx, t, T, k, E, my, nullptr);
+#pragma unroll
+    for (int j = 0; j < kMaxK; ++j) rank[j] = 0;
+    const unsigned lt = (1u << lane) - 1u;
+    for (int e = 0; e < E; ++e) {
+        unsigned b = __ballot_sync(0xffffffffu, holds(my, e));
+        if (lane == 0) wbase[warp][e] = __popc(b);
+#pragma unroll
+        for (int j = 0; j < kMaxK; ++j)
+            if (my[j] == e) rank[j] = __popc(b & lt);
+    }
+    __syncthreads();
+    for (int e = tid; e < E; e += kPermBlockTokens) {
+        int run = offsets[e] + block_base[(size_t)blockIdx.x * E + e];
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) {
+            int c = wbase[w][e];
+            wbase[w][e] = run;
+            run += c;
+        }
+    }
+    __syncthreads();
+#pragma unroll
+    for (int j = 0; j < kMaxK; ++j) {
+        if (my[j] >= 0) {
+            int pos = wbase[warp][my[j]] + rank[j];
+            if (pos < offsets[my[j] + 1])
+                row_src[pos] = t * k + j;
+            else
+                set_status(status, MOE_ERR_DEVICE, SITE_PERMUTE, pos);
+        }
+    }
+}
+
+// x_perm[r] = x[row_src[r] / k] for every real row r < offsets[E]; one warp
+// per row, 16-byte vectors.
+__global__ void __launch_bounds__(256) gather_rows_kernel(const uint4* __restrict__ x,
+                                                          int vec_per_row, int k,
+                                                          const int32_t* __restrict__ total_rows,
+                                                          const int32_t* __restrict__ row_src,
+                                                          uint4* __restrict__ x_perm) {
+    const int lane = threadIdx.x & 31;
+    const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int nw = (gridDim.x * blockDim.x) >> 5;
+    const int total = *total_rows;
+    for (int r = gw; r < total; r += nw) {
+        const int src = row_src[r];
+        if (src < 0) continue;
+        const uint4* s = x + (size_t)(src / k) * vec_per_row;
+        uint4* dst = x_perm + (size_t)r * vec_per_row;
+        for (int i = lane; i < vec_per_row; i += 32) dst[i] = __ldg(s + i);
+    }
+}
+
+// y[t] = slots[t*k + 0] + ... + slots[t*k + k-1], in that order (used when
+// there are no shared experts to fold the sum into).
+__global__ void __launch_bounds__(256) combine_slots_kernel(const float4* __restrict__ slots,
+                                                            int T, int d4, int k, void* y,
+                                                            int out_f32) {
+    const size_t n = (size_t)T * d4;
+    for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n;
+         i += (size_t)gridDim.x * blockDim.x) {
+        const size_t t = i / d4, c = i % d4;
+        float4 a = slots[(t * k) * d4 + c];
+        for (int j = 1; j < k; ++j) {
+            float4 b = slots[(t * k + j) * d4 + c];
+            a.x += b.x;
+            a.y += b.y;
+            a.z += b.z;
+            a.w += b.w;
+        }
+        if (out_f32) {
+            reinterpret_cast<float4*>(y)[i] = a;
+        } else {
+            uint2 p;
+            p.x = pack_bf16x2(a.x, a.y);
+            p.y = pack_bf16x2(a.z, a.w);
+            reinterpret_cast<uint2*>(y)[i] = p;
+        }
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_permute(const int32_t* idx, int T, int k, int E, int32_t* block_counts,
+                           int32_t* counts, int32_t* offsets, int32_t* row_src, int* status,
+                           cudaStream_t s) {
+    const int nb = (T + kPermBlockTokens - 1) / kPermBlockTokens;
+    perm_count_kernel<<<nb, kPermBlockTokens, 0, s>>>(idx, T, k, E, block_counts, status);
+    perm_scan_kernel<<<1, 1024, 0, s>>>(block_counts, nb, E, counts, offsets, row_src);
+    perm_rank_kernel<<<nb, kPermBlockTokens, 0, s>>>(idx, T, k, E, block_counts, offsets, row_src,
+                                                     status);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_gather_rows(const void* x, int d, int elem_bytes, int k,
+                               const int32_t* offsets_total, const int32_t* row_src,
+                               int rows_cap, void* x_perm, int num_sms, cudaStream_t s) {
+    const int vec = d * elem_bytes / 16;
+    int blocks = num_sms * 8;
+    const int need = (rows_cap + 7) / 8;
+    if (blocks > need) blocks = need > 0 ? need : 1;
+    gather_rows_kernel<<<blocks, 256, 0, s>>>(static_cast<const uint4*>(x), vec, k,
+                                              offsets_total, row_src,
+                                              static_cast<uint4*>(x_perm));
+    return cudaGetLastError();
+}
+
+cudaError_t launch_combine_slots(const float* slots, int T, int d, int k, void* y, int out_f32,
+                                 cudaStream_t s) {
+    const int d4 = d / 4;
+    size_t n = (size_t)T * d4;
+    int blocks = (int)((n + 255) / 256);
+    if (blocks > 148 * 16) blocks = 148 * 16;
+    if (blocks < 1) blocks = 1;
+    combine_slots_kernel<<<blocks, 256, 0, s>>>(reinterpret_cast<const float4*>(slots), T, d4, k,
+                                                y, out_f32);
+    return cudaGetLastError();
+}
+
+}  // namespace moe

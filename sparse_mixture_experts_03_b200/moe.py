@@ -1,0 +1,222 @@
+"""Thin Python binding of the C ABI in include/moe.h (libmoe_b200.so).
+
+Argument marshalling only: torch tensors are passed as raw device pointers
+with the current CUDA stream; every step of the layer runs in the library's
+kernels.  There is no fallback: if the library is missing or fails to load,
+every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Tuple
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmoe_b200.so")
+
+MOE_OK = 0
+MOE_ERR_INVALID_ARG = -1
+MOE_ERR_UNSUPPORTED = -2
+MOE_ERR_CUDA = -3
+MOE_ERR_WORKSPACE = -4
+MOE_ERR_TIMEOUT = -5
+MOE_ERR_DEVICE = -6
+MOE_F32, MOE_BF16 = 0, 1
+
+# workspace regions (indices into moe_workspace_layout)
+WS_REGIONS = ["status", "counts", "offsets", "block_counts", "topk_idx", "topk_w", "row_src",
+              "x_perm", "h", "h_shared", "slots"]
+WS_TOTAL = len(WS_REGIONS)
+ROW_ALIGN = 128
+
+# every entry point declared in include/moe.h
+SYMBOLS = ["moe_workspace_bytes", "moe_workspace_layout", "moe_route", "moe_forward",
+           "moe_get_device_status", "moe_clear_device_status", "moe_selftest_timeout",
+           "moe_set_stage_events", "moe_status_string", "moe_version"]
+N_STAGE_EVENTS = 7
+STAGES = ["route", "permute", "gate_up_routed", "gate_up_shared", "down_routed",
+          "down_shared_combine"]
+
+_lib = None
+
+
+class MoeError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {status_string(status)} ({status})")
+
+
+def lib() -> ctypes.CDLL:
+    """Load libmoe_b200.so (raises if it is missing: there is no other path)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"CUDA library not built: {LIB_PATH} "
+                               "(python -m sparse_mixture_experts_03_b200.build)")
+        L = ctypes.CDLL(LIB_PATH)
+        i, vp, sz = ctypes.c_int, ctypes.c_void_p, ctypes.c_size_t
+        L.moe_workspace_bytes.argtypes = [i] * 7
+        L.moe_workspace_bytes.restype = sz
+        L.moe_workspace_layout.argtypes = [i] * 7 + [ctypes.POINTER(sz), i]
+        L.moe_workspace_layout.restype = i
+        L.moe_route.argtypes = [vp, vp] + [i] * 7 + [vp, vp, vp]
+        L.moe_route.restype = i
+        L.moe_forward.argtypes = [vp] * 5 + [i] * 10 + [vp, vp, vp, vp, sz, vp]
+        L.moe_forward.restype = i
+        L.moe_get_device_status.argtypes = [vp, ctypes.POINTER(i), ctypes.POINTER(i), vp]
+        L.moe_get_device_status.restype = i
+        L.moe_clear_device_status.argtypes = [vp, vp]
+        L.moe_clear_device_status.restype = i
+        L.moe_selftest_timeout.argtypes = [vp, i, vp]
+        L.moe_selftest_timeout.restype = i
+        L.moe_set_stage_events.argtypes = [ctypes.POINTER(vp), i]
+        L.moe_set_stage_events.restype = i
+        L.moe_status_string.argtypes = [i]
+        L.moe_status_string.restype = ctypes.c_char_p
+        L.moe_version.restype = i
+        _lib = L
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().moe_status_string(status).decode()
+
+
+def _dt(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return MOE_BF16
+    if t.dtype == torch.float32:
+        return MOE_F32
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    if t is None:
+        return None
+    if not t.is_contiguous():
+        raise ValueError("tensors must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream: Optional[torch.cuda.Stream]):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check(status: int, what: str) -> None:
+    if status != MOE_OK:
+        raise MoeError(status, what)
+
+
+def workspace_bytes(T, d, E, k, inter, n_shared, dtype: torch.dtype) -> int:
+    n = lib().moe_workspace_bytes(T, d, E, k, inter, n_shared,
+                                  MOE_BF16 if dtype == torch.bfloat16 else MOE_F32)
+    if n == 0:
+        raise MoeError(MOE_ERR_INVALID_ARG, "moe_workspace_bytes")
+    return int(n)
+
+
+def workspace_layout(T, d, E, k, inter, n_shared, dtype: torch.dtype) -> dict:
+    arr = (ctypes.c_size_t * (WS_TOTAL + 1))()
+    _check(lib().moe_workspace_layout(T, d, E, k, inter, n_shared,
+                                      MOE_BF16 if dtype == torch.bfloat16 else MOE_F32,
+                                      arr, WS_TOTAL + 1), "moe_workspace_layout")
+    out = {name: int(arr[i]) for i, name in enumerate(WS_REGIONS)}
+    out["total"] = int(arr[WS_TOTAL])
+    return out
+
+
+def alloc_workspace(T, d, E, k, inter, n_shared, dtype, device="cuda") -> torch.Tensor:
+    return torch.empty(workspace_bytes(T, d, E, k, inter, n_shared, dtype), dtype=torch.uint8,
+                       device=device)
+
+
+def route(x: torch.Tensor, W_router: torch.Tensor, k: int, n_group: int, topk_group: int,
+          topk_idx: Optional[torch.Tensor] = None, topk_w: Optional[torch.Tensor] = None,
+          stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """moe_route: (topk_idx int32 [T,k], topk_w fp32 [T,k])."""
+    T, d = x.shape
+    E = W_router.shape[0]
+    if topk_idx is None:
+        topk_idx = torch.empty(T, k, dtype=torch.int32, device=x.device)
+    if topk_w is None:
+        topk_w = torch.empty(T, k, dtype=torch.float32, device=x.device)
+    _check(lib().moe_route(_ptr(x), _ptr(W_router), T, d, E, k, n_group, topk_group, _dt(x),
+                           _ptr(topk_idx), _ptr(topk_w), _stream(stream)), "moe_route")
+    return topk_idx, topk_w
+
+
+def forward(x: torch.Tensor, W_router: torch.Tensor, W_gate_up: torch.Tensor,
+            W_down: torch.Tensor, W_shared: Optional[torch.Tensor], k: int, n_group: int,
+            topk_group: int, inter: int, n_shared: int, out_dtype: torch.dtype = torch.float32,
+            y: Optional[torch.Tensor] = None, topk_idx: Optional[torch.Tensor] = None,
+            topk_w: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+            stream=None) -> torch.Tensor:
+    """moe_forward: y [T, d] in out_dtype (float32 or bfloat16)."""
+    T, d = x.shape
+    E = W_router.shape[0]
+    if y is None:
+        y = torch.empty(T, d, dtype=out_dtype, device=x.device)
+    if workspace is None:
+        workspace = alloc_workspace(T, d, E, k, inter, n_shared, x.dtype, x.device)
+    st = lib().moe_forward(_ptr(x), _ptr(W_router), _ptr(W_gate_up), _ptr(W_down),
+                           _ptr(W_shared), T, d, E, k, n_group, topk_group, inter, n_shared,
+                           _dt(x), _dt(y), _ptr(y), _ptr(topk_idx), _ptr(topk_w),
+                           _ptr(workspace), workspace.numel(), _stream(stream))
+    _check(st, "moe_forward")
+    return y
+
+
+def device_status(workspace: torch.Tensor, stream=None) -> Tuple[int, int]:
+    """(status, site) of the last moe_forward using `workspace` (synchronises)."""
+    s, w = ctypes.c_int(0), ctypes.c_int(0)
+    _check(lib().moe_get_device_status(_ptr(workspace), ctypes.byref(s), ctypes.byref(w),
+                                       _stream(stream)), "moe_get_device_status")
+    return s.value, w.value
+
+
+def clear_device_status(workspace: torch.Tensor, stream=None) -> None:
+    _check(lib().moe_clear_device_status(_ptr(workspace), _stream(stream)),
+           "moe_clear_device_status")
+
+
+def selftest_timeout(workspace: torch.Tensor, limit_us: int, stream=None) -> None:
+    _check(lib().moe_selftest_timeout(_ptr(workspace), limit_us, _stream(stream)),
+           "moe_selftest_timeout")
+
+
+def set_stage_events(events) -> None:
+    """Record torch.cuda.Event objects at stage boundaries of every following
+    forward (None turns it off).  The events must have been recorded once so
+    that their CUDA handles exist."""
+    if events is None:
+        _check(lib().moe_set_stage_events(None, 0), "moe_set_stage_events")
+        return
+    arr = (ctypes.c_void_p * len(events))(*[ctypes.c_void_p(e.cuda_event) for e in events])
+    _check(lib().moe_set_stage_events(arr, len(events)), "moe_set_stage_events")
+
+
+class MoELayer:
+    """Device-resident weights plus a reusable workspace for one layer shape."""
+
+    def __init__(self, x_example_T: int, W_router, W_gate_up, W_down, W_shared, k, n_group,
+                 topk_group, inter, n_shared, out_dtype=torch.float32):
+        self.W_router, self.W_gate_up, self.W_down, self.W_shared = (
+            W_router, W_gate_up, W_down, W_shared)
+        self.k, self.n_group, self.topk_group = k, n_group, topk_group
+        self.inter, self.n_shared, self.out_dtype = inter, n_shared, out_dtype
+        self.E, self.d = W_router.shape
+        self.T_cap = x_example_T
+        self.workspace = alloc_workspace(x_example_T, self.d, self.E, k, inter, n_shared,
+                                         W_router.dtype, W_router.device)
+
+    def __call__(self, x: torch.Tensor, y: Optional[torch.Tensor] = None, topk_idx=None,
+                 topk_w=None, stream=None) -> torch.Tensor:
+        if x.shape[0] > self.T_cap:
+            raise ValueError("more tokens than the workspace was sized for")
+        return forward(x, self.W_router, self.W_gate_up, self.W_down, self.W_shared, self.k,
+                       self.n_group, self.topk_group, self.inter, self.n_shared,
+                       self.out_dtype, y=y, topk_idx=topk_idx, topk_w=topk_w,
+                       workspace=self.workspace, stream=stream)
