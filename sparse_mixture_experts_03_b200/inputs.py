@@ -15,8 +15,10 @@ expert of inter I, so its down projection uses 1/I).
 Random streams: each tensor has a fixed stream id (x 0, W_router 1, W_gate_up
 2, W_down 3, shared gate_up 4, shared down 5, skew direction u 6) and is filled
 in chunks of 2**24 elements; chunk c of stream i is drawn by torch.randn from a
-CPU torch.Generator seeded with (seed << 40) | (i << 32) | c.  The values do
-not depend on how many threads fill the chunks.  Everything is drawn in fp32
+CPU torch.Generator seeded with the 32-bit value (seed << 24) | (i << 16) | c
+(the CPU generator keeps only 32 bits of a seed, so the fields are packed into
+32 bits: seed < 256, stream < 256, chunk < 65536).  The values do not depend
+on how many threads fill the chunks.  Everything is drawn in fp32
 and cast to bf16 with round-to-nearest-even where the workload is bf16.
 
 Layouts (all row-major, contiguous):
@@ -42,7 +44,7 @@ import torch
 # SKEW_ALPHA * u, where x = z + SKEW_SHIFT * u.  SKEW_ALPHA was chosen by
 # oracle/calibrate_skew.py so that about 40% of tokens route to expert 0.
 SKEW_SHIFT = 3.0
-SKEW_ALPHA = 0.4180
+SKEW_ALPHA = 0.4111
 
 
 @dataclasses.dataclass(frozen=True)
@@ -107,9 +109,11 @@ def _randn(shape, seed: int, stream: int, scale: float = 1.0) -> torch.Tensor:
     n = math.prod(shape)
     out = torch.empty(n, dtype=torch.float32)
     n_chunks = (n + CHUNK - 1) // CHUNK
+    if not (0 <= seed < 256 and 0 <= stream < 256 and n_chunks <= 65536):
+        raise ValueError("seed, stream or size outside the packed 32-bit seed fields")
 
     def fill(c: int) -> None:
-        g = torch.Generator(device="cpu").manual_seed((seed << 40) | (stream << 32) | c)
+        g = torch.Generator(device="cpu").manual_seed((seed << 24) | (stream << 16) | c)
         lo, hi = c * CHUNK, min(n, (c + 1) * CHUNK)
         out[lo:hi] = torch.randn(hi - lo, generator=g)
         if scale != 1.0:
