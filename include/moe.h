@@ -174,12 +174,12 @@ MOE_API int moe_selftest_timeout(void *workspace, int limit_us, void *stream);
  * events != NULL (n == MOE_N_STAGE_EVENTS handles of type cudaEvent_t, created
  * by the caller), every following moe_forward in this process records
  * events[i] on its stream: [0] start, [1] after routing, [2] after the
- * permutation, [3] after the routed gate/up GEMM, [4] after the shared gate/up
- * GEMM, [5] after the routed down GEMM, [6] at the end.  events == NULL turns
- * it off.  Process-wide setting, not thread-safe.  Returns MOE_OK or
+ * permutation, [3] after the gate/up GEMM (routed and shared experts, one
+ * launch), [4] after the routed down GEMM, [5] at the end.  events == NULL
+ * turns it off.  Process-wide setting, not thread-safe.  Returns MOE_OK or
  * MOE_ERR_INVALID_ARG.
  */
-#define MOE_N_STAGE_EVENTS 7
+#define MOE_N_STAGE_EVENTS 6
 MOE_API int moe_set_stage_events(void *const *events, int n);
 
 /* moe_status_string -- static text for a status code. */

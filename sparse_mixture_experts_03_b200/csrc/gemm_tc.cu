@@ -57,7 +57,7 @@ struct __align__(8) SmemTail {
     uint64_t drain;
     uint32_t tmem_base;
     int abort;
-    int offsets[kMaxOffsets];
+    int offsets[2][kMaxOffsets];
 };
 
 constexpr size_t kSmemBytes = 1024 /*alignment slack*/ + (size_t)kStages * kStageBytes +
@@ -79,10 +79,19 @@ __device__ __forceinline__ float silu_mul(float g, float u) {
     return __fdividef(g, 1.0f + __expf(-g)) * u;
 }
 
+// Tile t of the launch belongs to problem 0 when t < tiles0, else to problem 1
+// (tile t - tiles0).  Inside a problem: row block t / n_tiles, N tile t % n_tiles.
+struct TileRef {
+    int p, row0, nt, g;
+};
+
 template <int EPI>
 __global__ void __launch_bounds__(kThreads, 1)
-    grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
-                           const __grid_constant__ CUtensorMap tmB, const GemmArgs args) {
+    grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0,
+                           const __grid_constant__ CUtensorMap tmB0,
+                           const __grid_constant__ CUtensorMap tmA1,
+                           const __grid_constant__ CUtensorMap tmB1, const GemmArgs args0,
+                           const GemmArgs args1, int n_problems) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -90,7 +99,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     volatile int* abort_flag = &tail->abort;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int n_groups = args.offsets != nullptr ? args.n_groups : 1;
 
     if (tid == 0) {
         for (int s = 0; s < kStages; ++s) {
@@ -105,11 +113,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         tail->abort = 0;
         fence_barrier_init();
     }
-    if (args.offsets != nullptr) {
-        for (int i = tid; i <= n_groups; i += kThreads) tail->offsets[i] = args.offsets[i];
-    } else if (tid == 0) {
-        tail->offsets[0] = 0;
-        tail->offsets[1] = (args.static_rows + BM - 1) / BM * BM;
+    for (int p = 0; p < n_problems; ++p) {
+        const GemmArgs& a = p == 0 ? args0 : args1;
+        if (a.offsets != nullptr) {
+            for (int i = tid; i <= a.n_groups; i += kThreads) tail->offsets[p][i] = a.offsets[i];
+        } else if (tid == 0) {
+            tail->offsets[p][0] = 0;
+            tail->offsets[p][1] = (a.static_rows + BM - 1) / BM * BM;
+        }
     }
     if (warp == 1) {
         tmem_alloc(&tail->tmem_base, kTmemCols);
@@ -120,28 +131,48 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
 
     const uint32_t tmem_base = tail->tmem_base;
-    const int total_rows = tail->offsets[n_groups];
-    const int total_tiles = (total_rows / BM) * args.n_tiles;
-    const int kb_count = args.K / BK;
-    const uint64_t limit = args.wait_limit_ns;
+    const int ng0 = args0.offsets != nullptr ? args0.n_groups : 1;
+    const int ng1 = args1.offsets != nullptr ? args1.n_groups : 1;
+    const int tiles0 = (tail->offsets[0][ng0] / BM) * args0.n_tiles;
+    const int tiles1 = n_problems > 1 ? (tail->offsets[1][ng1] / BM) * args1.n_tiles : 0;
+    const int total_tiles = tiles0 + tiles1;
+    const uint64_t limit = args0.wait_limit_ns;
+    int* const status = args0.status;
+
+    auto tile_ref = [&](int tile) {
+        TileRef r;
+        r.p = tile < tiles0 ? 0 : 1;
+        const int lt = r.p == 0 ? tile : tile - tiles0;
+        const GemmArgs& a = r.p == 0 ? args0 : args1;
+        r.row0 = (lt / a.n_tiles) * BM;
+        r.nt = lt % a.n_tiles;
+        r.g = find_group(tail->offsets[r.p], r.p == 0 ? ng0 : ng1, r.row0);
+        return r;
+    };
 
     if (warp == 0) {
         // ------------------------------------------------ TMA producer
         if (lane == 0) {
-            tma_prefetch_desc(&tmA);
-            tma_prefetch_desc(&tmB);
+            tma_prefetch_desc(&tmA0);
+            tma_prefetch_desc(&tmB0);
+            if (n_problems > 1) {
+                tma_prefetch_desc(&tmA1);
+                tma_prefetch_desc(&tmB1);
+            }
             int s = 0;
             uint32_t ph = 0;
             bool ok = true;
             uint32_t issued = 0, issued_ph = 0;  // per stage: loaded at least once / parity
             for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x) {
-                const int mblk = tile / args.n_tiles, nt = tile % args.n_tiles;
-                const int row0 = mblk * BM;
-                const int g = find_group(tail->offsets, n_groups, row0);
-                const int b0 = (int)(g * args.b_group_stride) + nt * args.b_tile_step;
-                const int b1 = b0 + args.b_half_off;
+                const TileRef r = tile_ref(tile);
+                const GemmArgs& a = r.p == 0 ? args0 : args1;
+                const CUtensorMap* mA = r.p == 0 ? &tmA0 : &tmA1;
+                const CUtensorMap* mB = r.p == 0 ? &tmB0 : &tmB1;
+                const int b0 = (int)(r.g * a.b_group_stride) + r.nt * a.b_tile_step;
+                const int b1 = b0 + a.b_half_off;
+                const int kb_count = a.K / BK;
                 for (int kb = 0; kb < kb_count; ++kb) {
-                    if (!mbar_wait_bounded(&tail->empty[s], ph ^ 1u, abort_flag, args.status,
+                    if (!mbar_wait_bounded(&tail->empty[s], ph ^ 1u, abort_flag, status,
                                            SITE_GEMM_PRODUCER, limit)) {
                         ok = false;
                         break;
@@ -149,9 +180,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                     uint8_t* sa = smem + (size_t)s * kStageBytes;
                     uint8_t* sb = sa + kABytes;
                     mbar_arrive_expect_tx(&tail->full[s], kStageBytes);
-                    tma_load_2d(sa, &tmA, &tail->full[s], kb * BK, row0);
-                    tma_load_2d(sb, &tmB, &tail->full[s], kb * BK, b0);
-                    tma_load_2d(sb + kBBytes / 2, &tmB, &tail->full[s], kb * BK, b1);
+                    tma_load_2d(sa, mA, &tail->full[s], kb * BK, r.row0);
+                    tma_load_2d(sb, mB, &tail->full[s], kb * BK, b0);
+                    tma_load_2d(sb + kBBytes / 2, mB, &tail->full[s], kb * BK, b1);
                     issued |= 1u << s;
                     issued_ph = (issued_ph & ~(1u << s)) | (ph << s);
                     if (++s == kStages) {
@@ -178,7 +209,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x, ++it) {
                 const int acc = it & 1;
                 const uint32_t aph = (it >> 1) & 1;
-                if (!mbar_wait_bounded(&tail->tempty[acc], aph ^ 1u, abort_flag, args.status,
+                const int kb_count = (tile < tiles0 ? args0.K : args1.K) / BK;
+                if (!mbar_wait_bounded(&tail->tempty[acc], aph ^ 1u, abort_flag, status,
                                        SITE_GEMM_MMA, limit)) {
                     ok = false;
                     break;
@@ -186,7 +218,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BNB);
                 for (int kb = 0; kb < kb_count; ++kb) {
-                    if (!mbar_wait_bounded(&tail->full[s], ph, abort_flag, args.status,
+                    if (!mbar_wait_bounded(&tail->full[s], ph, abort_flag, status,
                                            SITE_GEMM_MMA, limit)) {
                         ok = false;
                         break;
@@ -211,7 +243,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             // all tensor-core work of this CTA is complete once `drain` fires
             tc_commit(&tail->drain);
-            mbar_wait_bounded(&tail->drain, 0u, nullptr, args.status, SITE_GEMM_DRAIN, limit);
+            mbar_wait_bounded(&tail->drain, 0u, nullptr, status, SITE_GEMM_DRAIN, limit);
         }
     } else {
         // ------------------------------------------------ epilogue (warps 2..5)
@@ -221,16 +253,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x, ++it) {
             const int acc = it & 1;
             const uint32_t aph = (it >> 1) & 1;
-            const bool got = mbar_wait_bounded(&tail->tfull[acc], aph, abort_flag, args.status,
+            const bool got = mbar_wait_bounded(&tail->tfull[acc], aph, abort_flag, status,
                                                SITE_GEMM_EPILOGUE, limit);
             // tcgen05.ld below is warp-collective: leave together or not at all
             if (!__all_sync(0xffffffffu, got)) break;
             tc_fence_after();
-            const int mblk = tile / args.n_tiles, nt = tile % args.n_tiles;
-            const int grow = mblk * BM + r_local;
+            const TileRef r = tile_ref(tile);
+            const GemmArgs& args = r.p == 0 ? args0 : args1;
+            const int grow = r.row0 + r_local;
             const uint32_t taddr =
                 tmem_base + (uint32_t)(acc * BNB) + ((uint32_t)(wq * 32) << 16);
-            const int col0 = nt * args.out_col_step;
+            const int col0 = r.nt * args.out_col_step;
 
             if constexpr (EPI == EPI_SWIGLU) {
                 const bool valid = grow < args.valid_rows;
@@ -350,9 +383,11 @@ __global__ void selftest_timeout_kernel(int* status, unsigned long long limit_ns
 
 size_t gemm_tc_smem_bytes() { return kSmemBytes; }
 
-cudaError_t launch_gemm_tc(int epi, const CUtensorMap& tmA, const CUtensorMap& tmB,
-                           const GemmArgs& a, int grid, cudaStream_t s) {
-    void (*kern)(const CUtensorMap, const CUtensorMap, const GemmArgs) = nullptr;
+cudaError_t launch_gemm_tc(int epi, const CUtensorMap& tmA0, const CUtensorMap& tmB0,
+                           const GemmArgs& a0, const CUtensorMap* tmA1, const CUtensorMap* tmB1,
+                           const GemmArgs* a1, int grid, cudaStream_t s) {
+    void (*kern)(const CUtensorMap, const CUtensorMap, const CUtensorMap, const CUtensorMap,
+                 const GemmArgs, const GemmArgs, int) = nullptr;
     switch (epi) {
         case EPI_SWIGLU: kern = grouped_gemm_tc_kernel<EPI_SWIGLU>; break;
         case EPI_SCATTER: kern = grouped_gemm_tc_kernel<EPI_SCATTER>; break;
@@ -362,7 +397,9 @@ cudaError_t launch_gemm_tc(int epi, const CUtensorMap& tmA, const CUtensorMap& t
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)kSmemBytes);
     if (e != cudaSuccess) return e;
-    kern<<<grid, kThreads, kSmemBytes, s>>>(tmA, tmB, a);
+    const int np = a1 != nullptr ? 2 : 1;
+    kern<<<grid, kThreads, kSmemBytes, s>>>(tmA0, tmB0, np > 1 ? *tmA1 : tmA0,
+                                            np > 1 ? *tmB1 : tmB0, a0, np > 1 ? *a1 : a0, np);
     return cudaGetLastError();
 }
 

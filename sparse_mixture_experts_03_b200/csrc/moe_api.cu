@@ -318,29 +318,30 @@ MOE_API int moe_forward(const void* x, const void* W_router, const void* W_gate_
 
     if (bf16) {
         const int rows_tiles = L.rows_cap / 128;
-        // 3. gate/up + SwiGLU, routed experts
+        // 3. gate/up + SwiGLU: routed experts, then the shared experts on all
+        //    tokens, as one persistent launch over both tile lists
         g1.n_tiles = inter / 128;
         g1.b_tile_step = 128;
         g1.out_col_step = 128;
-        CUtensorMap tA, tB;
+        CUtensorMap tA, tB, tA1, tB1;
         if (!make_map(&tA, x_perm, (uint64_t)L.rows_cap, d) ||
             !make_map(&tB, W_gate_up, (uint64_t)E * 2 * inter, d))
             return MOE_ERR_CUDA;
-        e = launch_gemm_tc(EPI_SWIGLU, tA, tB, g1, grid_for((long long)rows_tiles * g1.n_tiles), s);
-        if (e != cudaSuccess) return MOE_ERR_CUDA;
-        stage_mark(3, s);
-        // 4. gate/up + SwiGLU, shared experts (all tokens)
+        long long g1_tiles = (long long)rows_tiles * g1.n_tiles;
         if (n_shared > 0) {
             g1s.n_tiles = SI / 128;
             g1s.b_tile_step = 128;
             g1s.out_col_step = 128;
-            if (!make_map(&tA, x, (uint64_t)T, d) || !make_map(&tB, Wsh_gu, (uint64_t)2 * SI, d))
+            if (!make_map(&tA1, x, (uint64_t)T, d) || !make_map(&tB1, Wsh_gu, (uint64_t)2 * SI, d))
                 return MOE_ERR_CUDA;
-            e = launch_gemm_tc(EPI_SWIGLU, tA, tB, g1s,
-                               grid_for((long long)((T + 127) / 128) * g1s.n_tiles), s);
-            if (e != cudaSuccess) return MOE_ERR_CUDA;
+            g1_tiles += (long long)((T + 127) / 128) * g1s.n_tiles;
+            e = launch_gemm_tc(EPI_SWIGLU, tA, tB, g1, &tA1, &tB1, &g1s, grid_for(g1_tiles), s);
+        } else {
+            e = launch_gemm_tc(EPI_SWIGLU, tA, tB, g1, nullptr, nullptr, nullptr,
+                               grid_for(g1_tiles), s);
         }
-        stage_mark(4, s);
+        if (e != cudaSuccess) return MOE_ERR_CUDA;
+        stage_mark(3, s);
         // 5. down projection, routed: weighted scatter into token-order slots
         g2.n_tiles = d / 256;
         g2.b_tile_step = 256;
@@ -349,9 +350,10 @@ MOE_API int moe_forward(const void* x, const void* W_router, const void* W_gate_
         if (!make_map(&tA, h, (uint64_t)L.rows_cap, inter) ||
             !make_map(&tB, W_down, (uint64_t)E * d, inter))
             return MOE_ERR_CUDA;
-        e = launch_gemm_tc(EPI_SCATTER, tA, tB, g2, grid_for((long long)rows_tiles * g2.n_tiles), s);
+        e = launch_gemm_tc(EPI_SCATTER, tA, tB, g2, nullptr, nullptr, nullptr,
+                           grid_for((long long)rows_tiles * g2.n_tiles), s);
         if (e != cudaSuccess) return MOE_ERR_CUDA;
-        stage_mark(5, s);
+        stage_mark(4, s);
         // 6. down projection, shared, with the final fixed-order sum
         if (n_shared > 0) {
             g2s.n_tiles = d / 256;
@@ -360,14 +362,14 @@ MOE_API int moe_forward(const void* x, const void* W_router, const void* W_gate_
             g2s.out_col_step = 256;
             if (!make_map(&tA, h_sh, (uint64_t)T, SI) || !make_map(&tB, Wsh_dn, (uint64_t)d, SI))
                 return MOE_ERR_CUDA;
-            e = launch_gemm_tc(EPI_COMBINE, tA, tB, g2s,
+            e = launch_gemm_tc(EPI_COMBINE, tA, tB, g2s, nullptr, nullptr, nullptr,
                                grid_for((long long)((T + 127) / 128) * g2s.n_tiles), s);
             if (e != cudaSuccess) return MOE_ERR_CUDA;
         } else {
             e = launch_combine_slots(slots, T, d, k, y, out_f32, s);
             if (e != cudaSuccess) return MOE_ERR_CUDA;
         }
-        stage_mark(6, s);
+        stage_mark(5, s);
         return MOE_OK;
     }
 
@@ -379,7 +381,6 @@ MOE_API int moe_forward(const void* x, const void* W_router, const void* W_gate_
     g1.out_col_step = 64;
     e = launch_gemm_simt(EPI_SWIGLU, static_cast<const float*>(x_perm), Wgu, g1, L.rows_cap, s);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
-    stage_mark(3, s);
     if (n_shared > 0) {
         g1s.n_tiles = SI / 64;
         g1s.b_tile_step = 64;
@@ -389,14 +390,14 @@ MOE_API int moe_forward(const void* x, const void* W_router, const void* W_gate_
                              (T + 127) / 128 * 128, s);
         if (e != cudaSuccess) return MOE_ERR_CUDA;
     }
-    stage_mark(4, s);
+    stage_mark(3, s);
     g2.n_tiles = d / 64;
     g2.b_tile_step = 64;
     g2.b_half_off = 0;
     g2.out_col_step = 64;
     e = launch_gemm_simt(EPI_SCATTER, static_cast<const float*>(h), Wdn, g2, L.rows_cap, s);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
-    stage_mark(5, s);
+    stage_mark(4, s);
     if (n_shared > 0) {
         g2s.n_tiles = d / 64;
         g2s.b_tile_step = 64;
@@ -409,7 +410,7 @@ MOE_API int moe_forward(const void* x, const void* W_router, const void* W_gate_
         e = launch_combine_slots(slots, T, d, k, y, out_f32, s);
     }
     if (e != cudaSuccess) return MOE_ERR_CUDA;
-    stage_mark(6, s);
+    stage_mark(5, s);
     return MOE_OK;
 }
 

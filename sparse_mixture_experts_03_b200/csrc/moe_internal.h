@@ -67,9 +67,12 @@ cudaError_t launch_gemm_simt(int epi, const float* A, const float* B, const Gemm
                              int rows_cap, cudaStream_t s);
 
 // tcgen05 path.  tmA: A rows [*, K] bf16, box {64, 128}; tmB: B rows [*, K] bf16, box {64, 128}.
+// One launch runs problem 0 and, when a1 != nullptr, problem 1 (same epilogue
+// kind) over one persistent tile list: problem 0's tiles first.
 size_t gemm_tc_smem_bytes();
-cudaError_t launch_gemm_tc(int epi, const CUtensorMap& tmA, const CUtensorMap& tmB,
-                           const GemmArgs& a, int grid, cudaStream_t s);
+cudaError_t launch_gemm_tc(int epi, const CUtensorMap& tmA0, const CUtensorMap& tmB0,
+                           const GemmArgs& a0, const CUtensorMap* tmA1, const CUtensorMap* tmB1,
+                           const GemmArgs* a1, int grid, cudaStream_t s);
 
 cudaError_t launch_selftest_timeout(int* status, unsigned long long limit_ns, cudaStream_t s);
 

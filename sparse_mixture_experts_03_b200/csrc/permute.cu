@@ -67,35 +67,57 @@ __global__ void __launch_bounds__(kPermBlockTokens) perm_count_kernel(
 
 // One CTA: per expert, exclusive scan of the block histogram over blocks
 // (in place), total counts, 128-padded segment offsets, and row_src = -1 on
-// the padding rows.
+// the padding rows.  The histogram is staged through shared memory in
+// coalesced chunks so the per-expert scans run on-chip.
+constexpr int kScanChunkBlocks = 32;
+
 __global__ void __launch_bounds__(1024) perm_scan_kernel(int32_t* __restrict__ block_counts,
                                                          int nb, int E,
                                                          int32_t* __restrict__ counts,
                                                          int32_t* __restrict__ offsets,
                                                          int32_t* __restrict__ row_src) {
+    __shared__ int s_bc[kScanChunkBlocks * kMaxE];
     __shared__ int s_cnt[kMaxE];
     __shared__ int s_off[kMaxE + 1];
     const int tid = threadIdx.x;
-    for (int e = tid; e < E; e += blockDim.x) {
-        int run = 0;
-        for (int b = 0; b < nb; ++b) {
-            int c = block_counts[(size_t)b * E + e];
-            block_counts[(size_t)b * E + e] = run;
-            run += c;
+    for (int e = tid; e < E; e += blockDim.x) s_cnt[e] = 0;
+    for (int b0 = 0; b0 < nb; b0 += kScanChunkBlocks) {
+        const int nbc = min(kScanChunkBlocks, nb - b0);
+        __syncthreads();
+        for (int i = tid; i < nbc * E; i += blockDim.x) s_bc[i] = block_counts[(size_t)b0 * E + i];
+        __syncthreads();
+        for (int e = tid; e < E; e += blockDim.x) {
+            int run = s_cnt[e];
+            for (int b = 0; b < nbc; ++b) {
+                int c = s_bc[b * E + e];
+                s_bc[b * E + e] = run;
+                run += c;
+            }
+            s_cnt[e] = run;
         }
-        counts[e] = run;
-        s_cnt[e] = run;
+        __syncthreads();
+        for (int i = tid; i < nbc * E; i += blockDim.x) block_counts[(size_t)b0 * E + i] = s_bc[i];
     }
     __syncthreads();
-    if (tid == 0) {
-        int run = 0;
-        for (int e = 0; e < E; ++e) {
-            s_off[e] = run;
-            run += (s_cnt[e] + kRowAlign - 1) / kRowAlign * kRowAlign;
+    if (tid < 32) {
+        // warp scan of the padded segment sizes
+        int carry = 0;
+        for (int e0 = 0; e0 < E; e0 += 32) {
+            const int e = e0 + tid;
+            const int v = e < E ? (s_cnt[e] + kRowAlign - 1) / kRowAlign * kRowAlign : 0;
+            int incl = v;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                int n = __shfl_up_sync(0xffffffffu, incl, o);
+                if (tid >= o) incl += n;
+            }
+            if (e < E) s_off[e] = carry + incl - v;
+            carry += __shfl_sync(0xffffffffu, incl, 31);
         }
-        s_off[E] = run;
+        if (tid == 0) s_off[E] = carry;
     }
     __syncthreads();
+    for (int e = tid; e < E; e += blockDim.x) counts[e] = s_cnt[e];
     for (int e = tid; e <= E; e += blockDim.x) offsets[e] = s_off[e];
     for (int i = tid; i < E * kRowAlign; i += blockDim.x) {
         int e = i / kRowAlign, r = i % kRowAlign;

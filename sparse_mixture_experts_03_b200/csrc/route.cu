@@ -42,6 +42,78 @@ __device__ __forceinline__ void warp_argmax(float& v, int& i) {
     }
 }
 
+// Group-limited top-k of one token from its fp32 logits L[0..E) (shared
+// memory), by one warp.  Writes k expert ids (descending, ties to the lower
+// index) and the normalised sigmoid weights.
+template <int EJ>
+__device__ __forceinline__ void warp_topk(const float* L, int lane, int E, int k, int G, int TG,
+                                          int32_t* __restrict__ idx_out,
+                                          float* __restrict__ w_out) {
+    const int gsz = E / G;
+    // group scores: max logit of each group (lane g < G owns group g)
+    float gval = -INFINITY;
+    if (lane < G)
+        for (int e = lane * gsz; e < (lane + 1) * gsz; ++e) gval = fmaxf(gval, L[e]);
+    uint32_t kept = 0;
+    for (int r = 0; r < TG; ++r) {
+        float v = -INFINITY;
+        int i = INT_MAX;
+        if (lane < G && !((kept >> lane) & 1u)) {
+            v = gval;
+            i = lane;
+        }
+        warp_argmax(v, i);
+        kept |= 1u << i;
+    }
+    // candidates: experts lane + 32 j inside kept groups
+    float cv[EJ];
+    bool cand[EJ];
+#pragma unroll
+    for (int j = 0; j < EJ; ++j) {
+        int e = lane + 32 * j;
+        cand[j] = e < E && ((kept >> (e / gsz)) & 1u);
+        cv[j] = cand[j] ? L[e] : -INFINITY;
+    }
+    int sel_e[kMaxK];
+    float sel_l[kMaxK];
+#pragma unroll
+    for (int r = 0; r < kMaxK; ++r) {
+        if (r >= k) break;
+        float bv = -INFINITY;
+        int bi = INT_MAX;
+#pragma unroll
+        for (int j = 0; j < EJ; ++j) {
+            int e = lane + 32 * j;
+            if (cand[j] && beats(cv[j], e, bv, bi)) {
+                bv = cv[j];
+                bi = e;
+            }
+        }
+        warp_argmax(bv, bi);
+#pragma unroll
+        for (int j = 0; j < EJ; ++j)
+            if (lane + 32 * j == bi) cand[j] = false;
+        sel_e[r] = bi;
+        sel_l[r] = bv;
+    }
+    if (lane == 0) {
+        float s[kMaxK], sum = 0.f;
+#pragma unroll
+        for (int r = 0; r < kMaxK; ++r) {
+            if (r >= k) break;
+            s[r] = 1.f / (1.f + expf(-sel_l[r]));
+            sum += s[r];
+        }
+#pragma unroll
+        for (int r = 0; r < kMaxK; ++r) {
+            if (r >= k) break;
+            idx_out[r] = sel_e[r];
+            w_out[r] = s[r] / sum;
+        }
+    }
+}
+
+// CUDA-core router for any E <= 256 (fp32 or bf16 inputs): 32 tokens per CTA.
 template <typename TIn, int EJ>
 __global__ void __launch_bounds__(kRouteThreads) route_kernel(const TIn* __restrict__ x,
                                                               const TIn* __restrict__ Wr, int T,
@@ -66,7 +138,6 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const TIn* __restr
         for (int j = 0; j < EJ; ++j) acc[i][j] = 0.f;
 
     for (int c0 = 0; c0 < d; c0 += kRouteKChunk) {
-        // stage x [32 tokens][32] and W_router [E][32] as fp32
         for (int i = tid; i < kRouteTokens * kRouteKChunk; i += kRouteThreads) {
             int r = i / kRouteKChunk, c = i % kRouteKChunk;
             int t = t0 + r;
@@ -107,75 +178,187 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const TIn* __restr
             }
         }
     __syncthreads();
-
-    const int gsz = E / G;
     for (int tt = 0; tt < 4; ++tt) {
         const int tl = warp * 4 + tt;
         const int t = t0 + tl;
         if (t >= T) break;  // warp-uniform
-        const float* L = logit + tl * (E + 1);
-        // group scores: max logit of each group (lane g < G owns group g)
-        float gval = -INFINITY;
-        if (lane < G)
-            for (int e = lane * gsz; e < (lane + 1) * gsz; ++e) gval = fmaxf(gval, L[e]);
-        uint32_t kept = 0;
-        for (int r = 0; r < TG; ++r) {
-            float v = -INFINITY;
-            int i = INT_MAX;
-            if (lane < G && !((kept >> lane) & 1u)) {
-                v = gval;
-                i = lane;
-            }
-            warp_argmax(v, i);
-            kept |= 1u << i;
-        }
-        // candidates: experts lane + 32 j inside kept groups
-        float cv[EJ];
-        bool cand[EJ];
-#pragma unroll
-        for (int j = 0; j < EJ; ++j) {
-            int e = lane + 32 * j;
-            cand[j] = e < E && ((kept >> (e / gsz)) & 1u);
-            cv[j] = cand[j] ? L[e] : -INFINITY;
-        }
-        int sel_e[kMaxK];
-        float sel_l[kMaxK];
-#pragma unroll
-        for (int r = 0; r < kMaxK; ++r) {
-            if (r >= k) break;
-            float bv = -INFINITY;
-            int bi = INT_MAX;
-#pragma unroll
-            for (int j = 0; j < EJ; ++j) {
-                int e = lane + 32 * j;
-                if (cand[j] && beats(cv[j], e, bv, bi)) {
-                    bv = cv[j];
-                    bi = e;
-                }
-            }
-            warp_argmax(bv, bi);
-#pragma unroll
-            for (int j = 0; j < EJ; ++j)
-                if (lane + 32 * j == bi) cand[j] = false;
-            sel_e[r] = bi;
-            sel_l[r] = bv;
-        }
-        if (lane == 0) {
-            float s[kMaxK], sum = 0.f;
-#pragma unroll
-            for (int r = 0; r < kMaxK; ++r) {
-                if (r >= k) break;
-                s[r] = 1.f / (1.f + expf(-sel_l[r]));
-                sum += s[r];
-            }
-#pragma unroll
-            for (int r = 0; r < kMaxK; ++r) {
-                if (r >= k) break;
-                idx_out[(size_t)t * k + r] = sel_e[r];
-                w_out[(size_t)t * k + r] = s[r] / sum;
-            }
-        }
+        warp_topk<EJ>(logit + tl * (E + 1), lane, E, k, G, TG, idx_out + (size_t)t * k,
+                      w_out + (size_t)t * k);
     }
+}
+
+// ---------------------------------------------------------------------------
+// Tensor-core router for bf16, E <= 128, E % 16 == 0: mma.sync m16n8k16
+// (bf16 in, fp32 accumulate).  CTA = 8 warps over 32 tokens: warp (wm, wk)
+// computes tokens [16 wm, 16 wm + 16) x all E experts over the k-quarter wk of
+// every 256-wide chunk of d; the four partial sums are added in fixed order
+// (wk = 0..3) through shared memory, so the logits do not depend on timing.
+// x and W_router chunks are staged with cp.async (double buffered).
+constexpr int kMmaTokens = 32;
+constexpr int kMmaKC = 256;             // d per pipeline stage (4 warps x 64)
+constexpr int kMmaLd = kMmaKC + 8;      // padded smem row (bf16): conflict-free ldmatrix
+
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem, bool pred) {
+    const uint32_t s = smem_u32(smem);
+    const int n = pred ? 16 : 0;  // zero-fill when out of range
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(s), "l"(gmem), "r"(n)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+__device__ __forceinline__ void ldmatrix_x4(uint32_t (&r)[4], const void* p) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(smem_u32(p)));
+}
+
+__device__ __forceinline__ void mma_bf16_16816(float (&c)[4], const uint32_t (&a)[4],
+                                               uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, "
+        "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+template <int NT>  // NT = E / 8 n-tiles of 8 experts (E = 8 NT, NT even)
+__global__ void __launch_bounds__(256) route_mma_kernel(const __nv_bfloat16* __restrict__ x,
+                                                        const __nv_bfloat16* __restrict__ Wr,
+                                                        int T, int d, int E, int k, int G,
+                                                        int TG, int32_t* __restrict__ idx_out,
+                                                        float* __restrict__ w_out,
+                                                        int* status) {
+    extern __shared__ __align__(16) uint8_t rsm[];
+    __nv_bfloat16* xs = reinterpret_cast<__nv_bfloat16*>(rsm);  // [2][32][kMmaLd]
+    __nv_bfloat16* wsm = xs + 2 * kMmaTokens * kMmaLd;          // [2][E][kMmaLd]
+    float* red = reinterpret_cast<float*>(rsm);                // after the loop: [4][32][E+1]
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int wm = warp & 1, wk = warp >> 1;
+    const int t0 = blockIdx.x * kMmaTokens;
+    if (status != nullptr && blockIdx.x == 0 && tid < 4) status[tid] = 0;
+
+    auto load_chunk = [&](int stage, int c0) {
+        __nv_bfloat16* xd = xs + stage * kMmaTokens * kMmaLd;
+        __nv_bfloat16* wd = wsm + stage * E * kMmaLd;
+        // x: 32 rows x 256 cols = 1024 16-byte pieces
+        for (int i = tid; i < kMmaTokens * (kMmaKC / 8); i += 256) {
+            int r = i / (kMmaKC / 8), c = (i % (kMmaKC / 8)) * 8;
+            int t = t0 + r;
+            cp_async16(xd + r * kMmaLd + c, x + (size_t)(t < T ? t : 0) * d + c0 + c, t < T);
+        }
+        for (int i = tid; i < E * (kMmaKC / 8); i += 256) {
+            int r = i / (kMmaKC / 8), c = (i % (kMmaKC / 8)) * 8;
+            cp_async16(wd + r * kMmaLd + c, Wr + (size_t)r * d + c0 + c, true);
+        }
+        cp_async_commit();
+    };
+
+    float acc[NT][4];
+#pragma unroll
+    for (int n = 0; n < NT; ++n)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) acc[n][q] = 0.f;
+
+    const int n_chunks = d / kMmaKC;
+    load_chunk(0, 0);
+    for (int ch = 0; ch < n_chunks; ++ch) {
+        if (ch + 1 < n_chunks) {
+            load_chunk((ch + 1) & 1, (ch + 1) * kMmaKC);
+            cp_async_wait<1>();
+        } else {
+            cp_async_wait<0>();
+        }
+        __syncthreads();
+        const __nv_bfloat16* xc = xs + (ch & 1) * kMmaTokens * kMmaLd;
+        const __nv_bfloat16* wc = wsm + (ch & 1) * E * kMmaLd;
+#pragma unroll
+        for (int kk = 0; kk < 64; kk += 16) {
+            const int kb = wk * 64 + kk;
+            // A fragment: rows 16 wm + (lane & 15), columns kb + 8 (lane >> 4)
+            uint32_t a[4];
+            ldmatrix_x4(a, xc + (wm * 16 + (lane & 15)) * kMmaLd + kb + 8 * (lane >> 4));
+#pragma unroll
+            for (int n = 0; n < NT; n += 2) {
+                // B fragments of n-tiles n, n+1: expert rows 8n + (lane & 7) + 8 (lane >> 4),
+                // k halves by bit 3 of the lane
+                uint32_t b[4];
+                ldmatrix_x4(b, wc + (8 * n + (lane & 7) + 8 * (lane >> 4)) * kMmaLd + kb +
+                                   8 * ((lane >> 3) & 1));
+                mma_bf16_16816(acc[n], a, b[0], b[1]);
+                mma_bf16_16816(acc[n + 1], a, b[2], b[3]);
+            }
+        }
+        __syncthreads();
+    }
+    // partial logits of this warp's k-quarter -> red[wk][token][expert]
+    const int Ep = E + 1;
+#pragma unroll
+    for (int n = 0; n < NT; ++n) {
+        const int r0 = wm * 16 + (lane >> 2), col = 8 * n + 2 * (lane & 3);
+        float* base = red + (size_t)wk * kMmaTokens * Ep;
+        base[r0 * Ep + col] = acc[n][0];
+        base[r0 * Ep + col + 1] = acc[n][1];
+        base[(r0 + 8) * Ep + col] = acc[n][2];
+        base[(r0 + 8) * Ep + col + 1] = acc[n][3];
+    }
+    __syncthreads();
+    float* logit = red + (size_t)4 * kMmaTokens * Ep;  // [32][E+1]
+    for (int i = tid; i < kMmaTokens * E; i += 256) {
+        const int r = i / E, e = i % E;
+        float v = red[r * Ep + e];
+        v += red[(size_t)kMmaTokens * Ep + r * Ep + e];
+        v += red[(size_t)2 * kMmaTokens * Ep + r * Ep + e];
+        v += red[(size_t)3 * kMmaTokens * Ep + r * Ep + e];
+        logit[r * Ep + e] = (v != v) ? -INFINITY : v;
+    }
+    __syncthreads();
+    for (int tt = 0; tt < 4; ++tt) {
+        const int tl = warp * 4 + tt;
+        const int t = t0 + tl;
+        if (t >= T) break;  // warp-uniform
+        warp_topk<(NT * 8 + 31) / 32>(logit + tl * Ep, lane, E, k, G, TG,
+                                      idx_out + (size_t)t * k, w_out + (size_t)t * k);
+    }
+}
+
+size_t route_mma_smem(int E) {
+    const size_t stage = (size_t)2 * (kMmaTokens + E) * kMmaLd * sizeof(__nv_bfloat16);
+    const size_t red = (size_t)5 * kMmaTokens * (E + 1) * sizeof(float);
+    return stage > red ? stage : red;
+}
+
+cudaError_t launch_route_mma(const void* x, const void* Wr, int T, int d, int E, int k, int G,
+                             int TG, int32_t* idx, float* w, int* status, cudaStream_t s) {
+    const size_t smem = route_mma_smem(E);
+    const dim3 grid((T + kMmaTokens - 1) / kMmaTokens);
+    const __nv_bfloat16* xp = static_cast<const __nv_bfloat16*>(x);
+    const __nv_bfloat16* wp = static_cast<const __nv_bfloat16*>(Wr);
+#define MOE_ROUTE_MMA_CASE(NT)                                                                \
+    case NT: {                                                                                \
+        auto kern = route_mma_kernel<NT>;                                                     \
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, \
+                                             (int)smem);                                      \
+        if (e != cudaSuccess) return e;                                                       \
+        kern<<<grid, 256, smem, s>>>(xp, wp, T, d, E, k, G, TG, idx, w, status);              \
+        return cudaGetLastError();                                                            \
+    }
+    switch (E / 8) {
+        MOE_ROUTE_MMA_CASE(2)
+        MOE_ROUTE_MMA_CASE(4)
+        MOE_ROUTE_MMA_CASE(6)
+        MOE_ROUTE_MMA_CASE(8)
+        MOE_ROUTE_MMA_CASE(10)
+        MOE_ROUTE_MMA_CASE(12)
+        MOE_ROUTE_MMA_CASE(14)
+        MOE_ROUTE_MMA_CASE(16)
+        default:
+            return cudaErrorInvalidValue;
+    }
+#undef MOE_ROUTE_MMA_CASE
 }
 
 template <typename TIn>
@@ -216,6 +399,9 @@ cudaError_t launch_route(const void* x, const void* Wr, int T, int d, int E, int
 
 cudaError_t launch_route_bf16(const void* x, const void* Wr, int T, int d, int E, int k, int G,
                               int TG, int32_t* idx, float* w, int* status, cudaStream_t s) {
+    // tensor-core path for the shapes it tiles exactly; CUDA cores otherwise
+    if (E % 16 == 0 && E <= 128 && d % kMmaKC == 0)
+        return launch_route_mma(x, Wr, T, d, E, k, G, TG, idx, w, status, s);
     return launch_route<__nv_bfloat16>(x, Wr, T, d, E, k, G, TG, idx, w, status, s);
 }
 

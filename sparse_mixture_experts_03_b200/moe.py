@@ -35,9 +35,8 @@ ROW_ALIGN = 128
 SYMBOLS = ["moe_workspace_bytes", "moe_workspace_layout", "moe_route", "moe_forward",
            "moe_get_device_status", "moe_clear_device_status", "moe_selftest_timeout",
            "moe_set_stage_events", "moe_status_string", "moe_version"]
-N_STAGE_EVENTS = 7
-STAGES = ["route", "permute", "gate_up_routed", "gate_up_shared", "down_routed",
-          "down_shared_combine"]
+N_STAGE_EVENTS = 6
+STAGES = ["route", "permute", "gate_up", "down_routed", "down_shared_combine"]
 
 _lib = None
 
