@@ -175,7 +175,9 @@ MOE_API int moe_selftest_timeout(void *workspace, int limit_us, void *stream);
  * by the caller), every following moe_forward in this process records
  * events[i] on its stream: [0] start, [1] after routing, [2] after the
  * permutation, [3] after the gate/up GEMM (routed and shared experts, one
- * launch), [4] after the routed down GEMM, [5] at the end.  events == NULL
+ * launch), [4] after the down GEMM (routed experts, and the shared experts with
+ * the final sum, one launch), [5] at the end (after the separate final sum
+ * kernel that runs only when there are no shared experts).  events == NULL
  * turns it off.  Process-wide setting, not thread-safe.  Returns MOE_OK or
  * MOE_ERR_INVALID_ARG.
  */

@@ -49,7 +49,8 @@ constexpr int kEpiThreads = 128;
 constexpr uint32_t kIdesc = idesc_bf16_f32(BM, BNB);
 constexpr int kMaxOffsets = kMaxE + 1;
 
-struct __align__(8) SmemTail {
+struct __align__(16) SmemTail {
+    uint4 stage[kEpiThreads / 32][32 * 8];  // per epilogue warp: 32 rows x 128 B, swizzled
     uint64_t full[kStages];
     uint64_t empty[kStages];
     uint64_t tfull[2];
@@ -85,13 +86,142 @@ struct TileRef {
     int p, row0, nt, g;
 };
 
+// Epilogue of one tile for the rows of TMEM lane quarter wq (thread `lane`
+// holds row wq*32 + lane of the tile).
 template <int EPI>
+__device__ __forceinline__ void epilogue_tile(uint4* buf, uint32_t taddr, const TileRef& r,
+                                              const GemmArgs& args, int lane, int wq, int col0) {
+    const int grow = r.row0 + wq * 32 + lane;
+    // Epilogue stores go through a per-warp staging buffer: thread `lane`
+    // holds row wq*32 + lane after tcgen05.ld; it writes its 128-byte row
+    // piece to shared memory (16-byte units XOR-swizzled by row, so both
+    // the row-wise writes and the transposed reads are conflict-free),
+    // then each store instruction covers 4 rows x 128 contiguous bytes.
+    const int rr_lo = lane >> 3, q = lane & 7;
+    auto piece = [&](int i) -> uint4 {
+        const int rr = i * 4 + rr_lo;
+        return buf[rr * 8 + (q ^ (rr & 7))];
+    };
+    const int row_base = r.row0 + wq * 32;
+
+    if constexpr (EPI == EPI_SWIGLU) {
+#pragma unroll 1
+        for (int c = 0; c < BNB / 2; c += 64) {
+            uint32_t p[32];
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                uint32_t g[32], u[32];
+                tmem_ld32(taddr + c + 32 * half, g);
+                tmem_ld32(taddr + BNB / 2 + c + 32 * half, u);
+                tmem_ld_wait();
+#pragma unroll
+                for (int i = 0; i < 16; ++i)
+                    p[16 * half + i] = pack_bf16x2(
+                        silu_mul(__uint_as_float(g[2 * i]), __uint_as_float(u[2 * i])),
+                        silu_mul(__uint_as_float(g[2 * i + 1]),
+                                 __uint_as_float(u[2 * i + 1])));
+            }
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                buf[lane * 8 + (j ^ (lane & 7))] =
+                    make_uint4(p[4 * j], p[4 * j + 1], p[4 * j + 2], p[4 * j + 3]);
+            __syncwarp();
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const int row = row_base + i * 4 + rr_lo;
+                const uint4 v = piece(i);
+                if (row < args.valid_rows)
+                    *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(args.out) +
+                                              (size_t)row * args.out_ld + col0 + c +
+                                              8 * q) = v;
+            }
+            __syncwarp();
+        }
+    } else if constexpr (EPI == EPI_SCATTER) {
+        const int src = grow < args.valid_rows ? args.row_src[grow] : -1;
+        const float wv = src >= 0 ? args.topk_w[src] : 0.f;
+#pragma unroll 1
+        for (int c = 0; c < BNB; c += 32) {
+            uint32_t v[32];
+            tmem_ld32(taddr + c, v);
+            tmem_ld_wait();
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                buf[lane * 8 + (j ^ (lane & 7))] = make_uint4(
+                    __float_as_uint(wv * __uint_as_float(v[4 * j])),
+                    __float_as_uint(wv * __uint_as_float(v[4 * j + 1])),
+                    __float_as_uint(wv * __uint_as_float(v[4 * j + 2])),
+                    __float_as_uint(wv * __uint_as_float(v[4 * j + 3])));
+            __syncwarp();
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const int s_rr = __shfl_sync(0xffffffffu, src, i * 4 + rr_lo);
+                const uint4 val = piece(i);
+                if (s_rr >= 0)
+                    *reinterpret_cast<uint4*>(static_cast<float*>(args.out) +
+                                              (size_t)s_rr * args.out_ld + col0 + c +
+                                              4 * q) = val;
+            }
+            __syncwarp();
+        }
+    } else {  // EPI_COMBINE
+#pragma unroll 1
+        for (int c = 0; c < BNB; c += 32) {
+            uint32_t v[32];
+            tmem_ld32(taddr + c, v);
+            tmem_ld_wait();
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                buf[lane * 8 + (j ^ (lane & 7))] =
+                    make_uint4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+            __syncwarp();
+            float4 a[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const uint4 u = piece(i);
+                a[i] = make_float4(__uint_as_float(u.x), __uint_as_float(u.y),
+                                   __uint_as_float(u.z), __uint_as_float(u.w));
+            }
+            __syncwarp();
+            // y = shared + slot_0 + ... + slot_{k-1}, in that order
+            for (int j = 0; j < args.k; ++j) {
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const int t = row_base + i * 4 + rr_lo;
+                    if (t < args.valid_rows) {
+                        const float4 b = __ldcg(reinterpret_cast<const float4*>(
+                            args.slots + ((size_t)t * args.k + j) * args.out_ld + col0 +
+                            c + 4 * q));
+                        a[i].x += b.x;
+                        a[i].y += b.y;
+                        a[i].z += b.z;
+                        a[i].w += b.w;
+                    }
+                }
+            }
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const int t = row_base + i * 4 + rr_lo;
+                if (t >= args.valid_rows) continue;
+                const size_t o = (size_t)t * args.out_ld + col0 + c + 4 * q;
+                if (args.out_f32) {
+                    *reinterpret_cast<float4*>(static_cast<float*>(args.out) + o) = a[i];
+                } else {
+                    *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(args.out) + o) =
+                        make_uint2(pack_bf16x2(a[i].x, a[i].y), pack_bf16x2(a[i].z, a[i].w));
+                }
+            }
+        }
+    }
+}
+
+template <int EPI0, int EPI1>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0,
                            const __grid_constant__ CUtensorMap tmB0,
                            const __grid_constant__ CUtensorMap tmA1,
                            const __grid_constant__ CUtensorMap tmB1, const GemmArgs args0,
-                           const GemmArgs args1, int n_problems) {
+                           const GemmArgs args1, int n_problems, int* sync_counter) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -248,7 +378,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else {
         // ------------------------------------------------ epilogue (warps 2..5)
         const int wq = warp & 3;  // TMEM lane quarter this warp may access
-        const int r_local = wq * 32 + lane;
         int it = 0;
         for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x, ++it) {
             const int acc = it & 1;
@@ -260,98 +389,41 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_after();
             const TileRef r = tile_ref(tile);
             const GemmArgs& args = r.p == 0 ? args0 : args1;
-            const int grow = r.row0 + r_local;
             const uint32_t taddr =
                 tmem_base + (uint32_t)(acc * BNB) + ((uint32_t)(wq * 32) << 16);
             const int col0 = r.nt * args.out_col_step;
 
-            if constexpr (EPI == EPI_SWIGLU) {
-                const bool valid = grow < args.valid_rows;
-                __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(args.out) +
-                                      (size_t)grow * args.out_ld + col0;
-#pragma unroll 1
-                for (int c = 0; c < BNB / 2; c += 32) {
-                    uint32_t g[32], u[32];
-                    tmem_ld32(taddr + c, g);
-                    tmem_ld32(taddr + BNB / 2 + c, u);
-                    tmem_ld_wait();
-                    uint32_t p[16];
-#pragma unroll
-                    for (int i = 0; i < 16; ++i)
-                        p[i] = pack_bf16x2(
-                            silu_mul(__uint_as_float(g[2 * i]), __uint_as_float(u[2 * i])),
-                            silu_mul(__uint_as_float(g[2 * i + 1]),
-                                     __uint_as_float(u[2 * i + 1])));
-                    if (valid) {
-                        uint4* dst = reinterpret_cast<uint4*>(orow + c);
-#pragma unroll
-                        for (int q = 0; q < 4; ++q)
-                            dst[q] = make_uint4(p[4 * q], p[4 * q + 1], p[4 * q + 2], p[4 * q + 3]);
-                    }
-                }
-            } else if constexpr (EPI == EPI_SCATTER) {
-                const int src = grow < args.valid_rows ? args.row_src[grow] : -1;
-                const float wv = src >= 0 ? args.topk_w[src] : 0.f;
-                float* orow = static_cast<float*>(args.out) + (size_t)(src >= 0 ? src : 0) *
-                                                                  args.out_ld + col0;
-#pragma unroll 1
-                for (int c = 0; c < BNB; c += 32) {
-                    uint32_t v[32];
-                    tmem_ld32(taddr + c, v);
-                    tmem_ld_wait();
-                    if (src >= 0) {
-                        float4* dst = reinterpret_cast<float4*>(orow + c);
-#pragma unroll
-                        for (int q = 0; q < 8; ++q)
-                            dst[q] = make_float4(wv * __uint_as_float(v[4 * q]),
-                                                 wv * __uint_as_float(v[4 * q + 1]),
-                                                 wv * __uint_as_float(v[4 * q + 2]),
-                                                 wv * __uint_as_float(v[4 * q + 3]));
-                    }
-                }
-            } else {  // EPI_COMBINE
-                const bool valid = grow < args.valid_rows;
-                const size_t t = valid ? (size_t)grow : 0;
-#pragma unroll 1
-                for (int c = 0; c < BNB; c += 32) {
-                    uint32_t v[32];
-                    tmem_ld32(taddr + c, v);
-                    tmem_ld_wait();
-                    if (valid) {
-                        float a[32];
-#pragma unroll
-                        for (int i = 0; i < 32; ++i) a[i] = __uint_as_float(v[i]);
-                        for (int j = 0; j < args.k; ++j) {
-                            const float4* sp = reinterpret_cast<const float4*>(
-                                args.slots + (t * args.k + j) * args.out_ld + col0 + c);
-#pragma unroll
-                            for (int q = 0; q < 8; ++q) {
-                                float4 b = __ldg(sp + q);
-                                a[4 * q] += b.x;
-                                a[4 * q + 1] += b.y;
-                                a[4 * q + 2] += b.z;
-                                a[4 * q + 3] += b.w;
-                            }
+            if (sync_counter != nullptr && r.p == 1) {
+                // the combine reads slot rows written by problem 0's epilogues in
+                // other CTAs of this launch (all co-resident): wait until every
+                // epilogue warp of every problem-0 tile has published
+                bool ok = true;
+                if (lane == 0) {
+                    const int target = tiles0 * (kEpiThreads / 32);
+                    const uint64_t t0 = globaltimer_ns();
+                    while (ld_acquire(sync_counter) < target) {
+                        if (*abort_flag || globaltimer_ns() - t0 > limit) {
+                            ok = false;
+                            *abort_flag = 1;
+                            set_status(status, MOE_ERR_TIMEOUT, SITE_GEMM_EPILOGUE, 1);
+                            break;
                         }
-                        if (args.out_f32) {
-                            float4* dst = reinterpret_cast<float4*>(
-                                static_cast<float*>(args.out) + t * args.out_ld + col0 + c);
-#pragma unroll
-                            for (int q = 0; q < 8; ++q)
-                                dst[q] = make_float4(a[4 * q], a[4 * q + 1], a[4 * q + 2],
-                                                     a[4 * q + 3]);
-                        } else {
-                            uint4* dst = reinterpret_cast<uint4*>(
-                                static_cast<__nv_bfloat16*>(args.out) + t * args.out_ld + col0 + c);
-#pragma unroll
-                            for (int q = 0; q < 4; ++q)
-                                dst[q] = make_uint4(pack_bf16x2(a[8 * q], a[8 * q + 1]),
-                                                    pack_bf16x2(a[8 * q + 2], a[8 * q + 3]),
-                                                    pack_bf16x2(a[8 * q + 4], a[8 * q + 5]),
-                                                    pack_bf16x2(a[8 * q + 6], a[8 * q + 7]));
-                        }
+                        __nanosleep(256);
                     }
                 }
+                ok = __shfl_sync(0xffffffffu, ok, 0);
+                __syncwarp();
+                if (!ok) break;
+            }
+            if (r.p == 0)
+                epilogue_tile<EPI0>(tail->stage[wq], taddr, r, args0, lane, wq, col0);
+            else
+                epilogue_tile<EPI1>(tail->stage[wq], taddr, r, args1, lane, wq, col0);
+            if (sync_counter != nullptr && r.p == 0) {
+                // publish this warp's slot rows to the combine tiles of this launch
+                __threadfence();
+                __syncwarp();
+                if (lane == 0) atomicAdd(sync_counter, 1);
             }
             tc_fence_before();
             mbar_arrive(&tail->tempty[acc]);
@@ -385,22 +457,38 @@ size_t gemm_tc_smem_bytes() { return kSmemBytes; }
 
 cudaError_t launch_gemm_tc(int epi, const CUtensorMap& tmA0, const CUtensorMap& tmB0,
                            const GemmArgs& a0, const CUtensorMap* tmA1, const CUtensorMap* tmB1,
-                           const GemmArgs* a1, int grid, cudaStream_t s) {
-    void (*kern)(const CUtensorMap, const CUtensorMap, const CUtensorMap, const CUtensorMap,
-                 const GemmArgs, const GemmArgs, int) = nullptr;
+                           const GemmArgs* a1, int grid, cudaStream_t s, int* sync_counter) {
+    using Kern = void (*)(const CUtensorMap, const CUtensorMap, const CUtensorMap,
+                          const CUtensorMap, const GemmArgs, const GemmArgs, int, int*);
+    Kern kern = nullptr;
     switch (epi) {
-        case EPI_SWIGLU: kern = grouped_gemm_tc_kernel<EPI_SWIGLU>; break;
-        case EPI_SCATTER: kern = grouped_gemm_tc_kernel<EPI_SCATTER>; break;
-        case EPI_COMBINE: kern = grouped_gemm_tc_kernel<EPI_COMBINE>; break;
+        case EPI_SWIGLU: kern = grouped_gemm_tc_kernel<EPI_SWIGLU, EPI_SWIGLU>; break;
+        case EPI_SCATTER: kern = grouped_gemm_tc_kernel<EPI_SCATTER, EPI_COMBINE>; break;
+        case EPI_COMBINE: kern = grouped_gemm_tc_kernel<EPI_COMBINE, EPI_COMBINE>; break;
         default: return cudaErrorInvalidValue;
     }
+    if (sync_counter != nullptr && (epi != EPI_SCATTER || a1 == nullptr))
+        return cudaErrorInvalidValue;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)kSmemBytes);
     if (e != cudaSuccess) return e;
     const int np = a1 != nullptr ? 2 : 1;
-    kern<<<grid, kThreads, kSmemBytes, s>>>(tmA0, tmB0, np > 1 ? *tmA1 : tmA0,
-                                            np > 1 ? *tmB1 : tmB0, a0, np > 1 ? *a1 : a0, np);
-    return cudaGetLastError();
+    const CUtensorMap& mA1 = np > 1 ? *tmA1 : tmA0;
+    const CUtensorMap& mB1 = np > 1 ? *tmB1 : tmB0;
+    const GemmArgs& g1 = np > 1 ? *a1 : a0;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = kSmemBytes;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    // tiles of one launch wait on each other only through sync_counter; the
+    // cooperative attribute guarantees every CTA of the grid is resident
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = sync_counter != nullptr ? 1 : 0;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, tmA0, tmB0, mA1, mB1, a0, g1, np, sync_counter);
 }
 
 cudaError_t launch_selftest_timeout(int* status, unsigned long long limit_ns, cudaStream_t s) {

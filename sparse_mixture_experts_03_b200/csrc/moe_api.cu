@@ -342,7 +342,10 @@ MOE_API int moe_forward(const void* x, const void* W_router, const void* W_gate_
         }
         if (e != cudaSuccess) return MOE_ERR_CUDA;
         stage_mark(3, s);
-        // 5. down projection, routed: weighted scatter into token-order slots
+        // 5. down projections: routed experts with the weighted scatter into
+        //    token-order slots, then the shared experts with the fixed-order
+        //    final sum, as one cooperative launch (combine tiles wait for all
+        //    scatter tiles through a device counter)
         g2.n_tiles = d / 256;
         g2.b_tile_step = 256;
         g2.b_half_off = 128;
@@ -350,22 +353,24 @@ MOE_API int moe_forward(const void* x, const void* W_router, const void* W_gate_
         if (!make_map(&tA, h, (uint64_t)L.rows_cap, inter) ||
             !make_map(&tB, W_down, (uint64_t)E * d, inter))
             return MOE_ERR_CUDA;
-        e = launch_gemm_tc(EPI_SCATTER, tA, tB, g2, nullptr, nullptr, nullptr,
-                           grid_for((long long)rows_tiles * g2.n_tiles), s);
-        if (e != cudaSuccess) return MOE_ERR_CUDA;
-        stage_mark(4, s);
-        // 6. down projection, shared, with the final fixed-order sum
+        long long g2_tiles = (long long)rows_tiles * g2.n_tiles;
         if (n_shared > 0) {
             g2s.n_tiles = d / 256;
             g2s.b_tile_step = 256;
             g2s.b_half_off = 128;
             g2s.out_col_step = 256;
-            if (!make_map(&tA, h_sh, (uint64_t)T, SI) || !make_map(&tB, Wsh_dn, (uint64_t)d, SI))
+            if (!make_map(&tA1, h_sh, (uint64_t)T, SI) || !make_map(&tB1, Wsh_dn, (uint64_t)d, SI))
                 return MOE_ERR_CUDA;
-            e = launch_gemm_tc(EPI_COMBINE, tA, tB, g2s, nullptr, nullptr, nullptr,
-                               grid_for((long long)((T + 127) / 128) * g2s.n_tiles), s);
+            g2_tiles += (long long)((T + 127) / 128) * g2s.n_tiles;
+            e = launch_gemm_tc(EPI_SCATTER, tA, tB, g2, &tA1, &tB1, &g2s, grid_for(g2_tiles), s,
+                               status + kStatusSyncWord);
             if (e != cudaSuccess) return MOE_ERR_CUDA;
+            stage_mark(4, s);
         } else {
+            e = launch_gemm_tc(EPI_SCATTER, tA, tB, g2, nullptr, nullptr, nullptr,
+                               grid_for(g2_tiles), s);
+            if (e != cudaSuccess) return MOE_ERR_CUDA;
+            stage_mark(4, s);
             e = launch_combine_slots(slots, T, d, k, y, out_f32, s);
             if (e != cudaSuccess) return MOE_ERR_CUDA;
         }

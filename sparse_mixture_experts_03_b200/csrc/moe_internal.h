@@ -15,6 +15,7 @@ constexpr int kMaxK = 8;
 constexpr int kRowAlign = 128;         // expert segments of the permuted layout are padded to this
 constexpr int kPermBlockTokens = 256;  // tokens per block of the permutation kernels
 constexpr int kStatusWords = 64;       // int32 words of the status region of the workspace
+constexpr int kStatusSyncWord = 8;     // status word used as the scatter->combine tile counter
 
 // Epilogue variants of the grouped GEMMs.
 enum Epi : int {
@@ -70,9 +71,15 @@ cudaError_t launch_gemm_simt(int epi, const float* A, const float* B, const Gemm
 // One launch runs problem 0 and, when a1 != nullptr, problem 1 (same epilogue
 // kind) over one persistent tile list: problem 0's tiles first.
 size_t gemm_tc_smem_bytes();
+// epi selects the pair of epilogues: EPI_SWIGLU (both problems SwiGLU),
+// EPI_SCATTER (problem 0 scatter, problem 1 combine), EPI_COMBINE (combine).
+// With sync_counter (a zeroed device int; EPI_SCATTER with two problems
+// only), problem 1's epilogues wait until all of problem 0's have stored their
+// rows, and the grid is launched cooperatively so every CTA is resident.
 cudaError_t launch_gemm_tc(int epi, const CUtensorMap& tmA0, const CUtensorMap& tmB0,
                            const GemmArgs& a0, const CUtensorMap* tmA1, const CUtensorMap* tmB1,
-                           const GemmArgs* a1, int grid, cudaStream_t s);
+                           const GemmArgs* a1, int grid, cudaStream_t s,
+                           int* sync_counter = nullptr);
 
 cudaError_t launch_selftest_timeout(int* status, unsigned long long limit_ns, cudaStream_t s);
 

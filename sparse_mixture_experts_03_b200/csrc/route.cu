@@ -129,7 +129,7 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const TIn* __restr
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int t0 = blockIdx.x * kRouteTokens;
 
-    if (status != nullptr && blockIdx.x == 0 && tid < 4) status[tid] = 0;
+    if (status != nullptr && blockIdx.x == 0 && tid < 16) status[tid] = 0;
 
     float acc[4][EJ];
 #pragma unroll
@@ -239,7 +239,7 @@ __global__ void __launch_bounds__(256) route_mma_kernel(const __nv_bfloat16* __r
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int wm = warp & 1, wk = warp >> 1;
     const int t0 = blockIdx.x * kMmaTokens;
-    if (status != nullptr && blockIdx.x == 0 && tid < 4) status[tid] = 0;
+    if (status != nullptr && blockIdx.x == 0 && tid < 16) status[tid] = 0;
 
     auto load_chunk = [&](int stage, int c0) {
         __nv_bfloat16* xd = xs + stage * kMmaTokens * kMmaLd;

@@ -36,7 +36,7 @@ SYMBOLS = ["moe_workspace_bytes", "moe_workspace_layout", "moe_route", "moe_forw
            "moe_get_device_status", "moe_clear_device_status", "moe_selftest_timeout",
            "moe_set_stage_events", "moe_status_string", "moe_version"]
 N_STAGE_EVENTS = 6
-STAGES = ["route", "permute", "gate_up", "down_routed", "down_shared_combine"]
+STAGES = ["route", "permute", "gate_up", "down", "combine"]
 
 _lib = None
 
