@@ -93,7 +93,7 @@ enum {
     MOE_WS_X_PERM = 7,       /* in_dt[rows_cap, d] x rows in expert-contiguous order    */
     MOE_WS_H = 8,            /* in_dt[rows_cap, inter] silu(gate) * up, routed rows    */
     MOE_WS_H_SHARED = 9,     /* in_dt[T, n_shared*inter] the same for shared experts   */
-    MOE_WS_SLOTS = 10,       /* f32[T*k, d] w_j * expert output, token order            */
+    MOE_WS_SLOTS = 10,       /* in_dt[T*k, d] w_j * expert output, token order          */
     MOE_WS_TOTAL = 11        /* total size                                            */
 };
 /* rows_cap = T*k + 128*E (the padded permuted layout never needs more). */
@@ -135,12 +135,12 @@ MOE_API int moe_route(const void *x, const void *W_router, int T, int d, int E, 
  *   topk_idx_out, topk_w_out  device, optional (NULL = keep in workspace)
  *   workspace  device, >= moe_workspace_bytes(...) bytes, 256-byte aligned;
  *              its contents need no initialisation and are overwritten
- * Arithmetic: in_dt inputs, fp32 accumulation everywhere; the SwiGLU hidden
- * h is stored as in_dt between the two expert GEMMs; each routed expert's
- * output is scaled by its gate weight in fp32 and the final sum is
- * y = shared + slot_0 + ... + slot_{k-1} in that fixed order, so y is bitwise
- * reproducible from run to run.  bf16 uses tcgen05 tensor cores; f32 uses
- * CUDA cores.
+ * Arithmetic: in_dt inputs, fp32 accumulation in every GEMM; the SwiGLU
+ * hidden h is stored as in_dt between the two expert GEMMs; each routed
+ * expert's output row is scaled by its gate weight in fp32 and stored once as
+ * in_dt (a "slot"); the final sum is y = shared + slot_0 + ... + slot_{k-1}
+ * in fp32, in that fixed order, so y is bitwise reproducible from run to run.
+ * bf16 uses tcgen05 tensor cores; f32 uses CUDA cores.
  */
 MOE_API int moe_forward(const void *x, const void *W_router, const void *W_gate_up,
                         const void *W_down, const void *W_shared, int T, int d, int E, int k,

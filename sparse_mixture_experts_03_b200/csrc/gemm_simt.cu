@@ -96,7 +96,8 @@ __global__ void __launch_bounds__(256) grouped_gemm_simt_kernel(const float* __r
             for (int j = 0; j < 4; ++j) {
                 float a = acc0[i][j];
                 for (int s = 0; s < args.k; ++s)
-                    a += args.slots[((size_t)grow * args.k + s) * args.out_ld + col + j];
+                    a += static_cast<const float*>(
+                        args.slots)[((size_t)grow * args.k + s) * args.out_ld + col + j];
                 if (args.out_f32)
                     static_cast<float*>(args.out)[(size_t)grow * args.out_ld + col + j] = a;
                 else

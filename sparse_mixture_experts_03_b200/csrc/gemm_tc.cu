@@ -138,29 +138,35 @@ __device__ __forceinline__ void epilogue_tile(uint4* buf, uint32_t taddr, const 
             __syncwarp();
         }
     } else if constexpr (EPI == EPI_SCATTER) {
+        // slot rows are bf16: w * acc rounded once, 64 columns per staging round
         const int src = grow < args.valid_rows ? args.row_src[grow] : -1;
         const float wv = src >= 0 ? args.topk_w[src] : 0.f;
 #pragma unroll 1
-        for (int c = 0; c < BNB; c += 32) {
-            uint32_t v[32];
-            tmem_ld32(taddr + c, v);
-            tmem_ld_wait();
+        for (int c = 0; c < BNB; c += 64) {
+            uint32_t p[32];
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                uint32_t v[32];
+                tmem_ld32(taddr + c + 32 * half, v);
+                tmem_ld_wait();
+#pragma unroll
+                for (int i = 0; i < 16; ++i)
+                    p[16 * half + i] = pack_bf16x2(wv * __uint_as_float(v[2 * i]),
+                                                   wv * __uint_as_float(v[2 * i + 1]));
+            }
 #pragma unroll
             for (int j = 0; j < 8; ++j)
-                buf[lane * 8 + (j ^ (lane & 7))] = make_uint4(
-                    __float_as_uint(wv * __uint_as_float(v[4 * j])),
-                    __float_as_uint(wv * __uint_as_float(v[4 * j + 1])),
-                    __float_as_uint(wv * __uint_as_float(v[4 * j + 2])),
-                    __float_as_uint(wv * __uint_as_float(v[4 * j + 3])));
+                buf[lane * 8 + (j ^ (lane & 7))] =
+                    make_uint4(p[4 * j], p[4 * j + 1], p[4 * j + 2], p[4 * j + 3]);
             __syncwarp();
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
                 const int s_rr = __shfl_sync(0xffffffffu, src, i * 4 + rr_lo);
                 const uint4 val = piece(i);
                 if (s_rr >= 0)
-                    *reinterpret_cast<uint4*>(static_cast<float*>(args.out) +
-                                              (size_t)s_rr * args.out_ld + col0 + c +
-                                              4 * q) = val;
+                    *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(args.out) +
+                                              (size_t)s_rr * args.out_ld + col0 + c + 8 * q) =
+                        val;
             }
             __syncwarp();
         }
@@ -183,19 +189,33 @@ __device__ __forceinline__ void epilogue_tile(uint4* buf, uint32_t taddr, const 
                                    __uint_as_float(u.z), __uint_as_float(u.w));
             }
             __syncwarp();
-            // y = shared + slot_0 + ... + slot_{k-1}, in that order
-            for (int j = 0; j < args.k; ++j) {
+            // for 4 rows at a time: all k slot pieces (4 bf16 each) first, then
+            // y = shared + slot_0 + ... + slot_{k-1} in that order
 #pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const int t = row_base + i * 4 + rr_lo;
-                    if (t < args.valid_rows) {
-                        const float4 b = __ldcg(reinterpret_cast<const float4*>(
-                            args.slots + ((size_t)t * args.k + j) * args.out_ld + col0 +
-                            c + 4 * q));
-                        a[i].x += b.x;
-                        a[i].y += b.y;
-                        a[i].z += b.z;
-                        a[i].w += b.w;
+            for (int h4 = 0; h4 < 8; h4 += 4) {
+                uint2 sv[kMaxK][4];
+#pragma unroll
+                for (int j = 0; j < kMaxK; ++j) {
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const int t = row_base + (h4 + i) * 4 + rr_lo;
+                        sv[j][i] = make_uint2(0u, 0u);
+                        if (j < args.k && t < args.valid_rows)
+                            sv[j][i] = __ldcg(reinterpret_cast<const uint2*>(
+                                static_cast<const __nv_bfloat16*>(args.slots) +
+                                ((size_t)t * args.k + j) * args.out_ld + col0 + c + 4 * q));
+                    }
+                }
+#pragma unroll
+                for (int j = 0; j < kMaxK; ++j) {
+                    if (j >= args.k) break;
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        float4& ai = a[h4 + i];
+                        ai.x += __uint_as_float(sv[j][i].x << 16);
+                        ai.y += __uint_as_float(sv[j][i].x & 0xffff0000u);
+                        ai.z += __uint_as_float(sv[j][i].y << 16);
+                        ai.w += __uint_as_float(sv[j][i].y & 0xffff0000u);
                     }
                 }
             }

@@ -63,7 +63,7 @@ bool make_layout(int T, int d, int E, int k, int inter, int n_shared, int in_dt,
         esz * (size_t)L.rows_cap * d,                   // X_PERM
         esz * (size_t)L.rows_cap * inter,               // H
         esz * (size_t)T * n_shared * inter,             // H_SHARED
-        sizeof(float) * Tk * d,                         // SLOTS
+        esz * Tk * d,                                   // SLOTS (in_dt)
     };
     size_t o = 0;
     for (int i = 0; i < MOE_WS_TOTAL; ++i) {
@@ -243,7 +243,7 @@ MOE_API int moe_forward(const void* x, const void* W_router, const void* W_gate_
     void* x_perm = at<char>(workspace, L, MOE_WS_X_PERM);
     void* h = at<char>(workspace, L, MOE_WS_H);
     void* h_sh = at<char>(workspace, L, MOE_WS_H_SHARED);
-    float* slots = at<float>(workspace, L, MOE_WS_SLOTS);
+    void* slots = at<char>(workspace, L, MOE_WS_SLOTS);
     const int SI = n_shared * inter;
     const bool bf16 = in_dt == MOE_BF16;
     const int out_f32 = out_dt == MOE_F32 ? 1 : 0;
@@ -371,7 +371,7 @@ MOE_API int moe_forward(const void* x, const void* W_router, const void* W_gate_
                                grid_for(g2_tiles), s);
             if (e != cudaSuccess) return MOE_ERR_CUDA;
             stage_mark(4, s);
-            e = launch_combine_slots(slots, T, d, k, y, out_f32, s);
+            e = launch_combine_slots(slots, bf16 ? 1 : 0, T, d, k, y, out_f32, s);
             if (e != cudaSuccess) return MOE_ERR_CUDA;
         }
         stage_mark(5, s);
@@ -412,7 +412,7 @@ MOE_API int moe_forward(const void* x, const void* W_router, const void* W_gate_
                              reinterpret_cast<const float*>(Wsh_dn), g2s,
                              (T + 127) / 128 * 128, s);
     } else {
-        e = launch_combine_slots(slots, T, d, k, y, out_f32, s);
+        e = launch_combine_slots(slots, bf16 ? 1 : 0, T, d, k, y, out_f32, s);
     }
     if (e != cudaSuccess) return MOE_ERR_CUDA;
     stage_mark(5, s);

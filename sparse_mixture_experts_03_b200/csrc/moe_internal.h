@@ -20,7 +20,8 @@ constexpr int kStatusSyncWord = 8;     // status word used as the scatter->combi
 // Epilogue variants of the grouped GEMMs.
 enum Epi : int {
     EPI_SWIGLU = 0,   // out = bf16/f32 silu(gate) * up, columns [nt*cols, ...)
-    EPI_SCATTER = 1,  // slots[row_src[r]] = topk_w[row_src[r]] * acc  (rows with row_src < 0 skipped)
+    EPI_SCATTER = 1,  // slots[row_src[r]] = topk_w[row_src[r]] * acc  (rows with row_src < 0 skipped;
+                      // bf16 slots on the tensor-core path, f32 on CUDA cores)
     EPI_COMBINE = 2,  // y[t] = acc + slots[t*k + 0] + ... + slots[t*k + k-1]
 };
 
@@ -42,7 +43,7 @@ struct GemmArgs {
     int out_col_step;          // output columns per N tile
     const int32_t* row_src;    // SCATTER
     const float* topk_w;       // SCATTER
-    const float* slots;        // COMBINE
+    const void* slots;         // COMBINE (bf16 on the tensor-core path, f32 on CUDA cores)
     int k;                     // SCATTER/COMBINE
     int out_f32;               // COMBINE: y dtype (1 f32, 0 bf16); SWIGLU f32 path: 1
     int* status;
@@ -61,8 +62,8 @@ cudaError_t launch_permute(const int32_t* idx, int T, int k, int E, int32_t* blo
 cudaError_t launch_gather_rows(const void* x, int d, int elem_bytes, int k,
                                const int32_t* offsets_total, const int32_t* row_src,
                                int rows_cap, void* x_perm, int num_sms, cudaStream_t s);
-cudaError_t launch_combine_slots(const float* slots, int T, int d, int k, void* y, int out_f32,
-                                 cudaStream_t s);
+cudaError_t launch_combine_slots(const void* slots, int slots_bf16, int T, int d, int k, void* y,
+                                 int out_f32, cudaStream_t s);
 
 cudaError_t launch_gemm_simt(int epi, const float* A, const float* B, const GemmArgs& a,
                              int rows_cap, cudaStream_t s);

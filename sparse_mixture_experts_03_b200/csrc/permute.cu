@@ -190,30 +190,32 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint4* __restric
     }
 }
 
-// y[t] = slots[t*k + 0] + ... + slots[t*k + k-1], in that order (used when
-// there are no shared experts to fold the sum into).
-__global__ void __launch_bounds__(256) combine_slots_kernel(const float4* __restrict__ slots,
+// y[t] = slots[t*k + 0] + ... + slots[t*k + k-1], in that order, in fp32
+// (used when there are no shared experts to fold the sum into).  Slots are f32
+// or bf16; 4 columns per thread.
+template <typename TS>
+__global__ void __launch_bounds__(256) combine_slots_kernel(const TS* __restrict__ slots,
                                                             int T, int d4, int k, void* y,
                                                             int out_f32) {
     const size_t n = (size_t)T * d4;
     for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n;
          i += (size_t)gridDim.x * blockDim.x) {
         const size_t t = i / d4, c = i % d4;
-        float4 a = slots[(t * k) * d4 + c];
-        for (int j = 1; j < k; ++j) {
-            float4 b = slots[(t * k + j) * d4 + c];
-            a.x += b.x;
-            a.y += b.y;
-            a.z += b.z;
-            a.w += b.w;
+        float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int j = 0; j < k; ++j) {
+            const TS* p = slots + ((t * k + j) * d4 + c) * 4;
+            a.x += Elem<TS>::to_f(p[0]);
+            a.y += Elem<TS>::to_f(p[1]);
+            a.z += Elem<TS>::to_f(p[2]);
+            a.w += Elem<TS>::to_f(p[3]);
         }
         if (out_f32) {
             reinterpret_cast<float4*>(y)[i] = a;
         } else {
-            uint2 p;
-            p.x = pack_bf16x2(a.x, a.y);
-            p.y = pack_bf16x2(a.z, a.w);
-            reinterpret_cast<uint2*>(y)[i] = p;
+            uint2 pk;
+            pk.x = pack_bf16x2(a.x, a.y);
+            pk.y = pack_bf16x2(a.z, a.w);
+            reinterpret_cast<uint2*>(y)[i] = pk;
         }
     }
 }
@@ -244,15 +246,19 @@ cudaError_t launch_gather_rows(const void* x, int d, int elem_bytes, int k,
     return cudaGetLastError();
 }
 
-cudaError_t launch_combine_slots(const float* slots, int T, int d, int k, void* y, int out_f32,
-                                 cudaStream_t s) {
+cudaError_t launch_combine_slots(const void* slots, int slots_bf16, int T, int d, int k, void* y,
+                                 int out_f32, cudaStream_t s) {
     const int d4 = d / 4;
     size_t n = (size_t)T * d4;
     int blocks = (int)((n + 255) / 256);
     if (blocks > 148 * 16) blocks = 148 * 16;
     if (blocks < 1) blocks = 1;
-    combine_slots_kernel<<<blocks, 256, 0, s>>>(reinterpret_cast<const float4*>(slots), T, d4, k,
-                                                y, out_f32);
+    if (slots_bf16)
+        combine_slots_kernel<__nv_bfloat16><<<blocks, 256, 0, s>>>(
+            static_cast<const __nv_bfloat16*>(slots), T, d4, k, y, out_f32);
+    else
+        combine_slots_kernel<float><<<blocks, 256, 0, s>>>(static_cast<const float*>(slots), T,
+                                                           d4, k, y, out_f32);
     return cudaGetLastError();
 }
 

@@ -45,7 +45,7 @@ def test_workspace_layout_regions():
     rows_cap = T * k + moe.ROW_ALIGN * E
     assert lay["h"] - lay["x_perm"] >= rows_cap * d * 2
     assert lay["slots"] - lay["h_shared"] >= T * S * I * 2
-    assert lay["total"] - lay["slots"] >= T * k * d * 4
+    assert lay["total"] - lay["slots"] >= T * k * d * 2  # bf16 slots
     assert moe.workspace_bytes(T, d, E, k, I, S, torch.bfloat16) == lay["total"]
 
 
