@@ -40,7 +40,6 @@ constexpr int BM = 128;           // rows per tile (MMA M, TMEM lanes)
 constexpr int BK = 64;            // K per stage: one 128-byte swizzle atom of bf16
 constexpr int BNB = 256;          // B rows per tile (MMA N)
 constexpr int kStages = 4;
-constexpr int kPrefetchKB = 8;    // L2 prefetch distance of the producer, in k-blocks
 constexpr int kABytes = BM * BK * 2;        // 16 KiB
 constexpr int kBBytes = BNB * BK * 2;       // 32 KiB
 constexpr int kStageBytes = kABytes + kBBytes;
@@ -314,26 +313,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t ph = 0;
             bool ok = true;
             uint32_t issued = 0, issued_ph = 0;  // per stage: loaded at least once / parity
-            // L2 prefetch cursor: walks the same (tile, k-block) sequence
-            // kPrefetchKB k-blocks ahead of the loads, so operands that miss in L2
-            // start their trip from HBM before their stage is free
-            int pf_tile = blockIdx.x, pf_kb = 0;
-            auto prefetch_next = [&]() {
-                if (pf_tile >= total_tiles) return;
-                const TileRef pr = tile_ref(pf_tile);
-                const GemmArgs& pa = pr.p == 0 ? args0 : args1;
-                const CUtensorMap* pA = pr.p == 0 ? &tmA0 : &tmA1;
-                const CUtensorMap* pB = pr.p == 0 ? &tmB0 : &tmB1;
-                const int pb0 = (int)(pr.g * pa.b_group_stride) + pr.nt * pa.b_tile_step;
-                tma_prefetch_l2_2d(pA, pf_kb * BK, pr.row0);
-                tma_prefetch_l2_2d(pB, pf_kb * BK, pb0);
-                tma_prefetch_l2_2d(pB, pf_kb * BK, pb0 + pa.b_half_off);
-                if (++pf_kb == pa.K / BK) {
-                    pf_kb = 0;
-                    pf_tile += gridDim.x;
-                }
-            };
-            for (int i = 0; i < kPrefetchKB; ++i) prefetch_next();
             for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x) {
                 const TileRef r = tile_ref(tile);
                 const GemmArgs& a = r.p == 0 ? args0 : args1;
@@ -354,7 +333,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tma_load_2d(sa, mA, &tail->full[s], kb * BK, r.row0);
                     tma_load_2d(sb, mB, &tail->full[s], kb * BK, b0);
                     tma_load_2d(sb + kBBytes / 2, mB, &tail->full[s], kb * BK, b1);
-                    prefetch_next();
                     issued |= 1u << s;
                     issued_ph = (issued_ph & ~(1u << s)) | (ph << s);
                     if (++s == kStages) {

@@ -205,16 +205,9 @@ __device__ __forceinline__ void cp_async16(void* smem, const void* gmem, bool pr
                  : "memory");
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;"); }
-// wait until at most n (0..3) of this thread's cp.async groups are pending
-__device__ __forceinline__ void cp_async_wait_dyn(int n) {
-    if (n <= 0)
-        asm volatile("cp.async.wait_group 0;" ::: "memory");
-    else if (n == 1)
-        asm volatile("cp.async.wait_group 1;" ::: "memory");
-    else if (n == 2)
-        asm volatile("cp.async.wait_group 2;" ::: "memory");
-    else
-        asm volatile("cp.async.wait_group 3;" ::: "memory");
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
 __device__ __forceinline__ void ldmatrix_x4(uint32_t (&r)[4], const void* p) {
@@ -237,11 +230,11 @@ __global__ void __launch_bounds__(256) route_mma_kernel(const __nv_bfloat16* __r
                                                         const __nv_bfloat16* __restrict__ Wr,
                                                         int T, int d, int E, int k, int G,
                                                         int TG, int32_t* __restrict__ idx_out,
-                                                        float* __restrict__ w_out, int* status,
-                                                        int n_stages) {
+                                                        float* __restrict__ w_out,
+                                                        int* status) {
     extern __shared__ __align__(16) uint8_t rsm[];
-    __nv_bfloat16* xs = reinterpret_cast<__nv_bfloat16*>(rsm);  // [n_stages][32][kMmaLd]
-    __nv_bfloat16* wsm = xs + n_stages * kMmaTokens * kMmaLd;   // [n_stages][E][kMmaLd]
+    __nv_bfloat16* xs = reinterpret_cast<__nv_bfloat16*>(rsm);  // [2][32][kMmaLd]
+    __nv_bfloat16* wsm = xs + 2 * kMmaTokens * kMmaLd;          // [2][E][kMmaLd]
     float* red = reinterpret_cast<float*>(rsm);                // after the loop: [4][32][E+1]
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int wm = warp & 1, wk = warp >> 1;
@@ -270,21 +263,18 @@ __global__ void __launch_bounds__(256) route_mma_kernel(const __nv_bfloat16* __r
 #pragma unroll
         for (int q = 0; q < 4; ++q) acc[n][q] = 0.f;
 
-    // multistage cp.async pipeline: chunk ch lives in stage ch % n_stages;
-    // one commit group per chunk slot (empty groups keep the count uniform)
     const int n_chunks = d / kMmaKC;
-    for (int c = 0; c < n_stages - 1; ++c) {
-        if (c < n_chunks) load_chunk(c, c * kMmaKC);
-        cp_async_commit();
-    }
+    load_chunk(0, 0);
     for (int ch = 0; ch < n_chunks; ++ch) {
-        cp_async_wait_dyn(n_stages - 2);
+        if (ch + 1 < n_chunks) {
+            load_chunk((ch + 1) & 1, (ch + 1) * kMmaKC);
+            cp_async_wait<1>();
+        } else {
+            cp_async_wait<0>();
+        }
         __syncthreads();
-        const int pre = ch + n_stages - 1;
-        if (pre < n_chunks) load_chunk(pre % n_stages, pre * kMmaKC);
-        cp_async_commit();
-        const __nv_bfloat16* xc = xs + (ch % n_stages) * kMmaTokens * kMmaLd;
-        const __nv_bfloat16* wc = wsm + (size_t)(ch % n_stages) * E * kMmaLd;
+        const __nv_bfloat16* xc = xs + (ch & 1) * kMmaTokens * kMmaLd;
+        const __nv_bfloat16* wc = wsm + (ch & 1) * E * kMmaLd;
 #pragma unroll
         for (int kk = 0; kk < 64; kk += 16) {
             const int kb = wk * 64 + kk;
@@ -302,9 +292,8 @@ __global__ void __launch_bounds__(256) route_mma_kernel(const __nv_bfloat16* __r
                 mma_bf16_16816(acc[n + 1], a, b[2], b[3]);
             }
         }
+        __syncthreads();
     }
-    cp_async_wait_dyn(0);
-    __syncthreads();
     // partial logits of this warp's k-quarter -> red[wk][token][expert]
     const int Ep = E + 1;
 #pragma unroll
@@ -336,17 +325,8 @@ __global__ void __launch_bounds__(256) route_mma_kernel(const __nv_bfloat16* __r
     }
 }
 
-constexpr size_t kRouteSmemBudget = 200 * 1024;
-
-int route_mma_stages(int E) {
-    const size_t stage = (size_t)(kMmaTokens + E) * kMmaLd * sizeof(__nv_bfloat16);
-    int n = (int)(kRouteSmemBudget / stage);
-    return n < 2 ? 2 : (n > 4 ? 4 : n);
-}
-
 size_t route_mma_smem(int E) {
-    const size_t stage = (size_t)route_mma_stages(E) * (kMmaTokens + E) * kMmaLd *
-                         sizeof(__nv_bfloat16);
+    const size_t stage = (size_t)2 * (kMmaTokens + E) * kMmaLd * sizeof(__nv_bfloat16);
     const size_t red = (size_t)5 * kMmaTokens * (E + 1) * sizeof(float);
     return stage > red ? stage : red;
 }
@@ -363,8 +343,7 @@ cudaError_t launch_route_mma(const void* x, const void* Wr, int T, int d, int E,
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, \
                                              (int)smem);                                      \
         if (e != cudaSuccess) return e;                                                       \
-        kern<<<grid, 256, smem, s>>>(xp, wp, T, d, E, k, G, TG, idx, w, status,                 \
-                                     route_mma_stages(E));                                    \
+        kern<<<grid, 256, smem, s>>>(xp, wp, T, d, E, k, G, TG, idx, w, status);              \
         return cudaGetLastError();                                                            \
     }
     switch (E / 8) {
