@@ -171,7 +171,8 @@ __global__ void __launch_bounds__(kPermBlockTokens) perm_rank_kernel(
 }
 
 // x_perm[r] = x[row_src[r] / k] for every real row r < offsets[E]; one warp
-// per row, 16-byte vectors.
+// per row, 16-byte vectors, up to 8 vectors per lane loaded before any store
+// so each lane keeps 8 loads in flight.
 __global__ void __launch_bounds__(256) gather_rows_kernel(const uint4* __restrict__ x,
                                                           int vec_per_row, int k,
                                                           const int32_t* __restrict__ total_rows,
@@ -186,7 +187,19 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint4* __restric
         if (src < 0) continue;
         const uint4* s = x + (size_t)(src / k) * vec_per_row;
         uint4* dst = x_perm + (size_t)r * vec_per_row;
-        for (int i = lane; i < vec_per_row; i += 32) dst[i] = __ldg(s + i);
+        for (int i0 = 0; i0 < vec_per_row; i0 += 8 * 32) {
+            uint4 v[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int i = i0 + u * 32 + lane;
+                if (i < vec_per_row) v[u] = __ldg(s + i);
+            }
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int i = i0 + u * 32 + lane;
+                if (i < vec_per_row) dst[i] = v[u];
+            }
+        }
     }
 }
 

@@ -42,6 +42,19 @@ __device__ __forceinline__ void warp_argmax(float& v, int& i) {
     }
 }
 
+// Argmax over each aligned segment of 8 lanes (same tie rule as warp_argmax).
+__device__ __forceinline__ void seg8_argmax(float& v, int& i) {
+#pragma unroll
+    for (int off = 4; off > 0; off >>= 1) {
+        float ov = __shfl_xor_sync(0xffffffffu, v, off);
+        int oi = __shfl_xor_sync(0xffffffffu, i, off);
+        if (oi != INT_MAX && beats(ov, oi, v, i)) {
+            v = ov;
+            i = oi;
+        }
+    }
+}
+
 // Group-limited top-k of one token from its fp32 logits L[0..E) (shared
 // memory), by one warp.  Writes k expert ids (descending, ties to the lower
 // index) and the normalised sigmoid weights.
@@ -241,17 +254,20 @@ __global__ void __launch_bounds__(256) route_mma_kernel(const __nv_bfloat16* __r
     const int t0 = blockIdx.x * kMmaTokens;
     if (status != nullptr && blockIdx.x == 0 && tid < 16) status[tid] = 0;
 
+    // each thread copies fixed (row, 16-byte column) pieces of every chunk
     auto load_chunk = [&](int stage, int c0) {
         __nv_bfloat16* xd = xs + stage * kMmaTokens * kMmaLd;
         __nv_bfloat16* wd = wsm + stage * E * kMmaLd;
-        // x: 32 rows x 256 cols = 1024 16-byte pieces
-        for (int i = tid; i < kMmaTokens * (kMmaKC / 8); i += 256) {
-            int r = i / (kMmaKC / 8), c = (i % (kMmaKC / 8)) * 8;
-            int t = t0 + r;
+        // x: 32 rows x 256 cols = 1024 16-byte pieces, 4 per thread
+#pragma unroll
+        for (int m = 0; m < kMmaTokens * (kMmaKC / 8) / 256; ++m) {
+            const int i = tid + 256 * m;
+            const int r = i >> 5, c = (i & 31) * 8;
+            const int t = t0 + r;
             cp_async16(xd + r * kMmaLd + c, x + (size_t)(t < T ? t : 0) * d + c0 + c, t < T);
         }
         for (int i = tid; i < E * (kMmaKC / 8); i += 256) {
-            int r = i / (kMmaKC / 8), c = (i % (kMmaKC / 8)) * 8;
+            const int r = i >> 5, c = (i & 31) * 8;
             cp_async16(wd + r * kMmaLd + c, Wr + (size_t)r * d + c0 + c, true);
         }
         cp_async_commit();
@@ -316,12 +332,76 @@ __global__ void __launch_bounds__(256) route_mma_kernel(const __nv_bfloat16* __r
         logit[r * Ep + e] = (v != v) ? -INFINITY : v;
     }
     __syncthreads();
-    for (int tt = 0; tt < 4; ++tt) {
-        const int tl = warp * 4 + tt;
+    if (G <= 8 && 8 % G == 0) {
+        // 8 lanes per token, all 32 tokens at once: lane `sub` of a token owns
+        // experts [sub * NT, sub * NT + NT) (E / 8 = NT of them); a group of
+        // E / G experts spans 8 / G consecutive lanes
+        const int sub = lane & 7;
+        const int tl = warp * 4 + (lane >> 3);
         const int t = t0 + tl;
-        if (t >= T) break;  // warp-uniform
-        warp_topk<(NT * 8 + 31) / 32>(logit + tl * Ep, lane, E, k, G, TG,
-                                      idx_out + (size_t)t * k, w_out + (size_t)t * k);
+        const float* L = logit + tl * Ep;
+        float v[NT];
+#pragma unroll
+        for (int i = 0; i < NT; ++i) v[i] = L[sub * NT + i];
+        const int lanes_per_group = 8 / G;
+        const int gid = sub / lanes_per_group;
+        float gmax = v[0];
+#pragma unroll
+        for (int i = 1; i < NT; ++i) gmax = fmaxf(gmax, v[i]);
+        for (int o = 1; o < lanes_per_group; o <<= 1)
+            gmax = fmaxf(gmax, __shfl_xor_sync(0xffffffffu, gmax, o));
+        uint32_t kept = 0;
+        for (int r = 0; r < TG; ++r) {
+            float bv = ((kept >> gid) & 1u) ? -INFINITY : gmax;
+            int bi = ((kept >> gid) & 1u) ? INT_MAX : gid;
+            seg8_argmax(bv, bi);
+            kept |= 1u << bi;
+        }
+        const bool mine_kept = (kept >> gid) & 1u;
+        uint32_t taken = 0;  // bit i: expert sub * NT + i already chosen
+        int sel_e[kMaxK];
+        float sel_l[kMaxK];
+#pragma unroll
+        for (int r = 0; r < kMaxK; ++r) {
+            if (r >= k) break;
+            float bv = -INFINITY;
+            int bi = INT_MAX;
+            if (mine_kept) {
+#pragma unroll
+                for (int i = 0; i < NT; ++i)
+                    if (!((taken >> i) & 1u) && beats(v[i], sub * NT + i, bv, bi)) {
+                        bv = v[i];
+                        bi = sub * NT + i;
+                    }
+            }
+            seg8_argmax(bv, bi);
+            if (bi / NT == sub) taken |= 1u << (bi - sub * NT);
+            sel_e[r] = bi;
+            sel_l[r] = bv;
+        }
+        if (sub == 0 && t < T) {
+            float sc[kMaxK], sum = 0.f;
+#pragma unroll
+            for (int r = 0; r < kMaxK; ++r) {
+                if (r >= k) break;
+                sc[r] = 1.f / (1.f + expf(-sel_l[r]));
+                sum += sc[r];
+            }
+#pragma unroll
+            for (int r = 0; r < kMaxK; ++r) {
+                if (r >= k) break;
+                idx_out[(size_t)t * k + r] = sel_e[r];
+                w_out[(size_t)t * k + r] = sc[r] / sum;
+            }
+        }
+    } else {
+        for (int tt = 0; tt < 4; ++tt) {
+            const int tl = warp * 4 + tt;
+            const int t = t0 + tl;
+            if (t >= T) break;  // warp-uniform
+            warp_topk<(NT * 8 + 31) / 32>(logit + tl * Ep, lane, E, k, G, TG,
+                                          idx_out + (size_t)t * k, w_out + (size_t)t * k);
+        }
     }
 }
 
