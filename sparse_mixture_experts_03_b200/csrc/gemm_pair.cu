@@ -1,0 +1,569 @@
+// Grouped GEMM in "weights x tokens" orientation on CTA pairs (tcgen05
+// cta_group::2, sm_100a).
+//
+// Each expert GEMM out[t, f] = sum_c act[t, c] * W[f, c] is computed as
+// D[f, t] = W[f, :] . act[t, :]: the expert's weight rows are the MMA's M
+// operand (256 rows per CTA pair, 128 per CTA) and the expert's tokens are
+// the N operand (up to 256 per tile, any multiple of 16).  A ragged expert
+// therefore costs at most 15 padding columns, not a 128-row tile, and a
+// decode-sized batch (a few tokens per expert) becomes a stream of weight
+// tiles with a thin N.  The pair splits the weight rows (A) and the token
+// rows (B) between its two CTAs; each CTA loads only its own halves with TMA
+// into its own shared memory (no multicast), so per CTA a pipeline stage is
+// 16 KiB of weights + at most 16 KiB of tokens and 6 stages fit.
+//
+// Roles (both CTAs, 6 warps each): warp 0 lane 0 issues TMA loads into its
+// CTA's stage ring; the full-barrier of a stage lives in the pair's first CTA
+// (the MMA issuer) and receives the transaction bytes of both CTAs' loads;
+// warp 1 lane 0 of the first CTA issues tcgen05.mma.cta_group::2 and commits
+// the stage's empty barrier and the accumulator's full barrier in both CTAs;
+// warps 2..5 of each CTA read their 128 TMEM lanes (= weight rows) x N columns
+// (= tokens), transpose through shared memory and store token-major rows.
+//
+// Epilogues:
+//   SWIGLU  a CTA's 128 weight rows are 64 gate rows then the 64 matching up
+//           rows, so h = silu(gate) * up for 64 features is formed inside the
+//           CTA (SwiGLU: "大模型工程（一）：Transformer 到 MoE", section
+//           "变了什么，为什么变", item 3) and written as bf16 h[token][feature].
+//   SCATTER routed down projection: the row of token column t goes to slot
+//           row_src[b_row + t], scaled by its gate weight, stored bf16 (the
+//           weighted combine of the MoEBlock listing, section "混合专家：更多
+//           参数，相同 FLOPs").
+//   COMBINE shared down projection plus the final sum
+//           y = shared + slot_0 + ... + slot_{k-1}, fixed order, fp32.
+// Every wait is bounded (status word + early exit, never a trap).
+#include "moe_device.cuh"
+#include "moe_internal.h"
+
+namespace moe {
+
+namespace {
+
+constexpr int kBK = 64;                          // K per stage (one 128-byte swizzle atom)
+constexpr int kARows = 128;                      // weight rows per CTA (MMA M = 256 per pair)
+constexpr int kABytes = kARows * kBK * 2;        // 16 KiB
+constexpr int kBBox = 32;                        // token rows per B box
+constexpr int kBMaxRows = 128;                   // token rows per CTA (N <= 256 per pair)
+constexpr int kBBytes = kBMaxRows * kBK * 2;     // 16 KiB
+constexpr int kStageBytes = kABytes + kBBytes;   // 32 KiB
+constexpr int kStages = 6;
+constexpr int kNTile = 256;                      // tokens per tile
+constexpr int kTmemCols = 512;                   // 2 accumulators x 256 fp32 columns
+constexpr int kThreads = 192;
+constexpr int kEpiWarps = 4;
+constexpr int kMaxGroupsP = kMaxE + 1;
+
+struct __align__(16) PairTail {
+    // epilogue staging, reused per 32-token chunk:
+    //   SWIGLU:  up values [64][33] f32 (8448 B) + h [32][64] bf16 (4096 B)
+    //   SCATTER: [32 tokens][128] bf16 (8192 B)
+    //   COMBINE: [32 tokens][128 + 4] f32 (16896 B)
+    float stage[32 * 132];
+    int tile_src[kNTile];     // SCATTER: slot index of each token column (-1 beyond N)
+    float tile_w[kNTile];     // SCATTER: gate weight of each token column
+    uint64_t full[kStages];
+    uint64_t empty[kStages];
+    uint64_t tfull[2];
+    uint64_t tempty[2];
+    uint64_t drain;
+    uint32_t tmem_base;
+    int abort;
+    int seg_off[2][kMaxGroupsP];   // first token row of each group
+    int tile_off[2][kMaxGroupsP];  // first tile of each group
+};
+
+constexpr size_t kSmemBytes = 1024 + (size_t)kStages * kStageBytes + sizeof(PairTail);
+static_assert(kSmemBytes <= 232448, "shared memory per CTA");
+
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+// shared::cluster address of the same shared variable in CTA `rank` of the cluster
+__device__ __forceinline__ uint32_t map_to_rank(const void* p, uint32_t rank) {
+    uint32_t out;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(out) : "r"(smem_u32(p)), "r"(rank));
+    return out;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;"
+                 ::: "memory");
+}
+__device__ __forceinline__ void epi_bar() {  // the 4 epilogue warps only
+    asm volatile("bar.sync 1, %0;" ::"n"(kEpiWarps * 32) : "memory");
+}
+// AND of `ok` over the 4 epilogue warps (also a barrier among them)
+__device__ __forceinline__ bool epi_all(bool ok) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred q, o;\n\t"
+        "setp.ne.u32 q, %1, 0;\n\t"
+        "bar.red.and.pred o, 1, %2, q;\n\t"
+        "selp.u32 %0, 1, 0, o;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)ok), "n"(kEpiWarps * 32)
+        : "memory");
+    return r != 0;
+}
+// TMA 2-D tile load whose completion is reported to an mbarrier of either
+// CTA of the pair (shared::cluster address), no multicast.
+__device__ __forceinline__ void tma_load_2d_pair(void* smem_dst, const CUtensorMap* map,
+                                                 uint32_t bar_cluster, int c0, int c1) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(smem_dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster), "r"(c0), "r"(c1)
+        : "memory");
+}
+__device__ __forceinline__ void arrive_expect_tx_local(uint64_t* bar, uint32_t bytes) {
+    mbar_arrive_expect_tx(bar, bytes);
+}
+__device__ __forceinline__ void tc_mma_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                            uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+// arrive (once) on the mbarrier at shared::cluster address `bar` when all
+// previously issued tcgen05 operations of this thread have completed
+__device__ __forceinline__ void tc_commit_pair(uint32_t bar_cluster) {
+    asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                     bar_cluster)
+                 : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar_cluster) {
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster)
+                 : "memory");
+}
+
+struct Tile {
+    int p;      // problem
+    int g;      // group (expert)
+    int ft;     // feature tile
+    int b_row;  // first token row of the tile in the B tensor
+    int n_real; // tokens in the tile (1..256)
+    int n;      // MMA N: n_real rounded up to 16
+};
+
+__device__ __forceinline__ int upper_group(const int* off, int n, int v) {
+    // largest g in [0, n) with off[g] <= v
+    int lo = 0, hi = n - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (off[mid] <= v)
+            lo = mid;
+        else
+            hi = mid - 1;
+    }
+    return lo;
+}
+
+__device__ __forceinline__ float silu_mul(float g, float u) {
+    return __fdividef(g, 1.0f + __expf(-g)) * u;
+}
+
+template <int EPI>
+__device__ __forceinline__ void pair_epilogue(PairTail* tail, uint32_t taddr, const Tile& t,
+                                              const PairArgs& a, uint32_t cta, int ew, int lane) {
+    const int etid = ew * 32 + lane;  // 0..127 within the epilogue warps
+    if constexpr (EPI == EPI_SCATTER) {
+        // slot index and weight of every token column of the tile
+        for (int i = etid; i < kNTile; i += kEpiWarps * 32) {
+            int src = -1;
+            float wv = 0.f;
+            if (i < t.n_real) {
+                src = a.row_src[t.b_row + i];
+                wv = src >= 0 ? a.topk_w[src] : 0.f;
+            }
+            tail->tile_src[i] = src;
+            tail->tile_w[i] = wv;
+        }
+        epi_bar();
+    }
+    for (int c0 = 0; c0 < t.n; c0 += 32) {
+        uint32_t v[32];
+        tmem_ld32(taddr + (uint32_t)c0, v);  // my weight row (lane) x 32 tokens
+        tmem_ld_wait();
+        if constexpr (EPI == EPI_SWIGLU) {
+            float* up = tail->stage;                                          // [64][33]
+            __nv_bfloat16* hb = reinterpret_cast<__nv_bfloat16*>(tail->stage + 64 * 33);  // [32][64]
+            const int fl = (ew & 1) * 32 + lane;  // feature within this CTA's 64
+            if (ew >= 2) {
+#pragma unroll
+                for (int i = 0; i < 32; ++i) up[fl * 33 + i] = __uint_as_float(v[i]);
+            }
+            epi_bar();
+            if (ew < 2) {
+#pragma unroll
+                for (int i = 0; i < 32; ++i)
+                    hb[i * 64 + fl] = __float2bfloat16_rn(
+                        silu_mul(__uint_as_float(v[i]), up[fl * 33 + i]));
+            }
+            epi_bar();
+            // 32 tokens x 128 B: thread -> token etid / 4, 32-byte piece etid % 4
+            const int tk = etid >> 2, pc = etid & 3;
+            if (c0 + tk < t.n_real) {
+                const uint4* s = reinterpret_cast<const uint4*>(hb + tk * 64 + pc * 16);
+                uint4* d = reinterpret_cast<uint4*>(
+                    static_cast<__nv_bfloat16*>(a.out) + (size_t)(t.b_row + c0 + tk) * a.out_ld +
+                    t.ft * a.out_col_step + cta * 64 + pc * 16);
+                d[0] = s[0];
+                d[1] = s[1];
+            }
+            epi_bar();
+        } else if constexpr (EPI == EPI_SCATTER) {
+            __nv_bfloat16* sb = reinterpret_cast<__nv_bfloat16*>(tail->stage);  // [32][128]
+            const int fl = ew * 32 + lane;
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+                sb[i * 128 + fl] = __float2bfloat16_rn(tail->tile_w[c0 + i] * __uint_as_float(v[i]));
+            epi_bar();
+            // 32 tokens x 256 B: thread -> token etid / 4, 64-byte piece etid % 4
+            const int tk = etid >> 2, pc = etid & 3;
+            const int src = tail->tile_src[c0 + tk];
+            if (src >= 0) {
+                const uint4* s = reinterpret_cast<const uint4*>(sb + tk * 128 + pc * 32);
+                uint4* d = reinterpret_cast<uint4*>(
+                    static_cast<__nv_bfloat16*>(a.out) + (size_t)src * a.out_ld +
+                    t.ft * a.out_col_step + cta * 128 + pc * 32);
+#pragma unroll
+                for (int q = 0; q < 4; ++q) d[q] = s[q];
+            }
+            epi_bar();
+        } else {  // EPI_COMBINE
+            float* sf = tail->stage;  // [32][132]
+            const int fl = ew * 32 + lane;
+#pragma unroll
+            for (int i = 0; i < 32; ++i) sf[i * 132 + fl] = __uint_as_float(v[i]);
+            epi_bar();
+            // thread -> token etid / 4, 32 features (etid % 4) * 32
+            const int tk = etid >> 2, pc = etid & 3;
+            const int tok = t.b_row + c0 + tk;
+            if (c0 + tk < t.n_real) {
+                const int col = t.ft * a.out_col_step + cta * 128 + pc * 32;
+                float acc[32];
+#pragma unroll
+                for (int i = 0; i < 32; ++i) acc[i] = sf[tk * 132 + pc * 32 + i];
+                const __nv_bfloat16* slots = static_cast<const __nv_bfloat16*>(a.slots);
+                for (int j = 0; j < a.k; ++j) {
+                    const uint4* sp = reinterpret_cast<const uint4*>(
+                        slots + ((size_t)tok * a.k + j) * a.out_ld + col);
+                    uint4 q4[4];
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) q4[q] = __ldcg(sp + q);
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const uint32_t w4[4] = {q4[q].x, q4[q].y, q4[q].z, q4[q].w};
+#pragma unroll
+                        for (int h = 0; h < 4; ++h) {
+                            acc[q * 8 + 2 * h] += __uint_as_float(w4[h] << 16);
+                            acc[q * 8 + 2 * h + 1] += __uint_as_float(w4[h] & 0xffff0000u);
+                        }
+                    }
+                }
+                if (a.out_f32) {
+                    float4* d = reinterpret_cast<float4*>(static_cast<float*>(a.out) +
+                                                          (size_t)tok * a.out_ld + col);
+#pragma unroll
+                    for (int q = 0; q < 8; ++q)
+                        d[q] = make_float4(acc[4 * q], acc[4 * q + 1], acc[4 * q + 2], acc[4 * q + 3]);
+                } else {
+                    uint4* d = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.out) +
+                                                        (size_t)tok * a.out_ld + col);
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)
+                        d[q] = make_uint4(pack_bf16x2(acc[8 * q], acc[8 * q + 1]),
+                                          pack_bf16x2(acc[8 * q + 2], acc[8 * q + 3]),
+                                          pack_bf16x2(acc[8 * q + 4], acc[8 * q + 5]),
+                                          pack_bf16x2(acc[8 * q + 6], acc[8 * q + 7]));
+                }
+            }
+            epi_bar();
+        }
+    }
+}
+
+template <int EPI>
+__global__ void __launch_bounds__(kThreads, 1)
+    pair_gemm_kernel(const __grid_constant__ CUtensorMap tmA0,
+                     const __grid_constant__ CUtensorMap tmB0,
+                     const __grid_constant__ CUtensorMap tmA1,
+                     const __grid_constant__ CUtensorMap tmB1, const PairArgs args0,
+                     const PairArgs args1, int n_problems) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    PairTail* tail = reinterpret_cast<PairTail*>(smem + (size_t)kStages * kStageBytes);
+    volatile int* abort_flag = &tail->abort;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const uint32_t cta = cluster_ctarank();  // 0: MMA issuer of the pair
+    const int pair = blockIdx.x >> 1, n_pairs = gridDim.x >> 1;
+    int* const status = args0.status;
+    const uint64_t limit = args0.wait_limit_ns;
+
+    if (tid == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&tail->full[s], 1);   // used in CTA 0: its producer's expect_tx
+            mbar_init(&tail->empty[s], 1);  // one commit from the MMA issuer
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(&tail->tfull[a], 1);
+            mbar_init(&tail->tempty[a], 2 * kEpiWarps);  // used in CTA 0: both CTAs' warps
+        }
+        mbar_init(&tail->drain, 1);
+        tail->abort = 0;
+        fence_barrier_init();
+    }
+    // group offsets of both problems: rows and tiles (exclusive prefix sums)
+    if (warp == 0) {
+        for (int p = 0; p < n_problems; ++p) {
+            const PairArgs& a = p == 0 ? args0 : args1;
+            const int ng = a.counts != nullptr ? a.n_groups : 1;
+            int carry_r = 0, carry_t = 0;
+            for (int g0 = 0; g0 < ng; g0 += 32) {
+                const int g = g0 + lane;
+                const int c = g < ng ? (a.counts != nullptr ? a.counts[g] : a.static_rows) : 0;
+                const int tl = ((c + kNTile - 1) / kNTile) * a.n_ftiles;
+                int ir = c, it = tl;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const int nr = __shfl_up_sync(0xffffffffu, ir, o);
+                    const int nt = __shfl_up_sync(0xffffffffu, it, o);
+                    if (lane >= o) {
+                        ir += nr;
+                        it += nt;
+                    }
+                }
+                if (g < ng) {
+                    tail->seg_off[p][g] = carry_r + ir - c;
+                    tail->tile_off[p][g] = carry_t + it - tl;
+                }
+                carry_r += __shfl_sync(0xffffffffu, ir, 31);
+                carry_t += __shfl_sync(0xffffffffu, it, 31);
+            }
+            if (lane == 0) {
+                tail->seg_off[p][ng] = carry_r;
+                tail->tile_off[p][ng] = carry_t;
+            }
+        }
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         smem_u32(&tail->tmem_base)),
+                     "r"(kTmemCols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync_all();  // barrier init of both CTAs visible before any cross-CTA signal
+    tc_fence_after();
+
+    const uint32_t tmem_base = tail->tmem_base;
+    const int ng0 = args0.counts != nullptr ? args0.n_groups : 1;
+    const int ng1 = args1.counts != nullptr ? args1.n_groups : 1;
+    const int tiles0 = tail->tile_off[0][ng0];
+    const int tiles1 = n_problems > 1 ? tail->tile_off[1][ng1] : 0;
+    const int total_tiles = tiles0 + tiles1;
+
+    // tile -> (problem, expert, feature tile, token chunk); inside an expert the
+    // feature tile is the slow index so the token chunks of one weight tile are
+    // neighbours in the tile order (weights fetched from HBM once, re-read in L2)
+    auto decode = [&](int tile) {
+        Tile t;
+        t.p = tile < tiles0 ? 0 : 1;
+        const PairArgs& a = t.p == 0 ? args0 : args1;
+        const int lt = t.p == 0 ? tile : tile - tiles0;
+        const int ng = t.p == 0 ? ng0 : ng1;
+        t.g = upper_group(tail->tile_off[t.p], ng, lt);
+        const int cnt = tail->seg_off[t.p][t.g + 1] - tail->seg_off[t.p][t.g];
+        const int nch = (cnt + kNTile - 1) / kNTile;
+        const int local = lt - tail->tile_off[t.p][t.g];
+        t.ft = local / nch;
+        const int ch = local % nch;
+        t.b_row = a.b_row_base + tail->seg_off[t.p][t.g] + ch * kNTile;
+        t.n_real = min(kNTile, cnt - ch * kNTile);
+        t.n = (t.n_real + 15) & ~15;
+        return t;
+    };
+
+    if (warp == 0) {
+        // ------------------------------------------------ TMA producer (both CTAs)
+        if (lane == 0) {
+            tma_prefetch_desc(&tmA0);
+            tma_prefetch_desc(&tmB0);
+            if (n_problems > 1) {
+                tma_prefetch_desc(&tmA1);
+                tma_prefetch_desc(&tmB1);
+            }
+            int s = 0;
+            uint32_t ph = 0;
+            bool ok = true;
+            for (int tile = pair; ok && tile < total_tiles; tile += n_pairs) {
+                const Tile t = decode(tile);
+                const PairArgs& a = t.p == 0 ? args0 : args1;
+                const CUtensorMap* mA = t.p == 0 ? &tmA0 : &tmA1;
+                const CUtensorMap* mB = t.p == 0 ? &tmB0 : &tmB1;
+                const int a_row0 = (int)(t.g * a.a_group_stride) + t.ft * a.a_tile_step +
+                                   (int)cta * a.a_cta_step;
+                const int half_n = t.n >> 1;
+                const int b_row0 = t.b_row + (int)cta * half_n;
+                const int n_box = (half_n + kBBox - 1) / kBBox;
+                const uint32_t tx = 2u * (uint32_t)(kABytes + n_box * kBBox * kBK * 2);
+                const int kb_count = a.K / kBK;
+                for (int kb = 0; kb < kb_count; ++kb) {
+                    if (!mbar_wait_bounded(&tail->empty[s], ph ^ 1u, abort_flag, status,
+                                           SITE_GEMM_PRODUCER, limit)) {
+                        ok = false;
+                        break;
+                    }
+                    uint8_t* sa = smem + (size_t)s * kStageBytes;
+                    uint8_t* sb = sa + kABytes;
+                    if (cta == 0) arrive_expect_tx_local(&tail->full[s], tx);
+                    const uint32_t fb = map_to_rank(&tail->full[s], 0);
+                    tma_load_2d_pair(sa, mA, fb, kb * kBK, a_row0);
+                    tma_load_2d_pair(sa + kABytes / 2, mA, fb, kb * kBK, a_row0 + a.a_half_off);
+                    for (int i = 0; i < n_box; ++i)
+                        tma_load_2d_pair(sb + i * kBBox * kBK * 2, mB, fb, kb * kBK,
+                                         b_row0 + i * kBBox);
+                    if (++s == kStages) {
+                        s = 0;
+                        ph ^= 1u;
+                    }
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------ MMA issuer (CTA 0 of the pair)
+        if (lane == 0 && cta == 0) {
+            int s = 0;
+            uint32_t ph = 0;
+            int it = 0;
+            bool ok = true;
+            const uint32_t empty0 = smem_u32(&tail->empty[0]);
+            for (int tile = pair; ok && tile < total_tiles; tile += n_pairs, ++it) {
+                const Tile t = decode(tile);
+                const PairArgs& a = t.p == 0 ? args0 : args1;
+                const int acc = it & 1;
+                const uint32_t aph = (it >> 1) & 1;
+                if (!mbar_wait_bounded(&tail->tempty[acc], aph ^ 1u, abort_flag, status,
+                                       SITE_GEMM_MMA, limit)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + (uint32_t)(acc * kNTile);
+                const uint32_t idesc = idesc_bf16_f32(2 * kARows, t.n);
+                const int kb_count = a.K / kBK;
+                for (int kb = 0; kb < kb_count; ++kb) {
+                    if (!mbar_wait_bounded(&tail->full[s], ph, abort_flag, status, SITE_GEMM_MMA,
+                                           limit)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t a_addr = smem_u32(smem + (size_t)s * kStageBytes);
+                    const uint32_t b_addr = a_addr + kABytes;
+#pragma unroll
+                    for (int kk = 0; kk < kBK / 16; ++kk)
+                        tc_mma_pair(d_tmem, sw128_kmajor_desc(a_addr + kk * 32),
+                                    sw128_kmajor_desc(b_addr + kk * 32), idesc,
+                                    (kb | kk) != 0 ? 1u : 0u);
+                    // stage s free in both CTAs once these MMAs have read it
+                    tc_commit_pair(empty0 + (uint32_t)(s * 8));
+                    tc_commit_pair(map_to_rank(&tail->empty[s], 1));
+                    if (++s == kStages) {
+                        s = 0;
+                        ph ^= 1u;
+                    }
+                }
+                if (!ok) break;
+                tc_commit_pair(smem_u32(&tail->tfull[acc]));
+                tc_commit_pair(map_to_rank(&tail->tfull[acc], 1));
+            }
+            if (!ok) *abort_flag = 1;
+            // all tensor-core work of the pair is complete once `drain` fires
+            tc_commit_pair(smem_u32(&tail->drain));
+            mbar_wait_bounded(&tail->drain, 0u, nullptr, status, SITE_GEMM_DRAIN, limit);
+        }
+    } else {
+        // ------------------------------------------------ epilogue (warps 2..5, both CTAs)
+        const int wq = warp & 3;  // TMEM lane quarter this warp may access
+        int it = 0;
+        for (int tile = pair; tile < total_tiles; tile += n_pairs, ++it) {
+            const int acc = it & 1;
+            const uint32_t aph = (it >> 1) & 1;
+            const bool got = mbar_wait_bounded(&tail->tfull[acc], aph, abort_flag, status,
+                                               SITE_GEMM_EPILOGUE, limit);
+            // the epilogue warps synchronise on named barriers: leave together
+            if (!epi_all(got)) {
+                *abort_flag = 1;
+                break;
+            }
+            tc_fence_after();
+            const Tile t = decode(tile);
+            const uint32_t taddr =
+                tmem_base + (uint32_t)(acc * kNTile) + ((uint32_t)(wq * 32) << 16);
+            // lane quarter wq = weight rows 32 wq .. 32 wq + 31 of this CTA
+            if (t.p == 0)
+                pair_epilogue<EPI>(tail, taddr, t, args0, cta, wq, lane);
+            else
+                pair_epilogue<EPI>(tail, taddr, t, args1, cta, wq, lane);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(map_to_rank(&tail->tempty[acc], 0));
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync_all();  // no CTA leaves while its pair may still signal or read it
+    tc_fence_after();
+    if (warp == 1)
+        asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                     "r"(kTmemCols)
+                     : "memory");
+}
+
+}  // namespace
+
+size_t pair_gemm_smem_bytes() { return kSmemBytes; }
+
+cudaError_t launch_pair_gemm(int epi, const CUtensorMap& tmA0, const CUtensorMap& tmB0,
+                             const PairArgs& a0, const CUtensorMap* tmA1,
+                             const CUtensorMap* tmB1, const PairArgs* a1, int n_pairs,
+                             cudaStream_t s) {
+    using Kern = void (*)(const CUtensorMap, const CUtensorMap, const CUtensorMap,
+                          const CUtensorMap, const PairArgs, const PairArgs, int);
+    Kern kern = nullptr;
+    switch (epi) {
+        case EPI_SWIGLU: kern = pair_gemm_kernel<EPI_SWIGLU>; break;
+        case EPI_SCATTER: kern = pair_gemm_kernel<EPI_SCATTER>; break;
+        case EPI_COMBINE: kern = pair_gemm_kernel<EPI_COMBINE>; break;
+        default: return cudaErrorInvalidValue;
+    }
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)kSmemBytes);
+    if (e != cudaSuccess) return e;
+    const int np = a1 != nullptr ? 2 : 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * n_pairs);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = kSmemBytes;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, tmA0, tmB0, np > 1 ? *tmA1 : tmA0,
+                              np > 1 ? *tmB1 : tmB0, a0, np > 1 ? *a1 : a0, np);
+}
+
+}  // namespace moe

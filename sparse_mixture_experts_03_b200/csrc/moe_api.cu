@@ -8,6 +8,7 @@
 // moe_get_device_status, and nothing here allocates device memory.
 #include <cudaTypedefs.h>
 #include <limits.h>
+#include <stdlib.h>
 #include <string.h>
 
 #include "../../include/moe.h"
@@ -116,13 +117,15 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     return fn;
 }
 
-// bf16 matrix [rows, cols] row-major, TMA box of 64 columns x 128 rows, 128B swizzle.
-bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols) {
+// bf16 matrix [rows, cols] row-major, TMA box of 64 columns x box_rows rows,
+// 128B swizzle.
+bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
+              uint32_t box_rows = 128) {
     auto fn = encode_fn();
     if (fn == nullptr || rows == 0) return false;
     cuuint64_t dims[2] = {cols, rows};
     cuuint64_t strides[1] = {cols * 2};
-    cuuint32_t box[2] = {64, 128};
+    cuuint32_t box[2] = {64, box_rows};
     cuuint32_t estr[2] = {1, 1};
     CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
                     box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -142,6 +145,17 @@ bool g_stage_events_on = false;
 
 void stage_mark(int i, cudaStream_t s) {
     if (g_stage_events_on) cudaEventRecord(g_stage_events[i], s);
+}
+
+// Development switch: MOE_B200_GEMM=tile selects the 128-row tcgen05 tile
+// kernels instead of the CTA-pair kernels for bf16.
+bool use_tile_gemm() {
+    static int v = -1;
+    if (v < 0) {
+        const char* e = getenv("MOE_B200_GEMM");
+        v = (e != nullptr && strcmp(e, "tile") == 0) ? 1 : 0;
+    }
+    return v == 1;
 }
 
 int grid_for(long long tiles) {
@@ -257,7 +271,11 @@ MOE_API int moe_forward(const void* x, const void* W_router, const void* W_gate_
     if (e != cudaSuccess) return MOE_ERR_CUDA;
     stage_mark(1, s);
     // 2. permutation: histogram, scan, stable ranks, row gather
-    e = launch_permute(idx, T, k, E, block_counts, counts, offsets, row_src, status, s);
+    // the CTA-pair GEMMs take unpadded expert segments; the 128-row tile
+    // kernels (tcgen05 M-major, CUDA cores) take 128-padded ones
+    const bool pair_path = bf16 && !use_tile_gemm();
+    e = launch_permute(idx, T, k, E, block_counts, counts, offsets, row_src,
+                       pair_path ? 1 : kRowAlign, status, s);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
     e = launch_gather_rows(x, d, bf16 ? 2 : 4, k, offsets + E, row_src, L.rows_cap, x_perm,
                            num_sms(), s);
@@ -315,6 +333,92 @@ MOE_API int moe_forward(const void* x, const void* W_router, const void* W_gate_
     const char* Wsh_gu = static_cast<const char*>(W_shared);
     const char* Wsh_dn = Wsh_gu == nullptr ? nullptr
                                            : Wsh_gu + (size_t)2 * SI * d * (bf16 ? 2 : 4);
+
+    if (pair_path) {
+        // 3. gate/up + SwiGLU (routed experts, then shared experts on all tokens)
+        const int n_pairs = num_sms() / 2;
+        CUtensorMap a0, b0, a1, b1;
+        PairArgs p1{};
+        p1.K = d;
+        p1.n_ftiles = inter / 128;
+        p1.n_groups = E;
+        p1.counts = counts;
+        p1.a_group_stride = 2LL * inter;
+        p1.a_tile_step = 128;
+        p1.a_cta_step = 64;
+        p1.a_half_off = inter;
+        p1.out = h;
+        p1.out_ld = inter;
+        p1.out_col_step = 128;
+        p1.status = status;
+        p1.wait_limit_ns = kWaitLimitNs;
+        if (!make_map(&a0, W_gate_up, (uint64_t)E * 2 * inter, d, 64) ||
+            !make_map(&b0, x_perm, (uint64_t)T * k, d, 32))
+            return MOE_ERR_CUDA;
+        PairArgs p1s = p1;
+        if (n_shared > 0) {
+            p1s.n_ftiles = SI / 128;
+            p1s.counts = nullptr;
+            p1s.static_rows = T;
+            p1s.a_group_stride = 0;
+            p1s.a_half_off = SI;
+            p1s.out = h_sh;
+            p1s.out_ld = SI;
+            if (!make_map(&a1, Wsh_gu, (uint64_t)2 * SI, d, 64) || !make_map(&b1, x, (uint64_t)T, d, 32))
+                return MOE_ERR_CUDA;
+            e = launch_pair_gemm(EPI_SWIGLU, a0, b0, p1, &a1, &b1, &p1s, n_pairs, s);
+        } else {
+            e = launch_pair_gemm(EPI_SWIGLU, a0, b0, p1, nullptr, nullptr, nullptr, n_pairs, s);
+        }
+        if (e != cudaSuccess) return MOE_ERR_CUDA;
+        stage_mark(3, s);
+        // 4. routed down projection, weighted scatter into bf16 token-order slots
+        PairArgs p2{};
+        p2.K = inter;
+        p2.n_ftiles = d / 256;
+        p2.n_groups = E;
+        p2.counts = counts;
+        p2.a_group_stride = d;
+        p2.a_tile_step = 256;
+        p2.a_cta_step = 128;
+        p2.a_half_off = 64;
+        p2.out = slots;
+        p2.out_ld = d;
+        p2.out_col_step = 256;
+        p2.row_src = row_src;
+        p2.topk_w = w;
+        p2.k = k;
+        p2.status = status;
+        p2.wait_limit_ns = kWaitLimitNs;
+        if (!make_map(&a0, W_down, (uint64_t)E * d, inter, 64) ||
+            !make_map(&b0, h, (uint64_t)T * k, inter, 32))
+            return MOE_ERR_CUDA;
+        e = launch_pair_gemm(EPI_SCATTER, a0, b0, p2, nullptr, nullptr, nullptr, n_pairs, s);
+        if (e != cudaSuccess) return MOE_ERR_CUDA;
+        stage_mark(4, s);
+        // 5. shared down projection with y = shared + slot_0 + ... + slot_{k-1}
+        if (n_shared > 0) {
+            PairArgs p3 = p2;
+            p3.K = SI;
+            p3.counts = nullptr;
+            p3.static_rows = T;
+            p3.a_group_stride = 0;
+            p3.out = y;
+            p3.slots = slots;
+            p3.out_f32 = out_f32;
+            p3.row_src = nullptr;
+            p3.topk_w = nullptr;
+            if (!make_map(&a0, Wsh_dn, (uint64_t)d, SI, 64) ||
+                !make_map(&b0, h_sh, (uint64_t)T, SI, 32))
+                return MOE_ERR_CUDA;
+            e = launch_pair_gemm(EPI_COMBINE, a0, b0, p3, nullptr, nullptr, nullptr, n_pairs, s);
+        } else {
+            e = launch_combine_slots(slots, 1, T, d, k, y, out_f32, s);
+        }
+        if (e != cudaSuccess) return MOE_ERR_CUDA;
+        stage_mark(5, s);
+        return MOE_OK;
+    }
 
     if (bf16) {
         const int rows_tiles = L.rows_cap / 128;

@@ -56,9 +56,11 @@ cudaError_t launch_route_bf16(const void* x, const void* Wr, int T, int d, int E
 cudaError_t launch_route_f32(const void* x, const void* Wr, int T, int d, int E, int k, int G,
                              int TG, int32_t* idx, float* w, int* status, cudaStream_t s);
 
+// Segments of the permuted layout are padded to a multiple of `align` rows
+// (1: unpadded) with row_src = -1 on padding rows.
 cudaError_t launch_permute(const int32_t* idx, int T, int k, int E, int32_t* block_counts,
-                           int32_t* counts, int32_t* offsets, int32_t* row_src, int* status,
-                           cudaStream_t s);
+                           int32_t* counts, int32_t* offsets, int32_t* row_src, int align,
+                           int* status, cudaStream_t s);
 cudaError_t launch_gather_rows(const void* x, int d, int elem_bytes, int k,
                                const int32_t* offsets_total, const int32_t* row_src,
                                int rows_cap, void* x_perm, int num_sms, cudaStream_t s);
@@ -81,6 +83,41 @@ cudaError_t launch_gemm_tc(int epi, const CUtensorMap& tmA0, const CUtensorMap& 
                            const GemmArgs& a0, const CUtensorMap* tmA1, const CUtensorMap* tmB1,
                            const GemmArgs* a1, int grid, cudaStream_t s,
                            int* sync_counter = nullptr);
+
+// Weights x tokens grouped GEMM on CTA pairs (see gemm_pair.cu).  Group g of a
+// problem has counts[g] token rows (static_rows when counts == nullptr),
+// stored consecutively from row b_row_base in the B tensor; weight rows of
+// feature tile ft for the pair's CTA c: box 0 at
+//   g * a_group_stride + ft * a_tile_step + c * a_cta_step, box 1 at box 0 + a_half_off
+// (64 rows each).  Output columns of feature tile ft start at ft * out_col_step.
+struct PairArgs {
+    int K;
+    int n_ftiles;
+    int n_groups;
+    const int32_t* counts;
+    int static_rows;
+    int b_row_base;
+    long long a_group_stride;
+    int a_tile_step;
+    int a_cta_step;
+    int a_half_off;
+    void* out;
+    int out_ld;
+    int out_col_step;
+    const int32_t* row_src;  // SCATTER: permuted row -> t*k + j
+    const float* topk_w;     // SCATTER
+    const void* slots;       // COMBINE: bf16 [T*k, out_ld]
+    int k;
+    int out_f32;             // COMBINE
+    int* status;
+    unsigned long long wait_limit_ns;
+};
+size_t pair_gemm_smem_bytes();
+// tmA: weights, box {64 cols, 64 rows}; tmB: tokens, box {64 cols, 32 rows}.
+cudaError_t launch_pair_gemm(int epi, const CUtensorMap& tmA0, const CUtensorMap& tmB0,
+                             const PairArgs& a0, const CUtensorMap* tmA1,
+                             const CUtensorMap* tmB1, const PairArgs* a1, int n_pairs,
+                             cudaStream_t s);
 
 cudaError_t launch_selftest_timeout(int* status, unsigned long long limit_ns, cudaStream_t s);
 

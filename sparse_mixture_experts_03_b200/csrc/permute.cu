@@ -72,7 +72,7 @@ __global__ void __launch_bounds__(kPermBlockTokens) perm_count_kernel(
 constexpr int kScanChunkBlocks = 32;
 
 __global__ void __launch_bounds__(1024) perm_scan_kernel(int32_t* __restrict__ block_counts,
-                                                         int nb, int E,
+                                                         int nb, int E, int align,
                                                          int32_t* __restrict__ counts,
                                                          int32_t* __restrict__ offsets,
                                                          int32_t* __restrict__ row_src) {
@@ -104,7 +104,7 @@ __global__ void __launch_bounds__(1024) perm_scan_kernel(int32_t* __restrict__ b
         int carry = 0;
         for (int e0 = 0; e0 < E; e0 += 32) {
             const int e = e0 + tid;
-            const int v = e < E ? (s_cnt[e] + kRowAlign - 1) / kRowAlign * kRowAlign : 0;
+            const int v = e < E ? (s_cnt[e] + align - 1) / align * align : 0;
             int incl = v;
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
@@ -119,8 +119,8 @@ __global__ void __launch_bounds__(1024) perm_scan_kernel(int32_t* __restrict__ b
     __syncthreads();
     for (int e = tid; e < E; e += blockDim.x) counts[e] = s_cnt[e];
     for (int e = tid; e <= E; e += blockDim.x) offsets[e] = s_off[e];
-    for (int i = tid; i < E * kRowAlign; i += blockDim.x) {
-        int e = i / kRowAlign, r = i % kRowAlign;
+    for (int i = tid; i < E * align; i += blockDim.x) {
+        int e = i / align, r = i % align;
         int row = s_off[e] + s_cnt[e] + r;
         if (row < s_off[e + 1]) row_src[row] = -1;
     }
@@ -236,11 +236,11 @@ __global__ void __launch_bounds__(256) combine_slots_kernel(const TS* __restrict
 }  // namespace
 
 cudaError_t launch_permute(const int32_t* idx, int T, int k, int E, int32_t* block_counts,
-                           int32_t* counts, int32_t* offsets, int32_t* row_src, int* status,
-                           cudaStream_t s) {
+                           int32_t* counts, int32_t* offsets, int32_t* row_src, int align,
+                           int* status, cudaStream_t s) {
     const int nb = (T + kPermBlockTokens - 1) / kPermBlockTokens;
     perm_count_kernel<<<nb, kPermBlockTokens, 0, s>>>(idx, T, k, E, block_counts, status);
-    perm_scan_kernel<<<1, 1024, 0, s>>>(block_counts, nb, E, counts, offsets, row_src);
+    perm_scan_kernel<<<1, 1024, 0, s>>>(block_counts, nb, E, align, counts, offsets, row_src);
     perm_rank_kernel<<<nb, kPermBlockTokens, 0, s>>>(idx, T, k, E, block_counts, offsets, row_src,
                                                      status);
     return cudaGetLastError();
