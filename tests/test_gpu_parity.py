@@ -104,7 +104,9 @@ def test_empty_batch_is_a_no_op():
 
 def permutation_check(w, inp, idx, ws):
     """The permutation stage, bit-exact against a host computation from the
-    GPU's own routing: counts, padded offsets, stable row order, row copies."""
+    GPU's own routing: counts, segment offsets, stable row order, row copies.
+    bf16 layers use unpadded expert segments (the CTA-pair GEMMs tile tokens
+    as N in steps of 16); fp32 layers pad segments to 128 rows."""
     lay = moe.workspace_layout(w.T, w.d, w.E, w.k, w.inter, w.n_shared, inp.x.dtype)
     wsc = ws.cpu()
     i32 = lambda name, n: wsc[lay[name]:lay[name] + 4 * n].view(torch.int32).numpy()
@@ -113,7 +115,8 @@ def permutation_check(w, inp, idx, ws):
     counts = i32("counts", w.E)
     offsets = i32("offsets", w.E + 1)
     np.testing.assert_array_equal(counts, cnt_ref)
-    pad = (cnt_ref + 127) // 128 * 128
+    align = 1 if inp.x.dtype == torch.bfloat16 else 128
+    pad = (cnt_ref + align - 1) // align * align
     np.testing.assert_array_equal(offsets, np.concatenate([[0], np.cumsum(pad)]))
     rows_cap = w.T * w.k + 128 * w.E
     row_src = i32("row_src", rows_cap)
