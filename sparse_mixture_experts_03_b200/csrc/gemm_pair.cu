@@ -54,13 +54,7 @@ constexpr int kEpiWarps = 4;
 constexpr int kMaxGroupsP = kMaxE + 1;
 
 struct __align__(16) PairTail {
-    // epilogue staging, reused per 32-token chunk:
-    //   SWIGLU:  up values [64][33] f32 (8448 B) + h [32][64] bf16 (4096 B)
-    //   SCATTER: [32 tokens][128] bf16 (8192 B)
-    //   COMBINE: [32 tokens][128 + 4] f32 (16896 B)
-    float stage[32 * 132];
-    int tile_src[kNTile];     // SCATTER: slot index of each token column (-1 beyond N)
-    float tile_w[kNTile];     // SCATTER: gate weight of each token column
+    uint4 stage[kEpiWarps * 256];  // per epilogue warp: 32 rows x 128 B staging
     uint64_t full[kStages];
     uint64_t empty[kStages];
     uint64_t tfull[2];
@@ -166,114 +160,138 @@ __device__ __forceinline__ float silu_mul(float g, float u) {
     return __fdividef(g, 1.0f + __expf(-g)) * u;
 }
 
+// Per-warp staging: 32 rows x 128 B, 16-byte chunk q of row r stored at chunk
+// position q ^ (r & 7), so row-wise writes (one row per instruction, lanes
+// spread over the row) and transposed reads (one row per lane) are both free
+// of bank conflicts.
+__device__ __forceinline__ uint8_t* stage_chunk(uint8_t* wb, int row, int chunk) {
+    return wb + row * 128 + ((chunk ^ (row & 7)) << 4);
+}
+
+// Epilogue of one tile for warp quarter wq of this CTA: TMEM lanes 32 wq ..
+// 32 wq + 31 (weight rows) x the tile's N token columns.  Each warp works on
+// its own: tcgen05.ld of 32 columns (thread = weight row, registers = tokens),
+// transpose through its staging buffer, then thread = token for the stores.
 template <int EPI>
-__device__ __forceinline__ void pair_epilogue(PairTail* tail, uint32_t taddr, const Tile& t,
-                                              const PairArgs& a, uint32_t cta, int ew, int lane) {
-    const int etid = ew * 32 + lane;  // 0..127 within the epilogue warps
-    if constexpr (EPI == EPI_SCATTER) {
-        // slot index and weight of every token column of the tile
-        for (int i = etid; i < kNTile; i += kEpiWarps * 32) {
-            int src = -1;
-            float wv = 0.f;
-            if (i < t.n_real) {
-                src = a.row_src[t.b_row + i];
-                wv = src >= 0 ? a.topk_w[src] : 0.f;
-            }
-            tail->tile_src[i] = src;
-            tail->tile_w[i] = wv;
-        }
-        epi_bar();
-    }
+__device__ __forceinline__ void pair_epilogue(uint8_t* wb, uint32_t taddr, const Tile& t,
+                                              const PairArgs& a, uint32_t cta, int wq, int lane) {
     for (int c0 = 0; c0 < t.n; c0 += 32) {
         uint32_t v[32];
-        tmem_ld32(taddr + (uint32_t)c0, v);  // my weight row (lane) x 32 tokens
+        tmem_ld32(taddr + (uint32_t)c0, v);  // weight row (lane) x tokens c0 .. c0+31
         tmem_ld_wait();
+        const bool tok_ok = c0 + lane < t.n_real;  // after the transpose, lane = token
         if constexpr (EPI == EPI_SWIGLU) {
-            float* up = tail->stage;                                          // [64][33]
-            __nv_bfloat16* hb = reinterpret_cast<__nv_bfloat16*>(tail->stage + 64 * 33);  // [32][64]
-            const int fl = (ew & 1) * 32 + lane;  // feature within this CTA's 64
-            if (ew >= 2) {
+            // The CTA's weight rows are [16 gate, 16 up] per warp quarter: lane i < 16
+            // holds gate feature f = 16 wq + i, lane i + 16 the matching up row.  Lane
+            // i computes h for tokens 0..15 of feature f, lane i + 16 for tokens 16..31,
+            // each receiving the other half of SwiGLU by a register shuffle.
+            const bool is_gate = lane < 16;
+            __nv_bfloat16 h[16];
 #pragma unroll
-                for (int i = 0; i < 32; ++i) up[fl * 33 + i] = __uint_as_float(v[i]);
+            for (int i = 0; i < 16; ++i) {
+                const float send = __uint_as_float(is_gate ? v[16 + i] : v[i]);
+                const float recv = __shfl_xor_sync(0xffffffffu, send, 16);
+                const float g = is_gate ? __uint_as_float(v[i]) : recv;
+                const float u = is_gate ? recv : __uint_as_float(v[16 + i]);
+                h[i] = __float2bfloat16_rn(silu_mul(g, u));
             }
-            epi_bar();
-            if (ew < 2) {
+            const int f = lane & 15, tbase = is_gate ? 0 : 16;
 #pragma unroll
-                for (int i = 0; i < 32; ++i)
-                    hb[i * 64 + fl] = __float2bfloat16_rn(
-                        silu_mul(__uint_as_float(v[i]), up[fl * 33 + i]));
+            for (int i = 0; i < 16; ++i) {
+                // token row tbase + i: 16 features x 2 B = 32 B in chunks 0..1
+                __nv_bfloat16* row = reinterpret_cast<__nv_bfloat16*>(
+                    stage_chunk(wb, tbase + i, f >> 3));
+                row[f & 7] = h[i];
             }
-            epi_bar();
-            // 32 tokens x 128 B: thread -> token etid / 4, 32-byte piece etid % 4
-            const int tk = etid >> 2, pc = etid & 3;
-            if (c0 + tk < t.n_real) {
-                const uint4* s = reinterpret_cast<const uint4*>(hb + tk * 64 + pc * 16);
+            __syncwarp();
+            if (tok_ok) {
                 uint4* d = reinterpret_cast<uint4*>(
-                    static_cast<__nv_bfloat16*>(a.out) + (size_t)(t.b_row + c0 + tk) * a.out_ld +
-                    t.ft * a.out_col_step + cta * 64 + pc * 16);
-                d[0] = s[0];
-                d[1] = s[1];
+                    static_cast<__nv_bfloat16*>(a.out) + (size_t)(t.b_row + c0 + lane) * a.out_ld +
+                    t.ft * a.out_col_step + cta * 64 + wq * 16);
+                d[0] = *reinterpret_cast<const uint4*>(stage_chunk(wb, lane, 0));
+                d[1] = *reinterpret_cast<const uint4*>(stage_chunk(wb, lane, 1));
             }
-            epi_bar();
+            __syncwarp();
         } else if constexpr (EPI == EPI_SCATTER) {
-            __nv_bfloat16* sb = reinterpret_cast<__nv_bfloat16*>(tail->stage);  // [32][128]
-            const int fl = ew * 32 + lane;
+            // gate weight of token column i, fetched by lane i and broadcast
+            int src = -1;
+            float wv = 0.f;
+            if (tok_ok) {
+                src = a.row_src[t.b_row + c0 + lane];
+                wv = src >= 0 ? a.topk_w[src] : 0.f;
+            }
 #pragma unroll
-            for (int i = 0; i < 32; ++i)
-                sb[i * 128 + fl] = __float2bfloat16_rn(tail->tile_w[c0 + i] * __uint_as_float(v[i]));
-            epi_bar();
-            // 32 tokens x 256 B: thread -> token etid / 4, 64-byte piece etid % 4
-            const int tk = etid >> 2, pc = etid & 3;
-            const int src = tail->tile_src[c0 + tk];
+            for (int i = 0; i < 32; ++i) {
+                const float wi = __shfl_sync(0xffffffffu, wv, i);
+                // token row i: 32 features x 2 B = 64 B in chunks 0..3
+                __nv_bfloat16* row = reinterpret_cast<__nv_bfloat16*>(stage_chunk(wb, i, lane >> 3));
+                row[lane & 7] = __float2bfloat16_rn(wi * __uint_as_float(v[i]));
+            }
+            __syncwarp();
             if (src >= 0) {
-                const uint4* s = reinterpret_cast<const uint4*>(sb + tk * 128 + pc * 32);
                 uint4* d = reinterpret_cast<uint4*>(
                     static_cast<__nv_bfloat16*>(a.out) + (size_t)src * a.out_ld +
-                    t.ft * a.out_col_step + cta * 128 + pc * 32);
+                    t.ft * a.out_col_step + cta * 128 + wq * 32);
 #pragma unroll
-                for (int q = 0; q < 4; ++q) d[q] = s[q];
+                for (int q = 0; q < 4; ++q)
+                    d[q] = *reinterpret_cast<const uint4*>(stage_chunk(wb, lane, q));
             }
-            epi_bar();
+            __syncwarp();
         } else {  // EPI_COMBINE
-            float* sf = tail->stage;  // [32][132]
-            const int fl = ew * 32 + lane;
 #pragma unroll
-            for (int i = 0; i < 32; ++i) sf[i * 132 + fl] = __uint_as_float(v[i]);
-            epi_bar();
-            // thread -> token etid / 4, 32 features (etid % 4) * 32
-            const int tk = etid >> 2, pc = etid & 3;
-            const int tok = t.b_row + c0 + tk;
-            if (c0 + tk < t.n_real) {
-                const int col = t.ft * a.out_col_step + cta * 128 + pc * 32;
+            for (int i = 0; i < 32; ++i) {
+                // token row i: 32 features x 4 B = 128 B in chunks 0..7
+                float* row = reinterpret_cast<float*>(stage_chunk(wb, i, lane >> 2));
+                row[lane & 3] = __uint_as_float(v[i]);
+            }
+            __syncwarp();
+            if (tok_ok) {
+                const size_t tok = (size_t)(t.b_row + c0 + lane);
+                const int col = t.ft * a.out_col_step + cta * 128 + wq * 32;
                 float acc[32];
 #pragma unroll
-                for (int i = 0; i < 32; ++i) acc[i] = sf[tk * 132 + pc * 32 + i];
+                for (int q = 0; q < 8; ++q) {
+                    const float4 s4 = *reinterpret_cast<const float4*>(stage_chunk(wb, lane, q));
+                    acc[4 * q] = s4.x;
+                    acc[4 * q + 1] = s4.y;
+                    acc[4 * q + 2] = s4.z;
+                    acc[4 * q + 3] = s4.w;
+                }
+                // y = shared + slot_0 + ... + slot_{k-1}, in that order; all slot
+                // pieces of this token are loaded before the ordered sum
                 const __nv_bfloat16* slots = static_cast<const __nv_bfloat16*>(a.slots);
-                for (int j = 0; j < a.k; ++j) {
-                    const uint4* sp = reinterpret_cast<const uint4*>(
-                        slots + ((size_t)tok * a.k + j) * a.out_ld + col);
-                    uint4 q4[4];
+                uint4 sv[kMaxK][4];
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) q4[q] = __ldcg(sp + q);
+                for (int j = 0; j < kMaxK; ++j)
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)
+                        sv[j][q] = j < a.k ? __ldcg(reinterpret_cast<const uint4*>(
+                                                     slots + (tok * a.k + j) * a.out_ld + col) +
+                                                 q)
+                                           : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+                for (int j = 0; j < kMaxK; ++j) {
+                    if (j >= a.k) break;
 #pragma unroll
                     for (int q = 0; q < 4; ++q) {
-                        const uint32_t w4[4] = {q4[q].x, q4[q].y, q4[q].z, q4[q].w};
+                        const uint32_t w4[4] = {sv[j][q].x, sv[j][q].y, sv[j][q].z, sv[j][q].w};
 #pragma unroll
-                        for (int h = 0; h < 4; ++h) {
-                            acc[q * 8 + 2 * h] += __uint_as_float(w4[h] << 16);
-                            acc[q * 8 + 2 * h + 1] += __uint_as_float(w4[h] & 0xffff0000u);
+                        for (int hh = 0; hh < 4; ++hh) {
+                            acc[q * 8 + 2 * hh] += __uint_as_float(w4[hh] << 16);
+                            acc[q * 8 + 2 * hh + 1] += __uint_as_float(w4[hh] & 0xffff0000u);
                         }
                     }
                 }
                 if (a.out_f32) {
                     float4* d = reinterpret_cast<float4*>(static_cast<float*>(a.out) +
-                                                          (size_t)tok * a.out_ld + col);
+                                                          tok * a.out_ld + col);
 #pragma unroll
                     for (int q = 0; q < 8; ++q)
-                        d[q] = make_float4(acc[4 * q], acc[4 * q + 1], acc[4 * q + 2], acc[4 * q + 3]);
+                        d[q] = make_float4(acc[4 * q], acc[4 * q + 1], acc[4 * q + 2],
+                                           acc[4 * q + 3]);
                 } else {
                     uint4* d = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.out) +
-                                                        (size_t)tok * a.out_ld + col);
+                                                        tok * a.out_ld + col);
 #pragma unroll
                     for (int q = 0; q < 4; ++q)
                         d[q] = make_uint4(pack_bf16x2(acc[8 * q], acc[8 * q + 1]),
@@ -282,7 +300,7 @@ __device__ __forceinline__ void pair_epilogue(PairTail* tail, uint32_t taddr, co
                                           pack_bf16x2(acc[8 * q + 6], acc[8 * q + 7]));
                 }
             }
-            epi_bar();
+            __syncwarp();
         }
     }
 }
@@ -425,8 +443,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                     uint8_t* sb = sa + kABytes;
                     if (cta == 0) arrive_expect_tx_local(&tail->full[s], tx);
                     const uint32_t fb = map_to_rank(&tail->full[s], 0);
-                    tma_load_2d_pair(sa, mA, fb, kb * kBK, a_row0);
-                    tma_load_2d_pair(sa + kABytes / 2, mA, fb, kb * kBK, a_row0 + a.a_half_off);
+                    // 128 weight rows in boxes of a_box_rows; box b comes from row
+                    // a_row0 + (b / 2) * a_box_rows + (b % 2) * a_half_off, so with
+                    // 16-row boxes and a_half_off = the up block, each 32-row quarter
+                    // holds 16 gate rows then the 16 matching up rows
+                    const int a_boxes = kARows / a.a_box_rows;
+                    for (int b = 0; b < a_boxes; ++b)
+                        tma_load_2d_pair(sa + b * a.a_box_rows * kBK * 2, mA, fb, kb * kBK,
+                                         a_row0 + (b >> 1) * a.a_box_rows + (b & 1) * a.a_half_off);
                     for (int i = 0; i < n_box; ++i)
                         tma_load_2d_pair(sb + i * kBBox * kBK * 2, mB, fb, kb * kBK,
                                          b_row0 + i * kBBox);
@@ -493,6 +517,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else {
         // ------------------------------------------------ epilogue (warps 2..5, both CTAs)
         const int wq = warp & 3;  // TMEM lane quarter this warp may access
+        uint8_t* wstage = reinterpret_cast<uint8_t*>(tail->stage) + wq * 4096;
         int it = 0;
         for (int tile = pair; tile < total_tiles; tile += n_pairs, ++it) {
             const int acc = it & 1;
@@ -510,9 +535,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tmem_base + (uint32_t)(acc * kNTile) + ((uint32_t)(wq * 32) << 16);
             // lane quarter wq = weight rows 32 wq .. 32 wq + 31 of this CTA
             if (t.p == 0)
-                pair_epilogue<EPI>(tail, taddr, t, args0, cta, wq, lane);
+                pair_epilogue<EPI>(wstage, taddr, t, args0, cta, wq, lane);
             else
-                pair_epilogue<EPI>(tail, taddr, t, args1, cta, wq, lane);
+                pair_epilogue<EPI>(wstage, taddr, t, args1, cta, wq, lane);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(map_to_rank(&tail->tempty[acc], 0));

@@ -347,12 +347,13 @@ MOE_API int moe_forward(const void* x, const void* W_router, const void* W_gate_
         p1.a_tile_step = 128;
         p1.a_cta_step = 64;
         p1.a_half_off = inter;
+        p1.a_box_rows = 16;
         p1.out = h;
         p1.out_ld = inter;
         p1.out_col_step = 128;
         p1.status = status;
         p1.wait_limit_ns = kWaitLimitNs;
-        if (!make_map(&a0, W_gate_up, (uint64_t)E * 2 * inter, d, 64) ||
+        if (!make_map(&a0, W_gate_up, (uint64_t)E * 2 * inter, d, 16) ||
             !make_map(&b0, x_perm, (uint64_t)T * k, d, 32))
             return MOE_ERR_CUDA;
         PairArgs p1s = p1;
@@ -364,7 +365,7 @@ MOE_API int moe_forward(const void* x, const void* W_router, const void* W_gate_
             p1s.a_half_off = SI;
             p1s.out = h_sh;
             p1s.out_ld = SI;
-            if (!make_map(&a1, Wsh_gu, (uint64_t)2 * SI, d, 64) || !make_map(&b1, x, (uint64_t)T, d, 32))
+            if (!make_map(&a1, Wsh_gu, (uint64_t)2 * SI, d, 16) || !make_map(&b1, x, (uint64_t)T, d, 32))
                 return MOE_ERR_CUDA;
             e = launch_pair_gemm(EPI_SWIGLU, a0, b0, p1, &a1, &b1, &p1s, n_pairs, s);
         } else {
@@ -382,6 +383,7 @@ MOE_API int moe_forward(const void* x, const void* W_router, const void* W_gate_
         p2.a_tile_step = 256;
         p2.a_cta_step = 128;
         p2.a_half_off = 64;
+        p2.a_box_rows = 64;
         p2.out = slots;
         p2.out_ld = d;
         p2.out_col_step = 256;

@@ -87,9 +87,10 @@ cudaError_t launch_gemm_tc(int epi, const CUtensorMap& tmA0, const CUtensorMap& 
 // Weights x tokens grouped GEMM on CTA pairs (see gemm_pair.cu).  Group g of a
 // problem has counts[g] token rows (static_rows when counts == nullptr),
 // stored consecutively from row b_row_base in the B tensor; weight rows of
-// feature tile ft for the pair's CTA c: box 0 at
-//   g * a_group_stride + ft * a_tile_step + c * a_cta_step, box 1 at box 0 + a_half_off
-// (64 rows each).  Output columns of feature tile ft start at ft * out_col_step.
+// feature tile ft for the pair's CTA c start at
+//   a_row0 = g * a_group_stride + ft * a_tile_step + c * a_cta_step,
+// loaded as 128 / a_box_rows boxes, box b from a_row0 + (b / 2) * a_box_rows +
+// (b % 2) * a_half_off.  Output columns of feature tile ft start at ft * out_col_step.
 struct PairArgs {
     int K;
     int n_ftiles;
@@ -101,6 +102,7 @@ struct PairArgs {
     int a_tile_step;
     int a_cta_step;
     int a_half_off;
+    int a_box_rows;          // 16 (SwiGLU: gate/up interleaved per 16 rows) or 64
     void* out;
     int out_ld;
     int out_col_step;
@@ -113,7 +115,7 @@ struct PairArgs {
     unsigned long long wait_limit_ns;
 };
 size_t pair_gemm_smem_bytes();
-// tmA: weights, box {64 cols, 64 rows}; tmB: tokens, box {64 cols, 32 rows}.
+// tmA: weights, box {64 cols, a_box_rows rows}; tmB: tokens, box {64 cols, 32 rows}.
 cudaError_t launch_pair_gemm(int epi, const CUtensorMap& tmA0, const CUtensorMap& tmB0,
                              const PairArgs& a0, const CUtensorMap* tmA1,
                              const CUtensorMap* tmB1, const PairArgs* a1, int n_pairs,
