@@ -42,7 +42,7 @@ namespace {
 constexpr int kBK = 64;                          // K per stage (one 128-byte swizzle atom)
 constexpr int kARows = 128;                      // weight rows per CTA (MMA M = 256 per pair)
 constexpr int kABytes = kARows * kBK * 2;        // 16 KiB
-constexpr int kBBox = 32;                        // token rows per B box
+constexpr int kBBox = 64;                        // token rows per B box
 constexpr int kBMaxRows = 128;                   // token rows per CTA (N <= 256 per pair)
 constexpr int kBBytes = kBMaxRows * kBK * 2;     // 16 KiB
 constexpr int kStageBytes = kABytes + kBBytes;   // 32 KiB
@@ -108,6 +108,17 @@ __device__ __forceinline__ void tma_load_2d_pair(void* smem_dst, const CUtensorM
         "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
         " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(smem_dst)),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster), "r"(c0), "r"(c1)
+        : "memory");
+}
+// 5-D variant (weights with gate/up interleaving, see PairArgs::a_mode).
+__device__ __forceinline__ void tma_load_5d_pair(void* smem_dst, const CUtensorMap* map,
+                                                 uint32_t bar_cluster, int c0, int c1, int c2,
+                                                 int c3, int c4) {
+    asm volatile(
+        "cp.async.bulk.tensor.5d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(smem_u32(smem_dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster), "r"(c0), "r"(c1), "r"(c2),
+        "r"(c3), "r"(c4)
         : "memory");
 }
 __device__ __forceinline__ void arrive_expect_tx_local(uint64_t* bar, uint32_t bytes) {
@@ -401,8 +412,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int cnt = tail->seg_off[t.p][t.g + 1] - tail->seg_off[t.p][t.g];
         const int nch = (cnt + kNTile - 1) / kNTile;
         const int local = lt - tail->tile_off[t.p][t.g];
-        t.ft = local / nch;
-        const int ch = local % nch;
+        // routed experts: feature tile slow, token chunk fast (a weight tile's
+        // chunks are neighbours); dense problems: token chunk slow, feature tile
+        // fast (pairs running together cover whole token rows)
+        const bool dense = a.counts == nullptr;
+        t.ft = dense ? local % a.n_ftiles : local / nch;
+        const int ch = dense ? local / a.n_ftiles : local % nch;
         t.b_row = a.b_row_base + tail->seg_off[t.p][t.g] + ch * kNTile;
         t.n_real = min(kNTile, cnt - ch * kNTile);
         t.n = (t.n_real + 15) & ~15;
@@ -443,14 +458,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                     uint8_t* sb = sa + kABytes;
                     if (cta == 0) arrive_expect_tx_local(&tail->full[s], tx);
                     const uint32_t fb = map_to_rank(&tail->full[s], 0);
-                    // 128 weight rows in boxes of a_box_rows; box b comes from row
-                    // a_row0 + (b / 2) * a_box_rows + (b % 2) * a_half_off, so with
-                    // 16-row boxes and a_half_off = the up block, each 32-row quarter
-                    // holds 16 gate rows then the 16 matching up rows
-                    const int a_boxes = kARows / a.a_box_rows;
-                    for (int b = 0; b < a_boxes; ++b)
-                        tma_load_2d_pair(sa + b * a.a_box_rows * kBK * 2, mA, fb, kb * kBK,
-                                         a_row0 + (b >> 1) * a.a_box_rows + (b & 1) * a.a_half_off);
+                    if (a.a_mode == 0) {
+                        // 128 consecutive weight rows
+                        tma_load_2d_pair(sa, mA, fb, kb * kBK, a_row0);
+                    } else {
+                        // 4 blocks x (16 gate rows, 16 up rows) of features
+                        // ft * a_tile_step + cta * a_cta_step ... + 63 of group g
+                        tma_load_5d_pair(sa, mA, fb, kb * kBK, 0, 0,
+                                         (t.ft * a.a_tile_step + (int)cta * a.a_cta_step) >> 4,
+                                         t.g);
+                    }
                     for (int i = 0; i < n_box; ++i)
                         tma_load_2d_pair(sb + i * kBBox * kBK * 2, mB, fb, kb * kBK,
                                          b_row0 + i * kBBox);

@@ -133,6 +133,23 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
     return r == CUDA_SUCCESS;
 }
 
+// Gate/up weight [G][2][F][K] bf16 (per group: F gate rows, then F up rows)
+// seen as a 5-D tensor {K, 16, 2, F/16, G}; one box {64, 16, 2, 4, 1} brings 4
+// blocks of (16 gate rows, 16 up rows), i.e. 64 features with gate and up
+// interleaved per 16 rows, 128B swizzle.
+bool make_map_gate_up(CUtensorMap* m, const void* base, uint64_t G, uint64_t F, uint64_t K) {
+    auto fn = encode_fn();
+    if (fn == nullptr || F % 64 != 0) return false;
+    cuuint64_t dims[5] = {K, 16, 2, F / 16, G};
+    cuuint64_t strides[4] = {K * 2, F * K * 2, 16 * K * 2, 2 * F * K * 2};
+    cuuint32_t box[5] = {64, 16, 2, 4, 1};
+    cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(base), dims, strides,
+                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 int ret(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
 
 template <typename T>
@@ -346,15 +363,14 @@ MOE_API int moe_forward(const void* x, const void* W_router, const void* W_gate_
         p1.a_group_stride = 2LL * inter;
         p1.a_tile_step = 128;
         p1.a_cta_step = 64;
-        p1.a_half_off = inter;
-        p1.a_box_rows = 16;
+        p1.a_mode = 1;
         p1.out = h;
         p1.out_ld = inter;
         p1.out_col_step = 128;
         p1.status = status;
         p1.wait_limit_ns = kWaitLimitNs;
-        if (!make_map(&a0, W_gate_up, (uint64_t)E * 2 * inter, d, 16) ||
-            !make_map(&b0, x_perm, (uint64_t)T * k, d, 32))
+        if (!make_map_gate_up(&a0, W_gate_up, (uint64_t)E, inter, d) ||
+            !make_map(&b0, x_perm, (uint64_t)T * k, d, 64))
             return MOE_ERR_CUDA;
         PairArgs p1s = p1;
         if (n_shared > 0) {
@@ -362,10 +378,9 @@ MOE_API int moe_forward(const void* x, const void* W_router, const void* W_gate_
             p1s.counts = nullptr;
             p1s.static_rows = T;
             p1s.a_group_stride = 0;
-            p1s.a_half_off = SI;
             p1s.out = h_sh;
             p1s.out_ld = SI;
-            if (!make_map(&a1, Wsh_gu, (uint64_t)2 * SI, d, 16) || !make_map(&b1, x, (uint64_t)T, d, 32))
+            if (!make_map_gate_up(&a1, Wsh_gu, 1, SI, d) || !make_map(&b1, x, (uint64_t)T, d, 64))
                 return MOE_ERR_CUDA;
             e = launch_pair_gemm(EPI_SWIGLU, a0, b0, p1, &a1, &b1, &p1s, n_pairs, s);
         } else {
@@ -382,8 +397,7 @@ MOE_API int moe_forward(const void* x, const void* W_router, const void* W_gate_
         p2.a_group_stride = d;
         p2.a_tile_step = 256;
         p2.a_cta_step = 128;
-        p2.a_half_off = 64;
-        p2.a_box_rows = 64;
+        p2.a_mode = 0;
         p2.out = slots;
         p2.out_ld = d;
         p2.out_col_step = 256;
@@ -392,8 +406,8 @@ MOE_API int moe_forward(const void* x, const void* W_router, const void* W_gate_
         p2.k = k;
         p2.status = status;
         p2.wait_limit_ns = kWaitLimitNs;
-        if (!make_map(&a0, W_down, (uint64_t)E * d, inter, 64) ||
-            !make_map(&b0, h, (uint64_t)T * k, inter, 32))
+        if (!make_map(&a0, W_down, (uint64_t)E * d, inter, 128) ||
+            !make_map(&b0, h, (uint64_t)T * k, inter, 64))
             return MOE_ERR_CUDA;
         e = launch_pair_gemm(EPI_SCATTER, a0, b0, p2, nullptr, nullptr, nullptr, n_pairs, s);
         if (e != cudaSuccess) return MOE_ERR_CUDA;
@@ -410,8 +424,8 @@ MOE_API int moe_forward(const void* x, const void* W_router, const void* W_gate_
             p3.out_f32 = out_f32;
             p3.row_src = nullptr;
             p3.topk_w = nullptr;
-            if (!make_map(&a0, Wsh_dn, (uint64_t)d, SI, 64) ||
-                !make_map(&b0, h_sh, (uint64_t)T, SI, 32))
+            if (!make_map(&a0, Wsh_dn, (uint64_t)d, SI, 128) ||
+                !make_map(&b0, h_sh, (uint64_t)T, SI, 64))
                 return MOE_ERR_CUDA;
             e = launch_pair_gemm(EPI_COMBINE, a0, b0, p3, nullptr, nullptr, nullptr, n_pairs, s);
         } else {

@@ -88,9 +88,10 @@ cudaError_t launch_gemm_tc(int epi, const CUtensorMap& tmA0, const CUtensorMap& 
 // problem has counts[g] token rows (static_rows when counts == nullptr),
 // stored consecutively from row b_row_base in the B tensor; weight rows of
 // feature tile ft for the pair's CTA c start at
-//   a_row0 = g * a_group_stride + ft * a_tile_step + c * a_cta_step,
-// loaded as 128 / a_box_rows boxes, box b from a_row0 + (b / 2) * a_box_rows +
-// (b % 2) * a_half_off.  Output columns of feature tile ft start at ft * out_col_step.
+//   a_row0 = g * a_group_stride + ft * a_tile_step + c * a_cta_step
+// (a_mode 0), or are features ft * a_tile_step + c * a_cta_step .. + 63 of
+// group g, gate and up interleaved per 16 (a_mode 1).  Output columns of
+// feature tile ft start at ft * out_col_step.
 struct PairArgs {
     int K;
     int n_ftiles;
@@ -101,8 +102,9 @@ struct PairArgs {
     long long a_group_stride;
     int a_tile_step;
     int a_cta_step;
-    int a_half_off;
-    int a_box_rows;          // 16 (SwiGLU: gate/up interleaved per 16 rows) or 64
+    int a_mode;              // 0: 2-D map, 128 rows from a_row0
+                             // 1: 5-D map {K, 16, 2, F/16, G} of a [G][2][F][K] gate/up
+                             //    weight: 4 blocks of (16 gate, 16 up) rows per CTA
     void* out;
     int out_ld;
     int out_col_step;
@@ -115,7 +117,8 @@ struct PairArgs {
     unsigned long long wait_limit_ns;
 };
 size_t pair_gemm_smem_bytes();
-// tmA: weights, box {64 cols, a_box_rows rows}; tmB: tokens, box {64 cols, 32 rows}.
+// tmA: weights, a_mode 0: box {64, 128}; a_mode 1: box {64, 16, 2, 4, 1};
+// tmB: tokens, box {64 cols, 64 rows}.
 cudaError_t launch_pair_gemm(int epi, const CUtensorMap& tmA0, const CUtensorMap& tmB0,
                              const PairArgs& a0, const CUtensorMap* tmA1,
                              const CUtensorMap* tmB1, const PairArgs* a1, int n_pairs,
