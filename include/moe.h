@@ -94,7 +94,8 @@ enum {
     MOE_WS_H = 8,            /* in_dt[rows_cap, inter] silu(gate) * up, routed rows    */
     MOE_WS_H_SHARED = 9,     /* in_dt[T, n_shared*inter] the same for shared experts   */
     MOE_WS_SLOTS = 10,       /* in_dt[T*k, d] w_j * expert output, token order          */
-    MOE_WS_TOTAL = 11        /* total size                                            */
+    MOE_WS_Y_SHARED = 11,    /* bf16 with shared experts: f32[T, d] shared output        */
+    MOE_WS_TOTAL = 12        /* total size                                            */
 };
 /* rows_cap = T*k + 128*E (the padded permuted layout never needs more). */
 

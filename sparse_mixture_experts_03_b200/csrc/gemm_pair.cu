@@ -29,8 +29,9 @@
 //           row_src[b_row + t], scaled by its gate weight, stored bf16 (the
 //           weighted combine of the MoEBlock listing, section "混合专家：更多
 //           参数，相同 FLOPs").
-//   COMBINE shared down projection plus the final sum
-//           y = shared + slot_0 + ... + slot_{k-1}, fixed order, fp32.
+//   STORE_F32 shared down projection, fp32 rows; the final sum
+//           y = shared + slot_0 + ... + slot_{k-1} (fixed order) is a separate
+//           streaming kernel that reads whole slot rows.
 // Every wait is bounded (status word + early exit, never a trap).
 #include "moe_device.cuh"
 #include "moe_internal.h"
@@ -186,7 +187,21 @@ __device__ __forceinline__ uint8_t* stage_chunk(uint8_t* wb, int row, int chunk)
 template <int EPI>
 __device__ __forceinline__ void pair_epilogue(uint8_t* wb, uint32_t taddr, const Tile& t,
                                               const PairArgs& a, uint32_t cta, int wq, int lane) {
-    for (int c0 = 0; c0 < t.n; c0 += 32) {
+    // SCATTER: slot index and gate weight of every token column of the tile,
+    // loaded once per tile (lane l holds columns 32 c + l)
+    int srcs[kNTile / 32];
+    float wts[kNTile / 32];
+    if constexpr (EPI == EPI_SCATTER) {
+#pragma unroll
+        for (int c = 0; c < kNTile / 32; ++c)
+            srcs[c] = 32 * c + lane < t.n_real ? a.row_src[t.b_row + 32 * c + lane] : -1;
+#pragma unroll
+        for (int c = 0; c < kNTile / 32; ++c) wts[c] = srcs[c] >= 0 ? a.topk_w[srcs[c]] : 0.f;
+    }
+#pragma unroll
+    for (int cc = 0; cc < kNTile / 32; ++cc) {
+        const int c0 = 32 * cc;
+        if (c0 >= t.n) break;
         uint32_t v[32];
         tmem_ld32(taddr + (uint32_t)c0, v);  // weight row (lane) x tokens c0 .. c0+31
         tmem_ld_wait();
@@ -224,13 +239,8 @@ __device__ __forceinline__ void pair_epilogue(uint8_t* wb, uint32_t taddr, const
             }
             __syncwarp();
         } else if constexpr (EPI == EPI_SCATTER) {
-            // gate weight of token column i, fetched by lane i and broadcast
-            int src = -1;
-            float wv = 0.f;
-            if (tok_ok) {
-                src = a.row_src[t.b_row + c0 + lane];
-                wv = src >= 0 ? a.topk_w[src] : 0.f;
-            }
+            const int src = srcs[cc];
+            const float wv = wts[cc];
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
                 const float wi = __shfl_sync(0xffffffffu, wv, i);
@@ -248,7 +258,7 @@ __device__ __forceinline__ void pair_epilogue(uint8_t* wb, uint32_t taddr, const
                     d[q] = *reinterpret_cast<const uint4*>(stage_chunk(wb, lane, q));
             }
             __syncwarp();
-        } else {  // EPI_COMBINE
+        } else {  // EPI_STORE_F32: out[b_row + token][col] = acc, fp32
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
                 // token row i: 32 features x 4 B = 128 B in chunks 0..7
@@ -257,59 +267,12 @@ __device__ __forceinline__ void pair_epilogue(uint8_t* wb, uint32_t taddr, const
             }
             __syncwarp();
             if (tok_ok) {
-                const size_t tok = (size_t)(t.b_row + c0 + lane);
-                const int col = t.ft * a.out_col_step + cta * 128 + wq * 32;
-                float acc[32];
+                float4* d = reinterpret_cast<float4*>(
+                    static_cast<float*>(a.out) + (size_t)(t.b_row + c0 + lane) * a.out_ld +
+                    t.ft * a.out_col_step + cta * 128 + wq * 32);
 #pragma unroll
-                for (int q = 0; q < 8; ++q) {
-                    const float4 s4 = *reinterpret_cast<const float4*>(stage_chunk(wb, lane, q));
-                    acc[4 * q] = s4.x;
-                    acc[4 * q + 1] = s4.y;
-                    acc[4 * q + 2] = s4.z;
-                    acc[4 * q + 3] = s4.w;
-                }
-                // y = shared + slot_0 + ... + slot_{k-1}, in that order; all slot
-                // pieces of this token are loaded before the ordered sum
-                const __nv_bfloat16* slots = static_cast<const __nv_bfloat16*>(a.slots);
-                uint4 sv[kMaxK][4];
-#pragma unroll
-                for (int j = 0; j < kMaxK; ++j)
-#pragma unroll
-                    for (int q = 0; q < 4; ++q)
-                        sv[j][q] = j < a.k ? __ldcg(reinterpret_cast<const uint4*>(
-                                                     slots + (tok * a.k + j) * a.out_ld + col) +
-                                                 q)
-                                           : make_uint4(0u, 0u, 0u, 0u);
-#pragma unroll
-                for (int j = 0; j < kMaxK; ++j) {
-                    if (j >= a.k) break;
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        const uint32_t w4[4] = {sv[j][q].x, sv[j][q].y, sv[j][q].z, sv[j][q].w};
-#pragma unroll
-                        for (int hh = 0; hh < 4; ++hh) {
-                            acc[q * 8 + 2 * hh] += __uint_as_float(w4[hh] << 16);
-                            acc[q * 8 + 2 * hh + 1] += __uint_as_float(w4[hh] & 0xffff0000u);
-                        }
-                    }
-                }
-                if (a.out_f32) {
-                    float4* d = reinterpret_cast<float4*>(static_cast<float*>(a.out) +
-                                                          tok * a.out_ld + col);
-#pragma unroll
-                    for (int q = 0; q < 8; ++q)
-                        d[q] = make_float4(acc[4 * q], acc[4 * q + 1], acc[4 * q + 2],
-                                           acc[4 * q + 3]);
-                } else {
-                    uint4* d = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.out) +
-                                                        tok * a.out_ld + col);
-#pragma unroll
-                    for (int q = 0; q < 4; ++q)
-                        d[q] = make_uint4(pack_bf16x2(acc[8 * q], acc[8 * q + 1]),
-                                          pack_bf16x2(acc[8 * q + 2], acc[8 * q + 3]),
-                                          pack_bf16x2(acc[8 * q + 4], acc[8 * q + 5]),
-                                          pack_bf16x2(acc[8 * q + 6], acc[8 * q + 7]));
-                }
+                for (int q = 0; q < 8; ++q)
+                    d[q] = *reinterpret_cast<const float4*>(stage_chunk(wb, lane, q));
             }
             __syncwarp();
         }
@@ -585,7 +548,7 @@ cudaError_t launch_pair_gemm(int epi, const CUtensorMap& tmA0, const CUtensorMap
     switch (epi) {
         case EPI_SWIGLU: kern = pair_gemm_kernel<EPI_SWIGLU>; break;
         case EPI_SCATTER: kern = pair_gemm_kernel<EPI_SCATTER>; break;
-        case EPI_COMBINE: kern = pair_gemm_kernel<EPI_COMBINE>; break;
+        case EPI_STORE_F32: kern = pair_gemm_kernel<EPI_STORE_F32>; break;
         default: return cudaErrorInvalidValue;
     }
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,

@@ -65,6 +65,8 @@ bool make_layout(int T, int d, int E, int k, int inter, int n_shared, int in_dt,
         esz * (size_t)L.rows_cap * inter,               // H
         esz * (size_t)T * n_shared * inter,             // H_SHARED
         esz * Tk * d,                                   // SLOTS (in_dt)
+        // Y_SHARED: fp32 shared-expert output before the final sum (tensor-core path)
+        in_dt == MOE_BF16 ? sizeof(float) * (size_t)T * d * (n_shared > 0 ? 1 : 0) : 0,
     };
     size_t o = 0;
     for (int i = 0; i < MOE_WS_TOTAL; ++i) {
@@ -412,24 +414,26 @@ MOE_API int moe_forward(const void* x, const void* W_router, const void* W_gate_
         e = launch_pair_gemm(EPI_SCATTER, a0, b0, p2, nullptr, nullptr, nullptr, n_pairs, s);
         if (e != cudaSuccess) return MOE_ERR_CUDA;
         stage_mark(4, s);
-        // 5. shared down projection with y = shared + slot_0 + ... + slot_{k-1}
+        // 5. shared down projection (fp32 rows), then the streaming final sum
+        //    y = shared + slot_0 + ... + slot_{k-1}
         if (n_shared > 0) {
+            float* y_sh = at<float>(workspace, L, MOE_WS_Y_SHARED);
             PairArgs p3 = p2;
             p3.K = SI;
             p3.counts = nullptr;
             p3.static_rows = T;
             p3.a_group_stride = 0;
-            p3.out = y;
-            p3.slots = slots;
-            p3.out_f32 = out_f32;
+            p3.out = y_sh;
             p3.row_src = nullptr;
             p3.topk_w = nullptr;
             if (!make_map(&a0, Wsh_dn, (uint64_t)d, SI, 128) ||
                 !make_map(&b0, h_sh, (uint64_t)T, SI, 64))
                 return MOE_ERR_CUDA;
-            e = launch_pair_gemm(EPI_COMBINE, a0, b0, p3, nullptr, nullptr, nullptr, n_pairs, s);
+            e = launch_pair_gemm(EPI_STORE_F32, a0, b0, p3, nullptr, nullptr, nullptr, n_pairs, s);
+            if (e != cudaSuccess) return MOE_ERR_CUDA;
+            e = launch_combine_slots(slots, 1, y_sh, T, d, k, y, out_f32, s);
         } else {
-            e = launch_combine_slots(slots, 1, T, d, k, y, out_f32, s);
+            e = launch_combine_slots(slots, 1, nullptr, T, d, k, y, out_f32, s);
         }
         if (e != cudaSuccess) return MOE_ERR_CUDA;
         stage_mark(5, s);
@@ -491,7 +495,7 @@ MOE_API int moe_forward(const void* x, const void* W_router, const void* W_gate_
                                grid_for(g2_tiles), s);
             if (e != cudaSuccess) return MOE_ERR_CUDA;
             stage_mark(4, s);
-            e = launch_combine_slots(slots, bf16 ? 1 : 0, T, d, k, y, out_f32, s);
+            e = launch_combine_slots(slots, bf16 ? 1 : 0, nullptr, T, d, k, y, out_f32, s);
             if (e != cudaSuccess) return MOE_ERR_CUDA;
         }
         stage_mark(5, s);
@@ -532,7 +536,7 @@ MOE_API int moe_forward(const void* x, const void* W_router, const void* W_gate_
                              reinterpret_cast<const float*>(Wsh_dn), g2s,
                              (T + 127) / 128 * 128, s);
     } else {
-        e = launch_combine_slots(slots, bf16 ? 1 : 0, T, d, k, y, out_f32, s);
+        e = launch_combine_slots(slots, bf16 ? 1 : 0, nullptr, T, d, k, y, out_f32, s);
     }
     if (e != cudaSuccess) return MOE_ERR_CUDA;
     stage_mark(5, s);

@@ -23,6 +23,7 @@ enum Epi : int {
     EPI_SCATTER = 1,  // slots[row_src[r]] = topk_w[row_src[r]] * acc  (rows with row_src < 0 skipped;
                       // bf16 slots on the tensor-core path, f32 on CUDA cores)
     EPI_COMBINE = 2,  // y[t] = acc + slots[t*k + 0] + ... + slots[t*k + k-1]
+    EPI_STORE_F32 = 3,  // out[row] = acc, fp32 (CTA-pair kernel)
 };
 
 // One grouped GEMM  out[r, n] = sum_c A[r, c] * B[b_row(r, n), c]  over row
@@ -64,8 +65,10 @@ cudaError_t launch_permute(const int32_t* idx, int T, int k, int E, int32_t* blo
 cudaError_t launch_gather_rows(const void* x, int d, int elem_bytes, int k,
                                const int32_t* offsets_total, const int32_t* row_src,
                                int rows_cap, void* x_perm, int num_sms, cudaStream_t s);
-cudaError_t launch_combine_slots(const void* slots, int slots_bf16, int T, int d, int k, void* y,
-                                 int out_f32, cudaStream_t s);
+// y[t] = base[t] + slots[t*k + 0] + ... + slots[t*k + k-1] in fp32, in that
+// order (base: fp32 [T, d] or nullptr for none).
+cudaError_t launch_combine_slots(const void* slots, int slots_bf16, const float* base, int T,
+                                 int d, int k, void* y, int out_f32, cudaStream_t s);
 
 cudaError_t launch_gemm_simt(int epi, const float* A, const float* B, const GemmArgs& a,
                              int rows_cap, cudaStream_t s);

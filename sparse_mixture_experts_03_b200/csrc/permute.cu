@@ -203,32 +203,63 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint4* __restric
     }
 }
 
-// y[t] = slots[t*k + 0] + ... + slots[t*k + k-1], in that order, in fp32
-// (used when there are no shared experts to fold the sum into).  Slots are f32
-// or bf16; 4 columns per thread.
+// y[t] = base[t] + slots[t*k + 0] + ... + slots[t*k + k-1] in fp32, in that
+// order (base = shared-expert output, or none).  8 columns per thread: whole
+// slot rows are read with 16-byte loads (bf16) or 2 x 16-byte loads (fp32),
+// every slot load of a thread issued before the ordered sum.
 template <typename TS>
 __global__ void __launch_bounds__(256) combine_slots_kernel(const TS* __restrict__ slots,
-                                                            int T, int d4, int k, void* y,
+                                                            const float* __restrict__ base,
+                                                            int T, int d8, int k, void* y,
                                                             int out_f32) {
-    const size_t n = (size_t)T * d4;
+    const size_t n = (size_t)T * d8;
     for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n;
          i += (size_t)gridDim.x * blockDim.x) {
-        const size_t t = i / d4, c = i % d4;
-        float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int j = 0; j < k; ++j) {
-            const TS* p = slots + ((t * k + j) * d4 + c) * 4;
-            a.x += Elem<TS>::to_f(p[0]);
-            a.y += Elem<TS>::to_f(p[1]);
-            a.z += Elem<TS>::to_f(p[2]);
-            a.w += Elem<TS>::to_f(p[3]);
+        const size_t t = i / d8, c = (i % d8) * 8;
+        const size_t d = (size_t)d8 * 8;
+        float a[8];
+        if (base != nullptr) {
+            const float4 b0 = __ldcs(reinterpret_cast<const float4*>(base + t * d + c));
+            const float4 b1 = __ldcs(reinterpret_cast<const float4*>(base + t * d + c) + 1);
+            a[0] = b0.x; a[1] = b0.y; a[2] = b0.z; a[3] = b0.w;
+            a[4] = b1.x; a[5] = b1.y; a[6] = b1.z; a[7] = b1.w;
+        } else {
+#pragma unroll
+            for (int q = 0; q < 8; ++q) a[q] = 0.f;
+        }
+        float sv[kMaxK][8];
+#pragma unroll
+        for (int j = 0; j < kMaxK; ++j) {
+            if (j < k) {
+                const TS* p = slots + (t * k + j) * d + c;
+                if constexpr (sizeof(TS) == 2) {
+                    const uint4 u = __ldcs(reinterpret_cast<const uint4*>(p));
+                    const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+                    for (int h = 0; h < 4; ++h) {
+                        sv[j][2 * h] = __uint_as_float(w4[h] << 16);
+                        sv[j][2 * h + 1] = __uint_as_float(w4[h] & 0xffff0000u);
+                    }
+                } else {
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) sv[j][q] = Elem<TS>::to_f(p[q]);
+                }
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < kMaxK; ++j) {
+            if (j >= k) break;
+#pragma unroll
+            for (int q = 0; q < 8; ++q) a[q] += sv[j][q];
         }
         if (out_f32) {
-            reinterpret_cast<float4*>(y)[i] = a;
+            float4* o = reinterpret_cast<float4*>(static_cast<float*>(y) + t * d + c);
+            o[0] = make_float4(a[0], a[1], a[2], a[3]);
+            o[1] = make_float4(a[4], a[5], a[6], a[7]);
         } else {
-            uint2 pk;
-            pk.x = pack_bf16x2(a.x, a.y);
-            pk.y = pack_bf16x2(a.z, a.w);
-            reinterpret_cast<uint2*>(y)[i] = pk;
+            *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(y) + t * d + c) =
+                make_uint4(pack_bf16x2(a[0], a[1]), pack_bf16x2(a[2], a[3]),
+                           pack_bf16x2(a[4], a[5]), pack_bf16x2(a[6], a[7]));
         }
     }
 }
@@ -259,19 +290,19 @@ cudaError_t launch_gather_rows(const void* x, int d, int elem_bytes, int k,
     return cudaGetLastError();
 }
 
-cudaError_t launch_combine_slots(const void* slots, int slots_bf16, int T, int d, int k, void* y,
-                                 int out_f32, cudaStream_t s) {
-    const int d4 = d / 4;
-    size_t n = (size_t)T * d4;
+cudaError_t launch_combine_slots(const void* slots, int slots_bf16, const float* base, int T,
+                                 int d, int k, void* y, int out_f32, cudaStream_t s) {
+    const int d8 = d / 8;
+    const size_t n = (size_t)T * d8;
     int blocks = (int)((n + 255) / 256);
-    if (blocks > 148 * 16) blocks = 148 * 16;
+    if (blocks > 148 * 8) blocks = 148 * 8;
     if (blocks < 1) blocks = 1;
     if (slots_bf16)
         combine_slots_kernel<__nv_bfloat16><<<blocks, 256, 0, s>>>(
-            static_cast<const __nv_bfloat16*>(slots), T, d4, k, y, out_f32);
+            static_cast<const __nv_bfloat16*>(slots), base, T, d8, k, y, out_f32);
     else
-        combine_slots_kernel<float><<<blocks, 256, 0, s>>>(static_cast<const float*>(slots), T,
-                                                           d4, k, y, out_f32);
+        combine_slots_kernel<float><<<blocks, 256, 0, s>>>(static_cast<const float*>(slots), base,
+                                                           T, d8, k, y, out_f32);
     return cudaGetLastError();
 }
 

@@ -27,7 +27,7 @@ MOE_F32, MOE_BF16 = 0, 1
 
 # workspace regions (indices into moe_workspace_layout)
 WS_REGIONS = ["status", "counts", "offsets", "block_counts", "topk_idx", "topk_w", "row_src",
-              "x_perm", "h", "h_shared", "slots"]
+              "x_perm", "h", "h_shared", "slots", "y_shared"]
 WS_TOTAL = len(WS_REGIONS)
 ROW_ALIGN = 128
 
