@@ -134,6 +134,23 @@ __device__ __forceinline__ void tc_mma_pair(uint32_t d_tmem, uint64_t a_desc, ui
         "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
         : "memory");
 }
+// The 4 MMAs (K = 16 each) of one 64-deep k-block: descriptors of step kk
+// are the base descriptors + 2 kk (32 bytes further along the swizzled rows);
+// the first accumulates into D only if `accumulate`, the rest always do.
+__device__ __forceinline__ void tc_mma4_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                             uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "setp.eq.b32 q, %3, %3;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %5, %6, %3, q;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %7, %8, %3, q;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %9, %10, %3, q;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "l"(a_desc + 2), "l"(b_desc + 2),
+        "l"(a_desc + 4), "l"(b_desc + 4), "l"(a_desc + 6), "l"(b_desc + 6)
+        : "memory");
+}
 // arrive (once) on the mbarrier at shared::cluster address `bar` when all
 // previously issued tcgen05 operations of this thread have completed
 __device__ __forceinline__ void tc_commit_pair(uint32_t bar_cluster) {
@@ -381,8 +398,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bool dense = a.counts == nullptr;
         t.ft = dense ? local % a.n_ftiles : local / nch;
         const int ch = dense ? local / a.n_ftiles : local % nch;
-        t.b_row = a.b_row_base + tail->seg_off[t.p][t.g] + ch * kNTile;
-        t.n_real = min(kNTile, cnt - ch * kNTile);
+        // the expert's tokens split into nch nearly equal chunks (sizes differ by
+        // at most one row), so tiles of one expert take the same time
+        const int r0 = (int)((long long)ch * cnt / nch);
+        const int r1 = (int)((long long)(ch + 1) * cnt / nch);
+        t.b_row = a.b_row_base + tail->seg_off[t.p][t.g] + r0;
+        t.n_real = r1 - r0;
         t.n = (t.n_real + 15) & ~15;
         return t;
     };
@@ -448,7 +469,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t ph = 0;
             int it = 0;
             bool ok = true;
-            const uint32_t empty0 = smem_u32(&tail->empty[0]);
+            // everything the k-block loop needs is precomputed: the loop body is
+            // one barrier poll, one block of 4 MMAs and two commits (a single
+            // thread issues them, so its instruction count per MMA bounds the rate)
+            const uint32_t empty_loc0 = smem_u32(&tail->empty[0]);
+            const uint32_t empty_rem0 = map_to_rank(&tail->empty[0], 1);
+            const uint64_t desc0 = sw128_kmajor_desc(smem_u32(smem));
+            constexpr uint64_t kStageDesc = kStageBytes >> 4;  // descriptor step per stage
+            constexpr uint64_t kBDesc = kABytes >> 4;          // B tile after A tile
             for (int tile = pair; ok && tile < total_tiles; tile += n_pairs, ++it) {
                 const Tile t = decode(tile);
                 const PairArgs& a = t.p == 0 ? args0 : args1;
@@ -463,23 +491,21 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint32_t d_tmem = tmem_base + (uint32_t)(acc * kNTile);
                 const uint32_t idesc = idesc_bf16_f32(2 * kARows, t.n);
                 const int kb_count = a.K / kBK;
+                uint32_t accum = 0;
                 for (int kb = 0; kb < kb_count; ++kb) {
-                    if (!mbar_wait_bounded(&tail->full[s], ph, abort_flag, status, SITE_GEMM_MMA,
+                    if (!mbar_try_wait(&tail->full[s], ph) &&
+                        !mbar_wait_bounded(&tail->full[s], ph, abort_flag, status, SITE_GEMM_MMA,
                                            limit)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t a_addr = smem_u32(smem + (size_t)s * kStageBytes);
-                    const uint32_t b_addr = a_addr + kABytes;
-#pragma unroll
-                    for (int kk = 0; kk < kBK / 16; ++kk)
-                        tc_mma_pair(d_tmem, sw128_kmajor_desc(a_addr + kk * 32),
-                                    sw128_kmajor_desc(b_addr + kk * 32), idesc,
-                                    (kb | kk) != 0 ? 1u : 0u);
+                    const uint64_t ad = desc0 + (uint64_t)s * kStageDesc;
+                    tc_mma4_pair(d_tmem, ad, ad + kBDesc, idesc, accum);
+                    accum = 1;
                     // stage s free in both CTAs once these MMAs have read it
-                    tc_commit_pair(empty0 + (uint32_t)(s * 8));
-                    tc_commit_pair(map_to_rank(&tail->empty[s], 1));
+                    tc_commit_pair(empty_loc0 + (uint32_t)(s * 8));
+                    tc_commit_pair(empty_rem0 + (uint32_t)(s * 8));
                     if (++s == kStages) {
                         s = 0;
                         ph ^= 1u;
