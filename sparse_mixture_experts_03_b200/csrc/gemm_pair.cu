@@ -40,17 +40,22 @@ namespace moe {
 
 namespace {
 
-constexpr int kBK = 64;                          // K per stage (one 128-byte swizzle atom)
+constexpr int kAtoms = 2;                        // 128-byte swizzle atoms (64 bf16 of K) per stage
+constexpr int kBK = 64 * kAtoms;                 // K per stage
 constexpr int kARows = 128;                      // weight rows per CTA (MMA M = 256 per pair)
-constexpr int kABytes = kARows * kBK * 2;        // 16 KiB
-constexpr int kBBox = 64;                        // token rows per B box
+constexpr int kABytes = kARows * kBK * 2;        // 32 KiB: 2 atoms x 128 weight rows
 constexpr int kBMaxRows = 128;                   // token rows per CTA (N <= 256 per pair)
-constexpr int kBBytes = kBMaxRows * kBK * 2;     // 16 KiB
-constexpr int kStageBytes = kABytes + kBBytes;   // 32 KiB
-constexpr int kStages = 6;
+constexpr int kBBytes = kBMaxRows * kBK * 2;     // 32 KiB: 2 atoms x 128 token rows
+constexpr int kHalfStageBytes = kABytes;         // bytes one producer warp brings per stage
+constexpr int kStageBytes = kABytes + kBBytes;   // 64 KiB
+constexpr int kStages = 3;
+constexpr int kAtomBytesA = kARows * 128;        // 16 KiB between the atoms of a tile
+constexpr int kAtomBytesB = kBMaxRows * 128;
+static_assert(kABytes == kBBytes, "both producers bring the same bytes per stage");
 constexpr int kNTile = 256;                      // tokens per tile
 constexpr int kTmemCols = 512;                   // 2 accumulators x 256 fp32 columns
-constexpr int kThreads = 192;
+constexpr int kThreads = 224;                    // 7 warps: producers 0 and 6, MMA 1, epilogue 2..5
+constexpr int kBProducerWarp = 6;
 constexpr int kEpiWarps = 4;
 constexpr int kMaxGroupsP = kMaxE + 1;
 
@@ -101,14 +106,15 @@ __device__ __forceinline__ bool epi_all(bool ok) {
         : "memory");
     return r != 0;
 }
-// TMA 2-D tile load whose completion is reported to an mbarrier of either
-// CTA of the pair (shared::cluster address), no multicast.
-__device__ __forceinline__ void tma_load_2d_pair(void* smem_dst, const CUtensorMap* map,
-                                                 uint32_t bar_cluster, int c0, int c1) {
+// TMA 3-D tile load {64 columns, rows, k-atoms} whose completion is reported
+// to an mbarrier of either CTA of the pair (shared::cluster address), no
+// multicast.
+__device__ __forceinline__ void tma_load_3d_pair(void* smem_dst, const CUtensorMap* map,
+                                                 uint32_t bar_cluster, int c0, int c1, int c2) {
     asm volatile(
-        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(smem_dst)),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster), "r"(c0), "r"(c1)
+        "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_u32(smem_dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster), "r"(c0), "r"(c1), "r"(c2)
         : "memory");
 }
 // 5-D variant (weights with gate/up interleaving, see PairArgs::a_mode).
@@ -124,15 +130,6 @@ __device__ __forceinline__ void tma_load_5d_pair(void* smem_dst, const CUtensorM
 }
 __device__ __forceinline__ void arrive_expect_tx_local(uint64_t* bar, uint32_t bytes) {
     mbar_arrive_expect_tx(bar, bytes);
-}
-__device__ __forceinline__ void tc_mma_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
-                                            uint32_t idesc, uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-        : "memory");
 }
 // The 4 MMAs (K = 16 each) of one 64-deep k-block: descriptors of step kk
 // are the base descriptors + 2 kk (32 bytes further along the swizzled rows);
@@ -316,7 +313,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (tid == 0) {
         for (int s = 0; s < kStages; ++s) {
-            mbar_init(&tail->full[s], 1);   // used in CTA 0: its producer's expect_tx
+            mbar_init(&tail->full[s], 2);   // used in CTA 0: its two producers' expect_tx
             mbar_init(&tail->empty[s], 1);  // one commit from the MMA issuer
         }
         for (int a = 0; a < 2; ++a) {
@@ -408,29 +405,25 @@ __global__ void __launch_bounds__(kThreads, 1)
         return t;
     };
 
-    if (warp == 0) {
-        // ------------------------------------------------ TMA producer (both CTAs)
+    if (warp == 0 || warp == kBProducerWarp) {
+        // ------------------------------------------------ TMA producers (both CTAs)
+        // Warp 0 loads the weight tile, warp kBProducerWarp the token tile: each
+        // warp's bulk copies are processed one after another, so two issuing
+        // warps with one 32 KiB copy each per stage keep twice the bytes moving.
+        const bool is_a = warp == 0;
         if (lane == 0) {
-            tma_prefetch_desc(&tmA0);
-            tma_prefetch_desc(&tmB0);
-            if (n_problems > 1) {
-                tma_prefetch_desc(&tmA1);
-                tma_prefetch_desc(&tmB1);
-            }
+            tma_prefetch_desc(is_a ? &tmA0 : &tmB0);
+            if (n_problems > 1) tma_prefetch_desc(is_a ? &tmA1 : &tmB1);
             int s = 0;
             uint32_t ph = 0;
             bool ok = true;
             for (int tile = pair; ok && tile < total_tiles; tile += n_pairs) {
                 const Tile t = decode(tile);
                 const PairArgs& a = t.p == 0 ? args0 : args1;
-                const CUtensorMap* mA = t.p == 0 ? &tmA0 : &tmA1;
-                const CUtensorMap* mB = t.p == 0 ? &tmB0 : &tmB1;
+                const CUtensorMap* m = is_a ? (t.p == 0 ? &tmA0 : &tmA1) : (t.p == 0 ? &tmB0 : &tmB1);
                 const int a_row0 = (int)(t.g * a.a_group_stride) + t.ft * a.a_tile_step +
                                    (int)cta * a.a_cta_step;
-                const int half_n = t.n >> 1;
-                const int b_row0 = t.b_row + (int)cta * half_n;
-                const int n_box = (half_n + kBBox - 1) / kBBox;
-                const uint32_t tx = 2u * (uint32_t)(kABytes + n_box * kBBox * kBK * 2);
+                const int b_row0 = t.b_row + (int)cta * (t.n >> 1);
                 const int kb_count = a.K / kBK;
                 for (int kb = 0; kb < kb_count; ++kb) {
                     if (!mbar_wait_bounded(&tail->empty[s], ph ^ 1u, abort_flag, status,
@@ -439,22 +432,24 @@ __global__ void __launch_bounds__(kThreads, 1)
                         break;
                     }
                     uint8_t* sa = smem + (size_t)s * kStageBytes;
-                    uint8_t* sb = sa + kABytes;
-                    if (cta == 0) arrive_expect_tx_local(&tail->full[s], tx);
+                    // both CTAs' copies of this operand complete on CTA 0's barrier
+                    if (cta == 0) arrive_expect_tx_local(&tail->full[s], 2u * kHalfStageBytes);
                     const uint32_t fb = map_to_rank(&tail->full[s], 0);
-                    if (a.a_mode == 0) {
-                        // 128 consecutive weight rows
-                        tma_load_2d_pair(sa, mA, fb, kb * kBK, a_row0);
+                    const int atom = kb * kAtoms;
+                    if (!is_a) {
+                        // 128 token rows x 2 k-atoms (rows past the tile's N/2 unused)
+                        tma_load_3d_pair(sa + kABytes, m, fb, 0, b_row0, atom);
+                    } else if (a.a_mode == 0) {
+                        // 128 consecutive weight rows x 2 k-atoms
+                        tma_load_3d_pair(sa, m, fb, 0, a_row0, atom);
                     } else {
                         // 4 blocks x (16 gate rows, 16 up rows) of features
-                        // ft * a_tile_step + cta * a_cta_step ... + 63 of group g
-                        tma_load_5d_pair(sa, mA, fb, kb * kBK, 0, 0,
-                                         (t.ft * a.a_tile_step + (int)cta * a.a_cta_step) >> 4,
-                                         t.g);
+                        // ft * a_tile_step + cta * a_cta_step ... + 63 of group g, x 2 k-atoms
+                        tma_load_5d_pair(sa, m, fb, 0, 0, 0,
+                                         t.g * a.a_blocks_per_group +
+                                             ((t.ft * a.a_tile_step + (int)cta * a.a_cta_step) >> 4),
+                                         atom);
                     }
-                    for (int i = 0; i < n_box; ++i)
-                        tma_load_2d_pair(sb + i * kBBox * kBK * 2, mB, fb, kb * kBK,
-                                         b_row0 + i * kBBox);
                     if (++s == kStages) {
                         s = 0;
                         ph ^= 1u;
@@ -501,8 +496,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     tc_fence_after();
                     const uint64_t ad = desc0 + (uint64_t)s * kStageDesc;
-                    tc_mma4_pair(d_tmem, ad, ad + kBDesc, idesc, accum);
-                    accum = 1;
+#pragma unroll
+                    for (int at = 0; at < kAtoms; ++at) {
+                        tc_mma4_pair(d_tmem, ad + (uint64_t)at * (kAtomBytesA >> 4),
+                                     ad + kBDesc + (uint64_t)at * (kAtomBytesB >> 4), idesc, accum);
+                        accum = 1;
+                    }
                     // stage s free in both CTAs once these MMAs have read it
                     tc_commit_pair(empty_loc0 + (uint32_t)(s * 8));
                     tc_commit_pair(empty_rem0 + (uint32_t)(s * 8));

@@ -135,16 +135,33 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
     return r == CUDA_SUCCESS;
 }
 
+// bf16 matrix [rows, K] seen as {64, rows, K/64} (inner 64 columns, rows,
+// 128-byte k-atoms): one box {64, 128, 2} brings 128 rows x 128 of K as two
+// consecutive 128B-swizzled 16 KiB tiles.
+bool make_map_rows_atoms(CUtensorMap* m, const void* base, uint64_t rows, uint64_t K) {
+    auto fn = encode_fn();
+    if (fn == nullptr || rows == 0 || K % 128 != 0) return false;
+    cuuint64_t dims[3] = {64, rows, K / 64};
+    cuuint64_t strides[2] = {K * 2, 128};
+    cuuint32_t box[3] = {64, 128, 2};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
+                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 // Gate/up weight [G][2][F][K] bf16 (per group: F gate rows, then F up rows)
-// seen as a 5-D tensor {K, 16, 2, F/16, G}; one box {64, 16, 2, 4, 1} brings 4
-// blocks of (16 gate rows, 16 up rows), i.e. 64 features with gate and up
-// interleaved per 16 rows, 128B swizzle.
+// seen as {64, 16, 2, G*2F/16, K/64}: 16-row blocks of the whole weight, the
+// gate/up axis (F rows apart) and k-atoms.  One box {64, 16, 2, 4, 2} at block
+// b of a gate half brings, for 2 k-atoms, 4 x (16 gate rows, the 16 matching
+// up rows): 64 features with gate and up interleaved per 16 rows.
 bool make_map_gate_up(CUtensorMap* m, const void* base, uint64_t G, uint64_t F, uint64_t K) {
     auto fn = encode_fn();
-    if (fn == nullptr || F % 64 != 0) return false;
-    cuuint64_t dims[5] = {K, 16, 2, F / 16, G};
-    cuuint64_t strides[4] = {K * 2, F * K * 2, 16 * K * 2, 2 * F * K * 2};
-    cuuint32_t box[5] = {64, 16, 2, 4, 1};
+    if (fn == nullptr || F % 64 != 0 || K % 128 != 0) return false;
+    cuuint64_t dims[5] = {64, 16, 2, G * 2 * F / 16, K / 64};
+    cuuint64_t strides[4] = {K * 2, F * K * 2, 16 * K * 2, 128};
+    cuuint32_t box[5] = {64, 16, 2, 4, 2};
     cuuint32_t estr[5] = {1, 1, 1, 1, 1};
     CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(base), dims, strides,
                     box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -366,13 +383,14 @@ MOE_API int moe_forward(const void* x, const void* W_router, const void* W_gate_
         p1.a_tile_step = 128;
         p1.a_cta_step = 64;
         p1.a_mode = 1;
+        p1.a_blocks_per_group = 2 * inter / 16;
         p1.out = h;
         p1.out_ld = inter;
         p1.out_col_step = 128;
         p1.status = status;
         p1.wait_limit_ns = kWaitLimitNs;
         if (!make_map_gate_up(&a0, W_gate_up, (uint64_t)E, inter, d) ||
-            !make_map(&b0, x_perm, (uint64_t)T * k, d, 64))
+            !make_map_rows_atoms(&b0, x_perm, (uint64_t)T * k, d))
             return MOE_ERR_CUDA;
         PairArgs p1s = p1;
         if (n_shared > 0) {
@@ -382,7 +400,8 @@ MOE_API int moe_forward(const void* x, const void* W_router, const void* W_gate_
             p1s.a_group_stride = 0;
             p1s.out = h_sh;
             p1s.out_ld = SI;
-            if (!make_map_gate_up(&a1, Wsh_gu, 1, SI, d) || !make_map(&b1, x, (uint64_t)T, d, 64))
+            p1s.a_blocks_per_group = 2 * SI / 16;
+            if (!make_map_gate_up(&a1, Wsh_gu, 1, SI, d) || !make_map_rows_atoms(&b1, x, (uint64_t)T, d))
                 return MOE_ERR_CUDA;
             e = launch_pair_gemm(EPI_SWIGLU, a0, b0, p1, &a1, &b1, &p1s, n_pairs, s);
         } else {
@@ -408,8 +427,8 @@ MOE_API int moe_forward(const void* x, const void* W_router, const void* W_gate_
         p2.k = k;
         p2.status = status;
         p2.wait_limit_ns = kWaitLimitNs;
-        if (!make_map(&a0, W_down, (uint64_t)E * d, inter, 128) ||
-            !make_map(&b0, h, (uint64_t)T * k, inter, 64))
+        if (!make_map_rows_atoms(&a0, W_down, (uint64_t)E * d, inter) ||
+            !make_map_rows_atoms(&b0, h, (uint64_t)T * k, inter))
             return MOE_ERR_CUDA;
         e = launch_pair_gemm(EPI_SCATTER, a0, b0, p2, nullptr, nullptr, nullptr, n_pairs, s);
         if (e != cudaSuccess) return MOE_ERR_CUDA;
@@ -426,8 +445,8 @@ MOE_API int moe_forward(const void* x, const void* W_router, const void* W_gate_
             p3.out = y_sh;
             p3.row_src = nullptr;
             p3.topk_w = nullptr;
-            if (!make_map(&a0, Wsh_dn, (uint64_t)d, SI, 128) ||
-                !make_map(&b0, h_sh, (uint64_t)T, SI, 64))
+            if (!make_map_rows_atoms(&a0, Wsh_dn, (uint64_t)d, SI) ||
+                !make_map_rows_atoms(&b0, h_sh, (uint64_t)T, SI))
                 return MOE_ERR_CUDA;
             e = launch_pair_gemm(EPI_STORE_F32, a0, b0, p3, nullptr, nullptr, nullptr, n_pairs, s);
             if (e != cudaSuccess) return MOE_ERR_CUDA;

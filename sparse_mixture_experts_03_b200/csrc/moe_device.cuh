@@ -101,18 +101,24 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Wait until the phase with parity `parity` of `bar` has completed.  Gives up
-// after `limit_ns` nanoseconds, or as soon as *abort becomes non-zero (another
-// role of the same CTA gave up).  On giving up records MOE_ERR_TIMEOUT with
-// `site` (unless another role already aborted) and returns false.
+// after about `limit_ns` nanoseconds (measured in SM clock cycles at no more
+// than 2 GHz, so the real limit is between limit_ns and a few times that), or
+// as soon as *abort becomes non-zero (another role of the same CTA gave up).
+// On giving up records MOE_ERR_TIMEOUT with `site` (unless another role already
+// aborted) and returns false.  The barrier is polled 64 times between checks
+// of the clock and of *abort, so a completing phase is seen within one poll.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity,
                                                   volatile int* abort, int* status, int site,
                                                   uint64_t limit_ns) {
     if (mbar_try_wait(bar, parity)) return true;
-    const uint64_t t0 = globaltimer_ns();
+    const uint64_t t0 = clock64();
+    const uint64_t limit_cycles = limit_ns * 2;
     for (;;) {
-        if (mbar_try_wait(bar, parity)) return true;
+#pragma unroll 1
+        for (int i = 0; i < 64; ++i)
+            if (mbar_try_wait(bar, parity)) return true;
         if (abort != nullptr && *abort) return false;
-        if (globaltimer_ns() - t0 > limit_ns) {
+        if ((uint64_t)clock64() - t0 > limit_cycles) {
             if (abort != nullptr) *abort = 1;
             set_status(status, MOE_ERR_TIMEOUT, site);
             return false;

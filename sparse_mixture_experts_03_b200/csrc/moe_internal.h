@@ -105,9 +105,10 @@ struct PairArgs {
     long long a_group_stride;
     int a_tile_step;
     int a_cta_step;
-    int a_mode;              // 0: 2-D map, 128 rows from a_row0
-                             // 1: 5-D map {K, 16, 2, F/16, G} of a [G][2][F][K] gate/up
-                             //    weight: 4 blocks of (16 gate, 16 up) rows per CTA
+    int a_mode;              // 0: 3-D map {64, rows, K/64}: 128 rows from a_row0
+                             // 1: 5-D map {64, 16, 2, G*2F/16, K/64} of a [G][2][F][K]
+                             //    gate/up weight: 4 blocks of (16 gate, 16 up) rows
+    int a_blocks_per_group;  // a_mode 1: 16-row blocks per group (2F / 16)
     void* out;
     int out_ld;
     int out_col_step;
@@ -120,8 +121,9 @@ struct PairArgs {
     unsigned long long wait_limit_ns;
 };
 size_t pair_gemm_smem_bytes();
-// tmA: weights, a_mode 0: box {64, 128}; a_mode 1: box {64, 16, 2, 4, 1};
-// tmB: tokens, box {64 cols, 64 rows}.
+// Each stage covers 128 of K (two 64-column swizzle atoms).  tmA: weights,
+// a_mode 0: box {64, 128, 2}; a_mode 1: box {64, 16, 2, 4, 2}; tmB: tokens,
+// 3-D {64, rows, K/64}, box {64, 128, 2}.  K must be a multiple of 128.
 cudaError_t launch_pair_gemm(int epi, const CUtensorMap& tmA0, const CUtensorMap& tmB0,
                              const PairArgs& a0, const CUtensorMap* tmA1,
                              const CUtensorMap* tmB1, const PairArgs* a1, int n_pairs,
