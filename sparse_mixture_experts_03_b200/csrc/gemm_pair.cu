@@ -58,6 +58,13 @@ constexpr int kThreads = 224;                    // 7 warps: producers 0 and 6, 
 constexpr int kBProducerWarp = 6;
 constexpr int kEpiWarps = 4;
 constexpr int kMaxGroupsP = kMaxE + 1;
+// Tile ids reach every role of a pair through a ring in shared memory, filled
+// by CTA 0's weight producer from a global ticket counter (dynamic scheduling:
+// a pair takes its next tile when its producer is ready for one).
+constexpr int kSchedDepth = 8;
+// readers of each ring entry: in CTA 0 the token producer, the MMA issuer and
+// the 4 epilogue warps; in CTA 1 both producers and the 4 epilogue warps
+constexpr int kSchedReaders = 2 * (2 + kEpiWarps);
 
 struct __align__(16) PairTail {
     uint4 stage[kEpiWarps * 256];  // per epilogue warp: 32 rows x 128 B staging
@@ -66,6 +73,9 @@ struct __align__(16) PairTail {
     uint64_t tfull[2];
     uint64_t tempty[2];
     uint64_t drain;
+    uint64_t sched_full[kSchedDepth];   // one arrive from the scheduler per entry
+    uint64_t sched_empty[kSchedDepth];  // used in CTA 0: kSchedReaders arrives per entry
+    int sched_tile[kSchedDepth];
     uint32_t tmem_base;
     int abort;
     int seg_off[2][kMaxGroupsP];   // first token row of each group
@@ -89,9 +99,6 @@ __device__ __forceinline__ uint32_t map_to_rank(const void* p, uint32_t rank) {
 __device__ __forceinline__ void cluster_sync_all() {
     asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;"
                  ::: "memory");
-}
-__device__ __forceinline__ void epi_bar() {  // the 4 epilogue warps only
-    asm volatile("bar.sync 1, %0;" ::"n"(kEpiWarps * 32) : "memory");
 }
 // AND of `ok` over the 4 epilogue warps (also a barrier among them)
 __device__ __forceinline__ bool epi_all(bool ok) {
@@ -158,6 +165,66 @@ __device__ __forceinline__ void tc_commit_pair(uint32_t bar_cluster) {
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar_cluster) {
     asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster)
                  : "memory");
+}
+
+// Wait for phase `parity` of a local barrier whose arrivals may come from the
+// other CTA of the pair (acquire at cluster scope), bounded like
+// mbar_wait_bounded.
+__device__ __forceinline__ bool mbar_try_wait_cl(uint64_t* bar, uint32_t parity) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return done != 0;
+}
+__device__ __forceinline__ bool mbar_wait_cl(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                             int* status, int site, uint64_t limit_ns) {
+    if (mbar_try_wait_cl(bar, parity)) return true;
+    const uint64_t t0 = clock64();
+    const uint64_t limit_cycles = limit_ns * 2;
+    for (;;) {
+#pragma unroll 1
+        for (int i = 0; i < 64; ++i)
+            if (mbar_try_wait_cl(bar, parity)) return true;
+        if (abort != nullptr && *abort) return false;
+        if ((uint64_t)clock64() - t0 > limit_cycles) {
+            if (abort != nullptr) *abort = 1;
+            set_status(status, MOE_ERR_TIMEOUT, site);
+            return false;
+        }
+    }
+}
+
+// Scheduler side of the tile ring (CTA 0's weight producer): entry j of the
+// pair's tile sequence goes into both CTAs' rings once all readers are done
+// with entry j - kSchedDepth.
+__device__ __forceinline__ bool sched_put(PairTail* tail, int j, int tile, volatile int* abort,
+                                          int* status, uint64_t limit) {
+    const int slot = j % kSchedDepth;
+    const uint32_t ph = (uint32_t)(j / kSchedDepth) & 1u;
+    if (!mbar_wait_cl(&tail->sched_empty[slot], ph ^ 1u, abort, status, SITE_GEMM_PRODUCER, limit))
+        return false;
+    tail->sched_tile[slot] = tile;
+    asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(map_to_rank(&tail->sched_tile[slot], 1)),
+                 "r"(tile)
+                 : "memory");
+    mbar_arrive(&tail->sched_full[slot]);
+    mbar_arrive_cluster(map_to_rank(&tail->sched_full[slot], 1));
+    return true;
+}
+// Reader side: entry j of the tile sequence, then release it to the scheduler.
+__device__ __forceinline__ bool sched_get(PairTail* tail, int j, int& tile, volatile int* abort,
+                                          int* status, int site, uint64_t limit) {
+    const int slot = j % kSchedDepth;
+    const uint32_t ph = (uint32_t)(j / kSchedDepth) & 1u;
+    if (!mbar_wait_cl(&tail->sched_full[slot], ph, abort, status, site, limit)) return false;
+    tile = *reinterpret_cast<volatile int*>(&tail->sched_tile[slot]);
+    mbar_arrive_cluster(map_to_rank(&tail->sched_empty[slot], 0));
+    return true;
 }
 
 struct Tile {
@@ -293,7 +360,7 @@ __device__ __forceinline__ void pair_epilogue(uint8_t* wb, uint32_t taddr, const
     }
 }
 
-template <int EPI>
+template <int EPI0, int EPI1>
 __global__ void __launch_bounds__(kThreads, 1)
     pair_gemm_kernel(const __grid_constant__ CUtensorMap tmA0,
                      const __grid_constant__ CUtensorMap tmB0,
@@ -321,6 +388,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&tail->tempty[a], 2 * kEpiWarps);  // used in CTA 0: both CTAs' warps
         }
         mbar_init(&tail->drain, 1);
+        for (int i = 0; i < kSchedDepth; ++i) {
+            mbar_init(&tail->sched_full[i], 1);
+            mbar_init(&tail->sched_empty[i], kSchedReaders);
+        }
         tail->abort = 0;
         fence_barrier_init();
     }
@@ -410,14 +481,29 @@ __global__ void __launch_bounds__(kThreads, 1)
         // Warp 0 loads the weight tile, warp kBProducerWarp the token tile: each
         // warp's bulk copies are processed one after another, so two issuing
         // warps with one 32 KiB copy each per stage keep twice the bytes moving.
+        // CTA 0's weight producer is also the pair's scheduler: it draws the
+        // pair's tiles from the ticket counter (the first one is the pair's
+        // index) and publishes them; every other role reads the ring.
         const bool is_a = warp == 0;
+        const bool is_sched = is_a && cta == 0;
         if (lane == 0) {
             tma_prefetch_desc(is_a ? &tmA0 : &tmB0);
             if (n_problems > 1) tma_prefetch_desc(is_a ? &tmA1 : &tmB1);
             int s = 0;
             uint32_t ph = 0;
             bool ok = true;
-            for (int tile = pair; ok && tile < total_tiles; tile += n_pairs) {
+            int next = pair;
+            for (int j = 0; ok; ++j) {
+                int tile = next < total_tiles ? next : total_tiles;  // total_tiles: end
+                if (is_sched) {
+                    if (!sched_put(tail, j, tile, abort_flag, status, limit)) break;
+                    // the ticket's latency is hidden behind this tile's loads
+                    if (tile < total_tiles) next = n_pairs + atomicAdd(args0.sched_counter, 1);
+                } else if (!sched_get(tail, j, tile, abort_flag, status, SITE_GEMM_PRODUCER,
+                                      limit)) {
+                    break;
+                }
+                if (tile >= total_tiles) break;
                 const Tile t = decode(tile);
                 const PairArgs& a = t.p == 0 ? args0 : args1;
                 const CUtensorMap* m = is_a ? (t.p == 0 ? &tmA0 : &tmA1) : (t.p == 0 ? &tmB0 : &tmB1);
@@ -472,7 +558,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint64_t desc0 = sw128_kmajor_desc(smem_u32(smem));
             constexpr uint64_t kStageDesc = kStageBytes >> 4;  // descriptor step per stage
             constexpr uint64_t kBDesc = kABytes >> 4;          // B tile after A tile
-            for (int tile = pair; ok && tile < total_tiles; tile += n_pairs, ++it) {
+            for (;; ++it) {
+                int tile;
+                if (!sched_get(tail, it, tile, abort_flag, status, SITE_GEMM_MMA, limit)) {
+                    ok = false;
+                    break;
+                }
+                if (tile >= total_tiles) break;
                 const Tile t = decode(tile);
                 const PairArgs& a = t.p == 0 ? args0 : args1;
                 const int acc = it & 1;
@@ -523,8 +615,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ------------------------------------------------ epilogue (warps 2..5, both CTAs)
         const int wq = warp & 3;  // TMEM lane quarter this warp may access
         uint8_t* wstage = reinterpret_cast<uint8_t*>(tail->stage) + wq * 4096;
-        int it = 0;
-        for (int tile = pair; tile < total_tiles; tile += n_pairs, ++it) {
+        for (int it = 0;; ++it) {
+            int tile = 0;
+            bool sched_ok = true;
+            if (lane == 0)
+                sched_ok = sched_get(tail, it, tile, abort_flag, status, SITE_GEMM_EPILOGUE, limit);
+            sched_ok = __shfl_sync(0xffffffffu, (int)sched_ok, 0) != 0;
+            tile = __shfl_sync(0xffffffffu, tile, 0);
+            // the 4 warps read the same sequence: they vote before leaving so
+            // that none is left waiting on a named barrier
+            if (!epi_all(sched_ok)) {
+                *abort_flag = 1;
+                break;
+            }
+            if (tile >= total_tiles) break;
             const int acc = it & 1;
             const uint32_t aph = (it >> 1) & 1;
             const bool got = mbar_wait_bounded(&tail->tfull[acc], aph, abort_flag, status,
@@ -540,9 +644,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tmem_base + (uint32_t)(acc * kNTile) + ((uint32_t)(wq * 32) << 16);
             // lane quarter wq = weight rows 32 wq .. 32 wq + 31 of this CTA
             if (t.p == 0)
-                pair_epilogue<EPI>(wstage, taddr, t, args0, cta, wq, lane);
+                pair_epilogue<EPI0>(wstage, taddr, t, args0, cta, wq, lane);
             else
-                pair_epilogue<EPI>(wstage, taddr, t, args1, cta, wq, lane);
+                pair_epilogue<EPI1>(wstage, taddr, t, args1, cta, wq, lane);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(map_to_rank(&tail->tempty[acc], 0));
@@ -563,19 +667,22 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 size_t pair_gemm_smem_bytes() { return kSmemBytes; }
 
-cudaError_t launch_pair_gemm(int epi, const CUtensorMap& tmA0, const CUtensorMap& tmB0,
+cudaError_t launch_pair_gemm(int epi0, int epi1, const CUtensorMap& tmA0, const CUtensorMap& tmB0,
                              const PairArgs& a0, const CUtensorMap* tmA1,
                              const CUtensorMap* tmB1, const PairArgs* a1, int n_pairs,
                              cudaStream_t s) {
     using Kern = void (*)(const CUtensorMap, const CUtensorMap, const CUtensorMap,
                           const CUtensorMap, const PairArgs, const PairArgs, int);
     Kern kern = nullptr;
-    switch (epi) {
-        case EPI_SWIGLU: kern = pair_gemm_kernel<EPI_SWIGLU>; break;
-        case EPI_SCATTER: kern = pair_gemm_kernel<EPI_SCATTER>; break;
-        case EPI_STORE_F32: kern = pair_gemm_kernel<EPI_STORE_F32>; break;
-        default: return cudaErrorInvalidValue;
-    }
+    if (epi0 == EPI_SWIGLU && epi1 == EPI_SWIGLU)
+        kern = pair_gemm_kernel<EPI_SWIGLU, EPI_SWIGLU>;
+    else if (epi0 == EPI_STORE_F32 && epi1 == EPI_SCATTER)
+        kern = pair_gemm_kernel<EPI_STORE_F32, EPI_SCATTER>;
+    else if (epi0 == EPI_SCATTER && epi1 == EPI_SCATTER)
+        kern = pair_gemm_kernel<EPI_SCATTER, EPI_SCATTER>;
+    else
+        return cudaErrorInvalidValue;
+    if (a0.sched_counter == nullptr) return cudaErrorInvalidValue;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)kSmemBytes);
     if (e != cudaSuccess) return e;

@@ -371,89 +371,95 @@ MOE_API int moe_forward(const void* x, const void* W_router, const void* W_gate_
                                            : Wsh_gu + (size_t)2 * SI * d * (bf16 ? 2 : 4);
 
     if (pair_path) {
-        // 3. gate/up + SwiGLU (routed experts, then shared experts on all tokens)
+        // 3. gate/up + SwiGLU: shared experts on all tokens (problem 0: the
+        //    longest tiles are handed out first), routed experts (problem 1)
         const int n_pairs = num_sms() / 2;
         CUtensorMap a0, b0, a1, b1;
-        PairArgs p1{};
-        p1.K = d;
-        p1.n_ftiles = inter / 128;
-        p1.n_groups = E;
-        p1.counts = counts;
-        p1.a_group_stride = 2LL * inter;
-        p1.a_tile_step = 128;
-        p1.a_cta_step = 64;
-        p1.a_mode = 1;
-        p1.a_blocks_per_group = 2 * inter / 16;
-        p1.out = h;
-        p1.out_ld = inter;
-        p1.out_col_step = 128;
-        p1.status = status;
-        p1.wait_limit_ns = kWaitLimitNs;
-        if (!make_map_gate_up(&a0, W_gate_up, (uint64_t)E, inter, d) ||
-            !make_map_rows_atoms(&b0, x_perm, (uint64_t)T * k, d))
+        PairArgs pr{};
+        pr.K = d;
+        pr.n_ftiles = inter / 128;
+        pr.n_groups = E;
+        pr.counts = counts;
+        pr.a_group_stride = 2LL * inter;
+        pr.a_tile_step = 128;
+        pr.a_cta_step = 64;
+        pr.a_mode = 1;
+        pr.a_blocks_per_group = 2 * inter / 16;
+        pr.out = h;
+        pr.out_ld = inter;
+        pr.out_col_step = 128;
+        pr.status = status;
+        pr.sched_counter = status + kSchedWordGateUp;
+        pr.wait_limit_ns = kWaitLimitNs;
+        if (!make_map_gate_up(&a1, W_gate_up, (uint64_t)E, inter, d) ||
+            !make_map_rows_atoms(&b1, x_perm, (uint64_t)T * k, d))
             return MOE_ERR_CUDA;
-        PairArgs p1s = p1;
         if (n_shared > 0) {
-            p1s.n_ftiles = SI / 128;
-            p1s.counts = nullptr;
-            p1s.static_rows = T;
-            p1s.a_group_stride = 0;
-            p1s.out = h_sh;
-            p1s.out_ld = SI;
-            p1s.a_blocks_per_group = 2 * SI / 16;
-            if (!make_map_gate_up(&a1, Wsh_gu, 1, SI, d) || !make_map_rows_atoms(&b1, x, (uint64_t)T, d))
+            PairArgs ps = pr;
+            ps.n_ftiles = SI / 128;
+            ps.counts = nullptr;
+            ps.static_rows = T;
+            ps.a_group_stride = 0;
+            ps.out = h_sh;
+            ps.out_ld = SI;
+            ps.a_blocks_per_group = 2 * SI / 16;
+            if (!make_map_gate_up(&a0, Wsh_gu, 1, SI, d) ||
+                !make_map_rows_atoms(&b0, x, (uint64_t)T, d))
                 return MOE_ERR_CUDA;
-            e = launch_pair_gemm(EPI_SWIGLU, a0, b0, p1, &a1, &b1, &p1s, n_pairs, s);
+            e = launch_pair_gemm(EPI_SWIGLU, EPI_SWIGLU, a0, b0, ps, &a1, &b1, &pr, n_pairs, s);
         } else {
-            e = launch_pair_gemm(EPI_SWIGLU, a0, b0, p1, nullptr, nullptr, nullptr, n_pairs, s);
+            e = launch_pair_gemm(EPI_SWIGLU, EPI_SWIGLU, a1, b1, pr, nullptr, nullptr, nullptr,
+                                 n_pairs, s);
         }
         if (e != cudaSuccess) return MOE_ERR_CUDA;
         stage_mark(3, s);
-        // 4. routed down projection, weighted scatter into bf16 token-order slots
-        PairArgs p2{};
-        p2.K = inter;
-        p2.n_ftiles = d / 256;
-        p2.n_groups = E;
-        p2.counts = counts;
-        p2.a_group_stride = d;
-        p2.a_tile_step = 256;
-        p2.a_cta_step = 128;
-        p2.a_mode = 0;
-        p2.out = slots;
-        p2.out_ld = d;
-        p2.out_col_step = 256;
-        p2.row_src = row_src;
-        p2.topk_w = w;
-        p2.k = k;
-        p2.status = status;
-        p2.wait_limit_ns = kWaitLimitNs;
-        if (!make_map_rows_atoms(&a0, W_down, (uint64_t)E * d, inter) ||
-            !make_map_rows_atoms(&b0, h, (uint64_t)T * k, inter))
+        // 4. down projections: shared experts into fp32 rows (problem 0),
+        //    routed experts weighted into bf16 token-order slots (problem 1)
+        PairArgs qr{};
+        qr.K = inter;
+        qr.n_ftiles = d / 256;
+        qr.n_groups = E;
+        qr.counts = counts;
+        qr.a_group_stride = d;
+        qr.a_tile_step = 256;
+        qr.a_cta_step = 128;
+        qr.a_mode = 0;
+        qr.out = slots;
+        qr.out_ld = d;
+        qr.out_col_step = 256;
+        qr.row_src = row_src;
+        qr.topk_w = w;
+        qr.k = k;
+        qr.status = status;
+        qr.sched_counter = status + kSchedWordDown;
+        qr.wait_limit_ns = kWaitLimitNs;
+        if (!make_map_rows_atoms(&a1, W_down, (uint64_t)E * d, inter) ||
+            !make_map_rows_atoms(&b1, h, (uint64_t)T * k, inter))
             return MOE_ERR_CUDA;
-        e = launch_pair_gemm(EPI_SCATTER, a0, b0, p2, nullptr, nullptr, nullptr, n_pairs, s);
-        if (e != cudaSuccess) return MOE_ERR_CUDA;
-        stage_mark(4, s);
-        // 5. shared down projection (fp32 rows), then the streaming final sum
-        //    y = shared + slot_0 + ... + slot_{k-1}
+        float* y_sh = nullptr;
         if (n_shared > 0) {
-            float* y_sh = at<float>(workspace, L, MOE_WS_Y_SHARED);
-            PairArgs p3 = p2;
-            p3.K = SI;
-            p3.counts = nullptr;
-            p3.static_rows = T;
-            p3.a_group_stride = 0;
-            p3.out = y_sh;
-            p3.row_src = nullptr;
-            p3.topk_w = nullptr;
+            y_sh = at<float>(workspace, L, MOE_WS_Y_SHARED);
+            PairArgs qs = qr;
+            qs.K = SI;
+            qs.counts = nullptr;
+            qs.static_rows = T;
+            qs.a_group_stride = 0;
+            qs.out = y_sh;
+            qs.row_src = nullptr;
+            qs.topk_w = nullptr;
             if (!make_map_rows_atoms(&a0, Wsh_dn, (uint64_t)d, SI) ||
                 !make_map_rows_atoms(&b0, h_sh, (uint64_t)T, SI))
                 return MOE_ERR_CUDA;
-            e = launch_pair_gemm(EPI_STORE_F32, a0, b0, p3, nullptr, nullptr, nullptr, n_pairs, s);
-            if (e != cudaSuccess) return MOE_ERR_CUDA;
-            e = launch_combine_slots(slots, 1, y_sh, T, d, k, y, out_f32, s);
+            e = launch_pair_gemm(EPI_STORE_F32, EPI_SCATTER, a0, b0, qs, &a1, &b1, &qr, n_pairs,
+                                 s);
         } else {
-            e = launch_combine_slots(slots, 1, nullptr, T, d, k, y, out_f32, s);
+            e = launch_pair_gemm(EPI_SCATTER, EPI_SCATTER, a1, b1, qr, nullptr, nullptr, nullptr,
+                                 n_pairs, s);
         }
+        if (e != cudaSuccess) return MOE_ERR_CUDA;
+        stage_mark(4, s);
+        // 5. the streaming final sum y = shared + slot_0 + ... + slot_{k-1}
+        e = launch_combine_slots(slots, 1, y_sh, T, d, k, y, out_f32, s);
         if (e != cudaSuccess) return MOE_ERR_CUDA;
         stage_mark(5, s);
         return MOE_OK;

@@ -16,6 +16,10 @@ constexpr int kRowAlign = 128;         // expert segments of the permuted layout
 constexpr int kPermBlockTokens = 256;  // tokens per block of the permutation kernels
 constexpr int kStatusWords = 64;       // int32 words of the status region of the workspace
 constexpr int kStatusSyncWord = 8;     // status word used as the scatter->combine tile counter
+// status words used as tile ticket counters of the CTA-pair GEMM launches
+// (reset to 0, with words 0..15, by the routing kernel at the start of a forward)
+constexpr int kSchedWordGateUp = 12;
+constexpr int kSchedWordDown = 13;
 
 // Epilogue variants of the grouped GEMMs.
 enum Epi : int {
@@ -118,13 +122,16 @@ struct PairArgs {
     int k;
     int out_f32;             // COMBINE
     int* status;
+    int* sched_counter;      // problem 0's: tile tickets of the launch, 0 at launch
     unsigned long long wait_limit_ns;
 };
 size_t pair_gemm_smem_bytes();
 // Each stage covers 128 of K (two 64-column swizzle atoms).  tmA: weights,
 // a_mode 0: box {64, 128, 2}; a_mode 1: box {64, 16, 2, 4, 2}; tmB: tokens,
 // 3-D {64, rows, K/64}, box {64, 128, 2}.  K must be a multiple of 128.
-cudaError_t launch_pair_gemm(int epi, const CUtensorMap& tmA0, const CUtensorMap& tmB0,
+// Epilogue pairs (epi0 for problem 0, epi1 for problem 1): SWIGLU/SWIGLU,
+// STORE_F32/SCATTER, SCATTER/SCATTER.
+cudaError_t launch_pair_gemm(int epi0, int epi1, const CUtensorMap& tmA0, const CUtensorMap& tmB0,
                              const PairArgs& a0, const CUtensorMap* tmA1,
                              const CUtensorMap* tmB1, const PairArgs* a1, int n_pairs,
                              cudaStream_t s);

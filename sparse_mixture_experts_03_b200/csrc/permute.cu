@@ -264,6 +264,48 @@ __global__ void __launch_bounds__(256) combine_slots_kernel(const TS* __restrict
     }
 }
 
+// bf16 slots, k fixed at compile time: one thread per (token, 8 columns), its
+// k slot loads (16 B each) and the base loads all issued before the ordered
+// sum; nothing is held beyond the raw loads, so a full SM of threads keeps
+// enough bytes in flight to stream at HBM speed.
+template <int K>
+__global__ void __launch_bounds__(256) combine_slots_bf16_kernel(
+    const uint4* __restrict__ slots, const float4* __restrict__ base, int T, int d8, void* y,
+    int out_f32) {
+    const size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x;
+    if (i >= (size_t)T * d8) return;
+    const size_t t = i / d8, c8 = i % d8;
+    uint4 raw[K];
+#pragma unroll
+    for (int j = 0; j < K; ++j) raw[j] = __ldcs(slots + (t * K + j) * d8 + c8);
+    float a[8];
+    if (base != nullptr) {
+        const float4 b0 = __ldcs(base + 2 * i), b1 = __ldcs(base + 2 * i + 1);
+        a[0] = b0.x; a[1] = b0.y; a[2] = b0.z; a[3] = b0.w;
+        a[4] = b1.x; a[5] = b1.y; a[6] = b1.z; a[7] = b1.w;
+    } else {
+#pragma unroll
+        for (int q = 0; q < 8; ++q) a[q] = 0.f;
+    }
+#pragma unroll
+    for (int j = 0; j < K; ++j) {
+        const uint32_t w4[4] = {raw[j].x, raw[j].y, raw[j].z, raw[j].w};
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+            a[2 * h] += __uint_as_float(w4[h] << 16);
+            a[2 * h + 1] += __uint_as_float(w4[h] & 0xffff0000u);
+        }
+    }
+    if (out_f32) {
+        float4* o = static_cast<float4*>(y) + 2 * i;
+        __stcs(o, make_float4(a[0], a[1], a[2], a[3]));
+        __stcs(o + 1, make_float4(a[4], a[5], a[6], a[7]));
+    } else {
+        static_cast<uint4*>(y)[i] = make_uint4(pack_bf16x2(a[0], a[1]), pack_bf16x2(a[2], a[3]),
+                                               pack_bf16x2(a[4], a[5]), pack_bf16x2(a[6], a[7]));
+    }
+}
+
 }  // namespace
 
 cudaError_t launch_permute(const int32_t* idx, int T, int k, int E, int32_t* block_counts,
@@ -294,15 +336,28 @@ cudaError_t launch_combine_slots(const void* slots, int slots_bf16, const float*
                                  int d, int k, void* y, int out_f32, cudaStream_t s) {
     const int d8 = d / 8;
     const size_t n = (size_t)T * d8;
+    if (slots_bf16) {
+        if (n == 0) return cudaSuccess;
+        const unsigned blocks16 = (unsigned)((n + 255) / 256);
+        const uint4* sl = static_cast<const uint4*>(slots);
+        const float4* b4 = reinterpret_cast<const float4*>(base);
+        switch (k) {
+#define MOE_COMBINE_K(KK)                                                                   \
+    case KK:                                                                                \
+        combine_slots_bf16_kernel<KK><<<blocks16, 256, 0, s>>>(sl, b4, T, d8, y, out_f32); \
+        break;
+            MOE_COMBINE_K(1) MOE_COMBINE_K(2) MOE_COMBINE_K(3) MOE_COMBINE_K(4)
+            MOE_COMBINE_K(5) MOE_COMBINE_K(6) MOE_COMBINE_K(7) MOE_COMBINE_K(8)
+#undef MOE_COMBINE_K
+            default: return cudaErrorInvalidValue;
+        }
+        return cudaGetLastError();
+    }
     int blocks = (int)((n + 255) / 256);
     if (blocks > 148 * 8) blocks = 148 * 8;
     if (blocks < 1) blocks = 1;
-    if (slots_bf16)
-        combine_slots_kernel<__nv_bfloat16><<<blocks, 256, 0, s>>>(
-            static_cast<const __nv_bfloat16*>(slots), base, T, d8, k, y, out_f32);
-    else
-        combine_slots_kernel<float><<<blocks, 256, 0, s>>>(static_cast<const float*>(slots), base,
-                                                           T, d8, k, y, out_f32);
+    combine_slots_kernel<float><<<blocks, 256, 0, s>>>(static_cast<const float*>(slots), base, T,
+                                                       d8, k, y, out_f32);
     return cudaGetLastError();
 }
 
