@@ -66,6 +66,19 @@ constexpr int kSchedDepth = 8;
 // the 4 epilogue warps; in CTA 1 both producers and the 4 epilogue warps
 constexpr int kSchedReaders = 2 * (2 + kEpiWarps);
 
+// One tile of a launch, decoded once by the scheduler and passed through the
+// ring as two 16-byte words.
+struct __align__(16) Tile {
+    int p;       // problem
+    int g;       // group (expert)
+    int ft;      // feature tile
+    int b_row;   // first token row of the tile in the B tensor
+    int n_real;  // tokens in the tile (1..256)
+    int n;       // MMA N: n_real rounded up to 16
+    int end;     // 1: no more tiles for this pair
+    int pad;
+};
+
 struct __align__(16) PairTail {
     uint4 stage[kEpiWarps * 256];  // per epilogue warp: 32 rows x 128 B staging
     uint64_t full[kStages];
@@ -75,7 +88,7 @@ struct __align__(16) PairTail {
     uint64_t drain;
     uint64_t sched_full[kSchedDepth];   // one arrive from the scheduler per entry
     uint64_t sched_empty[kSchedDepth];  // used in CTA 0: kSchedReaders arrives per entry
-    int sched_tile[kSchedDepth];
+    Tile sched_tile[kSchedDepth];
     uint32_t tmem_base;
     int abort;
     int seg_off[2][kMaxGroupsP];   // first token row of each group
@@ -162,6 +175,15 @@ __device__ __forceinline__ void tc_commit_pair(uint32_t bar_cluster) {
                      bar_cluster)
                  : "memory");
 }
+// Arrive on the barrier at this shared address in both CTAs of the pair once
+// the tcgen05 ops issued so far are complete (one commit, CTA mask 0b11).
+__device__ __forceinline__ void tc_commit_both(uint32_t bar_local) {
+    asm volatile(
+        "{\n\t.reg .b16 m;\n\tmov.b16 m, 3;\n\t"
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+        " [%0], m;\n\t}" ::"r"(bar_local)
+        : "memory");
+}
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar_cluster) {
     asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster)
                  : "memory");
@@ -199,42 +221,52 @@ __device__ __forceinline__ bool mbar_wait_cl(uint64_t* bar, uint32_t parity, vol
     }
 }
 
+__device__ __forceinline__ void st_cluster_v4(uint32_t addr, const int4& v) {
+    asm volatile("st.shared::cluster.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x),
+                 "r"(v.y), "r"(v.z), "r"(v.w)
+                 : "memory");
+}
+__device__ __forceinline__ int4 ld_shared_v4(const void* p) {
+    int4 v;
+    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "r"(smem_u32(p))
+                 : "memory");
+    return v;
+}
+
 // Scheduler side of the tile ring (CTA 0's weight producer): entry j of the
 // pair's tile sequence goes into both CTAs' rings once all readers are done
 // with entry j - kSchedDepth.
-__device__ __forceinline__ bool sched_put(PairTail* tail, int j, int tile, volatile int* abort,
-                                          int* status, uint64_t limit) {
+__device__ __forceinline__ bool sched_put(PairTail* tail, int j, const Tile& t,
+                                          volatile int* abort, int* status, uint64_t limit) {
     const int slot = j % kSchedDepth;
     const uint32_t ph = (uint32_t)(j / kSchedDepth) & 1u;
     if (!mbar_wait_cl(&tail->sched_empty[slot], ph ^ 1u, abort, status, SITE_GEMM_PRODUCER, limit))
         return false;
-    tail->sched_tile[slot] = tile;
-    asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(map_to_rank(&tail->sched_tile[slot], 1)),
-                 "r"(tile)
-                 : "memory");
+    const int4* w = reinterpret_cast<const int4*>(&t);
+    int4* dst = reinterpret_cast<int4*>(&tail->sched_tile[slot]);
+    dst[0] = w[0];
+    dst[1] = w[1];
+    const uint32_t remote = map_to_rank(&tail->sched_tile[slot], 1);
+    st_cluster_v4(remote, w[0]);
+    st_cluster_v4(remote + 16, w[1]);
     mbar_arrive(&tail->sched_full[slot]);
     mbar_arrive_cluster(map_to_rank(&tail->sched_full[slot], 1));
     return true;
 }
 // Reader side: entry j of the tile sequence, then release it to the scheduler.
-__device__ __forceinline__ bool sched_get(PairTail* tail, int j, int& tile, volatile int* abort,
+__device__ __forceinline__ bool sched_get(PairTail* tail, int j, Tile& t, volatile int* abort,
                                           int* status, int site, uint64_t limit) {
     const int slot = j % kSchedDepth;
     const uint32_t ph = (uint32_t)(j / kSchedDepth) & 1u;
     if (!mbar_wait_cl(&tail->sched_full[slot], ph, abort, status, site, limit)) return false;
-    tile = *reinterpret_cast<volatile int*>(&tail->sched_tile[slot]);
+    int4* w = reinterpret_cast<int4*>(&t);
+    w[0] = ld_shared_v4(&tail->sched_tile[slot]);
+    w[1] = ld_shared_v4(reinterpret_cast<const int4*>(&tail->sched_tile[slot]) + 1);
     mbar_arrive_cluster(map_to_rank(&tail->sched_empty[slot], 0));
     return true;
 }
-
-struct Tile {
-    int p;      // problem
-    int g;      // group (expert)
-    int ft;     // feature tile
-    int b_row;  // first token row of the tile in the B tensor
-    int n_real; // tokens in the tile (1..256)
-    int n;      // MMA N: n_real rounded up to 16
-};
 
 __device__ __forceinline__ int upper_group(const int* off, int n, int v) {
     // largest g in [0, n) with off[g] <= v
@@ -473,17 +505,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         t.b_row = a.b_row_base + tail->seg_off[t.p][t.g] + r0;
         t.n_real = r1 - r0;
         t.n = (t.n_real + 15) & ~15;
+        t.end = 0;
+        t.pad = 0;
         return t;
     };
 
     if (warp == 0 || warp == kBProducerWarp) {
         // ------------------------------------------------ TMA producers (both CTAs)
-        // Warp 0 loads the weight tile, warp kBProducerWarp the token tile: each
-        // warp's bulk copies are processed one after another, so two issuing
-        // warps with one 32 KiB copy each per stage keep twice the bytes moving.
-        // CTA 0's weight producer is also the pair's scheduler: it draws the
-        // pair's tiles from the ticket counter (the first one is the pair's
-        // index) and publishes them; every other role reads the ring.
+        // Warp 0 loads the weight tile, warp kBProducerWarp the token tile, one
+        // 32 KiB copy each per stage.  CTA 0's weight producer is also the
+        // pair's scheduler: it draws the pair's tiles from the ticket counter
+        // (the first one is the pair's index) and publishes them; every other
+        // role reads the ring.
         const bool is_a = warp == 0;
         const bool is_sched = is_a && cta == 0;
         if (lane == 0) {
@@ -494,17 +527,21 @@ __global__ void __launch_bounds__(kThreads, 1)
             bool ok = true;
             int next = pair;
             for (int j = 0; ok; ++j) {
-                int tile = next < total_tiles ? next : total_tiles;  // total_tiles: end
+                Tile t;
                 if (is_sched) {
-                    if (!sched_put(tail, j, tile, abort_flag, status, limit)) break;
-                    // the ticket's latency is hidden behind this tile's loads
-                    if (tile < total_tiles) next = n_pairs + atomicAdd(args0.sched_counter, 1);
-                } else if (!sched_get(tail, j, tile, abort_flag, status, SITE_GEMM_PRODUCER,
-                                      limit)) {
+                    if (next < total_tiles) {
+                        t = decode(next);
+                        // the ticket's latency is hidden behind this tile's loads
+                        next = n_pairs + atomicAdd(args0.sched_counter, 1);
+                    } else {
+                        t = Tile{};
+                        t.end = 1;
+                    }
+                    if (!sched_put(tail, j, t, abort_flag, status, limit)) break;
+                } else if (!sched_get(tail, j, t, abort_flag, status, SITE_GEMM_PRODUCER, limit)) {
                     break;
                 }
-                if (tile >= total_tiles) break;
-                const Tile t = decode(tile);
+                if (t.end) break;
                 const PairArgs& a = t.p == 0 ? args0 : args1;
                 const CUtensorMap* m = is_a ? (t.p == 0 ? &tmA0 : &tmA1) : (t.p == 0 ? &tmB0 : &tmB1);
                 const int a_row0 = (int)(t.g * a.a_group_stride) + t.ft * a.a_tile_step +
@@ -554,18 +591,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             // one barrier poll, one block of 4 MMAs and two commits (a single
             // thread issues them, so its instruction count per MMA bounds the rate)
             const uint32_t empty_loc0 = smem_u32(&tail->empty[0]);
-            const uint32_t empty_rem0 = map_to_rank(&tail->empty[0], 1);
             const uint64_t desc0 = sw128_kmajor_desc(smem_u32(smem));
             constexpr uint64_t kStageDesc = kStageBytes >> 4;  // descriptor step per stage
             constexpr uint64_t kBDesc = kABytes >> 4;          // B tile after A tile
             for (;; ++it) {
-                int tile;
-                if (!sched_get(tail, it, tile, abort_flag, status, SITE_GEMM_MMA, limit)) {
+                Tile t;
+                if (!sched_get(tail, it, t, abort_flag, status, SITE_GEMM_MMA, limit)) {
                     ok = false;
                     break;
                 }
-                if (tile >= total_tiles) break;
-                const Tile t = decode(tile);
+                if (t.end) break;
                 const PairArgs& a = t.p == 0 ? args0 : args1;
                 const int acc = it & 1;
                 const uint32_t aph = (it >> 1) & 1;
@@ -595,16 +630,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                         accum = 1;
                     }
                     // stage s free in both CTAs once these MMAs have read it
-                    tc_commit_pair(empty_loc0 + (uint32_t)(s * 8));
-                    tc_commit_pair(empty_rem0 + (uint32_t)(s * 8));
+                    tc_commit_both(empty_loc0 + (uint32_t)(s * 8));
                     if (++s == kStages) {
                         s = 0;
                         ph ^= 1u;
                     }
                 }
                 if (!ok) break;
-                tc_commit_pair(smem_u32(&tail->tfull[acc]));
-                tc_commit_pair(map_to_rank(&tail->tfull[acc], 1));
+                tc_commit_both(smem_u32(&tail->tfull[acc]));
             }
             if (!ok) *abort_flag = 1;
             // all tensor-core work of the pair is complete once `drain` fires
@@ -616,19 +649,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int wq = warp & 3;  // TMEM lane quarter this warp may access
         uint8_t* wstage = reinterpret_cast<uint8_t*>(tail->stage) + wq * 4096;
         for (int it = 0;; ++it) {
-            int tile = 0;
+            Tile t{};
             bool sched_ok = true;
             if (lane == 0)
-                sched_ok = sched_get(tail, it, tile, abort_flag, status, SITE_GEMM_EPILOGUE, limit);
+                sched_ok = sched_get(tail, it, t, abort_flag, status, SITE_GEMM_EPILOGUE, limit);
             sched_ok = __shfl_sync(0xffffffffu, (int)sched_ok, 0) != 0;
-            tile = __shfl_sync(0xffffffffu, tile, 0);
+            {
+                int* w = reinterpret_cast<int*>(&t);
+#pragma unroll
+                for (int q = 0; q < 8; ++q) w[q] = __shfl_sync(0xffffffffu, w[q], 0);
+            }
             // the 4 warps read the same sequence: they vote before leaving so
             // that none is left waiting on a named barrier
             if (!epi_all(sched_ok)) {
                 *abort_flag = 1;
                 break;
             }
-            if (tile >= total_tiles) break;
+            if (t.end) break;
             const int acc = it & 1;
             const uint32_t aph = (it >> 1) & 1;
             const bool got = mbar_wait_bounded(&tail->tfull[acc], aph, abort_flag, status,
@@ -639,7 +676,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                 break;
             }
             tc_fence_after();
-            const Tile t = decode(tile);
             const uint32_t taddr =
                 tmem_base + (uint32_t)(acc * kNTile) + ((uint32_t)(wq * 32) << 16);
             // lane quarter wq = weight rows 32 wq .. 32 wq + 31 of this CTA
