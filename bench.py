@@ -334,7 +334,7 @@ def main():
                            "frac": roof_ms / ms, "peak_tflops": pk["bf16_tflops"],
                            "hbm_gbs": pk["hbm_gbs"], "alg_bytes": bytes_alg,
                            "touched_experts": n_touched, "peak_source": pk["source"]},
-        "roofline": {"bound": "tensor", "kernel": "grouped_gemm_tc_kernel<0> (gate/up + SwiGLU, routed and shared)",
+        "roofline": {"bound": "tensor", "kernel": "pair_gemm_kernel<SWIGLU,SWIGLU> (gate/up + SwiGLU, shared and routed experts)",
                      "achieved": dom_ach, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
                      "frac": dom_ach / pk["bf16_tflops"], "traffic": None,
                      "flops_per_launch": g1_flops, "avg_launch_ms": dom_ms,

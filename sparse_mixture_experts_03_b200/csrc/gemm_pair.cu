@@ -699,9 +699,27 @@ __global__ void __launch_bounds__(kThreads, 1)
                      : "memory");
 }
 
+// A bounded wait on a barrier that nothing signals: it must end with
+// MOE_ERR_TIMEOUT in the status word (site SITE_SELFTEST), not hang.
+__global__ void selftest_timeout_kernel(int* status, unsigned long long limit_ns) {
+    __shared__ uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        abort_flag = 0;
+        fence_barrier_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0)
+        mbar_wait_bounded(&bar, 0u, &abort_flag, status, SITE_SELFTEST, limit_ns);
+}
+
 }  // namespace
 
-size_t pair_gemm_smem_bytes() { return kSmemBytes; }
+cudaError_t launch_selftest_timeout(int* status, unsigned long long limit_ns, cudaStream_t s) {
+    selftest_timeout_kernel<<<1, 32, 0, s>>>(status, limit_ns);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_pair_gemm(int epi0, int epi1, const CUtensorMap& tmA0, const CUtensorMap& tmB0,
                              const PairArgs& a0, const CUtensorMap* tmA1,

@@ -1,7 +1,7 @@
 // Grouped GEMM for fp32 inputs on CUDA cores (no tensor cores: fp32 operands
-// keep their full precision), with the same three epilogues and the same
-// padded, expert-contiguous row layout as the tcgen05 kernel.  Used for fp32
-// layers, which are small; bf16 layers take the tensor-core path.
+// keep their full precision) over expert segments padded to 128 rows, with
+// SwiGLU, weighted-scatter and combine epilogues.  Used for fp32 layers,
+// which are small; bf16 layers take the CTA-pair tcgen05 kernel.
 #include "moe_device.cuh"
 #include "moe_internal.h"
 

@@ -65,7 +65,7 @@ bool make_layout(int T, int d, int E, int k, int inter, int n_shared, int in_dt,
         esz * (size_t)L.rows_cap * inter,               // H
         esz * (size_t)T * n_shared * inter,             // H_SHARED
         esz * Tk * d,                                   // SLOTS (in_dt)
-        // Y_SHARED: fp32 shared-expert output before the final sum (tensor-core path)
+        // Y_SHARED: fp32 shared-expert output before the final sum (bf16 layers)
         in_dt == MOE_BF16 ? sizeof(float) * (size_t)T * d * (n_shared > 0 ? 1 : 0) : 0,
     };
     size_t o = 0;
@@ -119,22 +119,6 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     return fn;
 }
 
-// bf16 matrix [rows, cols] row-major, TMA box of 64 columns x box_rows rows,
-// 128B swizzle.
-bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
-              uint32_t box_rows = 128) {
-    auto fn = encode_fn();
-    if (fn == nullptr || rows == 0) return false;
-    cuuint64_t dims[2] = {cols, rows};
-    cuuint64_t strides[1] = {cols * 2};
-    cuuint32_t box[2] = {64, box_rows};
-    cuuint32_t estr[2] = {1, 1};
-    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
-                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS;
-}
-
 // bf16 matrix [rows, K] seen as {64, rows, K/64} (inner 64 columns, rows,
 // 128-byte k-atoms): one box {64, 128, 2} brings 128 rows x 128 of K as two
 // consecutive 128B-swizzled 16 KiB tiles.
@@ -181,22 +165,6 @@ bool g_stage_events_on = false;
 
 void stage_mark(int i, cudaStream_t s) {
     if (g_stage_events_on) cudaEventRecord(g_stage_events[i], s);
-}
-
-// Development switch: MOE_B200_GEMM=tile selects the 128-row tcgen05 tile
-// kernels instead of the CTA-pair kernels for bf16.
-bool use_tile_gemm() {
-    static int v = -1;
-    if (v < 0) {
-        const char* e = getenv("MOE_B200_GEMM");
-        v = (e != nullptr && strcmp(e, "tile") == 0) ? 1 : 0;
-    }
-    return v == 1;
-}
-
-int grid_for(long long tiles) {
-    const int n = num_sms();
-    return (int)(tiles < n ? (tiles > 0 ? tiles : 1) : n);
 }
 
 }  // namespace
@@ -307,70 +275,21 @@ MOE_API int moe_forward(const void* x, const void* W_router, const void* W_gate_
     if (e != cudaSuccess) return MOE_ERR_CUDA;
     stage_mark(1, s);
     // 2. permutation: histogram, scan, stable ranks, row gather
-    // the CTA-pair GEMMs take unpadded expert segments; the 128-row tile
-    // kernels (tcgen05 M-major, CUDA cores) take 128-padded ones
-    const bool pair_path = bf16 && !use_tile_gemm();
+    // the CTA-pair GEMMs (bf16) take unpadded expert segments; the CUDA-core
+    // kernels (fp32) take segments padded to their 128-row tiles
     e = launch_permute(idx, T, k, E, block_counts, counts, offsets, row_src,
-                       pair_path ? 1 : kRowAlign, status, s);
+                       bf16 ? 1 : kRowAlign, status, s);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
     e = launch_gather_rows(x, d, bf16 ? 2 : 4, k, offsets + E, row_src, L.rows_cap, x_perm,
                            num_sms(), s);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
     stage_mark(2, s);
 
-    GemmArgs g1{};
-    g1.K = d;
-    g1.n_groups = E;
-    g1.offsets = offsets;
-    g1.b_group_stride = 2LL * inter;
-    g1.b_half_off = inter;
-    g1.valid_rows = INT_MAX;
-    g1.out = h;
-    g1.out_ld = inter;
-    g1.out_f32 = bf16 ? 0 : 1;
-    g1.status = status;
-    g1.wait_limit_ns = kWaitLimitNs;
-
-    GemmArgs g1s = g1;
-    g1s.offsets = nullptr;
-    g1s.n_groups = 1;
-    g1s.static_rows = T;
-    g1s.b_group_stride = 0;
-    g1s.b_half_off = SI;
-    g1s.valid_rows = T;
-    g1s.out = h_sh;
-    g1s.out_ld = SI;
-
-    GemmArgs g2{};
-    g2.K = inter;
-    g2.n_groups = E;
-    g2.offsets = offsets;
-    g2.b_group_stride = d;
-    g2.valid_rows = INT_MAX;
-    g2.out = slots;
-    g2.out_ld = d;
-    g2.row_src = row_src;
-    g2.topk_w = w;
-    g2.k = k;
-    g2.status = status;
-    g2.wait_limit_ns = kWaitLimitNs;
-
-    GemmArgs g2s = g2;
-    g2s.K = SI;
-    g2s.offsets = nullptr;
-    g2s.n_groups = 1;
-    g2s.static_rows = T;
-    g2s.b_group_stride = 0;
-    g2s.valid_rows = T;
-    g2s.out = y;
-    g2s.slots = slots;
-    g2s.out_f32 = out_f32;
-
     const char* Wsh_gu = static_cast<const char*>(W_shared);
     const char* Wsh_dn = Wsh_gu == nullptr ? nullptr
                                            : Wsh_gu + (size_t)2 * SI * d * (bf16 ? 2 : 4);
 
-    if (pair_path) {
+    if (bf16) {
         // 3. gate/up + SwiGLU: shared experts on all tokens (problem 0: the
         //    longest tiles are handed out first), routed experts (problem 1)
         const int n_pairs = num_sms() / 2;
@@ -465,67 +384,53 @@ MOE_API int moe_forward(const void* x, const void* W_router, const void* W_gate_
         return MOE_OK;
     }
 
-    if (bf16) {
-        const int rows_tiles = L.rows_cap / 128;
-        // 3. gate/up + SwiGLU: routed experts, then the shared experts on all
-        //    tokens, as one persistent launch over both tile lists
-        g1.n_tiles = inter / 128;
-        g1.b_tile_step = 128;
-        g1.out_col_step = 128;
-        CUtensorMap tA, tB, tA1, tB1;
-        if (!make_map(&tA, x_perm, (uint64_t)L.rows_cap, d) ||
-            !make_map(&tB, W_gate_up, (uint64_t)E * 2 * inter, d))
-            return MOE_ERR_CUDA;
-        long long g1_tiles = (long long)rows_tiles * g1.n_tiles;
-        if (n_shared > 0) {
-            g1s.n_tiles = SI / 128;
-            g1s.b_tile_step = 128;
-            g1s.out_col_step = 128;
-            if (!make_map(&tA1, x, (uint64_t)T, d) || !make_map(&tB1, Wsh_gu, (uint64_t)2 * SI, d))
-                return MOE_ERR_CUDA;
-            g1_tiles += (long long)((T + 127) / 128) * g1s.n_tiles;
-            e = launch_gemm_tc(EPI_SWIGLU, tA, tB, g1, &tA1, &tB1, &g1s, grid_for(g1_tiles), s);
-        } else {
-            e = launch_gemm_tc(EPI_SWIGLU, tA, tB, g1, nullptr, nullptr, nullptr,
-                               grid_for(g1_tiles), s);
-        }
-        if (e != cudaSuccess) return MOE_ERR_CUDA;
-        stage_mark(3, s);
-        // 5. down projections: routed experts with the weighted scatter into
-        //    token-order slots, then the shared experts with the fixed-order
-        //    final sum, as one cooperative launch (combine tiles wait for all
-        //    scatter tiles through a device counter)
-        g2.n_tiles = d / 256;
-        g2.b_tile_step = 256;
-        g2.b_half_off = 128;
-        g2.out_col_step = 256;
-        if (!make_map(&tA, h, (uint64_t)L.rows_cap, inter) ||
-            !make_map(&tB, W_down, (uint64_t)E * d, inter))
-            return MOE_ERR_CUDA;
-        long long g2_tiles = (long long)rows_tiles * g2.n_tiles;
-        if (n_shared > 0) {
-            g2s.n_tiles = d / 256;
-            g2s.b_tile_step = 256;
-            g2s.b_half_off = 128;
-            g2s.out_col_step = 256;
-            if (!make_map(&tA1, h_sh, (uint64_t)T, SI) || !make_map(&tB1, Wsh_dn, (uint64_t)d, SI))
-                return MOE_ERR_CUDA;
-            g2_tiles += (long long)((T + 127) / 128) * g2s.n_tiles;
-            e = launch_gemm_tc(EPI_SCATTER, tA, tB, g2, &tA1, &tB1, &g2s, grid_for(g2_tiles), s,
-                               status + kStatusSyncWord);
-            if (e != cudaSuccess) return MOE_ERR_CUDA;
-            stage_mark(4, s);
-        } else {
-            e = launch_gemm_tc(EPI_SCATTER, tA, tB, g2, nullptr, nullptr, nullptr,
-                               grid_for(g2_tiles), s);
-            if (e != cudaSuccess) return MOE_ERR_CUDA;
-            stage_mark(4, s);
-            e = launch_combine_slots(slots, bf16 ? 1 : 0, nullptr, T, d, k, y, out_f32, s);
-            if (e != cudaSuccess) return MOE_ERR_CUDA;
-        }
-        stage_mark(5, s);
-        return MOE_OK;
-    }
+    GemmArgs g1{};
+    g1.K = d;
+    g1.n_groups = E;
+    g1.offsets = offsets;
+    g1.b_group_stride = 2LL * inter;
+    g1.b_half_off = inter;
+    g1.valid_rows = INT_MAX;
+    g1.out = h;
+    g1.out_ld = inter;
+    g1.out_f32 = bf16 ? 0 : 1;
+    g1.status = status;
+    g1.wait_limit_ns = kWaitLimitNs;
+
+    GemmArgs g1s = g1;
+    g1s.offsets = nullptr;
+    g1s.n_groups = 1;
+    g1s.static_rows = T;
+    g1s.b_group_stride = 0;
+    g1s.b_half_off = SI;
+    g1s.valid_rows = T;
+    g1s.out = h_sh;
+    g1s.out_ld = SI;
+
+    GemmArgs g2{};
+    g2.K = inter;
+    g2.n_groups = E;
+    g2.offsets = offsets;
+    g2.b_group_stride = d;
+    g2.valid_rows = INT_MAX;
+    g2.out = slots;
+    g2.out_ld = d;
+    g2.row_src = row_src;
+    g2.topk_w = w;
+    g2.k = k;
+    g2.status = status;
+    g2.wait_limit_ns = kWaitLimitNs;
+
+    GemmArgs g2s = g2;
+    g2s.K = SI;
+    g2s.offsets = nullptr;
+    g2s.n_groups = 1;
+    g2s.static_rows = T;
+    g2s.b_group_stride = 0;
+    g2s.valid_rows = T;
+    g2s.out = y;
+    g2s.slots = slots;
+    g2s.out_f32 = out_f32;
 
     // fp32: CUDA-core grouped GEMMs, 64-column output tiles
     const float* Wgu = static_cast<const float*>(W_gate_up);

@@ -15,7 +15,6 @@ constexpr int kMaxK = 8;
 constexpr int kRowAlign = 128;         // expert segments of the permuted layout are padded to this
 constexpr int kPermBlockTokens = 256;  // tokens per block of the permutation kernels
 constexpr int kStatusWords = 64;       // int32 words of the status region of the workspace
-constexpr int kStatusSyncWord = 8;     // status word used as the scatter->combine tile counter
 // status words used as tile ticket counters of the CTA-pair GEMM launches
 // (reset to 0, with words 0..15, by the routing kernel at the start of a forward)
 constexpr int kSchedWordGateUp = 12;
@@ -23,14 +22,14 @@ constexpr int kSchedWordDown = 13;
 
 // Epilogue variants of the grouped GEMMs.
 enum Epi : int {
-    EPI_SWIGLU = 0,   // out = bf16/f32 silu(gate) * up, columns [nt*cols, ...)
-    EPI_SCATTER = 1,  // slots[row_src[r]] = topk_w[row_src[r]] * acc  (rows with row_src < 0 skipped;
-                      // bf16 slots on the tensor-core path, f32 on CUDA cores)
-    EPI_COMBINE = 2,  // y[t] = acc + slots[t*k + 0] + ... + slots[t*k + k-1]
+    EPI_SWIGLU = 0,     // out = silu(gate) * up (bf16 on the CTA-pair kernel, f32 on CUDA cores)
+    EPI_SCATTER = 1,    // slots[row_src[r]] = topk_w[row_src[r]] * acc, rows with row_src < 0
+                        // skipped (bf16 slots on the CTA-pair kernel, f32 on CUDA cores)
+    EPI_COMBINE = 2,    // y[t] = acc + slots[t*k + 0] + ... + slots[t*k + k-1] (CUDA cores)
     EPI_STORE_F32 = 3,  // out[row] = acc, fp32 (CTA-pair kernel)
 };
 
-// One grouped GEMM  out[r, n] = sum_c A[r, c] * B[b_row(r, n), c]  over row
+// CUDA-core (fp32 layers) grouped GEMM  out[r, n] = sum_c A[r, c] * B[b_row(r, n), c]  over row
 // groups.  Rows of group g are [off[g], off[g+1]) of A (a multiple of 128
 // rows each); with offsets == nullptr there is one group of static_rows rows.
 struct GemmArgs {
@@ -48,7 +47,7 @@ struct GemmArgs {
     int out_col_step;          // output columns per N tile
     const int32_t* row_src;    // SCATTER
     const float* topk_w;       // SCATTER
-    const void* slots;         // COMBINE (bf16 on the tensor-core path, f32 on CUDA cores)
+    const void* slots;         // COMBINE: f32 slots
     int k;                     // SCATTER/COMBINE
     int out_f32;               // COMBINE: y dtype (1 f32, 0 bf16); SWIGLU f32 path: 1
     int* status;
@@ -76,20 +75,6 @@ cudaError_t launch_combine_slots(const void* slots, int slots_bf16, const float*
 
 cudaError_t launch_gemm_simt(int epi, const float* A, const float* B, const GemmArgs& a,
                              int rows_cap, cudaStream_t s);
-
-// tcgen05 path.  tmA: A rows [*, K] bf16, box {64, 128}; tmB: B rows [*, K] bf16, box {64, 128}.
-// One launch runs problem 0 and, when a1 != nullptr, problem 1 (same epilogue
-// kind) over one persistent tile list: problem 0's tiles first.
-size_t gemm_tc_smem_bytes();
-// epi selects the pair of epilogues: EPI_SWIGLU (both problems SwiGLU),
-// EPI_SCATTER (problem 0 scatter, problem 1 combine), EPI_COMBINE (combine).
-// With sync_counter (a zeroed device int; EPI_SCATTER with two problems
-// only), problem 1's epilogues wait until all of problem 0's have stored their
-// rows, and the grid is launched cooperatively so every CTA is resident.
-cudaError_t launch_gemm_tc(int epi, const CUtensorMap& tmA0, const CUtensorMap& tmB0,
-                           const GemmArgs& a0, const CUtensorMap* tmA1, const CUtensorMap* tmB1,
-                           const GemmArgs* a1, int grid, cudaStream_t s,
-                           int* sync_counter = nullptr);
 
 // Weights x tokens grouped GEMM on CTA pairs (see gemm_pair.cu).  Group g of a
 // problem has counts[g] token rows (static_rows when counts == nullptr),
@@ -125,7 +110,6 @@ struct PairArgs {
     int* sched_counter;      // problem 0's: tile tickets of the launch, 0 at launch
     unsigned long long wait_limit_ns;
 };
-size_t pair_gemm_smem_bytes();
 // Each stage covers 128 of K (two 64-column swizzle atoms).  tmA: weights,
 // a_mode 0: box {64, 128, 2}; a_mode 1: box {64, 16, 2, 4, 2}; tmB: tokens,
 // 3-D {64, rows, K/64}, box {64, 128, 2}.  K must be a multiple of 128.
