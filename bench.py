@@ -108,35 +108,54 @@ class ClockSampler:
                 "reasons": sorted(self.reasons), "samples": len(self.samples)}
 
 
-def dist_setup():
+def dist_setup(backend: str = "nccl", timeout_s: float = 120.0):
+    """One process per GPU: rank, world size and local rank from the launcher's
+    environment.  The process group (NCCL on GPUs, gloo for host-side tests)
+    carries only barriers and the max-over-ranks of the timings."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
+    if backend == "nccl":
+        torch.cuda.set_device(local)
     if world > 1:
         import datetime
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
-    else:
-        torch.cuda.set_device(local)
+        kw = {"device_id": torch.device("cuda", local)} if backend == "nccl" else {}
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=timeout_s), **kw)
     return world, rank, local
 
 
-def max_over_ranks(v: float, world: int) -> float:
+def max_over_ranks(v: float, world: int, device: str = "cuda") -> float:
     if world == 1:
         return v
     import torch.distributed as dist
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    t = torch.tensor([v], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 
 
-def barrier(world: int):
+def barrier(world: int, cuda: bool = True):
     if world > 1:
         import torch.distributed as dist
         dist.barrier()
-    torch.cuda.synchronize()
+    if cuda:
+        torch.cuda.synchronize()
+
+
+def rank_batch(w, inp, rank: int) -> torch.Tensor:
+    """Token batch of one rank (host tensor): rank 0 takes the workload's x,
+    rank r > 0 its own draw (seed + r); the weights are the same on every rank."""
+    if rank == 0:
+        return inp.x
+    return _randn((w.T, w.d), w.seed + rank, 0).to(inp.x.dtype)
+
+
+def run_config(w, world: int) -> dict:
+    """The `config` object of the JSON line (both arms)."""
+    return {"workload": f"{w.name}: {w.describe()}", "global_batch": world * w.T,
+            "tokens_per_gpu": w.T, "parallelism": f"token-parallel x{world} (replicas)",
+            "l2": "flushed between timed steps (512 MB write); weights 1.28 GB > L2",
+            "out_dtype": "f32"}
 
 
 def cpu_baseline(w, inp, budget_s: float = 15.0):
@@ -196,8 +215,7 @@ def run_reference(args, w):
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": sec * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": f"{w.name}: {w.describe()}", "tokens_per_step": n,
-                   "l2": "host CPU run"},
+        "config": run_config(w, world),
         "tflops": flops / sec / 1e12,
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": nthreads, "kind": "oracle",
                          "sample": f"{n} random tokens of {w.T} per step"},
@@ -226,9 +244,7 @@ def main():
     world, rank, local = dist_setup()
     dev = torch.device("cuda", local)
     inp = make_inputs(w)
-    if rank > 0:  # each rank its own batch of tokens, same weights
-        x = _randn((w.T, w.d), w.seed + rank, 0)
-        inp.x = x.to(inp.x.dtype)
+    inp.x = rank_batch(w, inp, rank)  # each rank its own batch of tokens, same weights
     x = inp.x.to(dev)
     Wr, Wgu, Wd = inp.W_router.to(dev), inp.W_gate_up.to(dev), inp.W_down.to(dev)
     Wsh = inp.W_shared.to(dev) if inp.W_shared is not None else None
@@ -325,10 +341,7 @@ def main():
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded N(0,1) activations, N(0,1/fan_in) weights; no dataset)",
-        "config": {"workload": f"{w.name}: {w.describe()}", "global_batch": world * w.T,
-                   "tokens_per_gpu": w.T, "parallelism": f"token-parallel x{world} (replicas)",
-                   "l2": "flushed between timed steps (512 MB write); weights 1.28 GB > L2",
-                   "out_dtype": "f32"},
+        "config": run_config(w, world),
         "tflops": tflops,
         "roofline_layer": {"bound": "tensor", "roofline_ms": roof_ms,
                            "frac": roof_ms / ms, "peak_tflops": pk["bf16_tflops"],
