@@ -175,15 +175,40 @@ MOE_API int moe_selftest_timeout(void *workspace, int limit_us, void *stream);
  * events != NULL (n == MOE_N_STAGE_EVENTS handles of type cudaEvent_t, created
  * by the caller), every following moe_forward in this process records
  * events[i] on its stream: [0] start, [1] after routing, [2] after the
- * permutation, [3] after the gate/up GEMM (routed and shared experts, one
- * launch), [4] after the down GEMM (routed experts, and the shared experts with
- * the final sum, one launch), [5] at the end (after the separate final sum
- * kernel that runs only when there are no shared experts).  events == NULL
+ * permutation, [3] after the gate/up GEMM (shared and routed experts, one
+ * launch), [4] after the down GEMM (shared and routed experts, one launch),
+ * [5] at the end (after the final sum y = shared + slots).  events == NULL
  * turns it off.  Process-wide setting, not thread-safe.  Returns MOE_OK or
  * MOE_ERR_INVALID_ARG.
  */
 #define MOE_N_STAGE_EVENTS 6
 MOE_API int moe_set_stage_events(void *const *events, int n);
+
+/*
+ * moe_expert_counts_noalloc -- per-expert token counts and segment offsets
+ * of a routing result, for callers that must not allocate device memory or
+ * pass a workspace on the call path (e.g. a serving step whose device memory
+ * is planned once up front).  The pages have no counterpart of this entry
+ * point: it is the histogram + scan of the permutation stage ("开源混合架构大模
+ * 型技术解析", section 四: tokens grouped by the expert they go to), exposed on
+ * its own with its scratch in a fixed device array of the library.
+ *   topk_idx  device, int32[T, k]: expert ids (ids outside [0, E) are not
+ *             counted)
+ *   counts    device, int32[E]   out: tokens routed to each expert
+ *   offsets   device, int32[E+1] out: exclusive prefix sum of counts
+ *             (unpadded segments; offsets[E] = number of counted ids)
+ * Limits: 1 <= k <= 8, k <= E <= 256, ceil(T/256) * E <= 65536 (the fixed
+ * scratch: 256 KiB; e.g. T <= 262144 at E = 64).  Larger sizes return
+ * MOE_ERR_WORKSPACE before any launch; bad arguments MOE_ERR_INVALID_ARG.
+ * Allocates nothing.  The first call on a device (with it current) looks up
+ * the scratch array's device address; make that first call before any stream
+ * capture.  All calls share the one array: calls that overlap in time (two
+ * streams, two host threads) race and must be serialised by the caller.
+ * Nothing in the array needs to start at zero.  Queues work on `stream` and
+ * returns without synchronising.
+ */
+MOE_API int moe_expert_counts_noalloc(const int32_t *topk_idx, int T, int k, int E,
+                                      int32_t *counts, int32_t *offsets, void *stream);
 
 /* moe_status_string -- static text for a status code. */
 MOE_API const char *moe_status_string(int status);

@@ -70,6 +70,12 @@ cudaError_t launch_gather_rows(const void* x, int d, int elem_bytes, int k,
                                int rows_cap, void* x_perm, int num_sms, cudaStream_t s);
 // y[t] = base[t] + slots[t*k + 0] + ... + slots[t*k + k-1] in fp32, in that
 // order (base: fp32 [T, d] or nullptr for none).
+// Per-expert counts and unpadded segment offsets of a routing result
+// (histogram + scan only); block_counts holds ceil(T/256) * E int32.  Expert
+// ids outside [0, E) are not counted.
+cudaError_t launch_expert_counts(const int32_t* idx, int T, int k, int E,
+                                 int32_t* block_counts, int32_t* counts, int32_t* offsets,
+                                 cudaStream_t s);
 cudaError_t launch_combine_slots(const void* slots, int slots_bf16, const float* base, int T,
                                  int d, int k, void* y, int out_f32, cudaStream_t s);
 

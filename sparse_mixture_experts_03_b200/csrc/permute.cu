@@ -6,9 +6,11 @@
 // tokens that route to different experts).
 //
 // Layout produced: expert e owns rows [offsets[e], offsets[e+1]) of x_perm,
-// a segment padded to a multiple of 128 rows.  Inside a segment the real rows
-// come first, in increasing token order (stable), then padding rows whose
-// row_src is -1.  row_src[r] = t*k + j for the row holding slot j of token t.
+// a segment padded to a multiple of `align` rows (1 for the CTA-pair GEMMs of
+// bf16 layers, 128 for the CUDA-core GEMMs of fp32 layers).  Inside a segment
+// the real rows come first, in increasing token order (stable), then padding
+// rows whose row_src is -1.  row_src[r] = t*k + j for the row holding slot j
+// of token t.
 #include "moe_device.cuh"
 #include "moe_internal.h"
 
@@ -316,6 +318,17 @@ cudaError_t launch_permute(const int32_t* idx, int T, int k, int E, int32_t* blo
     perm_scan_kernel<<<1, 1024, 0, s>>>(block_counts, nb, E, align, counts, offsets, row_src);
     perm_rank_kernel<<<nb, kPermBlockTokens, 0, s>>>(idx, T, k, E, block_counts, offsets, row_src,
                                                      status);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_expert_counts(const int32_t* idx, int T, int k, int E,
+                                 int32_t* block_counts, int32_t* counts, int32_t* offsets,
+                                 cudaStream_t s) {
+    const int nb = (T + kPermBlockTokens - 1) / kPermBlockTokens;
+    if (nb > 0)
+        perm_count_kernel<<<nb, kPermBlockTokens, 0, s>>>(idx, T, k, E, block_counts, nullptr);
+    // align 1: no padding rows, so the scan writes no row_src entry
+    perm_scan_kernel<<<1, 1024, 0, s>>>(block_counts, nb, E, 1, counts, offsets, nullptr);
     return cudaGetLastError();
 }
 

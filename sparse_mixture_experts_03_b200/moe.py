@@ -34,7 +34,8 @@ ROW_ALIGN = 128
 # every entry point declared in include/moe.h
 SYMBOLS = ["moe_workspace_bytes", "moe_workspace_layout", "moe_route", "moe_forward",
            "moe_get_device_status", "moe_clear_device_status", "moe_selftest_timeout",
-           "moe_set_stage_events", "moe_status_string", "moe_version"]
+           "moe_set_stage_events", "moe_status_string", "moe_version",
+           "moe_expert_counts_noalloc"]
 N_STAGE_EVENTS = 6
 STAGES = ["route", "permute", "gate_up", "down", "combine"]
 
@@ -75,6 +76,8 @@ def lib() -> ctypes.CDLL:
         L.moe_status_string.argtypes = [i]
         L.moe_status_string.restype = ctypes.c_char_p
         L.moe_version.restype = i
+        L.moe_expert_counts_noalloc.argtypes = [vp, i, i, i, vp, vp, vp]
+        L.moe_expert_counts_noalloc.restype = i
         _lib = L
     return _lib
 
@@ -145,6 +148,15 @@ def route(x: torch.Tensor, W_router: torch.Tensor, k: int, n_group: int, topk_gr
     _check(lib().moe_route(_ptr(x), _ptr(W_router), T, d, E, k, n_group, topk_group, _dt(x),
                            _ptr(topk_idx), _ptr(topk_w), _stream(stream)), "moe_route")
     return topk_idx, topk_w
+
+
+def expert_counts_noalloc(topk_idx: torch.Tensor, E: int, counts: torch.Tensor,
+                          offsets: torch.Tensor, stream=None) -> None:
+    """moe_expert_counts_noalloc: counts int32 [E] and offsets int32 [E+1] of a
+    routing result, into the caller's tensors; the library allocates nothing."""
+    T, k = topk_idx.shape
+    _check(lib().moe_expert_counts_noalloc(_ptr(topk_idx), T, k, E, _ptr(counts), _ptr(offsets),
+                                           _stream(stream)), "moe_expert_counts_noalloc")
 
 
 def forward(x: torch.Tensor, W_router: torch.Tensor, W_gate_up: torch.Tensor,
