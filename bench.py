@@ -150,6 +150,27 @@ def rank_batch(w, inp, rank: int) -> torch.Tensor:
     return _randn((w.T, w.d), w.seed + rank, 0).to(inp.x.dtype)
 
 
+def profiled_traffic(w):
+    """DRAM bytes per launch of the gate/up GEMM from the committed ncu summary,
+    or None when the workload differs or the kernel source changed since."""
+    import hashlib
+    if w.name != "prefill":
+        return None
+    csrc = os.path.join(ROOT, "sparse_mixture_experts_03_b200", "csrc")
+    try:
+        with open(os.path.join(csrc, "gemm_pair.cu"), "rb") as f:
+            src = f.read()
+        with open(os.path.join(csrc, "moe_device.cuh"), "rb") as f:
+            src += f.read()
+        with open(os.path.join(ROOT, "profiles", "pair_gemm_prefill_T4096.md")) as f:
+            fields = dict(l.strip().split(": ", 1) for l in f if ": " in l and l.startswith("    "))
+        if fields.get("kernel_source_sha256") != hashlib.sha256(src).hexdigest():
+            return None
+        return int(fields["traffic_bytes_per_launch"])
+    except (OSError, KeyError, ValueError):
+        return None
+
+
 def run_config(w, world: int) -> dict:
     """The `config` object of the JSON line (both arms)."""
     return {"workload": f"{w.name}: {w.describe()}", "global_batch": world * w.T,
@@ -349,7 +370,7 @@ def main():
                            "touched_experts": n_touched, "peak_source": pk["source"]},
         "roofline": {"bound": "tensor", "kernel": "pair_gemm_kernel<SWIGLU,SWIGLU> (gate/up + SwiGLU, shared and routed experts)",
                      "achieved": dom_ach, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
-                     "frac": dom_ach / pk["bf16_tflops"], "traffic": None,
+                     "frac": dom_ach / pk["bf16_tflops"], "traffic": profiled_traffic(w),
                      "flops_per_launch": g1_flops, "avg_launch_ms": dom_ms,
                      "peak_kind": f"bf16 burst ({pk['source']})"},
         "stage_ms": stage,
