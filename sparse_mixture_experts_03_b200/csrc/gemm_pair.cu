@@ -45,13 +45,10 @@ constexpr int kBK = 64 * kAtoms;                 // K per stage
 constexpr int kARows = 128;                      // weight rows per CTA (MMA M = 256 per pair)
 constexpr int kABytes = kARows * kBK * 2;        // 32 KiB: 2 atoms x 128 weight rows
 constexpr int kBMaxRows = 128;                   // token rows per CTA (N <= 256 per pair)
-constexpr int kBBytes = kBMaxRows * kBK * 2;     // 32 KiB: 2 atoms x 128 token rows
-constexpr int kHalfStageBytes = kABytes;         // bytes one producer warp brings per stage
+constexpr int kBBytes = kBMaxRows * kBK * 2;     // up to 32 KiB: 2 atoms x 16 rb token rows
 constexpr int kStageBytes = kABytes + kBBytes;   // 64 KiB
 constexpr int kStages = 3;
 constexpr int kAtomBytesA = kARows * 128;        // 16 KiB between the atoms of a tile
-constexpr int kAtomBytesB = kBMaxRows * 128;
-static_assert(kABytes == kBBytes, "both producers bring the same bytes per stage");
 constexpr int kNTile = 256;                      // tokens per tile
 constexpr int kTmemCols = 512;                   // 2 accumulators x 256 fp32 columns
 constexpr int kThreads = 224;                    // 7 warps: producers 0 and 6, MMA 1, epilogue 2..5
@@ -394,10 +391,7 @@ __device__ __forceinline__ void pair_epilogue(uint8_t* wb, uint32_t taddr, const
 
 template <int EPI0, int EPI1>
 __global__ void __launch_bounds__(kThreads, 1)
-    pair_gemm_kernel(const __grid_constant__ CUtensorMap tmA0,
-                     const __grid_constant__ CUtensorMap tmB0,
-                     const __grid_constant__ CUtensorMap tmA1,
-                     const __grid_constant__ CUtensorMap tmB1, const PairArgs args0,
+    pair_gemm_kernel(const __grid_constant__ PairMaps maps, const PairArgs args0,
                      const PairArgs args1, int n_problems) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -520,8 +514,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bool is_a = warp == 0;
         const bool is_sched = is_a && cta == 0;
         if (lane == 0) {
-            tma_prefetch_desc(is_a ? &tmA0 : &tmB0);
-            if (n_problems > 1) tma_prefetch_desc(is_a ? &tmA1 : &tmB1);
+            for (int p = 0; p < n_problems; ++p) {
+                if (is_a) {
+                    tma_prefetch_desc(&maps.a[p]);
+                } else {
+                    for (int j = 0; j < kTokenBoxes; ++j) tma_prefetch_desc(&maps.b[p][j]);
+                }
+            }
             int s = 0;
             uint32_t ph = 0;
             bool ok = true;
@@ -543,7 +542,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 if (t.end) break;
                 const PairArgs& a = t.p == 0 ? args0 : args1;
-                const CUtensorMap* m = is_a ? (t.p == 0 ? &tmA0 : &tmA1) : (t.p == 0 ? &tmB0 : &tmB1);
+                // token rows per CTA: N/2, loaded with the box of 16 rb rows
+                const int rb = ((t.n >> 1) + 15) >> 4;
+                const CUtensorMap* m = is_a ? &maps.a[t.p] : &maps.b[t.p][rb - 1];
+                const uint32_t op_bytes = is_a ? (uint32_t)kABytes : (uint32_t)rb * 4096u;
                 const int a_row0 = (int)(t.g * a.a_group_stride) + t.ft * a.a_tile_step +
                                    (int)cta * a.a_cta_step;
                 const int b_row0 = t.b_row + (int)cta * (t.n >> 1);
@@ -556,11 +558,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     uint8_t* sa = smem + (size_t)s * kStageBytes;
                     // both CTAs' copies of this operand complete on CTA 0's barrier
-                    if (cta == 0) arrive_expect_tx_local(&tail->full[s], 2u * kHalfStageBytes);
+                    if (cta == 0) arrive_expect_tx_local(&tail->full[s], 2u * op_bytes);
                     const uint32_t fb = map_to_rank(&tail->full[s], 0);
                     const int atom = kb * kAtoms;
                     if (!is_a) {
-                        // 128 token rows x 2 k-atoms (rows past the tile's N/2 unused)
+                        // 16 rb token rows x 2 k-atoms (rows past the tile's N/2 unused)
                         tma_load_3d_pair(sa + kABytes, m, fb, 0, b_row0, atom);
                     } else if (a.a_mode == 0) {
                         // 128 consecutive weight rows x 2 k-atoms
@@ -612,6 +614,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + (uint32_t)(acc * kNTile);
                 const uint32_t idesc = idesc_bf16_f32(2 * kARows, t.n);
+                // the token tile's second k-atom starts 16 rb rows x 128 B after its first
+                const uint64_t b_atom_desc = (uint64_t)(((t.n >> 1) + 15) >> 4) * (2048 >> 4);
                 const int kb_count = a.K / kBK;
                 uint32_t accum = 0;
                 for (int kb = 0; kb < kb_count; ++kb) {
@@ -626,7 +630,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                     for (int at = 0; at < kAtoms; ++at) {
                         tc_mma4_pair(d_tmem, ad + (uint64_t)at * (kAtomBytesA >> 4),
-                                     ad + kBDesc + (uint64_t)at * (kAtomBytesB >> 4), idesc, accum);
+                                     ad + kBDesc + (uint64_t)at * b_atom_desc, idesc, accum);
                         accum = 1;
                     }
                     // stage s free in both CTAs once these MMAs have read it
@@ -721,12 +725,9 @@ cudaError_t launch_selftest_timeout(int* status, unsigned long long limit_ns, cu
     return cudaGetLastError();
 }
 
-cudaError_t launch_pair_gemm(int epi0, int epi1, const CUtensorMap& tmA0, const CUtensorMap& tmB0,
-                             const PairArgs& a0, const CUtensorMap* tmA1,
-                             const CUtensorMap* tmB1, const PairArgs* a1, int n_pairs,
-                             cudaStream_t s) {
-    using Kern = void (*)(const CUtensorMap, const CUtensorMap, const CUtensorMap,
-                          const CUtensorMap, const PairArgs, const PairArgs, int);
+cudaError_t launch_pair_gemm(int epi0, int epi1, const PairMaps& maps, const PairArgs& a0,
+                             const PairArgs* a1, int n_pairs, cudaStream_t s) {
+    using Kern = void (*)(const PairMaps, const PairArgs, const PairArgs, int);
     Kern kern = nullptr;
     if (epi0 == EPI_SWIGLU && epi1 == EPI_SWIGLU)
         kern = pair_gemm_kernel<EPI_SWIGLU, EPI_SWIGLU>;
@@ -753,8 +754,7 @@ cudaError_t launch_pair_gemm(int epi0, int epi1, const CUtensorMap& tmA0, const 
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kern, tmA0, tmB0, np > 1 ? *tmA1 : tmA0,
-                              np > 1 ? *tmB1 : tmB0, a0, np > 1 ? *a1 : a0, np);
+    return cudaLaunchKernelEx(&cfg, kern, maps, a0, np > 1 ? *a1 : a0, np);
 }
 
 }  // namespace moe

@@ -120,19 +120,27 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 }
 
 // bf16 matrix [rows, K] seen as {64, rows, K/64} (inner 64 columns, rows,
-// 128-byte k-atoms): one box {64, 128, 2} brings 128 rows x 128 of K as two
-// consecutive 128B-swizzled 16 KiB tiles.
-bool make_map_rows_atoms(CUtensorMap* m, const void* base, uint64_t rows, uint64_t K) {
+// 128-byte k-atoms): one box {64, box_rows, 2} brings box_rows rows x 128 of
+// K as two consecutive 128B-swizzled tiles of box_rows x 128 bytes.
+bool make_map_rows_atoms(CUtensorMap* m, const void* base, uint64_t rows, uint64_t K,
+                         uint32_t box_rows = 128) {
     auto fn = encode_fn();
     if (fn == nullptr || rows == 0 || K % 128 != 0) return false;
     cuuint64_t dims[3] = {64, rows, K / 64};
     cuuint64_t strides[2] = {K * 2, 128};
-    cuuint32_t box[3] = {64, 128, 2};
+    cuuint32_t box[3] = {64, box_rows, 2};
     cuuint32_t estr[3] = {1, 1, 1};
     CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
                     box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
+}
+
+// The token maps of one problem: boxes of 16, 32, ..., 128 rows.
+bool make_token_maps(CUtensorMap (&m)[kTokenBoxes], const void* base, uint64_t rows, uint64_t K) {
+    for (int j = 0; j < kTokenBoxes; ++j)
+        if (!make_map_rows_atoms(&m[j], base, rows, K, 16u * (j + 1))) return false;
+    return true;
 }
 
 // Gate/up weight [G][2][F][K] bf16 (per group: F gate rows, then F up rows)
@@ -293,7 +301,7 @@ MOE_API int moe_forward(const void* x, const void* W_router, const void* W_gate_
         // 3. gate/up + SwiGLU: shared experts on all tokens (problem 0: the
         //    longest tiles are handed out first), routed experts (problem 1)
         const int n_pairs = num_sms() / 2;
-        CUtensorMap a0, b0, a1, b1;
+        PairMaps mp{};
         PairArgs pr{};
         pr.K = d;
         pr.n_ftiles = inter / 128;
@@ -310,8 +318,10 @@ MOE_API int moe_forward(const void* x, const void* W_router, const void* W_gate_
         pr.status = status;
         pr.sched_counter = status + kSchedWordGateUp;
         pr.wait_limit_ns = kWaitLimitNs;
-        if (!make_map_gate_up(&a1, W_gate_up, (uint64_t)E, inter, d) ||
-            !make_map_rows_atoms(&b1, x_perm, (uint64_t)T * k, d))
+        // problem 1 (routed) goes in slot 1 when there are shared experts, else slot 0
+        const int pr_slot = n_shared > 0 ? 1 : 0;
+        if (!make_map_gate_up(&mp.a[pr_slot], W_gate_up, (uint64_t)E, inter, d) ||
+            !make_token_maps(mp.b[pr_slot], x_perm, (uint64_t)T * k, d))
             return MOE_ERR_CUDA;
         if (n_shared > 0) {
             PairArgs ps = pr;
@@ -322,13 +332,12 @@ MOE_API int moe_forward(const void* x, const void* W_router, const void* W_gate_
             ps.out = h_sh;
             ps.out_ld = SI;
             ps.a_blocks_per_group = 2 * SI / 16;
-            if (!make_map_gate_up(&a0, Wsh_gu, 1, SI, d) ||
-                !make_map_rows_atoms(&b0, x, (uint64_t)T, d))
+            if (!make_map_gate_up(&mp.a[0], Wsh_gu, 1, SI, d) ||
+                !make_token_maps(mp.b[0], x, (uint64_t)T, d))
                 return MOE_ERR_CUDA;
-            e = launch_pair_gemm(EPI_SWIGLU, EPI_SWIGLU, a0, b0, ps, &a1, &b1, &pr, n_pairs, s);
+            e = launch_pair_gemm(EPI_SWIGLU, EPI_SWIGLU, mp, ps, &pr, n_pairs, s);
         } else {
-            e = launch_pair_gemm(EPI_SWIGLU, EPI_SWIGLU, a1, b1, pr, nullptr, nullptr, nullptr,
-                                 n_pairs, s);
+            e = launch_pair_gemm(EPI_SWIGLU, EPI_SWIGLU, mp, pr, nullptr, n_pairs, s);
         }
         if (e != cudaSuccess) return MOE_ERR_CUDA;
         stage_mark(3, s);
@@ -352,8 +361,9 @@ MOE_API int moe_forward(const void* x, const void* W_router, const void* W_gate_
         qr.status = status;
         qr.sched_counter = status + kSchedWordDown;
         qr.wait_limit_ns = kWaitLimitNs;
-        if (!make_map_rows_atoms(&a1, W_down, (uint64_t)E * d, inter) ||
-            !make_map_rows_atoms(&b1, h, (uint64_t)T * k, inter))
+        const int qr_slot = n_shared > 0 ? 1 : 0;
+        if (!make_map_rows_atoms(&mp.a[qr_slot], W_down, (uint64_t)E * d, inter) ||
+            !make_token_maps(mp.b[qr_slot], h, (uint64_t)T * k, inter))
             return MOE_ERR_CUDA;
         float* y_sh = nullptr;
         if (n_shared > 0) {
@@ -366,14 +376,12 @@ MOE_API int moe_forward(const void* x, const void* W_router, const void* W_gate_
             qs.out = y_sh;
             qs.row_src = nullptr;
             qs.topk_w = nullptr;
-            if (!make_map_rows_atoms(&a0, Wsh_dn, (uint64_t)d, SI) ||
-                !make_map_rows_atoms(&b0, h_sh, (uint64_t)T, SI))
+            if (!make_map_rows_atoms(&mp.a[0], Wsh_dn, (uint64_t)d, SI) ||
+                !make_token_maps(mp.b[0], h_sh, (uint64_t)T, SI))
                 return MOE_ERR_CUDA;
-            e = launch_pair_gemm(EPI_STORE_F32, EPI_SCATTER, a0, b0, qs, &a1, &b1, &qr, n_pairs,
-                                 s);
+            e = launch_pair_gemm(EPI_STORE_F32, EPI_SCATTER, mp, qs, &qr, n_pairs, s);
         } else {
-            e = launch_pair_gemm(EPI_SCATTER, EPI_SCATTER, a1, b1, qr, nullptr, nullptr, nullptr,
-                                 n_pairs, s);
+            e = launch_pair_gemm(EPI_SCATTER, EPI_SCATTER, mp, qr, nullptr, n_pairs, s);
         }
         if (e != cudaSuccess) return MOE_ERR_CUDA;
         stage_mark(4, s);

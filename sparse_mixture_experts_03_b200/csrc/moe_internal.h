@@ -116,15 +116,20 @@ struct PairArgs {
     int* sched_counter;      // problem 0's: tile tickets of the launch, 0 at launch
     unsigned long long wait_limit_ns;
 };
-// Each stage covers 128 of K (two 64-column swizzle atoms).  tmA: weights,
-// a_mode 0: box {64, 128, 2}; a_mode 1: box {64, 16, 2, 4, 2}; tmB: tokens,
-// 3-D {64, rows, K/64}, box {64, 128, 2}.  K must be a multiple of 128.
+// Tensor maps of one launch.  Each stage covers 128 of K (two 64-column
+// swizzle atoms).  a[p]: weights of problem p, a_mode 0: box {64, 128, 2};
+// a_mode 1: box {64, 16, 2, 4, 2}.  b[p][j]: tokens of problem p, 3-D
+// {64, rows, K/64}, box {64, 16 (j + 1), 2}: a tile of N tokens loads N/2 rows
+// per CTA with the smallest box that covers them.  K must be a multiple of 128.
+constexpr int kTokenBoxes = 8;
+struct PairMaps {
+    CUtensorMap a[2];
+    CUtensorMap b[2][kTokenBoxes];
+};
 // Epilogue pairs (epi0 for problem 0, epi1 for problem 1): SWIGLU/SWIGLU,
-// STORE_F32/SCATTER, SCATTER/SCATTER.
-cudaError_t launch_pair_gemm(int epi0, int epi1, const CUtensorMap& tmA0, const CUtensorMap& tmB0,
-                             const PairArgs& a0, const CUtensorMap* tmA1,
-                             const CUtensorMap* tmB1, const PairArgs* a1, int n_pairs,
-                             cudaStream_t s);
+// STORE_F32/SCATTER, SCATTER/SCATTER.  a1 == nullptr: one problem.
+cudaError_t launch_pair_gemm(int epi0, int epi1, const PairMaps& maps, const PairArgs& a0,
+                             const PairArgs* a1, int n_pairs, cudaStream_t s);
 
 cudaError_t launch_selftest_timeout(int* status, unsigned long long limit_ns, cudaStream_t s);
 
