@@ -177,9 +177,11 @@ MOE_API int moe_selftest_timeout(void *workspace, int limit_us, void *stream);
  * events[i] on its stream: [0] start, [1] after routing, [2] after the
  * permutation, [3] after the gate/up GEMM (shared and routed experts, one
  * launch), [4] after the down GEMM (shared and routed experts, one launch),
- * [5] at the end (after the final sum y = shared + slots).  events == NULL
- * turns it off.  Process-wide setting, not thread-safe.  Returns MOE_OK or
- * MOE_ERR_INVALID_ARG.
+ * [5] at the end (after the final sum y = shared + slots).  A NULL entry is
+ * not recorded (an event record between two kernels keeps the second from
+ * starting early, so a timing run records only the boundaries it needs).
+ * events == NULL turns it off.  Process-wide setting, not thread-safe.
+ * Returns MOE_OK or MOE_ERR_INVALID_ARG.
  */
 #define MOE_N_STAGE_EVENTS 6
 MOE_API int moe_set_stage_events(void *const *events, int n);

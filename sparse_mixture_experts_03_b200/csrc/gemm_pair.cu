@@ -421,6 +421,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         tail->abort = 0;
         fence_barrier_init();
     }
+    // everything below reads or writes memory of earlier kernels (counts,
+    // token rows, outputs): wait until the previous kernel has completed
+    pdl_wait();
     // group offsets of both problems: rows and tiles (exclusive prefix sums)
     if (warp == 0) {
         for (int p = 0; p < n_problems; ++p) {
@@ -693,6 +696,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     }
 
+    pdl_trigger();
     tc_fence_before();
     __syncthreads();
     cluster_sync_all();  // no CTA leaves while its pair may still signal or read it
@@ -742,19 +746,8 @@ cudaError_t launch_pair_gemm(int epi0, int epi1, const PairMaps& maps, const Pai
                                          (int)kSmemBytes);
     if (e != cudaSuccess) return e;
     const int np = a1 != nullptr ? 2 : 1;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(2 * n_pairs);
-    cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = kSmemBytes;
-    cfg.stream = s;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 2;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kern, maps, a0, np > 1 ? *a1 : a0, np);
+    return launch_pdl(kern, dim3(2 * n_pairs), dim3(kThreads), kSmemBytes, s, 2, maps, a0,
+                      np > 1 ? *a1 : a0, np);
 }
 
 }  // namespace moe

@@ -17,6 +17,7 @@ __global__ void __launch_bounds__(256) grouped_gemm_simt_kernel(const float* __r
                                                                 const GemmArgs args, int a_rows) {
     __shared__ float As[TK][TM + 4];
     __shared__ float Bs[2][TK][TN + 4];
+    pdl_wait();
     const int n_groups = args.offsets != nullptr ? args.n_groups : 1;
     const int total_rows = args.offsets != nullptr
                                ? args.offsets[n_groups]
@@ -106,6 +107,7 @@ __global__ void __launch_bounds__(256) grouped_gemm_simt_kernel(const float* __r
             }
         }
     }
+    pdl_trigger();
 }
 
 }  // namespace
@@ -119,18 +121,17 @@ cudaError_t launch_gemm_simt(int epi, const float* A, const float* B, const Gemm
     const int a_rows = a.offsets != nullptr ? rows_cap : a.static_rows;
     switch (epi) {
         case EPI_SWIGLU:
-            grouped_gemm_simt_kernel<EPI_SWIGLU><<<grid, 256, 0, s>>>(A, B, a, a_rows);
-            break;
+            return launch_pdl(grouped_gemm_simt_kernel<EPI_SWIGLU>, grid, dim3(256), 0, s, 1, A, B,
+                              a, a_rows);
         case EPI_SCATTER:
-            grouped_gemm_simt_kernel<EPI_SCATTER><<<grid, 256, 0, s>>>(A, B, a, a_rows);
-            break;
+            return launch_pdl(grouped_gemm_simt_kernel<EPI_SCATTER>, grid, dim3(256), 0, s, 1, A,
+                              B, a, a_rows);
         case EPI_COMBINE:
-            grouped_gemm_simt_kernel<EPI_COMBINE><<<grid, 256, 0, s>>>(A, B, a, a_rows);
-            break;
+            return launch_pdl(grouped_gemm_simt_kernel<EPI_COMBINE>, grid, dim3(256), 0, s, 1, A,
+                              B, a, a_rows);
         default:
             return cudaErrorInvalidValue;
     }
-    return cudaGetLastError();
 }
 
 }  // namespace moe

@@ -172,7 +172,7 @@ cudaEvent_t g_stage_events[MOE_N_STAGE_EVENTS];
 bool g_stage_events_on = false;
 
 void stage_mark(int i, cudaStream_t s) {
-    if (g_stage_events_on) cudaEventRecord(g_stage_events[i], s);
+    if (g_stage_events_on && g_stage_events[i] != nullptr) cudaEventRecord(g_stage_events[i], s);
 }
 
 }  // namespace
@@ -487,10 +487,7 @@ MOE_API int moe_set_stage_events(void* const* events, int n) {
         return MOE_OK;
     }
     if (n != MOE_N_STAGE_EVENTS) return MOE_ERR_INVALID_ARG;
-    for (int i = 0; i < n; ++i) {
-        if (events[i] == nullptr) return MOE_ERR_INVALID_ARG;
-        g_stage_events[i] = static_cast<cudaEvent_t>(events[i]);
-    }
+    for (int i = 0; i < n; ++i) g_stage_events[i] = static_cast<cudaEvent_t>(events[i]);
     g_stage_events_on = true;
     return MOE_OK;
 }

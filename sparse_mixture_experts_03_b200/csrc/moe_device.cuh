@@ -34,6 +34,17 @@ __device__ __forceinline__ void set_status(int* status, int code, int where, int
     }
 }
 
+// ---------------------------------------------------------------- launch order
+// Wait until the previous kernel of the stream has completed and its memory
+// writes are visible (no-op for a kernel launched without programmatic
+// dependent launch).
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+// This CTA's work that later kernels depend on is done: the next kernel may be
+// scheduled once every CTA of this grid has signalled or exited.
+__device__ __forceinline__ void pdl_trigger() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---------------------------------------------------------------- elements
 template <typename T> struct Elem;
 template <> struct Elem<float> {

@@ -7,7 +7,40 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <utility>
+
 namespace moe {
+
+// Every kernel of the forward is launched with programmatic dependent launch:
+// its CTAs may be scheduled while the previous kernel in the stream is
+// finishing (hiding the launch latency between the small stages), and each
+// kernel waits (griddepcontrol.wait, which returns once the previous grid has
+// completed and its writes are visible) before it reads or writes memory.
+// cluster_x > 1 adds a cluster dimension.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t s, int cluster_x, Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[2];
+    int n = 0;
+    attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[n].val.programmaticStreamSerializationAllowed = 1;
+    ++n;
+    if (cluster_x > 1) {
+        attr[n].id = cudaLaunchAttributeClusterDimension;
+        attr[n].val.clusterDim.x = (unsigned)cluster_x;
+        attr[n].val.clusterDim.y = 1;
+        attr[n].val.clusterDim.z = 1;
+        ++n;
+    }
+    cfg.attrs = attr;
+    cfg.numAttrs = (unsigned)n;
+    return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
 
 constexpr int kMaxE = 256;
 constexpr int kMaxGroups = 32;

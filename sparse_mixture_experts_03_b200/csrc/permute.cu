@@ -52,6 +52,7 @@ __global__ void __launch_bounds__(kPermBlockTokens) perm_count_kernel(
     __shared__ int wcnt[kWarps][kMaxE];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int t = blockIdx.x * kPermBlockTokens + tid;
+    pdl_wait();
     int my[kMaxK];
     load_slots(idx, t, T, k, E, my, status);
     for (int e = 0; e < E; ++e) {
@@ -65,6 +66,7 @@ __global__ void __launch_bounds__(kPermBlockTokens) perm_count_kernel(
         for (int w = 0; w < kWarps; ++w) s += wcnt[w][e];
         block_counts[(size_t)blockIdx.x * E + e] = s;
     }
+    pdl_trigger();
 }
 
 // One CTA: per expert, exclusive scan of the block histogram over blocks
@@ -82,6 +84,7 @@ __global__ void __launch_bounds__(1024) perm_scan_kernel(int32_t* __restrict__ b
     __shared__ int s_cnt[kMaxE];
     __shared__ int s_off[kMaxE + 1];
     const int tid = threadIdx.x;
+    pdl_wait();
     for (int e = tid; e < E; e += blockDim.x) s_cnt[e] = 0;
     for (int b0 = 0; b0 < nb; b0 += kScanChunkBlocks) {
         const int nbc = min(kScanChunkBlocks, nb - b0);
@@ -126,6 +129,7 @@ __global__ void __launch_bounds__(1024) perm_scan_kernel(int32_t* __restrict__ b
         int row = s_off[e] + s_cnt[e] + r;
         if (row < s_off[e + 1]) row_src[row] = -1;
     }
+    pdl_trigger();
 }
 
 // Stable rank of every (token, slot) inside its expert, and row_src of the
@@ -138,6 +142,7 @@ __global__ void __launch_bounds__(kPermBlockTokens) perm_rank_kernel(
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int t = blockIdx.x * kPermBlockTokens + tid;
     int my[kMaxK], rank[kMaxK];
+    pdl_wait();
     load_slots(idx, t, T, k, E, my, nullptr);
 #pragma unroll
     for (int j = 0; j < kMaxK; ++j) rank[j] = 0;
@@ -170,6 +175,7 @@ __global__ void __launch_bounds__(kPermBlockTokens) perm_rank_kernel(
                 set_status(status, MOE_ERR_DEVICE, SITE_PERMUTE, pos);
         }
     }
+    pdl_trigger();
 }
 
 // x_perm[r] = x[row_src[r] / k] for every real row r < offsets[E]; one warp
@@ -183,6 +189,7 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint4* __restric
     const int lane = threadIdx.x & 31;
     const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int nw = (gridDim.x * blockDim.x) >> 5;
+    pdl_wait();
     const int total = *total_rows;
     for (int r = gw; r < total; r += nw) {
         const int src = row_src[r];
@@ -203,6 +210,7 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint4* __restric
             }
         }
     }
+    pdl_trigger();
 }
 
 // y[t] = base[t] + slots[t*k + 0] + ... + slots[t*k + k-1] in fp32, in that
@@ -215,6 +223,7 @@ __global__ void __launch_bounds__(256) combine_slots_kernel(const TS* __restrict
                                                             int T, int d8, int k, void* y,
                                                             int out_f32) {
     const size_t n = (size_t)T * d8;
+    pdl_wait();
     for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n;
          i += (size_t)gridDim.x * blockDim.x) {
         const size_t t = i / d8, c = (i % d8) * 8;
@@ -264,6 +273,7 @@ __global__ void __launch_bounds__(256) combine_slots_kernel(const TS* __restrict
                            pack_bf16x2(a[4], a[5]), pack_bf16x2(a[6], a[7]));
         }
     }
+    pdl_trigger();
 }
 
 // bf16 slots, k fixed at compile time: one thread per (token, 8 columns), its
@@ -275,6 +285,7 @@ __global__ void __launch_bounds__(256) combine_slots_bf16_kernel(
     const uint4* __restrict__ slots, const float4* __restrict__ base, int T, int d8, void* y,
     int out_f32) {
     const size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x;
+    pdl_wait();
     if (i >= (size_t)T * d8) return;
     const size_t t = i / d8, c8 = i % d8;
     uint4 raw[K];
@@ -306,6 +317,7 @@ __global__ void __launch_bounds__(256) combine_slots_bf16_kernel(
         static_cast<uint4*>(y)[i] = make_uint4(pack_bf16x2(a[0], a[1]), pack_bf16x2(a[2], a[3]),
                                                pack_bf16x2(a[4], a[5]), pack_bf16x2(a[6], a[7]));
     }
+    pdl_trigger();
 }
 
 }  // namespace
@@ -314,11 +326,15 @@ cudaError_t launch_permute(const int32_t* idx, int T, int k, int E, int32_t* blo
                            int32_t* counts, int32_t* offsets, int32_t* row_src, int align,
                            int* status, cudaStream_t s) {
     const int nb = (T + kPermBlockTokens - 1) / kPermBlockTokens;
-    perm_count_kernel<<<nb, kPermBlockTokens, 0, s>>>(idx, T, k, E, block_counts, status);
-    perm_scan_kernel<<<1, 1024, 0, s>>>(block_counts, nb, E, align, counts, offsets, row_src);
-    perm_rank_kernel<<<nb, kPermBlockTokens, 0, s>>>(idx, T, k, E, block_counts, offsets, row_src,
-                                                     status);
-    return cudaGetLastError();
+    cudaError_t e = launch_pdl(perm_count_kernel, dim3(nb), dim3(kPermBlockTokens), 0, s, 1, idx,
+                               T, k, E, block_counts, status);
+    if (e != cudaSuccess) return e;
+    e = launch_pdl(perm_scan_kernel, dim3(1), dim3(1024), 0, s, 1, block_counts, nb, E, align,
+                   counts, offsets, row_src);
+    if (e != cudaSuccess) return e;
+    return launch_pdl(perm_rank_kernel, dim3(nb), dim3(kPermBlockTokens), 0, s, 1, idx, T, k, E,
+                      static_cast<const int32_t*>(block_counts),
+                      static_cast<const int32_t*>(offsets), row_src, status);
 }
 
 cudaError_t launch_expert_counts(const int32_t* idx, int T, int k, int E,
@@ -339,10 +355,9 @@ cudaError_t launch_gather_rows(const void* x, int d, int elem_bytes, int k,
     int blocks = num_sms * 8;
     const int need = (rows_cap + 7) / 8;
     if (blocks > need) blocks = need > 0 ? need : 1;
-    gather_rows_kernel<<<blocks, 256, 0, s>>>(static_cast<const uint4*>(x), vec, k,
-                                              offsets_total, row_src,
-                                              static_cast<uint4*>(x_perm));
-    return cudaGetLastError();
+    return launch_pdl(gather_rows_kernel, dim3(blocks), dim3(256), 0, s, 1,
+                      static_cast<const uint4*>(x), vec, k, offsets_total, row_src,
+                      static_cast<uint4*>(x_perm));
 }
 
 cudaError_t launch_combine_slots(const void* slots, int slots_bf16, const float* base, int T,
@@ -355,23 +370,21 @@ cudaError_t launch_combine_slots(const void* slots, int slots_bf16, const float*
         const uint4* sl = static_cast<const uint4*>(slots);
         const float4* b4 = reinterpret_cast<const float4*>(base);
         switch (k) {
-#define MOE_COMBINE_K(KK)                                                                   \
-    case KK:                                                                                \
-        combine_slots_bf16_kernel<KK><<<blocks16, 256, 0, s>>>(sl, b4, T, d8, y, out_f32); \
-        break;
+#define MOE_COMBINE_K(KK)                                                                 \
+    case KK:                                                                              \
+        return launch_pdl(combine_slots_bf16_kernel<KK>, dim3(blocks16), dim3(256), 0, s, 1, \
+                          sl, b4, T, d8, y, out_f32);
             MOE_COMBINE_K(1) MOE_COMBINE_K(2) MOE_COMBINE_K(3) MOE_COMBINE_K(4)
             MOE_COMBINE_K(5) MOE_COMBINE_K(6) MOE_COMBINE_K(7) MOE_COMBINE_K(8)
 #undef MOE_COMBINE_K
             default: return cudaErrorInvalidValue;
         }
-        return cudaGetLastError();
     }
     int blocks = (int)((n + 255) / 256);
     if (blocks > 148 * 8) blocks = 148 * 8;
     if (blocks < 1) blocks = 1;
-    combine_slots_kernel<float><<<blocks, 256, 0, s>>>(static_cast<const float*>(slots), base, T,
-                                                       d8, k, y, out_f32);
-    return cudaGetLastError();
+    return launch_pdl(combine_slots_kernel<float>, dim3(blocks), dim3(256), 0, s, 1,
+                      static_cast<const float*>(slots), base, T, d8, k, y, out_f32);
 }
 
 }  // namespace moe

@@ -142,6 +142,7 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const TIn* __restr
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int t0 = blockIdx.x * kRouteTokens;
 
+    pdl_wait();
     if (status != nullptr && blockIdx.x == 0 && tid < 16) status[tid] = 0;
 
     float acc[4][EJ];
@@ -198,6 +199,7 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const TIn* __restr
         warp_topk<EJ>(logit + tl * (E + 1), lane, E, k, G, TG, idx_out + (size_t)t * k,
                       w_out + (size_t)t * k);
     }
+    pdl_trigger();
 }
 
 // ---------------------------------------------------------------------------
@@ -252,6 +254,7 @@ __global__ void __launch_bounds__(256) route_mma_kernel(const __nv_bfloat16* __r
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int wm = warp & 1, wk = warp >> 1;
     const int t0 = blockIdx.x * kMmaTokens;
+    pdl_wait();
     if (status != nullptr && blockIdx.x == 0 && tid < 16) status[tid] = 0;
 
     // each thread copies fixed (row, 16-byte column) pieces of every chunk
@@ -403,6 +406,169 @@ __global__ void __launch_bounds__(256) route_mma_kernel(const __nv_bfloat16* __r
                                           idx_out + (size_t)t * k, w_out + (size_t)t * k);
         }
     }
+    pdl_trigger();
+}
+
+// ---------------------------------------------------------------------------
+// Cluster router for bf16 with d = 256 S (S = 2, 4 or 8 CTAs per cluster):
+// the S CTAs of a cluster share 32 tokens and split d, CTA r taking columns
+// [256 r, 256 r + 256).  Each CTA loads its x and W_router slices once
+// (48 KB at E = 64, d = 2048), forms its partial logits with mma.sync (k
+// quarters added in fixed order), and after a cluster barrier CTA r sums the
+// S partials of tokens [r 32/S, (r + 1) 32/S) over distributed shared memory
+// in rank order and selects their experts.  Every SM streams only a 1/S slice
+// of W_router, so small batches are not limited by one SM reading all of it.
+__device__ __forceinline__ uint32_t cluster_rank_u32() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ float ld_cluster_f32(const float* local, uint32_t rank) {
+    uint32_t a;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(a) : "r"(smem_u32(local)), "r"(rank));
+    float v;
+    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(a) : "memory");
+    return v;
+}
+__device__ __forceinline__ void cluster_barrier() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;"
+                 ::: "memory");
+}
+
+template <int NT, int S>
+__global__ void __launch_bounds__(256) route_split_kernel(const __nv_bfloat16* __restrict__ x,
+                                                          const __nv_bfloat16* __restrict__ Wr,
+                                                          int T, int d, int E, int k, int G,
+                                                          int TG, int32_t* __restrict__ idx_out,
+                                                          float* __restrict__ w_out,
+                                                          int* status) {
+    extern __shared__ __align__(16) uint8_t rsm[];
+    constexpr int kTokPerCta = kMmaTokens / S;
+    const int Ep = E + 1;
+    __nv_bfloat16* xs = reinterpret_cast<__nv_bfloat16*>(rsm);  // [32][kMmaLd]
+    __nv_bfloat16* wsm = xs + kMmaTokens * kMmaLd;              // [E][kMmaLd]
+    float* red = reinterpret_cast<float*>(rsm);                // after the MMAs: [4][32][E+1]
+    const size_t stage_bytes = (size_t)(kMmaTokens + E) * kMmaLd * sizeof(__nv_bfloat16);
+    const size_t red_bytes = (size_t)4 * kMmaTokens * Ep * sizeof(float);
+    float* part = reinterpret_cast<float*>(rsm + (stage_bytes > red_bytes ? stage_bytes : red_bytes));
+    float* lg = part + kMmaTokens * Ep;  // [kTokPerCta][E+1] summed logits
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int wm = warp & 1, wk = warp >> 1;
+    const uint32_t rank = cluster_rank_u32();
+    const int t0 = (blockIdx.x / S) * kMmaTokens;
+    const int c0 = (int)rank * kMmaKC;
+    pdl_wait();
+    if (status != nullptr && blockIdx.x == 0 && tid < 16) status[tid] = 0;
+
+#pragma unroll
+    for (int m = 0; m < kMmaTokens * (kMmaKC / 8) / 256; ++m) {
+        const int i = tid + 256 * m;
+        const int r = i >> 5, c = (i & 31) * 8;
+        const int t = t0 + r;
+        cp_async16(xs + r * kMmaLd + c, x + (size_t)(t < T ? t : 0) * d + c0 + c, t < T);
+    }
+    for (int i = tid; i < E * (kMmaKC / 8); i += 256) {
+        const int r = i >> 5, c = (i & 31) * 8;
+        cp_async16(wsm + r * kMmaLd + c, Wr + (size_t)r * d + c0 + c, true);
+    }
+    cp_async_commit();
+    cp_async_wait<0>();
+    __syncthreads();
+
+    float acc[NT][4];
+#pragma unroll
+    for (int n = 0; n < NT; ++n)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) acc[n][q] = 0.f;
+#pragma unroll
+    for (int kk = 0; kk < 64; kk += 16) {
+        const int kb = wk * 64 + kk;
+        uint32_t a[4];
+        ldmatrix_x4(a, xs + (wm * 16 + (lane & 15)) * kMmaLd + kb + 8 * (lane >> 4));
+#pragma unroll
+        for (int n = 0; n < NT; n += 2) {
+            uint32_t b[4];
+            ldmatrix_x4(b, wsm + (8 * n + (lane & 7) + 8 * (lane >> 4)) * kMmaLd + kb +
+                               8 * ((lane >> 3) & 1));
+            mma_bf16_16816(acc[n], a, b[0], b[1]);
+            mma_bf16_16816(acc[n + 1], a, b[2], b[3]);
+        }
+    }
+    __syncthreads();  // the stage buffers become the k-quarter partials
+#pragma unroll
+    for (int n = 0; n < NT; ++n) {
+        const int r0 = wm * 16 + (lane >> 2), col = 8 * n + 2 * (lane & 3);
+        float* base = red + (size_t)wk * kMmaTokens * Ep;
+        base[r0 * Ep + col] = acc[n][0];
+        base[r0 * Ep + col + 1] = acc[n][1];
+        base[(r0 + 8) * Ep + col] = acc[n][2];
+        base[(r0 + 8) * Ep + col + 1] = acc[n][3];
+    }
+    __syncthreads();
+    for (int i = tid; i < kMmaTokens * E; i += 256) {
+        const int r = i / E, e = i % E;
+        float v = red[r * Ep + e];
+        v += red[(size_t)kMmaTokens * Ep + r * Ep + e];
+        v += red[(size_t)2 * kMmaTokens * Ep + r * Ep + e];
+        v += red[(size_t)3 * kMmaTokens * Ep + r * Ep + e];
+        part[r * Ep + e] = v;
+    }
+    cluster_barrier();  // every CTA's partial logits are ready
+    for (int i = tid; i < kTokPerCta * E; i += 256) {
+        const int r = i / E, e = i % E;
+        const float* src = part + ((int)rank * kTokPerCta + r) * Ep + e;
+        float v = ld_cluster_f32(src, 0);
+#pragma unroll
+        for (int q = 1; q < S; ++q) v += ld_cluster_f32(src, (uint32_t)q);
+        lg[r * Ep + e] = (v != v) ? -INFINITY : v;
+    }
+    __syncthreads();
+    for (int tt = warp; tt < kTokPerCta; tt += 8) {
+        const int t = t0 + (int)rank * kTokPerCta + tt;
+        if (t < T)  // warp-uniform
+            warp_topk<(NT * 8 + 31) / 32>(lg + tt * Ep, lane, E, k, G, TG,
+                                          idx_out + (size_t)t * k, w_out + (size_t)t * k);
+    }
+    pdl_trigger();
+    cluster_barrier();  // no CTA leaves while another may still read its partials
+}
+
+size_t route_split_smem(int E, int S) {
+    const size_t stage = (size_t)(kMmaTokens + E) * kMmaLd * sizeof(__nv_bfloat16);
+    const size_t red = (size_t)4 * kMmaTokens * (E + 1) * sizeof(float);
+    return (stage > red ? stage : red) +
+           (size_t)(kMmaTokens + kMmaTokens / S) * (E + 1) * sizeof(float);
+}
+
+template <int S>
+cudaError_t launch_route_split(const void* x, const void* Wr, int T, int d, int E, int k, int G,
+                               int TG, int32_t* idx, float* w, int* status, cudaStream_t s) {
+    const size_t smem = route_split_smem(E, S);
+    const __nv_bfloat16* xp = static_cast<const __nv_bfloat16*>(x);
+    const __nv_bfloat16* wp = static_cast<const __nv_bfloat16*>(Wr);
+    const dim3 grid((unsigned)(((T + kMmaTokens - 1) / kMmaTokens) * S));
+#define MOE_ROUTE_SPLIT_CASE(NT)                                                              \
+    case NT: {                                                                                \
+        auto kern = route_split_kernel<NT, S>;                                                \
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, \
+                                             (int)smem);                                      \
+        if (e != cudaSuccess) return e;                                                       \
+        return launch_pdl(kern, grid, dim3(256), smem, s, S, xp, wp, T, d, E, k, G, TG, idx, w, \
+                          status);                                                            \
+    }
+    switch (E / 8) {
+        MOE_ROUTE_SPLIT_CASE(2)
+        MOE_ROUTE_SPLIT_CASE(4)
+        MOE_ROUTE_SPLIT_CASE(6)
+        MOE_ROUTE_SPLIT_CASE(8)
+        MOE_ROUTE_SPLIT_CASE(10)
+        MOE_ROUTE_SPLIT_CASE(12)
+        MOE_ROUTE_SPLIT_CASE(14)
+        MOE_ROUTE_SPLIT_CASE(16)
+        default:
+            return cudaErrorInvalidValue;
+    }
+#undef MOE_ROUTE_SPLIT_CASE
 }
 
 size_t route_mma_smem(int E) {
@@ -423,8 +589,8 @@ cudaError_t launch_route_mma(const void* x, const void* Wr, int T, int d, int E,
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, \
                                              (int)smem);                                      \
         if (e != cudaSuccess) return e;                                                       \
-        kern<<<grid, 256, smem, s>>>(xp, wp, T, d, E, k, G, TG, idx, w, status);              \
-        return cudaGetLastError();                                                            \
+        return launch_pdl(kern, grid, dim3(256), smem, s, 1, xp, wp, T, d, E, k, G, TG, idx, w, \
+                          status);                                                            \
     }
     switch (E / 8) {
         MOE_ROUTE_MMA_CASE(2)
@@ -457,8 +623,8 @@ cudaError_t launch_route(const void* x, const void* Wr, int T, int d, int E, int
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, \
                                              (int)smem);                                    \
         if (e != cudaSuccess) return e;                                                     \
-        kern<<<grid, kRouteThreads, smem, s>>>(xp, wp, T, d, E, k, G, TG, idx, w, status);  \
-        return cudaGetLastError();                                                          \
+        return launch_pdl(kern, grid, dim3(kRouteThreads), smem, s, 1, xp, wp, T, d, E, k, G, \
+                          TG, idx, w, status);                                              \
     }
     switch (ej) {
         MOE_ROUTE_CASE(1)
@@ -480,8 +646,19 @@ cudaError_t launch_route(const void* x, const void* Wr, int T, int d, int E, int
 cudaError_t launch_route_bf16(const void* x, const void* Wr, int T, int d, int E, int k, int G,
                               int TG, int32_t* idx, float* w, int* status, cudaStream_t s) {
     // tensor-core path for the shapes it tiles exactly; CUDA cores otherwise
-    if (E % 16 == 0 && E <= 128 && d % kMmaKC == 0)
+    if (E % 16 == 0 && E <= 128 && d % kMmaKC == 0) {
+        // small batches: d split over a cluster of S CTAs when d = 256 S (the
+        // whole-d kernel's few CTAs would each stream all of W_router); from
+        // about 2048 tokens on, the whole-d kernel fills the GPU and is faster
+        if (T > 1024) return launch_route_mma(x, Wr, T, d, E, k, G, TG, idx, w, status, s);
+        if (d == 8 * kMmaKC)
+            return launch_route_split<8>(x, Wr, T, d, E, k, G, TG, idx, w, status, s);
+        if (d == 4 * kMmaKC)
+            return launch_route_split<4>(x, Wr, T, d, E, k, G, TG, idx, w, status, s);
+        if (d == 2 * kMmaKC)
+            return launch_route_split<2>(x, Wr, T, d, E, k, G, TG, idx, w, status, s);
         return launch_route_mma(x, Wr, T, d, E, k, G, TG, idx, w, status, s);
+    }
     return launch_route<__nv_bfloat16>(x, Wr, T, d, E, k, G, TG, idx, w, status, s);
 }
 

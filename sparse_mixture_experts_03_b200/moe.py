@@ -205,7 +205,8 @@ def set_stage_events(events) -> None:
     if events is None:
         _check(lib().moe_set_stage_events(None, 0), "moe_set_stage_events")
         return
-    arr = (ctypes.c_void_p * len(events))(*[ctypes.c_void_p(e.cuda_event) for e in events])
+    arr = (ctypes.c_void_p * len(events))(
+        *[ctypes.c_void_p(e.cuda_event if e is not None else None) for e in events])
     _check(lib().moe_set_stage_events(arr, len(events)), "moe_set_stage_events")
 
 
