@@ -36,10 +36,11 @@ def lib() -> ctypes.CDLL:
         path = _build.build()
         L = ctypes.CDLL(path)
         vp, i32, dp = ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p
-        L.oracle_route.argtypes = [vp, vp, i32, i32, i32, i32, i32, i32, i32, dp, dp, dp, dp, dp, i32]
+        L.oracle_route.argtypes = [vp, vp, i32, i32, i32, i32, i32, i32, i32, i32, dp, dp, dp, dp,
+                                   dp, dp, i32]
         L.oracle_route.restype = i32
         L.oracle_forward.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, i32,
-                                     i32, dp, i32, dp, dp, dp, dp, i32]
+                                     i32, i32, dp, dp, i32, dp, dp, dp, dp, i32]
         L.oracle_forward.restype = i32
         L.oracle_max_threads.restype = i32
         L.oracle_check_args.argtypes = [i32] * 6
@@ -74,11 +75,25 @@ def _np_ptr(a: Optional[np.ndarray]):
     return ctypes.c_void_p(a.ctypes.data)
 
 
+SCORE_FUNCS = {"sigmoid": 0, "softmax": 1}
+
+
+def _bias(bias, E):
+    """Selection bias as a contiguous fp64 array (the exact fp32 values given to
+    the GPU), or None."""
+    if bias is None:
+        return None
+    b = np.ascontiguousarray(np.asarray(bias, dtype=np.float32).astype(np.float64))
+    assert b.shape == (E,)
+    return b
+
+
 class Routing:
-    """Oracle routing of T tokens: idx [T,k] int32 (descending score, ties to
-    the lower index), w [T,k] fp64, scores [T,E] fp64 (sigmoid gate scores),
-    gap_e / gap_g [T] fp64 (score gap at the k-th expert boundary inside the
-    kept groups, and at the topk_group-th group boundary)."""
+    """Oracle routing of T tokens: idx [T,k] int32 (descending key, ties to
+    the lower index), w [T,k] fp64, scores [T,E] fp64 (selection keys: the
+    gate score -- sigmoid, or the logit for softmax gating -- plus the
+    selection bias), gap_e / gap_g [T] fp64 (key gap at the k-th expert
+    boundary inside the kept groups, and at the topk_group-th group boundary)."""
 
     def __init__(self, idx, w, scores, gap_e, gap_g):
         self.idx, self.w, self.scores, self.gap_e, self.gap_g = idx, w, scores, gap_e, gap_g
@@ -88,8 +103,9 @@ class Routing:
 
 
 def route(x: torch.Tensor, W_router: torch.Tensor, k: int, n_group: int, topk_group: int,
-          with_scores: bool = True, nthreads: int = 0) -> Routing:
-    """Steps 1-5 (router, sigmoid, group limit, top-k, normalise) for every token."""
+          with_scores: bool = True, nthreads: int = 0, score_func: str = "sigmoid",
+          bias=None) -> Routing:
+    """Steps 1-5 (router, gate, group limit, top-k, weights) for every token."""
     T, d = x.shape
     E = W_router.shape[0]
     assert W_router.shape[1] == d and W_router.dtype == x.dtype
@@ -98,9 +114,10 @@ def route(x: torch.Tensor, W_router: torch.Tensor, k: int, n_group: int, topk_gr
     scores = np.zeros((T, E), np.float64) if with_scores else None
     ge = np.zeros(T, np.float64)
     gg = np.zeros(T, np.float64)
+    b = _bias(bias, E)
     rc = lib().oracle_route(_ptr(x), _ptr(W_router), _dt(x), T, d, E, k, n_group, topk_group,
-                            _np_ptr(idx), _np_ptr(w), _np_ptr(scores), _np_ptr(ge), _np_ptr(gg),
-                            nthreads)
+                            SCORE_FUNCS[score_func], _np_ptr(b), _np_ptr(idx), _np_ptr(w),
+                            _np_ptr(scores), _np_ptr(ge), _np_ptr(gg), nthreads)
     if rc != 0:
         raise ValueError("oracle_route: invalid arguments")
     return Routing(idx, w, scores, ge, gg)
@@ -109,7 +126,7 @@ def route(x: torch.Tensor, W_router: torch.Tensor, k: int, n_group: int, topk_gr
 def forward(x: torch.Tensor, W_router: torch.Tensor, W_gate_up: torch.Tensor,
             W_down: torch.Tensor, W_shared: Optional[torch.Tensor], k: int, n_group: int,
             topk_group: int, inter: int, n_shared: int, tokens=None, forced_idx=None,
-            nthreads: int = 0):
+            nthreads: int = 0, score_func: str = "sigmoid", bias=None):
     """Full layer forward (steps 1-7) for the listed tokens (default: all).
 
     Returns (y [n,d] fp64, idx [n,k] int32, w [n,k] fp64).  With forced_idx
@@ -134,10 +151,11 @@ def forward(x: torch.Tensor, W_router: torch.Tensor, W_gate_up: torch.Tensor,
     if forced_idx is not None:
         fi = np.ascontiguousarray(np.asarray(forced_idx, dtype=np.int32))
         assert fi.shape == (n, k)
+    b = _bias(bias, E)
     rc = lib().oracle_forward(_ptr(x), _ptr(W_router), _ptr(W_gate_up), _ptr(W_down),
                               _ptr(W_shared), dt, T, d, E, k, n_group, topk_group, inter,
-                              n_shared, _np_ptr(tokens), n, _np_ptr(fi), _np_ptr(y),
-                              _np_ptr(idx), _np_ptr(w), nthreads)
+                              n_shared, SCORE_FUNCS[score_func], _np_ptr(b), _np_ptr(tokens), n,
+                              _np_ptr(fi), _np_ptr(y), _np_ptr(idx), _np_ptr(w), nthreads)
     if rc != 0:
         raise ValueError("oracle_forward: invalid arguments")
     return y, idx, w

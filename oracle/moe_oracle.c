@@ -44,6 +44,17 @@
  *        [FusionLLM] "模型配置与规模"; always-on shared experts in [Arch]
  *        "Mixtral、Qwen3-MoE 与 DeepSeek-V3 架构对比")
  *
+ * Gating variants (the pages' other gates, selected by score_func and bias):
+ *   score_func 0  the FusionLLM gate above (sigmoid scores, weights s / sum s)
+ *   score_func 1  softmax over the chosen experts ([Arch] "MoE 数学：路由、容量
+ *                 与平衡详解" and the MoEBlock listing: top-k of the router
+ *                 logits, weights = softmax of those k logits)
+ *   bias b[E]     selection-only expert bias ([Arch], the aux-loss-free
+ *                 balancing of DeepSeek-V3 in "MoE 数学" and "Mixtral、Qwen3-MoE
+ *                 与 DeepSeek-V3 架构对比"): the group limit and the top-k
+ *                 compare gate score + b_e (gate score = s_e for score_func 0,
+ *                 l_e for 1); the weights use the unbiased gate scores.
+ *
  * Inputs are read as the exact values handed to the GPU: fp32, or bf16 bit
  * patterns widened to fp32 (a bf16 value is the top 16 bits of an fp32).
  * Nothing is rounded to bf16 inside the oracle; h stays fp64.
@@ -95,19 +106,41 @@ int oracle_check_args(int T, int d, int E, int k, int G, int TG) {
     return 0;
 }
 
+/* Routing weights of the experts idx[0..k) from the gate scores g[E]. */
+static void gate_weights(const double *g, const int32_t *idx, int k, int score_func,
+                         double *w) {
+    if (score_func == 0) {
+        double sum = 0.0;
+        for (int j = 0; j < k; ++j) sum += g[idx[j]];
+        for (int j = 0; j < k; ++j) w[j] = g[idx[j]] / sum;
+    } else {
+        double m = g[idx[0]];
+        for (int j = 1; j < k; ++j)
+            if (g[idx[j]] > m) m = g[idx[j]];
+        double sum = 0.0;
+        for (int j = 0; j < k; ++j) sum += exp(g[idx[j]] - m);
+        for (int j = 0; j < k; ++j) w[j] = exp(g[idx[j]] - m) / sum;
+    }
+}
+
 /*
- * Steps 1-5 for one token.  s: [E] scratch/output scores.  Writes idx[k],
- * w[k], and the two decision gaps used to flag near-ties:
- *   gap_e = s of the k-th chosen expert minus the best score not chosen among
+ * Steps 1-5 for one token.  g: [E] gate scores (out), s: [E] selection keys
+ * (out; gate score + bias).  Writes idx[k], w[k], and the two decision gaps
+ * used to flag near-ties:
+ *   gap_e = key of the k-th chosen expert minus the best key not chosen among
  *           the experts of the kept groups (+inf when there is none),
- *   gap_g = group score of the TG-th kept group minus the best score of a
+ *   gap_g = group key of the TG-th kept group minus the best key of a
  *           dropped group (+inf when every group is kept).
  */
 static void route_token(const double *xt, const void *Wr, int dt, int d, int E, int k,
-                        int G, int TG, double *s, int32_t *idx, double *w,
-                        double *gap_e, double *gap_g) {
+                        int G, int TG, int score_func, const double *bias, double *g,
+                        double *s, int32_t *idx, double *w, double *gap_e, double *gap_g) {
     int gsz = E / G;
-    for (int e = 0; e < E; ++e) s[e] = sigmoid(dot_row(Wr, dt, (size_t)e * d, xt, d));
+    for (int e = 0; e < E; ++e) {
+        double l = dot_row(Wr, dt, (size_t)e * d, xt, d);
+        g[e] = score_func == 0 ? sigmoid(l) : l;
+        s[e] = g[e] + (bias ? bias[e] : 0.0);
+    }
 
     /* group scores and the kept groups */
     double *gs = (double *)malloc(sizeof(double) * G);
@@ -133,7 +166,6 @@ static void route_token(const double *xt, const void *Wr, int dt, int d, int E, 
 
     /* top-k inside the kept groups */
     char *taken = (char *)calloc(E, 1);
-    double sum = 0.0;
     for (int j = 0; j < k; ++j) {
         int best = -1;
         for (int e = 0; e < E; ++e) {
@@ -142,7 +174,6 @@ static void route_token(const double *xt, const void *Wr, int dt, int d, int E, 
         }
         taken[best] = 1;
         idx[j] = best;
-        sum += s[best];
     }
     double best_left = -INFINITY;
     int n_left = 0;
@@ -152,7 +183,7 @@ static void route_token(const double *xt, const void *Wr, int dt, int d, int E, 
         if (s[e] > best_left) best_left = s[e];
     }
     *gap_e = n_left ? s[idx[k - 1]] - best_left : INFINITY;
-    for (int j = 0; j < k; ++j) w[j] = s[idx[j]] / sum;
+    gate_weights(g, idx, k, score_func, w);
     free(gs);
     free(gkeep);
     free(taken);
@@ -163,20 +194,22 @@ static void load_row(const void *x, int dt, size_t off, int d, double *out) {
 }
 
 /*
- * Routing only (steps 1-5) for all T tokens.
- * idx [T,k] int32, w [T,k] fp64, scores [T,E] fp64 (nullable),
- * gap_e / gap_g [T] fp64 (nullable).  Returns 0, or -1 on invalid arguments.
+ * Routing only (steps 1-5) for all T tokens.  score_func / bias: the gating
+ * variant (bias [E] nullable).  idx [T,k] int32, w [T,k] fp64, scores [T,E]
+ * fp64 selection keys (nullable), gap_e / gap_g [T] fp64 (nullable).
+ * Returns 0, or -1 on invalid arguments.
  */
 int oracle_route(const void *x, const void *Wr, int dt, int T, int d, int E, int k, int G,
-                 int TG, int32_t *idx, double *w, double *scores, double *gap_e,
-                 double *gap_g, int nthreads) {
-    if (oracle_check_args(T, d, E, k, G, TG)) return -1;
+                 int TG, int score_func, const double *bias, int32_t *idx, double *w,
+                 double *scores, double *gap_e, double *gap_g, int nthreads) {
+    if (oracle_check_args(T, d, E, k, G, TG) || score_func < 0 || score_func > 1) return -1;
 #ifdef _OPENMP
     if (nthreads > 0) omp_set_num_threads(nthreads);
 #pragma omp parallel
 #endif
     {
         double *xt = (double *)malloc(sizeof(double) * d);
+        double *g = (double *)malloc(sizeof(double) * E);
         double *s = (double *)malloc(sizeof(double) * E);
 #ifdef _OPENMP
 #pragma omp for schedule(dynamic, 16)
@@ -184,13 +217,14 @@ int oracle_route(const void *x, const void *Wr, int dt, int T, int d, int E, int
         for (int t = 0; t < T; ++t) {
             double ge, gg;
             load_row(x, dt, (size_t)t * d, d, xt);
-            route_token(xt, Wr, dt, d, E, k, G, TG, s, idx + (size_t)t * k, w + (size_t)t * k,
-                        &ge, &gg);
+            route_token(xt, Wr, dt, d, E, k, G, TG, score_func, bias, g, s, idx + (size_t)t * k,
+                        w + (size_t)t * k, &ge, &gg);
             if (scores) memcpy(scores + (size_t)t * E, s, sizeof(double) * E);
             if (gap_e) gap_e[t] = ge;
             if (gap_g) gap_g[t] = gg;
         }
         free(xt);
+        free(g);
         free(s);
     }
     return 0;
@@ -224,9 +258,11 @@ static void swiglu_hidden(const void *Wgu, int dt, size_t base, size_t g_row0, s
  */
 int oracle_forward(const void *x, const void *Wr, const void *Wgu, const void *Wd,
                    const void *Wsh, int dt, int T, int d, int E, int k, int G, int TG, int I,
-                   int S, const int32_t *tokens, int n_tok, const int32_t *forced_idx,
-                   double *y, int32_t *idx_out, double *w_out, int nthreads) {
+                   int S, int score_func, const double *bias, const int32_t *tokens, int n_tok,
+                   const int32_t *forced_idx, double *y, int32_t *idx_out, double *w_out,
+                   int nthreads) {
     if (oracle_check_args(T, d, E, k, G, TG) || I <= 0 || S < 0) return -1;
+    if (score_func < 0 || score_func > 1) return -1;
     if (S > 0 && !Wsh) return -1;
     for (int n = 0; n < n_tok; ++n)
         if (tokens[n] < 0 || tokens[n] >= T) return -1;
@@ -240,6 +276,7 @@ int oracle_forward(const void *x, const void *Wr, const void *Wgu, const void *W
 #endif
     {
         double *xt = (double *)malloc(sizeof(double) * d);
+        double *g = (double *)malloc(sizeof(double) * E);
         double *s = (double *)malloc(sizeof(double) * E);
         double *h = (double *)malloc(sizeof(double) * (I > SI ? I : SI) + 8);
         int32_t *idx = (int32_t *)malloc(sizeof(int32_t) * k);
@@ -251,14 +288,10 @@ int oracle_forward(const void *x, const void *Wr, const void *Wgu, const void *W
             int t = tokens[n];
             double ge, gg, *yt = y + (size_t)n * d;
             load_row(x, dt, (size_t)t * d, d, xt);
-            route_token(xt, Wr, dt, d, E, k, G, TG, s, idx, w, &ge, &gg);
+            route_token(xt, Wr, dt, d, E, k, G, TG, score_func, bias, g, s, idx, w, &ge, &gg);
             if (forced_idx) {
-                double sum = 0.0;
-                for (int j = 0; j < k; ++j) {
-                    idx[j] = forced_idx[(size_t)n * k + j];
-                    sum += s[idx[j]];
-                }
-                for (int j = 0; j < k; ++j) w[j] = s[idx[j]] / sum;
+                for (int j = 0; j < k; ++j) idx[j] = forced_idx[(size_t)n * k + j];
+                gate_weights(g, idx, k, score_func, w);
             }
             for (int c = 0; c < d; ++c) yt[c] = 0.0;
             for (int j = 0; j < k; ++j) {
@@ -278,6 +311,7 @@ int oracle_forward(const void *x, const void *Wr, const void *Wgu, const void *W
             if (w_out) memcpy(w_out + (size_t)n * k, w, sizeof(double) * k);
         }
         free(xt);
+        free(g);
         free(s);
         free(h);
         free(idx);

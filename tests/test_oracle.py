@@ -300,3 +300,97 @@ def test_empty_token_batch():
     assert r.idx.shape == (0, 2)
     y, idx, w = oracle.forward(x, Wr, Wgu, Wd, None, 2, 1, 1, 4, 0, tokens=[])
     assert y.shape == (0, 8)
+
+
+# ---------------------------------------------------------------- gating variants
+# softmax over the chosen experts (Mixtral-style gate) and the selection-only
+# expert bias (aux-loss-free balancing), both from "大模型工程（一）：Transformer
+# 到 MoE", section "MoE 数学：路由、容量与平衡详解"
+
+
+@pytest.mark.parametrize("E,G,TG,k", [(8, 1, 1, 2), (8, 2, 1, 3), (8, 4, 2, 3), (6, 3, 2, 2)])
+def test_softmax_gate_brute_force(E, G, TG, k):
+    """Softmax gating: the chosen set is the exhaustive optimum of the logits,
+    the weights are torch.softmax over the chosen logits."""
+    T, d = 30, 16
+    x, Wr, *_ = rand_case(T, d, E, 8, 0, seed=7 + E * 10 + k, router_scale=3.0)
+    r = oracle.route(x, Wr, k, G, TG, score_func="softmax")
+    logits = x.double() @ Wr.double().T
+    np.testing.assert_allclose(r.scores, logits.numpy(), rtol=0, atol=1e-15)
+    for t in range(T):
+        want = brute_force_select(list(logits[t].numpy()), G, TG, k)
+        assert list(r.idx[t]) == want
+        w = torch.softmax(logits[t, want], dim=0).numpy()
+        np.testing.assert_allclose(r.w[t], w, rtol=1e-13)
+
+
+def test_softmax_gate_all_experts_is_full_softmax():
+    """k = E, one group: the weights are the softmax of every logit."""
+    T, d, E = 12, 8, 6
+    x, Wr, *_ = rand_case(T, d, E, 4, 0, seed=3)
+    r = oracle.route(x, Wr, E, 1, 1, score_func="softmax")
+    full = torch.softmax(x.double() @ Wr.double().T, dim=1).numpy()
+    for t in range(T):
+        np.testing.assert_allclose(r.w[t], full[t, r.idx[t]], rtol=1e-13)
+    np.testing.assert_allclose(r.w.sum(axis=1), 1.0, rtol=0, atol=1e-14)
+
+
+@pytest.mark.parametrize("score_func", ["sigmoid", "softmax"])
+def test_selection_bias_brute_force(score_func):
+    """Selection bias: groups and experts are chosen on gate score + bias
+    (exhaustive optimum), the weights use the unbiased gate scores."""
+    E, G, TG, k, T, d = 8, 4, 2, 3, 30, 16
+    x, Wr, *_ = rand_case(T, d, E, 8, 0, seed=11, router_scale=3.0)
+    bias = np.linspace(-0.3, 0.4, E).astype(np.float32)
+    r = oracle.route(x, Wr, k, G, TG, score_func=score_func, bias=bias)
+    logits = x.double() @ Wr.double().T
+    gate = torch.sigmoid(logits) if score_func == "sigmoid" else logits
+    keys = gate.numpy() + bias.astype(np.float64)
+    np.testing.assert_allclose(r.scores, keys, rtol=0, atol=1e-15)
+    for t in range(T):
+        want = brute_force_select(list(keys[t]), G, TG, k)
+        assert list(r.idx[t]) == want
+        g = gate[t, want]
+        w = (g / g.sum()) if score_func == "sigmoid" else torch.softmax(g, dim=0)
+        np.testing.assert_allclose(r.w[t], w.numpy(), rtol=1e-13)
+
+
+def test_zero_bias_is_no_bias_and_large_bias_forces_an_expert():
+    E, G, TG, k, T, d = 8, 2, 1, 2, 20, 16
+    x, Wr, *_ = rand_case(T, d, E, 8, 0, seed=5)
+    r0 = oracle.route(x, Wr, k, G, TG)
+    rz = oracle.route(x, Wr, k, G, TG, bias=np.zeros(E, np.float32))
+    assert (r0.idx == rz.idx).all() and (r0.w == rz.w).all()
+    bias = np.zeros(E, np.float32)
+    bias[5] = 10.0  # sigmoid scores are < 1: expert 5 (group 1) always wins
+    rb = oracle.route(x, Wr, k, G, TG, bias=bias)
+    assert (rb.idx[:, 0] == 5).all() and (rb.idx // (E // G) == 1).all()
+    s = torch.sigmoid(x.double() @ Wr.double().T).numpy()
+    for t in range(T):
+        np.testing.assert_allclose(rb.w[t], s[t, rb.idx[t]] / s[t, rb.idx[t]].sum(), rtol=1e-14)
+
+
+def test_forward_gating_variants_match_library_composition():
+    """Whole layer with softmax gating and a bias: the torch fp64 composition
+    of the stated steps on the oracle's own routing."""
+    T, d, E, k, G, TG, I, S = 10, 16, 8, 2, 2, 1, 8, 1
+    x, Wr, Wgu, Wd, Wsh = rand_case(T, d, E, I, S, seed=21, router_scale=2.0)
+    bias = np.linspace(0.2, -0.2, E).astype(np.float32)
+    for sf in ("sigmoid", "softmax"):
+        y, idx, w = oracle.forward(x, Wr, Wgu, Wd, Wsh, k, G, TG, I, S, score_func=sf, bias=bias)
+        r = oracle.route(x, Wr, k, G, TG, score_func=sf, bias=bias)
+        assert (idx == r.idx).all()
+        np.testing.assert_allclose(w, r.w, rtol=1e-15)
+        x64 = x.double()
+        ref = np.zeros((T, d))
+        for t in range(T):
+            for j in range(k):
+                e = idx[t, j]
+                ref[t] += w[t, j] * swiglu_lib(x64[t:t + 1], Wgu[e, :I].double(),
+                                               Wgu[e, I:].double(), Wd[e].double()).numpy()[0]
+        sh = Wsh.double()
+        Wg_s = sh[:S * I * d].reshape(S * I, d)
+        Wu_s = sh[S * I * d:2 * S * I * d].reshape(S * I, d)
+        Wd_s = sh[2 * S * I * d:].reshape(d, S * I)
+        ref += swiglu_lib(x64, Wg_s, Wu_s, Wd_s).numpy()
+        np.testing.assert_allclose(y, ref, rtol=1e-12, atol=1e-12)
