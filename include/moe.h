@@ -51,6 +51,14 @@
 #endif
 #define MOE_API MOE_EXTERN __attribute__((visibility("default")))
 
+/* Gates (routing weights).  MOE_GATE_SIGMOID is the FusionLLM gate
+ * ("FusionLLM：融合 MLA、GDN 与 MoE 的高效混合架构大模型训练框架", section
+ * "混合专家（MoE）"): sigmoid scores, weights = scores of the chosen experts
+ * normalised to sum 1.  MOE_GATE_SOFTMAX_TOPK is the Mixtral-style gate of
+ * "大模型工程（一）：Transformer 到 MoE", section "MoE 数学：路由、容量与平衡详解":
+ * the k largest logits, weights = softmax of those k logits. */
+typedef enum { MOE_GATE_SIGMOID = 0, MOE_GATE_SOFTMAX_TOPK = 1 } moe_gate;
+
 typedef enum {
     MOE_OK = 0,
     MOE_ERR_INVALID_ARG = -1, /* a size, pointer or alignment check failed          */
@@ -148,6 +156,37 @@ MOE_API int moe_forward(const void *x, const void *W_router, const void *W_gate_
                         int n_group, int topk_group, int inter, int n_shared, int in_dt,
                         int out_dt, void *y, int32_t *topk_idx_out, float *topk_w_out,
                         void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * moe_route_ex / moe_forward_ex -- moe_route / moe_forward with the gating
+ * variants of "大模型工程（一）：Transformer 到 MoE", section "MoE 数学：路由、容量
+ * 与平衡详解" (moe_route and moe_forward are these with MOE_GATE_SIGMOID, no
+ * bias and no load output):
+ *   gate         MOE_GATE_SIGMOID or MOE_GATE_SOFTMAX_TOPK (see moe_gate)
+ *   expert_bias  device f32[E] or NULL: selection-only bias (the aux-loss-free
+ *                load balancing of DeepSeek-V3 described there): the group
+ *                limit and the top-k compare gate score + expert_bias[e]
+ *                (gate score = sigmoid(logit) for MOE_GATE_SIGMOID, the logit
+ *                for MOE_GATE_SOFTMAX_TOPK); the weights use the unbiased
+ *                scores.  The caller updates the bias between steps from the
+ *                expert loads.
+ *   expert_load  (moe_forward_ex) device int32[E] or NULL, out: tokens routed
+ *                to each expert in this call (sum = T * k), the load figure
+ *                that such a bias update reads.
+ * Other arguments, layouts, ownership and errors as moe_route / moe_forward;
+ * an unknown gate or a host pointer for expert_bias / expert_load returns
+ * MOE_ERR_INVALID_ARG before any launch.
+ */
+MOE_API int moe_route_ex(const void *x, const void *W_router, int T, int d, int E, int k,
+                         int n_group, int topk_group, int in_dt, int gate,
+                         const float *expert_bias, int32_t *topk_idx, float *topk_w,
+                         void *stream);
+MOE_API int moe_forward_ex(const void *x, const void *W_router, const void *W_gate_up,
+                           const void *W_down, const void *W_shared, int T, int d, int E, int k,
+                           int n_group, int topk_group, int inter, int n_shared, int in_dt,
+                           int out_dt, int gate, const float *expert_bias, void *y,
+                           int32_t *topk_idx_out, float *topk_w_out, int32_t *expert_load,
+                           void *workspace, size_t workspace_bytes, void *stream);
 
 /*
  * moe_get_device_status -- synchronise `stream`, then copy the status word

@@ -210,14 +210,32 @@ MOE_API int moe_workspace_layout(int T, int d, int E, int k, int inter, int n_sh
     return MOE_OK;
 }
 
+// gate and optional selection bias / expert-load output: shared checks
+int check_gating(int gate, const float* bias, const int32_t* load) {
+    if (gate != MOE_GATE_SIGMOID && gate != MOE_GATE_SOFTMAX_TOPK) return MOE_ERR_INVALID_ARG;
+    if (bias != nullptr && (!is_device_ptr(bias) || !aligned(bias, 4))) return MOE_ERR_INVALID_ARG;
+    if (load != nullptr && (!is_device_ptr(load) || !aligned(load, 4))) return MOE_ERR_INVALID_ARG;
+    return MOE_OK;
+}
+
 MOE_API int moe_route(const void* x, const void* W_router, int T, int d, int E, int k,
                       int n_group, int topk_group, int in_dt, int32_t* topk_idx, float* topk_w,
                       void* stream) {
+    return moe_route_ex(x, W_router, T, d, E, k, n_group, topk_group, in_dt, MOE_GATE_SIGMOID,
+                        nullptr, topk_idx, topk_w, stream);
+}
+
+MOE_API int moe_route_ex(const void* x, const void* W_router, int T, int d, int E, int k,
+                         int n_group, int topk_group, int in_dt, int gate,
+                         const float* expert_bias, int32_t* topk_idx, float* topk_w,
+                         void* stream) {
     int st = check_sizes(T, d, E, k, 128, 0, in_dt);
     if (st != MOE_OK) return st;
     st = check_routing(E, k, n_group, topk_group);
     if (st != MOE_OK) return st;
     if (T == 0) return MOE_OK;
+    st = check_gating(gate, expert_bias, nullptr);
+    if (st != MOE_OK) return st;
     if (!is_device_ptr(x) || !is_device_ptr(W_router) || !is_device_ptr(topk_idx) ||
         !is_device_ptr(topk_w))
         return MOE_ERR_INVALID_ARG;
@@ -226,10 +244,10 @@ MOE_API int moe_route(const void* x, const void* W_router, int T, int d, int E, 
         return MOE_ERR_INVALID_ARG;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (in_dt == MOE_BF16)
-        return ret(launch_route_bf16(x, W_router, T, d, E, k, n_group, topk_group, topk_idx,
-                                     topk_w, nullptr, s));
-    return ret(launch_route_f32(x, W_router, T, d, E, k, n_group, topk_group, topk_idx, topk_w,
-                                nullptr, s));
+        return ret(launch_route_bf16(x, W_router, T, d, E, k, n_group, topk_group, gate,
+                                     expert_bias, topk_idx, topk_w, nullptr, s));
+    return ret(launch_route_f32(x, W_router, T, d, E, k, n_group, topk_group, gate, expert_bias,
+                                topk_idx, topk_w, nullptr, s));
 }
 
 MOE_API int moe_forward(const void* x, const void* W_router, const void* W_gate_up,
@@ -237,6 +255,18 @@ MOE_API int moe_forward(const void* x, const void* W_router, const void* W_gate_
                         int n_group, int topk_group, int inter, int n_shared, int in_dt,
                         int out_dt, void* y, int32_t* topk_idx_out, float* topk_w_out,
                         void* workspace, size_t workspace_bytes, void* stream) {
+    return moe_forward_ex(x, W_router, W_gate_up, W_down, W_shared, T, d, E, k, n_group,
+                          topk_group, inter, n_shared, in_dt, out_dt, MOE_GATE_SIGMOID, nullptr,
+                          y, topk_idx_out, topk_w_out, nullptr, workspace, workspace_bytes,
+                          stream);
+}
+
+MOE_API int moe_forward_ex(const void* x, const void* W_router, const void* W_gate_up,
+                           const void* W_down, const void* W_shared, int T, int d, int E, int k,
+                           int n_group, int topk_group, int inter, int n_shared, int in_dt,
+                           int out_dt, int gate, const float* expert_bias, void* y,
+                           int32_t* topk_idx_out, float* topk_w_out, int32_t* expert_load,
+                           void* workspace, size_t workspace_bytes, void* stream) {
     int st = check_sizes(T, d, E, k, inter, n_shared, in_dt);
     if (st != MOE_OK) return st;
     st = check_routing(E, k, n_group, topk_group);
@@ -247,7 +277,14 @@ MOE_API int moe_forward(const void* x, const void* W_router, const void* W_gate_
     Layout L;
     make_layout(T, d, E, k, inter, n_shared, in_dt, L);
     if (workspace == nullptr || workspace_bytes < L.off[MOE_WS_TOTAL]) return MOE_ERR_WORKSPACE;
-    if (T == 0) return MOE_OK;
+    st = check_gating(gate, expert_bias, expert_load);
+    if (st != MOE_OK) return st;
+    if (T == 0) {
+        if (expert_load != nullptr)
+            return ret(cudaMemsetAsync(expert_load, 0, sizeof(int32_t) * E,
+                                       static_cast<cudaStream_t>(stream)));
+        return MOE_OK;
+    }
     const void* dev_ptrs[] = {x, W_router, W_gate_up, W_down, y, workspace};
     for (const void* p : dev_ptrs)
         if (!is_device_ptr(p) || !aligned(p, 16)) return MOE_ERR_INVALID_ARG;
@@ -276,17 +313,17 @@ MOE_API int moe_forward(const void* x, const void* W_router, const void* W_gate_
 
     stage_mark(0, s);
     // 1. routing (also resets the status word)
-    cudaError_t e = bf16 ? launch_route_bf16(x, W_router, T, d, E, k, n_group, topk_group, idx, w,
-                                             status, s)
-                         : launch_route_f32(x, W_router, T, d, E, k, n_group, topk_group, idx, w,
-                                            status, s);
+    cudaError_t e = bf16 ? launch_route_bf16(x, W_router, T, d, E, k, n_group, topk_group, gate,
+                                             expert_bias, idx, w, status, s)
+                         : launch_route_f32(x, W_router, T, d, E, k, n_group, topk_group, gate,
+                                            expert_bias, idx, w, status, s);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
     stage_mark(1, s);
     // 2. permutation: histogram, scan, stable ranks, row gather
     // the CTA-pair GEMMs (bf16) take unpadded expert segments; the CUDA-core
     // kernels (fp32) take segments padded to their 128-row tiles
     e = launch_permute(idx, T, k, E, block_counts, counts, offsets, row_src,
-                       bf16 ? 1 : kRowAlign, status, s);
+                       bf16 ? 1 : kRowAlign, expert_load, status, s);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
     e = launch_gather_rows(x, d, bf16 ? 2 : 4, k, offsets + E, row_src, L.rows_cap, x_perm,
                            num_sms(), s);

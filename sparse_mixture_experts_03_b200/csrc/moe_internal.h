@@ -88,16 +88,20 @@ struct GemmArgs {
 };
 
 // ---- launchers (return a cudaError_t from the launch)
+// gate: MOE_GATE_SIGMOID or MOE_GATE_SOFTMAX_TOPK; bias: device f32[E] selection-only
+// expert bias, or nullptr.
 cudaError_t launch_route_bf16(const void* x, const void* Wr, int T, int d, int E, int k, int G,
-                              int TG, int32_t* idx, float* w, int* status, cudaStream_t s);
+                              int TG, int gate, const float* bias, int32_t* idx, float* w,
+                              int* status, cudaStream_t s);
 cudaError_t launch_route_f32(const void* x, const void* Wr, int T, int d, int E, int k, int G,
-                             int TG, int32_t* idx, float* w, int* status, cudaStream_t s);
+                             int TG, int gate, const float* bias, int32_t* idx, float* w,
+                             int* status, cudaStream_t s);
 
 // Segments of the permuted layout are padded to a multiple of `align` rows
 // (1: unpadded) with row_src = -1 on padding rows.
 cudaError_t launch_permute(const int32_t* idx, int T, int k, int E, int32_t* block_counts,
                            int32_t* counts, int32_t* offsets, int32_t* row_src, int align,
-                           int* status, cudaStream_t s);
+                           int32_t* load_out, int* status, cudaStream_t s);
 cudaError_t launch_gather_rows(const void* x, int d, int elem_bytes, int k,
                                const int32_t* offsets_total, const int32_t* row_src,
                                int rows_cap, void* x_perm, int num_sms, cudaStream_t s);

@@ -79,7 +79,8 @@ __global__ void __launch_bounds__(1024) perm_scan_kernel(int32_t* __restrict__ b
                                                          int nb, int E, int align,
                                                          int32_t* __restrict__ counts,
                                                          int32_t* __restrict__ offsets,
-                                                         int32_t* __restrict__ row_src) {
+                                                         int32_t* __restrict__ row_src,
+                                                         int32_t* __restrict__ load_out) {
     __shared__ int s_bc[kScanChunkBlocks * kMaxE];
     __shared__ int s_cnt[kMaxE];
     __shared__ int s_off[kMaxE + 1];
@@ -122,7 +123,10 @@ __global__ void __launch_bounds__(1024) perm_scan_kernel(int32_t* __restrict__ b
         if (tid == 0) s_off[E] = carry;
     }
     __syncthreads();
-    for (int e = tid; e < E; e += blockDim.x) counts[e] = s_cnt[e];
+    for (int e = tid; e < E; e += blockDim.x) {
+        counts[e] = s_cnt[e];
+        if (load_out != nullptr) load_out[e] = s_cnt[e];
+    }
     for (int e = tid; e <= E; e += blockDim.x) offsets[e] = s_off[e];
     for (int i = tid; i < E * align; i += blockDim.x) {
         int e = i / align, r = i % align;
@@ -187,7 +191,8 @@ constexpr int kSmallWarps = kSmallTokens / 32;
 
 __global__ void __launch_bounds__(kSmallTokens) perm_small_kernel(
     const int32_t* __restrict__ idx, int T, int k, int E, int align, int32_t* __restrict__ counts,
-    int32_t* __restrict__ offsets, int32_t* __restrict__ row_src, int* status) {
+    int32_t* __restrict__ offsets, int32_t* __restrict__ row_src, int32_t* __restrict__ load_out,
+    int* status) {
     __shared__ int wcnt[kSmallWarps][kMaxE];  // per-warp counts, then per-warp bases
     __shared__ int s_cnt[kMaxE];
     __shared__ int s_off[kMaxE + 1];
@@ -238,6 +243,7 @@ __global__ void __launch_bounds__(kSmallTokens) perm_small_kernel(
             run += c;
         }
         counts[e] = s_cnt[e];
+        if (load_out != nullptr) load_out[e] = s_cnt[e];
     }
     for (int e = tid; e <= E; e += nthr) offsets[e] = s_off[e];
     for (int i = tid; i < E * align; i += nthr) {
@@ -398,16 +404,16 @@ __global__ void __launch_bounds__(256) combine_slots_bf16_kernel(
 
 cudaError_t launch_permute(const int32_t* idx, int T, int k, int E, int32_t* block_counts,
                            int32_t* counts, int32_t* offsets, int32_t* row_src, int align,
-                           int* status, cudaStream_t s) {
+                           int32_t* load_out, int* status, cudaStream_t s) {
     if (T <= kSmallTokens)
         return launch_pdl(perm_small_kernel, dim3(1), dim3((unsigned)((T + 31) / 32 * 32)), 0, s,
-                          1, idx, T, k, E, align, counts, offsets, row_src, status);
+                          1, idx, T, k, E, align, counts, offsets, row_src, load_out, status);
     const int nb = (T + kPermBlockTokens - 1) / kPermBlockTokens;
     cudaError_t e = launch_pdl(perm_count_kernel, dim3(nb), dim3(kPermBlockTokens), 0, s, 1, idx,
                                T, k, E, block_counts, status);
     if (e != cudaSuccess) return e;
     e = launch_pdl(perm_scan_kernel, dim3(1), dim3(1024), 0, s, 1, block_counts, nb, E, align,
-                   counts, offsets, row_src);
+                   counts, offsets, row_src, load_out);
     if (e != cudaSuccess) return e;
     return launch_pdl(perm_rank_kernel, dim3(nb), dim3(kPermBlockTokens), 0, s, 1, idx, T, k, E,
                       static_cast<const int32_t*>(block_counts),
@@ -421,7 +427,7 @@ cudaError_t launch_expert_counts(const int32_t* idx, int T, int k, int E,
     if (nb > 0)
         perm_count_kernel<<<nb, kPermBlockTokens, 0, s>>>(idx, T, k, E, block_counts, nullptr);
     // align 1: no padding rows, so the scan writes no row_src entry
-    perm_scan_kernel<<<1, 1024, 0, s>>>(block_counts, nb, E, 1, counts, offsets, nullptr);
+    perm_scan_kernel<<<1, 1024, 0, s>>>(block_counts, nb, E, 1, counts, offsets, nullptr, nullptr);
     return cudaGetLastError();
 }
 

@@ -10,6 +10,12 @@
 // Selection compares fp32 logits: sigmoid is monotone, so the kept groups and
 // the chosen experts are the ones a comparison of sigmoid scores would pick,
 // without the ties that rounding sigmoid(l) to fp32 near 0 or 1 would create.
+//
+// Gating variants of "大模型工程（一）：Transformer 到 MoE", section "MoE 数学：路由、
+// 容量与平衡详解": MOE_GATE_SOFTMAX_TOPK (select on the logits, weights =
+// softmax of the k chosen logits) and a selection-only expert bias b[E]
+// (aux-loss-free balancing: select on gate score + b, weigh with the unbiased
+// scores; gate score = sigmoid(l) for the sigmoid gate, l for softmax).
 #include <float.h>
 #include <limits.h>
 
@@ -23,6 +29,41 @@ namespace {
 constexpr int kRouteTokens = 32;   // tokens per CTA
 constexpr int kRouteKChunk = 32;   // reduction chunk staged in shared memory
 constexpr int kRouteThreads = 256;
+
+// Selection key of expert e from its fp32 logit l.
+__device__ __forceinline__ float sel_key(float l, int e, int gate, const float* bias) {
+    if (bias == nullptr) return l;  // monotone in the gate score for both gates
+    const float g = gate == MOE_GATE_SIGMOID ? 1.f / (1.f + expf(-l)) : l;
+    return g + bias[e];
+}
+
+// Weights of the k chosen experts from their logits (one thread).
+__device__ __forceinline__ void gate_weights(const float (&l)[kMaxK], int k, int gate,
+                                             float (&w)[kMaxK]) {
+    float sum = 0.f;
+    if (gate == MOE_GATE_SIGMOID) {
+#pragma unroll
+        for (int r = 0; r < kMaxK; ++r) {
+            if (r >= k) break;
+            w[r] = 1.f / (1.f + expf(-l[r]));
+            sum += w[r];
+        }
+    } else {
+        float m = l[0];
+#pragma unroll
+        for (int r = 1; r < kMaxK; ++r)
+            if (r < k) m = fmaxf(m, l[r]);
+#pragma unroll
+        for (int r = 0; r < kMaxK; ++r) {
+            if (r >= k) break;
+            w[r] = expf(l[r] - m);
+            sum += w[r];
+        }
+    }
+#pragma unroll
+    for (int r = 0; r < kMaxK; ++r)
+        if (r < k) w[r] /= sum;
+}
 
 // (v, i) beats (bv, bi): larger value, ties to the lower index; bi == INT_MAX
 // marks "nothing yet".
@@ -60,13 +101,15 @@ __device__ __forceinline__ void seg8_argmax(float& v, int& i) {
 // index) and the normalised sigmoid weights.
 template <int EJ>
 __device__ __forceinline__ void warp_topk(const float* L, int lane, int E, int k, int G, int TG,
+                                          int gate, const float* __restrict__ bias,
                                           int32_t* __restrict__ idx_out,
                                           float* __restrict__ w_out) {
     const int gsz = E / G;
-    // group scores: max logit of each group (lane g < G owns group g)
+    // group scores: max key of each group (lane g < G owns group g)
     float gval = -INFINITY;
     if (lane < G)
-        for (int e = lane * gsz; e < (lane + 1) * gsz; ++e) gval = fmaxf(gval, L[e]);
+        for (int e = lane * gsz; e < (lane + 1) * gsz; ++e)
+            gval = fmaxf(gval, sel_key(L[e], e, gate, bias));
     uint32_t kept = 0;
     for (int r = 0; r < TG; ++r) {
         float v = -INFINITY;
@@ -85,7 +128,7 @@ __device__ __forceinline__ void warp_topk(const float* L, int lane, int E, int k
     for (int j = 0; j < EJ; ++j) {
         int e = lane + 32 * j;
         cand[j] = e < E && ((kept >> (e / gsz)) & 1u);
-        cv[j] = cand[j] ? L[e] : -INFINITY;
+        cv[j] = cand[j] ? sel_key(L[e], e, gate, bias) : -INFINITY;
     }
     int sel_e[kMaxK];
     float sel_l[kMaxK];
@@ -107,21 +150,18 @@ __device__ __forceinline__ void warp_topk(const float* L, int lane, int E, int k
         for (int j = 0; j < EJ; ++j)
             if (lane + 32 * j == bi) cand[j] = false;
         sel_e[r] = bi;
-        sel_l[r] = bv;
     }
     if (lane == 0) {
-        float s[kMaxK], sum = 0.f;
 #pragma unroll
-        for (int r = 0; r < kMaxK; ++r) {
-            if (r >= k) break;
-            s[r] = 1.f / (1.f + expf(-sel_l[r]));
-            sum += s[r];
-        }
+        for (int r = 0; r < kMaxK; ++r)
+            if (r < k) sel_l[r] = L[sel_e[r]];
+        float wv[kMaxK];
+        gate_weights(sel_l, k, gate, wv);
 #pragma unroll
         for (int r = 0; r < kMaxK; ++r) {
             if (r >= k) break;
             idx_out[r] = sel_e[r];
-            w_out[r] = s[r] / sum;
+            w_out[r] = wv[r];
         }
     }
 }
@@ -131,6 +171,8 @@ template <typename TIn, int EJ>
 __global__ void __launch_bounds__(kRouteThreads) route_kernel(const TIn* __restrict__ x,
                                                               const TIn* __restrict__ Wr, int T,
                                                               int d, int E, int k, int G, int TG,
+                                                              int gate,
+                                                              const float* __restrict__ bias,
                                                               int32_t* __restrict__ idx_out,
                                                               float* __restrict__ w_out,
                                                               int* status) {
@@ -196,7 +238,7 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const TIn* __restr
         const int tl = warp * 4 + tt;
         const int t = t0 + tl;
         if (t >= T) break;  // warp-uniform
-        warp_topk<EJ>(logit + tl * (E + 1), lane, E, k, G, TG, idx_out + (size_t)t * k,
+        warp_topk<EJ>(logit + tl * (E + 1), lane, E, k, G, TG, gate, bias, idx_out + (size_t)t * k,
                       w_out + (size_t)t * k);
     }
     pdl_trigger();
@@ -244,7 +286,9 @@ template <int NT>  // NT = E / 8 n-tiles of 8 experts (E = 8 NT, NT even)
 __global__ void __launch_bounds__(256) route_mma_kernel(const __nv_bfloat16* __restrict__ x,
                                                         const __nv_bfloat16* __restrict__ Wr,
                                                         int T, int d, int E, int k, int G,
-                                                        int TG, int32_t* __restrict__ idx_out,
+                                                        int TG, int gate,
+                                                        const float* __restrict__ bias,
+                                                        int32_t* __restrict__ idx_out,
                                                         float* __restrict__ w_out,
                                                         int* status) {
     extern __shared__ __align__(16) uint8_t rsm[];
@@ -345,7 +389,7 @@ __global__ void __launch_bounds__(256) route_mma_kernel(const __nv_bfloat16* __r
         const float* L = logit + tl * Ep;
         float v[NT];
 #pragma unroll
-        for (int i = 0; i < NT; ++i) v[i] = L[sub * NT + i];
+        for (int i = 0; i < NT; ++i) v[i] = sel_key(L[sub * NT + i], sub * NT + i, gate, bias);
         const int lanes_per_group = 8 / G;
         const int gid = sub / lanes_per_group;
         float gmax = v[0];
@@ -380,21 +424,18 @@ __global__ void __launch_bounds__(256) route_mma_kernel(const __nv_bfloat16* __r
             seg8_argmax(bv, bi);
             if (bi / NT == sub) taken |= 1u << (bi - sub * NT);
             sel_e[r] = bi;
-            sel_l[r] = bv;
         }
         if (sub == 0 && t < T) {
-            float sc[kMaxK], sum = 0.f;
 #pragma unroll
-            for (int r = 0; r < kMaxK; ++r) {
-                if (r >= k) break;
-                sc[r] = 1.f / (1.f + expf(-sel_l[r]));
-                sum += sc[r];
-            }
+            for (int r = 0; r < kMaxK; ++r)
+                if (r < k) sel_l[r] = L[sel_e[r]];
+            float wv[kMaxK];
+            gate_weights(sel_l, k, gate, wv);
 #pragma unroll
             for (int r = 0; r < kMaxK; ++r) {
                 if (r >= k) break;
                 idx_out[(size_t)t * k + r] = sel_e[r];
-                w_out[(size_t)t * k + r] = sc[r] / sum;
+                w_out[(size_t)t * k + r] = wv[r];
             }
         }
     } else {
@@ -402,7 +443,7 @@ __global__ void __launch_bounds__(256) route_mma_kernel(const __nv_bfloat16* __r
             const int tl = warp * 4 + tt;
             const int t = t0 + tl;
             if (t >= T) break;  // warp-uniform
-            warp_topk<(NT * 8 + 31) / 32>(logit + tl * Ep, lane, E, k, G, TG,
+            warp_topk<(NT * 8 + 31) / 32>(logit + tl * Ep, lane, E, k, G, TG, gate, bias,
                                           idx_out + (size_t)t * k, w_out + (size_t)t * k);
         }
     }
@@ -439,7 +480,9 @@ template <int NT, int S>
 __global__ void __launch_bounds__(256) route_split_kernel(const __nv_bfloat16* __restrict__ x,
                                                           const __nv_bfloat16* __restrict__ Wr,
                                                           int T, int d, int E, int k, int G,
-                                                          int TG, int32_t* __restrict__ idx_out,
+                                                          int TG, int gate,
+                                                          const float* __restrict__ bias,
+                                                          int32_t* __restrict__ idx_out,
                                                           float* __restrict__ w_out,
                                                           int* status) {
     extern __shared__ __align__(16) uint8_t rsm[];
@@ -526,7 +569,7 @@ __global__ void __launch_bounds__(256) route_split_kernel(const __nv_bfloat16* _
     for (int tt = warp; tt < kTokPerCta; tt += 8) {
         const int t = t0 + (int)rank * kTokPerCta + tt;
         if (t < T)  // warp-uniform
-            warp_topk<(NT * 8 + 31) / 32>(lg + tt * Ep, lane, E, k, G, TG,
+            warp_topk<(NT * 8 + 31) / 32>(lg + tt * Ep, lane, E, k, G, TG, gate, bias,
                                           idx_out + (size_t)t * k, w_out + (size_t)t * k);
     }
     pdl_trigger();
@@ -542,7 +585,8 @@ size_t route_split_smem(int E, int S) {
 
 template <int S>
 cudaError_t launch_route_split(const void* x, const void* Wr, int T, int d, int E, int k, int G,
-                               int TG, int32_t* idx, float* w, int* status, cudaStream_t s) {
+                               int TG, int gate, const float* bias, int32_t* idx, float* w,
+                               int* status, cudaStream_t s) {
     const size_t smem = route_split_smem(E, S);
     const __nv_bfloat16* xp = static_cast<const __nv_bfloat16*>(x);
     const __nv_bfloat16* wp = static_cast<const __nv_bfloat16*>(Wr);
@@ -553,8 +597,8 @@ cudaError_t launch_route_split(const void* x, const void* Wr, int T, int d, int 
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, \
                                              (int)smem);                                      \
         if (e != cudaSuccess) return e;                                                       \
-        return launch_pdl(kern, grid, dim3(256), smem, s, S, xp, wp, T, d, E, k, G, TG, idx, w, \
-                          status);                                                            \
+        return launch_pdl(kern, grid, dim3(256), smem, s, S, xp, wp, T, d, E, k, G, TG, gate, \
+                          bias, idx, w, status);                                              \
     }
     switch (E / 8) {
         MOE_ROUTE_SPLIT_CASE(2)
@@ -578,7 +622,8 @@ size_t route_mma_smem(int E) {
 }
 
 cudaError_t launch_route_mma(const void* x, const void* Wr, int T, int d, int E, int k, int G,
-                             int TG, int32_t* idx, float* w, int* status, cudaStream_t s) {
+                             int TG, int gate, const float* bias, int32_t* idx, float* w,
+                               int* status, cudaStream_t s) {
     const size_t smem = route_mma_smem(E);
     const dim3 grid((T + kMmaTokens - 1) / kMmaTokens);
     const __nv_bfloat16* xp = static_cast<const __nv_bfloat16*>(x);
@@ -589,8 +634,8 @@ cudaError_t launch_route_mma(const void* x, const void* Wr, int T, int d, int E,
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, \
                                              (int)smem);                                      \
         if (e != cudaSuccess) return e;                                                       \
-        return launch_pdl(kern, grid, dim3(256), smem, s, 1, xp, wp, T, d, E, k, G, TG, idx, w, \
-                          status);                                                            \
+        return launch_pdl(kern, grid, dim3(256), smem, s, 1, xp, wp, T, d, E, k, G, TG, gate, \
+                          bias, idx, w, status);                                              \
     }
     switch (E / 8) {
         MOE_ROUTE_MMA_CASE(2)
@@ -609,7 +654,8 @@ cudaError_t launch_route_mma(const void* x, const void* Wr, int T, int d, int E,
 
 template <typename TIn>
 cudaError_t launch_route(const void* x, const void* Wr, int T, int d, int E, int k, int G,
-                         int TG, int32_t* idx, float* w, int* status, cudaStream_t s) {
+                         int TG, int gate, const float* bias, int32_t* idx, float* w,
+                               int* status, cudaStream_t s) {
     const int ej = (E + 31) / 32;
     const size_t p1 = (size_t)(kRouteTokens + E) * (kRouteKChunk + 1);
     const size_t p2 = (size_t)kRouteTokens * (E + 1);
@@ -624,7 +670,7 @@ cudaError_t launch_route(const void* x, const void* Wr, int T, int d, int E, int
                                              (int)smem);                                    \
         if (e != cudaSuccess) return e;                                                     \
         return launch_pdl(kern, grid, dim3(kRouteThreads), smem, s, 1, xp, wp, T, d, E, k, G, \
-                          TG, idx, w, status);                                              \
+                          TG, gate, bias, idx, w, status);                                              \
     }
     switch (ej) {
         MOE_ROUTE_CASE(1)
@@ -644,27 +690,30 @@ cudaError_t launch_route(const void* x, const void* Wr, int T, int d, int E, int
 }  // namespace
 
 cudaError_t launch_route_bf16(const void* x, const void* Wr, int T, int d, int E, int k, int G,
-                              int TG, int32_t* idx, float* w, int* status, cudaStream_t s) {
+                              int TG, int gate, const float* bias, int32_t* idx, float* w,
+                               int* status, cudaStream_t s) {
     // tensor-core path for the shapes it tiles exactly; CUDA cores otherwise
     if (E % 16 == 0 && E <= 128 && d % kMmaKC == 0) {
         // small batches: d split over a cluster of S CTAs when d = 256 S (the
         // whole-d kernel's few CTAs would each stream all of W_router); from
         // about 2048 tokens on, the whole-d kernel fills the GPU and is faster
-        if (T > 1024) return launch_route_mma(x, Wr, T, d, E, k, G, TG, idx, w, status, s);
+        if (T > 1024)
+            return launch_route_mma(x, Wr, T, d, E, k, G, TG, gate, bias, idx, w, status, s);
         if (d == 8 * kMmaKC)
-            return launch_route_split<8>(x, Wr, T, d, E, k, G, TG, idx, w, status, s);
+            return launch_route_split<8>(x, Wr, T, d, E, k, G, TG, gate, bias, idx, w, status, s);
         if (d == 4 * kMmaKC)
-            return launch_route_split<4>(x, Wr, T, d, E, k, G, TG, idx, w, status, s);
+            return launch_route_split<4>(x, Wr, T, d, E, k, G, TG, gate, bias, idx, w, status, s);
         if (d == 2 * kMmaKC)
-            return launch_route_split<2>(x, Wr, T, d, E, k, G, TG, idx, w, status, s);
-        return launch_route_mma(x, Wr, T, d, E, k, G, TG, idx, w, status, s);
+            return launch_route_split<2>(x, Wr, T, d, E, k, G, TG, gate, bias, idx, w, status, s);
+        return launch_route_mma(x, Wr, T, d, E, k, G, TG, gate, bias, idx, w, status, s);
     }
-    return launch_route<__nv_bfloat16>(x, Wr, T, d, E, k, G, TG, idx, w, status, s);
+    return launch_route<__nv_bfloat16>(x, Wr, T, d, E, k, G, TG, gate, bias, idx, w, status, s);
 }
 
 cudaError_t launch_route_f32(const void* x, const void* Wr, int T, int d, int E, int k, int G,
-                             int TG, int32_t* idx, float* w, int* status, cudaStream_t s) {
-    return launch_route<float>(x, Wr, T, d, E, k, G, TG, idx, w, status, s);
+                             int TG, int gate, const float* bias, int32_t* idx, float* w,
+                               int* status, cudaStream_t s) {
+    return launch_route<float>(x, Wr, T, d, E, k, G, TG, gate, bias, idx, w, status, s);
 }
 
 }  // namespace moe

@@ -35,7 +35,8 @@ ROW_ALIGN = 128
 SYMBOLS = ["moe_workspace_bytes", "moe_workspace_layout", "moe_route", "moe_forward",
            "moe_get_device_status", "moe_clear_device_status", "moe_selftest_timeout",
            "moe_set_stage_events", "moe_status_string", "moe_version",
-           "moe_expert_counts_noalloc"]
+           "moe_expert_counts_noalloc", "moe_route_ex", "moe_forward_ex"]
+GATES = {"sigmoid": 0, "softmax": 1}  # MOE_GATE_SIGMOID, MOE_GATE_SOFTMAX_TOPK
 N_STAGE_EVENTS = 6
 STAGES = ["route", "permute", "gate_up", "down", "combine"]
 
@@ -78,6 +79,10 @@ def lib() -> ctypes.CDLL:
         L.moe_version.restype = i
         L.moe_expert_counts_noalloc.argtypes = [vp, i, i, i, vp, vp, vp]
         L.moe_expert_counts_noalloc.restype = i
+        L.moe_route_ex.argtypes = [vp, vp] + [i] * 8 + [vp, vp, vp, vp]
+        L.moe_route_ex.restype = i
+        L.moe_forward_ex.argtypes = [vp] * 5 + [i] * 11 + [vp, vp, vp, vp, vp, vp, sz, vp]
+        L.moe_forward_ex.restype = i
         _lib = L
     return _lib
 
@@ -137,16 +142,19 @@ def alloc_workspace(T, d, E, k, inter, n_shared, dtype, device="cuda") -> torch.
 
 def route(x: torch.Tensor, W_router: torch.Tensor, k: int, n_group: int, topk_group: int,
           topk_idx: Optional[torch.Tensor] = None, topk_w: Optional[torch.Tensor] = None,
-          stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
-    """moe_route: (topk_idx int32 [T,k], topk_w fp32 [T,k])."""
+          stream=None, gate: str = "sigmoid",
+          expert_bias: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """moe_route_ex: (topk_idx int32 [T,k], topk_w fp32 [T,k]); gate "sigmoid"
+    or "softmax", expert_bias a device float32 [E] selection-only bias."""
     T, d = x.shape
     E = W_router.shape[0]
     if topk_idx is None:
         topk_idx = torch.empty(T, k, dtype=torch.int32, device=x.device)
     if topk_w is None:
         topk_w = torch.empty(T, k, dtype=torch.float32, device=x.device)
-    _check(lib().moe_route(_ptr(x), _ptr(W_router), T, d, E, k, n_group, topk_group, _dt(x),
-                           _ptr(topk_idx), _ptr(topk_w), _stream(stream)), "moe_route")
+    _check(lib().moe_route_ex(_ptr(x), _ptr(W_router), T, d, E, k, n_group, topk_group, _dt(x),
+                              GATES[gate], _ptr(expert_bias), _ptr(topk_idx), _ptr(topk_w),
+                              _stream(stream)), "moe_route_ex")
     return topk_idx, topk_w
 
 
@@ -164,19 +172,24 @@ def forward(x: torch.Tensor, W_router: torch.Tensor, W_gate_up: torch.Tensor,
             topk_group: int, inter: int, n_shared: int, out_dtype: torch.dtype = torch.float32,
             y: Optional[torch.Tensor] = None, topk_idx: Optional[torch.Tensor] = None,
             topk_w: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
-            stream=None) -> torch.Tensor:
-    """moe_forward: y [T, d] in out_dtype (float32 or bfloat16)."""
+            stream=None, gate: str = "sigmoid", expert_bias: Optional[torch.Tensor] = None,
+            expert_load: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """moe_forward_ex: y [T, d] in out_dtype (float32 or bfloat16).  gate
+    "sigmoid" (the FusionLLM gate) or "softmax" (over the chosen k);
+    expert_bias: device float32 [E] selection-only bias; expert_load: device
+    int32 [E] filled with the tokens routed to each expert."""
     T, d = x.shape
     E = W_router.shape[0]
     if y is None:
         y = torch.empty(T, d, dtype=out_dtype, device=x.device)
     if workspace is None:
         workspace = alloc_workspace(T, d, E, k, inter, n_shared, x.dtype, x.device)
-    st = lib().moe_forward(_ptr(x), _ptr(W_router), _ptr(W_gate_up), _ptr(W_down),
-                           _ptr(W_shared), T, d, E, k, n_group, topk_group, inter, n_shared,
-                           _dt(x), _dt(y), _ptr(y), _ptr(topk_idx), _ptr(topk_w),
-                           _ptr(workspace), workspace.numel(), _stream(stream))
-    _check(st, "moe_forward")
+    st = lib().moe_forward_ex(_ptr(x), _ptr(W_router), _ptr(W_gate_up), _ptr(W_down),
+                              _ptr(W_shared), T, d, E, k, n_group, topk_group, inter, n_shared,
+                              _dt(x), _dt(y), GATES[gate], _ptr(expert_bias), _ptr(y),
+                              _ptr(topk_idx), _ptr(topk_w), _ptr(expert_load),
+                              _ptr(workspace), workspace.numel(), _stream(stream))
+    _check(st, "moe_forward_ex")
     return y
 
 

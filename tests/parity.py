@@ -83,7 +83,8 @@ def check_output(y: np.ndarray, y_ref: np.ndarray, dtype: str):
     return max_abs, rel
 
 
-def oracle_outputs(inp, w, tokens, gpu_idx_rows, ref_routing, nthreads=0):
+def oracle_outputs(inp, w, tokens, gpu_idx_rows, ref_routing, nthreads=0, score_func="sigmoid",
+                   bias=None):
     """Oracle y for `tokens`; near-tie tokens whose GPU set differs are
     evaluated on the GPU's set (forced), the rest on the oracle's own."""
     tokens = np.asarray(tokens, dtype=np.int32)
@@ -92,12 +93,14 @@ def oracle_outputs(inp, w, tokens, gpu_idx_rows, ref_routing, nthreads=0):
     if same.any():
         y_ref[same], _, _ = oracle.forward(inp.x, inp.W_router, inp.W_gate_up, inp.W_down,
                                            inp.W_shared, w.k, w.n_group, w.topk_group, w.inter,
-                                           w.n_shared, tokens=tokens[same], nthreads=nthreads)
+                                           w.n_shared, tokens=tokens[same], nthreads=nthreads,
+                                           score_func=score_func, bias=bias)
     if (~same).any():
         y_ref[~same], _, _ = oracle.forward(inp.x, inp.W_router, inp.W_gate_up, inp.W_down,
                                             inp.W_shared, w.k, w.n_group, w.topk_group,
                                             w.inter, w.n_shared, tokens=tokens[~same],
-                                            forced_idx=gpu_idx_rows[~same], nthreads=nthreads)
+                                            forced_idx=gpu_idx_rows[~same], nthreads=nthreads,
+                                            score_func=score_func, bias=bias)
     return y_ref
 
 
