@@ -317,55 +317,65 @@ __device__ __forceinline__ void pair_epilogue(uint8_t* wb, uint32_t taddr, const
         tmem_ld_wait();
         const bool tok_ok = c0 + lane < t.n_real;  // after the transpose, lane = token
         if constexpr (EPI == EPI_SWIGLU) {
-            // The CTA's weight rows are [16 gate, 16 up] per warp quarter: lane i < 16
-            // holds gate feature f = 16 wq + i, lane i + 16 the matching up row.  Lane
-            // i computes h for tokens 0..15 of feature f, lane i + 16 for tokens 16..31,
-            // each receiving the other half of SwiGLU by a register shuffle.
-            const bool is_gate = lane < 16;
-            __nv_bfloat16 h[16];
+            // The CTA's weight rows are [16 gate, 16 up] per warp quarter: lane
+            // i < 16 holds gate feature 16 wq + i, lane i + 16 the matching up
+            // row.  fp32 transpose through the staging buffer, then lane = token:
+            // h_f = silu(g_f) * u_f for its 16 features, one 32-byte store.
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                const float send = __uint_as_float(is_gate ? v[16 + i] : v[i]);
-                const float recv = __shfl_xor_sync(0xffffffffu, send, 16);
-                const float g = is_gate ? __uint_as_float(v[i]) : recv;
-                const float u = is_gate ? recv : __uint_as_float(v[16 + i]);
-                h[i] = __float2bfloat16_rn(silu_mul(g, u));
-            }
-            const int f = lane & 15, tbase = is_gate ? 0 : 16;
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                // token row tbase + i: 16 features x 2 B = 32 B in chunks 0..1
-                __nv_bfloat16* row = reinterpret_cast<__nv_bfloat16*>(
-                    stage_chunk(wb, tbase + i, f >> 3));
-                row[f & 7] = h[i];
+            for (int i = 0; i < 32; ++i) {
+                float* row = reinterpret_cast<float*>(stage_chunk(wb, i, lane >> 2));
+                row[lane & 3] = __uint_as_float(v[i]);
             }
             __syncwarp();
             if (tok_ok) {
+                float f[32];
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    const float4 c4 = *reinterpret_cast<const float4*>(stage_chunk(wb, lane, q));
+                    f[4 * q] = c4.x;
+                    f[4 * q + 1] = c4.y;
+                    f[4 * q + 2] = c4.z;
+                    f[4 * q + 3] = c4.w;
+                }
+                uint32_t packed[8];
+#pragma unroll
+                for (int p = 0; p < 8; ++p)
+                    packed[p] = pack_bf16x2(silu_mul(f[2 * p], f[16 + 2 * p]),
+                                            silu_mul(f[2 * p + 1], f[16 + 2 * p + 1]));
                 uint4* d = reinterpret_cast<uint4*>(
                     static_cast<__nv_bfloat16*>(a.out) + (size_t)(t.b_row + c0 + lane) * a.out_ld +
                     t.ft * a.out_col_step + cta * 64 + wq * 16);
-                d[0] = *reinterpret_cast<const uint4*>(stage_chunk(wb, lane, 0));
-                d[1] = *reinterpret_cast<const uint4*>(stage_chunk(wb, lane, 1));
+                d[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+                d[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
             }
             __syncwarp();
         } else if constexpr (EPI == EPI_SCATTER) {
+            // fp32 transpose through the staging buffer (token row i: 32 features x
+            // 4 B), then lane = token: its 32 features times its own gate weight,
+            // rounded to bf16, one 64-byte store into the token's slot row
             const int src = srcs[cc];
             const float wv = wts[cc];
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
-                const float wi = __shfl_sync(0xffffffffu, wv, i);
-                // token row i: 32 features x 2 B = 64 B in chunks 0..3
-                __nv_bfloat16* row = reinterpret_cast<__nv_bfloat16*>(stage_chunk(wb, i, lane >> 3));
-                row[lane & 7] = __float2bfloat16_rn(wi * __uint_as_float(v[i]));
+                float* row = reinterpret_cast<float*>(stage_chunk(wb, i, lane >> 2));
+                row[lane & 3] = __uint_as_float(v[i]);
             }
             __syncwarp();
             if (src >= 0) {
+                uint32_t packed[16];
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    const float4 f = *reinterpret_cast<const float4*>(stage_chunk(wb, lane, q));
+                    packed[2 * q] = pack_bf16x2(wv * f.x, wv * f.y);
+                    packed[2 * q + 1] = pack_bf16x2(wv * f.z, wv * f.w);
+                }
                 uint4* d = reinterpret_cast<uint4*>(
                     static_cast<__nv_bfloat16*>(a.out) + (size_t)src * a.out_ld +
                     t.ft * a.out_col_step + cta * 128 + wq * 32);
 #pragma unroll
                 for (int q = 0; q < 4; ++q)
-                    d[q] = *reinterpret_cast<const uint4*>(stage_chunk(wb, lane, q));
+                    d[q] = make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2],
+                                      packed[4 * q + 3]);
             }
             __syncwarp();
         } else {  // EPI_STORE_F32: out[b_row + token][col] = acc, fp32
