@@ -171,29 +171,48 @@ def profiled_traffic(w):
         return None
 
 
-def run_config(w, world: int) -> dict:
+def bias_ramp(w, gate: str) -> np.ndarray:
+    """The selection bias used with --expert-bias: a fixed, shuffled ramp on
+    the scale of the gate scores (sigmoid scores in (0, 1); logits of order 1)."""
+    span = 0.1 if gate == "sigmoid" else 0.5
+    return np.random.default_rng(0).permutation(np.linspace(-span, span, w.E)).astype(np.float32)
+
+
+def oracle_gating(args, w) -> dict:
+    """The oracle's gating keyword arguments for the bench options."""
+    return {"score_func": getattr(args, "gate", "sigmoid"),
+            "bias": bias_ramp(w, args.gate) if getattr(args, "expert_bias", False) else None}
+
+
+def run_config(w, world: int, args=None) -> dict:
     """The `config` object of the JSON line (both arms)."""
-    return {"workload": f"{w.name}: {w.describe()}", "global_batch": world * w.T,
+    gating = ""
+    if args is not None and (getattr(args, "gate", "sigmoid") != "sigmoid" or
+                             getattr(args, "expert_bias", False)):
+        gating = f" gate={args.gate}" + (" expert_bias=on" if args.expert_bias else "")
+    return {"workload": f"{w.name}: {w.describe()}{gating}", "global_batch": world * w.T,
             "tokens_per_gpu": w.T, "parallelism": f"token-parallel x{world} (replicas)",
             "l2": "flushed between timed steps (512 MB write); weights 1.28 GB > L2",
             "out_dtype": "f32"}
 
 
-def cpu_baseline(w, inp, budget_s: float = 15.0):
+def cpu_baseline(w, inp, args, budget_s: float = 15.0):
     """Time the CPU oracle (as it stands) on a bounded sample of the workload's tokens."""
     import oracle
     nthreads = os.cpu_count() or 1
     probe = np.arange(min(w.T, max(8, nthreads)), dtype=np.int32)
     t0 = time.perf_counter()
     oracle.forward(inp.x, inp.W_router, inp.W_gate_up, inp.W_down, inp.W_shared, w.k,
-                   w.n_group, w.topk_group, w.inter, w.n_shared, tokens=probe, nthreads=nthreads)
+                   w.n_group, w.topk_group, w.inter, w.n_shared, tokens=probe, nthreads=nthreads,
+                   **oracle_gating(args, w))
     per_tok = (time.perf_counter() - t0) / len(probe)
     n = int(min(w.T, max(len(probe), budget_s / max(per_tok, 1e-9))))
     n = max(nthreads, n // nthreads * nthreads) if n >= nthreads else n
     toks = np.linspace(0, w.T - 1, n).astype(np.int32)
     t0 = time.perf_counter()
     oracle.forward(inp.x, inp.W_router, inp.W_gate_up, inp.W_down, inp.W_shared, w.k,
-                   w.n_group, w.topk_group, w.inter, w.n_shared, tokens=toks, nthreads=nthreads)
+                   w.n_group, w.topk_group, w.inter, w.n_shared, tokens=toks, nthreads=nthreads,
+                   **oracle_gating(args, w))
     dt = time.perf_counter() - t0
     return {"value": n / dt, "unit": "tokens/s", "cores": nthreads, "kind": "oracle",
             "sample": f"{n} of {w.T} tokens of the {w.name} workload (full layer per token, "
@@ -213,7 +232,8 @@ def run_reference(args, w):
     probe = np.arange(min(w.T, max(4, nthreads)), dtype=np.int32)
     t0 = time.perf_counter()
     oracle.forward(inp.x, inp.W_router, inp.W_gate_up, inp.W_down, inp.W_shared, w.k,
-                   w.n_group, w.topk_group, w.inter, w.n_shared, tokens=probe, nthreads=nthreads)
+                   w.n_group, w.topk_group, w.inter, w.n_shared, tokens=probe, nthreads=nthreads,
+                   **oracle_gating(args, w))
     per_tok = (time.perf_counter() - t0) / len(probe)
     total_steps = args.steps + args.warmup
     per_step_budget = 150.0 / max(total_steps, 1)
@@ -225,7 +245,7 @@ def run_reference(args, w):
         t0 = time.perf_counter()
         oracle.forward(inp.x, inp.W_router, inp.W_gate_up, inp.W_down, inp.W_shared, w.k,
                        w.n_group, w.topk_group, w.inter, w.n_shared, tokens=toks,
-                       nthreads=nthreads)
+                       nthreads=nthreads, **oracle_gating(args, w))
         if s >= args.warmup:
             times.append(time.perf_counter() - t0)
     sec = sum(times) / len(times)
@@ -236,7 +256,7 @@ def run_reference(args, w):
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": sec * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": run_config(w, world),
+        "config": run_config(w, world, args),
         "tflops": flops / sec / 1e12,
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": nthreads, "kind": "oracle",
                          "sample": f"{n} random tokens of {w.T} per step"},
@@ -254,6 +274,10 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="prefill", choices=sorted(WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--gate", default="sigmoid", choices=["sigmoid", "softmax"],
+                    help="routing gate (the FusionLLM sigmoid gate is the headline)")
+    ap.add_argument("--expert-bias", action="store_true",
+                    help="add a selection-only expert bias (and read back the expert loads)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -276,8 +300,15 @@ def main():
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream()
 
+    bias = None
+    load = None
+    if args.expert_bias:
+        bias = torch.from_numpy(bias_ramp(w, args.gate)).to(dev)
+        load = torch.empty(w.E, dtype=torch.int32, device=dev)
+
     def step(xin=x, yout=y):
         moe.forward(xin, Wr, Wgu, Wd, Wsh, w.k, w.n_group, w.topk_group, w.inter, w.n_shared,
+                    gate=args.gate, expert_bias=bias, expert_load=load,
                     y=yout, topk_idx=idx, topk_w=wt, workspace=ws)
 
     for _ in range(args.warmup):
@@ -382,7 +413,7 @@ def main():
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded N(0,1) activations, N(0,1/fan_in) weights; no dataset)",
-        "config": run_config(w, world),
+        "config": run_config(w, world, args),
         "tflops": tflops,
         "roofline_layer": {"bound": "tensor", "roofline_ms": roof_ms,
                            "frac": roof_ms / ms, "peak_tflops": pk["bf16_tflops"],
@@ -404,7 +435,7 @@ def main():
         "clocks": clocks.summary(),
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        out["cpu_baseline"] = cpu_baseline(w, inp)
+        out["cpu_baseline"] = cpu_baseline(w, inp, args)
     if rank == 0:
         print(json.dumps(out), flush=True)
     if world > 1:
