@@ -44,10 +44,7 @@ constexpr int kAtoms = 2;                        // 128-byte swizzle atoms (64 b
 constexpr int kBK = 64 * kAtoms;                 // K per stage
 constexpr int kARows = 128;                      // weight rows per CTA (MMA M = 256 per pair)
 constexpr int kABytes = kARows * kBK * 2;        // 32 KiB: 2 atoms x 128 weight rows
-constexpr int kBMaxRows = 128;                   // token rows per CTA (N <= 256 per pair)
-constexpr int kBBytes = kBMaxRows * kBK * 2;     // up to 32 KiB: 2 atoms x 16 rb token rows
-constexpr int kStageBytes = kABytes + kBBytes;   // 64 KiB
-constexpr int kStages = 3;
+constexpr int kMaxStages = 6;
 constexpr int kAtomBytesA = kARows * 128;        // 16 KiB between the atoms of a tile
 constexpr int kNTile = 256;                      // tokens per tile
 constexpr int kTmemCols = 512;                   // 2 accumulators x 256 fp32 columns
@@ -78,8 +75,8 @@ struct __align__(16) Tile {
 
 struct __align__(16) PairTail {
     uint4 stage[kEpiWarps * 256];  // per epilogue warp: 32 rows x 128 B staging
-    uint64_t full[kStages];
-    uint64_t empty[kStages];
+    uint64_t full[kMaxStages];
+    uint64_t empty[kMaxStages];
     uint64_t tfull[2];
     uint64_t tempty[2];
     uint64_t drain;
@@ -92,8 +89,23 @@ struct __align__(16) PairTail {
     int tile_off[2][kMaxGroupsP];  // first tile of each group
 };
 
-constexpr size_t kSmemBytes = 1024 + (size_t)kStages * kStageBytes + sizeof(PairTail);
-static_assert(kSmemBytes <= 232448, "shared memory per CTA");
+// Load-ring shapes.  A stage holds the weight tile (32 KiB) and up to BMAX
+// token rows per CTA (tiles of N <= 2 BMAX tokens); smaller token tiles leave
+// room for more stages in flight.
+template <int STAGES, int BMAX>
+struct Ring {
+    static constexpr int kStages = STAGES;
+    static constexpr int kBMaxRows = BMAX;
+    static constexpr int kBBytes = BMAX * kBK * 2;
+    static constexpr int kStageBytes = kABytes + kBBytes;
+    static constexpr size_t kSmemBytes = 1024 + (size_t)STAGES * kStageBytes + sizeof(PairTail);
+    static_assert(STAGES <= kMaxStages, "stages");
+    static_assert(kStageBytes % 1024 == 0, "stages stay 1024-byte aligned (128B swizzle)");
+    static_assert(kSmemBytes <= 232448, "shared memory per CTA");
+};
+using WideRing = Ring<3, 128>;   // tiles of up to 256 tokens: 3 stages of 64 KiB
+using MidRing = Ring<4, 64>;     // tiles of up to 128 tokens: 4 stages of 48 KiB
+using NarrowRing = Ring<5, 32>;  // tiles of up to 64 tokens: 5 stages of 40 KiB
 
 __device__ __forceinline__ uint32_t cluster_ctarank() {
     uint32_t r;
@@ -399,13 +411,15 @@ __device__ __forceinline__ void pair_epilogue(uint8_t* wb, uint32_t taddr, const
     }
 }
 
-template <int EPI0, int EPI1>
+template <int EPI0, int EPI1, class RING>
 __global__ void __launch_bounds__(kThreads, 1)
     pair_gemm_kernel(const __grid_constant__ PairMaps maps, const PairArgs args0,
                      const PairArgs args1, int n_problems) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    constexpr int kStages = RING::kStages;
+    constexpr int kStageBytes = RING::kStageBytes;
     PairTail* tail = reinterpret_cast<PairTail*>(smem + (size_t)kStages * kStageBytes);
     volatile int* abort_flag = &tail->abort;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -543,6 +557,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (is_sched) {
                     if (next < total_tiles) {
                         t = decode(next);
+                        if (t.n > 2 * RING::kBMaxRows) {
+                            // a token tile larger than this ring's stages: the
+                            // launch chose the wrong ring; stop every role cleanly
+                            set_status(status, MOE_ERR_DEVICE, SITE_GEMM_BOUNDS, t.n);
+                            t = Tile{};
+                            t.end = 1;
+                            next = total_tiles;
+                        }
                         // the ticket's latency is hidden behind this tile's loads
                         next = n_pairs + atomicAdd(args0.sched_counter, 1);
                     } else {
@@ -739,25 +761,38 @@ cudaError_t launch_selftest_timeout(int* status, unsigned long long limit_ns, cu
     return cudaGetLastError();
 }
 
-cudaError_t launch_pair_gemm(int epi0, int epi1, const PairMaps& maps, const PairArgs& a0,
+namespace {
+template <class RING>
+cudaError_t launch_pair_ring(int epi0, int epi1, const PairMaps& maps, const PairArgs& a0,
                              const PairArgs* a1, int n_pairs, cudaStream_t s) {
     using Kern = void (*)(const PairMaps, const PairArgs, const PairArgs, int);
     Kern kern = nullptr;
     if (epi0 == EPI_SWIGLU && epi1 == EPI_SWIGLU)
-        kern = pair_gemm_kernel<EPI_SWIGLU, EPI_SWIGLU>;
+        kern = pair_gemm_kernel<EPI_SWIGLU, EPI_SWIGLU, RING>;
     else if (epi0 == EPI_STORE_F32 && epi1 == EPI_SCATTER)
-        kern = pair_gemm_kernel<EPI_STORE_F32, EPI_SCATTER>;
+        kern = pair_gemm_kernel<EPI_STORE_F32, EPI_SCATTER, RING>;
     else if (epi0 == EPI_SCATTER && epi1 == EPI_SCATTER)
-        kern = pair_gemm_kernel<EPI_SCATTER, EPI_SCATTER>;
+        kern = pair_gemm_kernel<EPI_SCATTER, EPI_SCATTER, RING>;
     else
         return cudaErrorInvalidValue;
-    if (a0.sched_counter == nullptr) return cudaErrorInvalidValue;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)kSmemBytes);
+                                         (int)RING::kSmemBytes);
     if (e != cudaSuccess) return e;
     const int np = a1 != nullptr ? 2 : 1;
-    return launch_pdl(kern, dim3(2 * n_pairs), dim3(kThreads), kSmemBytes, s, 2, maps, a0,
+    return launch_pdl(kern, dim3(2 * n_pairs), dim3(kThreads), RING::kSmemBytes, s, 2, maps, a0,
                       np > 1 ? *a1 : a0, np);
+}
+}  // namespace
+
+cudaError_t launch_pair_gemm(int epi0, int epi1, const PairMaps& maps, const PairArgs& a0,
+                             const PairArgs* a1, int n_pairs, int max_tile_tokens,
+                             cudaStream_t s) {
+    if (a0.sched_counter == nullptr) return cudaErrorInvalidValue;
+    if (max_tile_tokens <= 2 * NarrowRing::kBMaxRows)
+        return launch_pair_ring<NarrowRing>(epi0, epi1, maps, a0, a1, n_pairs, s);
+    if (max_tile_tokens <= 2 * MidRing::kBMaxRows)
+        return launch_pair_ring<MidRing>(epi0, epi1, maps, a0, a1, n_pairs, s);
+    return launch_pair_ring<WideRing>(epi0, epi1, maps, a0, a1, n_pairs, s);
 }
 
 }  // namespace moe

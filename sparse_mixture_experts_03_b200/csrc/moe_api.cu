@@ -372,9 +372,9 @@ MOE_API int moe_forward_ex(const void* x, const void* W_router, const void* W_ga
             if (!make_map_gate_up(&mp.a[0], Wsh_gu, 1, SI, d) ||
                 !make_token_maps(mp.b[0], x, (uint64_t)T, d))
                 return MOE_ERR_CUDA;
-            e = launch_pair_gemm(EPI_SWIGLU, EPI_SWIGLU, mp, ps, &pr, n_pairs, s);
+            e = launch_pair_gemm(EPI_SWIGLU, EPI_SWIGLU, mp, ps, &pr, n_pairs, T, s);
         } else {
-            e = launch_pair_gemm(EPI_SWIGLU, EPI_SWIGLU, mp, pr, nullptr, n_pairs, s);
+            e = launch_pair_gemm(EPI_SWIGLU, EPI_SWIGLU, mp, pr, nullptr, n_pairs, T, s);
         }
         if (e != cudaSuccess) return MOE_ERR_CUDA;
         stage_mark(3, s);
@@ -416,9 +416,9 @@ MOE_API int moe_forward_ex(const void* x, const void* W_router, const void* W_ga
             if (!make_map_rows_atoms(&mp.a[0], Wsh_dn, (uint64_t)d, SI) ||
                 !make_token_maps(mp.b[0], h_sh, (uint64_t)T, SI))
                 return MOE_ERR_CUDA;
-            e = launch_pair_gemm(EPI_STORE_F32, EPI_SCATTER, mp, qs, &qr, n_pairs, s);
+            e = launch_pair_gemm(EPI_STORE_F32, EPI_SCATTER, mp, qs, &qr, n_pairs, T, s);
         } else {
-            e = launch_pair_gemm(EPI_SCATTER, EPI_SCATTER, mp, qr, nullptr, n_pairs, s);
+            e = launch_pair_gemm(EPI_SCATTER, EPI_SCATTER, mp, qr, nullptr, n_pairs, T, s);
         }
         if (e != cudaSuccess) return MOE_ERR_CUDA;
         stage_mark(4, s);

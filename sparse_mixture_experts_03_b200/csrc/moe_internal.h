@@ -165,8 +165,12 @@ struct PairMaps {
 };
 // Epilogue pairs (epi0 for problem 0, epi1 for problem 1): SWIGLU/SWIGLU,
 // STORE_F32/SCATTER, SCATTER/SCATTER.  a1 == nullptr: one problem.
+// max_tile_tokens: an upper bound on the tokens of any tile (the batch size,
+// capped at 256); up to 128 (and again up to 64) the launch uses a deeper ring
+// of smaller stages.
 cudaError_t launch_pair_gemm(int epi0, int epi1, const PairMaps& maps, const PairArgs& a0,
-                             const PairArgs* a1, int n_pairs, cudaStream_t s);
+                             const PairArgs* a1, int n_pairs, int max_tile_tokens,
+                             cudaStream_t s);
 
 cudaError_t launch_selftest_timeout(int* status, unsigned long long limit_ns, cudaStream_t s);
 

@@ -57,6 +57,9 @@ SMALL = [
     # d = 1024: the small-batch router splits d over a cluster of 4 CTAs
     ("bf16_d1024", Workload("bf16_d1024", T=200, d=1024, E=16, k=4, n_group=4, topk_group=2,
                             inter=256, n_shared=1, dtype="bf16")),
+    # T = 100: the GEMMs' 4-stage ring (tiles of at most 128 tokens)
+    ("bf16_T100", Workload("bf16_T100", T=100, d=512, E=16, k=4, n_group=4, topk_group=2,
+                           inter=256, n_shared=2, dtype="bf16")),
     # T > 1024 with d = 512: the whole-d router
     ("bf16_T1500", Workload("bf16_T1500", T=1500, d=512, E=32, k=4, n_group=4, topk_group=2,
                             inter=128, n_shared=1, dtype="bf16")),
