@@ -9,22 +9,26 @@
 // decode-sized batch (a few tokens per expert) becomes a stream of weight
 // tiles with a thin N.  The pair splits the weight rows (A) and the token
 // rows (B) between its two CTAs; each CTA loads only its own halves with TMA
-// into its own shared memory (no multicast), so per CTA a pipeline stage is
-// 16 KiB of weights + at most 16 KiB of tokens and 6 stages fit.
+// into its own shared memory (no multicast).  A pipeline stage covers 128 of
+// K: 32 KiB of weights and N/2 token rows per CTA; the ring has 3 stages of
+// 64 KiB, or 4 / 5 smaller ones when the batch bounds N by 128 / 64.
 //
-// Roles (both CTAs, 6 warps each): warp 0 lane 0 issues TMA loads into its
-// CTA's stage ring; the full-barrier of a stage lives in the pair's first CTA
-// (the MMA issuer) and receives the transaction bytes of both CTAs' loads;
-// warp 1 lane 0 of the first CTA issues tcgen05.mma.cta_group::2 and commits
-// the stage's empty barrier and the accumulator's full barrier in both CTAs;
-// warps 2..5 of each CTA read their 128 TMEM lanes (= weight rows) x N columns
-// (= tokens), transpose through shared memory and store token-major rows.
+// Roles (both CTAs, 7 warps each): warps 0 (weights) and 6 (tokens) issue
+// one TMA copy each per stage; a stage's full barrier lives in the pair's
+// first CTA (the MMA issuer) and receives the transaction bytes of both
+// CTAs' copies; warp 1 lane 0 of the first CTA issues tcgen05.mma.cta_group::2
+// and frees the stage in both CTAs with one multicast commit; warps 2..5 of
+// each CTA read their 32 TMEM lanes (= weight rows) x N columns (= tokens),
+// transpose through shared memory and store token-major rows.  Tiles are
+// handed out dynamically (a ticket counter, and a ring of decoded tiles that
+// every role of the pair reads).
 //
 // Epilogues:
-//   SWIGLU  a CTA's 128 weight rows are 64 gate rows then the 64 matching up
-//           rows, so h = silu(gate) * up for 64 features is formed inside the
-//           CTA (SwiGLU: "大模型工程（一）：Transformer 到 MoE", section
-//           "变了什么，为什么变", item 3) and written as bf16 h[token][feature].
+//   SWIGLU  each warp's 32 weight rows are 16 gate rows and the 16 matching
+//           up rows (the gate/up tensor map interleaves them per 16 rows), so
+//           h = silu(gate) * up is formed per warp (SwiGLU: "大模型工程（一）：
+//           Transformer 到 MoE", section "变了什么，为什么变", item 3) and
+//           written as bf16 h[token][feature].
 //   SCATTER routed down projection: the row of token column t goes to slot
 //           row_src[b_row + t], scaled by its gate weight, stored bf16 (the
 //           weighted combine of the MoEBlock listing, section "混合专家：更多
