@@ -282,7 +282,8 @@ __device__ __forceinline__ void mma_bf16_16816(float (&c)[4], const uint32_t (&a
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-template <int NT>  // NT = E / 8 n-tiles of 8 experts (E = 8 NT, NT even)
+// NT = E / 8 n-tiles of 8 experts (E = 8 NT, NT even); S cp.async stages
+template <int NT, int S>
 __global__ void __launch_bounds__(256) route_mma_kernel(const __nv_bfloat16* __restrict__ x,
                                                         const __nv_bfloat16* __restrict__ Wr,
                                                         int T, int d, int E, int k, int G,
@@ -292,8 +293,8 @@ __global__ void __launch_bounds__(256) route_mma_kernel(const __nv_bfloat16* __r
                                                         float* __restrict__ w_out,
                                                         int* status) {
     extern __shared__ __align__(16) uint8_t rsm[];
-    __nv_bfloat16* xs = reinterpret_cast<__nv_bfloat16*>(rsm);  // [2][32][kMmaLd]
-    __nv_bfloat16* wsm = xs + 2 * kMmaTokens * kMmaLd;          // [2][E][kMmaLd]
+    __nv_bfloat16* xs = reinterpret_cast<__nv_bfloat16*>(rsm);  // [S][32][kMmaLd]
+    __nv_bfloat16* wsm = xs + S * kMmaTokens * kMmaLd;          // [S][E][kMmaLd]
     float* red = reinterpret_cast<float*>(rsm);                // after the loop: [4][32][E+1]
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int wm = warp & 1, wk = warp >> 1;
@@ -326,18 +327,27 @@ __global__ void __launch_bounds__(256) route_mma_kernel(const __nv_bfloat16* __r
 #pragma unroll
         for (int q = 0; q < 4; ++q) acc[n][q] = 0.f;
 
+    // S-deep cp.async ring: one commit group per chunk (empty groups past the
+    // end keep the count uniform), so waiting until S-1 groups are pending
+    // means chunk ch has landed
     const int n_chunks = d / kMmaKC;
-    load_chunk(0, 0);
+#pragma unroll
+    for (int st = 0; st < S - 1; ++st) {
+        if (st < n_chunks)
+            load_chunk(st, st * kMmaKC);
+        else
+            cp_async_commit();
+    }
     for (int ch = 0; ch < n_chunks; ++ch) {
-        if (ch + 1 < n_chunks) {
-            load_chunk((ch + 1) & 1, (ch + 1) * kMmaKC);
-            cp_async_wait<1>();
-        } else {
-            cp_async_wait<0>();
-        }
+        const int nx = ch + S - 1;
+        if (nx < n_chunks)
+            load_chunk(nx % S, nx * kMmaKC);  // the buffer chunk ch - 1 has been read from
+        else
+            cp_async_commit();
+        cp_async_wait<S - 1>();
         __syncthreads();
-        const __nv_bfloat16* xc = xs + (ch & 1) * kMmaTokens * kMmaLd;
-        const __nv_bfloat16* wc = wsm + (ch & 1) * E * kMmaLd;
+        const __nv_bfloat16* xc = xs + (ch % S) * kMmaTokens * kMmaLd;
+        const __nv_bfloat16* wc = wsm + (ch % S) * E * kMmaLd;
 #pragma unroll
         for (int kk = 0; kk < 64; kk += 16) {
             const int kb = wk * 64 + kk;
@@ -615,22 +625,23 @@ cudaError_t launch_route_split(const void* x, const void* Wr, int T, int d, int 
 #undef MOE_ROUTE_SPLIT_CASE
 }
 
-size_t route_mma_smem(int E) {
-    const size_t stage = (size_t)2 * (kMmaTokens + E) * kMmaLd * sizeof(__nv_bfloat16);
+size_t route_mma_smem(int E, int S) {
+    const size_t stage = (size_t)S * (kMmaTokens + E) * kMmaLd * sizeof(__nv_bfloat16);
     const size_t red = (size_t)5 * kMmaTokens * (E + 1) * sizeof(float);
     return stage > red ? stage : red;
 }
 
-cudaError_t launch_route_mma(const void* x, const void* Wr, int T, int d, int E, int k, int G,
-                             int TG, int gate, const float* bias, int32_t* idx, float* w,
+template <int S>
+cudaError_t launch_route_mma_s(const void* x, const void* Wr, int T, int d, int E, int k, int G,
+                               int TG, int gate, const float* bias, int32_t* idx, float* w,
                                int* status, cudaStream_t s) {
-    const size_t smem = route_mma_smem(E);
+    const size_t smem = route_mma_smem(E, S);
     const dim3 grid((T + kMmaTokens - 1) / kMmaTokens);
     const __nv_bfloat16* xp = static_cast<const __nv_bfloat16*>(x);
     const __nv_bfloat16* wp = static_cast<const __nv_bfloat16*>(Wr);
 #define MOE_ROUTE_MMA_CASE(NT)                                                                \
     case NT: {                                                                                \
-        auto kern = route_mma_kernel<NT>;                                                     \
+        auto kern = route_mma_kernel<NT, S>;                                                  \
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, \
                                              (int)smem);                                      \
         if (e != cudaSuccess) return e;                                                       \
@@ -650,6 +661,19 @@ cudaError_t launch_route_mma(const void* x, const void* Wr, int T, int d, int E,
             return cudaErrorInvalidValue;
     }
 #undef MOE_ROUTE_MMA_CASE
+}
+
+// 4 cp.async stages (one CTA per SM) when the grid fits on the GPU at once
+// and E <= 64; otherwise 2 stages, two CTAs per SM
+cudaError_t launch_route_mma(const void* x, const void* Wr, int T, int d, int E, int k, int G,
+                             int TG, int gate, const float* bias, int32_t* idx, float* w,
+                             int* status, cudaStream_t s) {
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess)
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (E <= 64 && (T + kMmaTokens - 1) / kMmaTokens <= sms)
+        return launch_route_mma_s<4>(x, Wr, T, d, E, k, G, TG, gate, bias, idx, w, status, s);
+    return launch_route_mma_s<2>(x, Wr, T, d, E, k, G, TG, gate, bias, idx, w, status, s);
 }
 
 template <typename TIn>
