@@ -60,6 +60,12 @@ SMALL = [
     # T = 100: the GEMMs' 4-stage ring (tiles of at most 128 tokens)
     ("bf16_T100", Workload("bf16_T100", T=100, d=512, E=16, k=4, n_group=4, topk_group=2,
                            inter=256, n_shared=2, dtype="bf16")),
+    # the largest expert counts the kernels take: E = 256 in 32 groups, k = 8
+    ("bf16_E256", Workload("bf16_E256", T=600, d=256, E=256, k=8, n_group=32, topk_group=4,
+                           inter=128, n_shared=1, dtype="bf16")),
+    # E = 128 (the tensor-core router's widest tile, 2 cp.async stages)
+    ("bf16_E128_T1100", Workload("bf16_E128_T1100", T=1100, d=512, E=128, k=4, n_group=8,
+                                 topk_group=2, inter=128, n_shared=0, dtype="bf16")),
     # T > 1024 with d = 512: the whole-d router
     ("bf16_T1500", Workload("bf16_T1500", T=1500, d=512, E=32, k=4, n_group=4, topk_group=2,
                             inter=128, n_shared=1, dtype="bf16")),
