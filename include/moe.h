@@ -27,7 +27,8 @@
  *     stream).  Calls are asynchronous unless stated otherwise: they return
  *     after queueing work and never synchronise the stream.
  *   - The caller owns every buffer.  The library allocates no device memory;
- *     it keeps only per-process caches (kernel attributes).
+ *     it keeps only per-process caches (kernel attributes) and one fixed
+ *     256 KiB device array that only moe_expert_counts_noalloc uses.
  *   - All matrices are row-major and contiguous.  Device pointers must be
  *     16-byte aligned; `workspace` must be 256-byte aligned.
  *   - Errors: invalid arguments are reported synchronously, before anything
@@ -36,7 +37,10 @@
  *     a bounds check) do not trap: the kernel records a code in the status
  *     word at the start of the workspace, returns early, and the host reads
  *     it with moe_get_device_status().
- *   - T = 0 is valid and queues nothing.
+ *   - T = 0 is valid and queues nothing (moe_forward_ex with an expert_load
+ *     buffer queues the zeroing of that buffer).
+ *   - moe_forward can be captured in a CUDA graph: every replay resets the
+ *     status word and its internal counters itself.
  */
 #ifndef MOE_B200_H
 #define MOE_B200_H
@@ -93,7 +97,7 @@ enum {
     MOE_WS_STATUS = 0,       /* int32[64]: [0] status code, [1] where, [2..3] info     */
     MOE_WS_COUNTS = 1,       /* int32[E]   tokens routed to each expert                */
     MOE_WS_OFFSETS = 2,      /* int32[E+1] first row of each expert in the permuted
-                                layout; segments are padded to 128 rows              */
+                                layout (bf16: unpadded; f32: padded to 128 rows)     */
     MOE_WS_BLOCK_COUNTS = 3, /* int32[ceil(T/256) * E] per-block histogram / bases     */
     MOE_WS_TOPK_IDX = 4,     /* int32[T*k] chosen experts (used when no output given)  */
     MOE_WS_TOPK_W = 5,       /* f32[T*k]   gate weights                               */
