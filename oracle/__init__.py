@@ -1,4 +1,5 @@
-"""CPU oracle for the fine-grained MoE layer forward -- TEST INFRASTRUCTURE ONLY.
+"""CPU oracle for the fine-grained MoE layer (forward and backward) -- TEST
+INFRASTRUCTURE ONLY.
 
 Only tests/, the smoke check in __graft_entry__ and the benchmark's CPU-baseline
 leg may import this package.  It never imports the CUDA package and the CUDA
@@ -13,7 +14,8 @@ Two independent formulations live here:
     to cross-check the sparse form.
 
 Inputs are torch CPU tensors in float32 or bfloat16 (the exact values given to
-the GPU); outputs are numpy float64 / int32 arrays.
+the GPU), or float64 (the finite-difference checks of the backward); outputs
+are numpy float64 / int32 arrays.
 """
 from __future__ import annotations
 
@@ -27,7 +29,7 @@ import torch
 from . import build as _build
 
 _LIB = None
-OR_F32, OR_BF16 = 0, 1
+OR_F32, OR_BF16, OR_F64 = 0, 1, 2
 
 
 def lib() -> ctypes.CDLL:
@@ -42,6 +44,13 @@ def lib() -> ctypes.CDLL:
         L.oracle_forward.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, i32,
                                      i32, i32, dp, dp, i32, dp, dp, dp, dp, i32]
         L.oracle_forward.restype = i32
+        L.oracle_backward.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, i32,
+                                      i32, i32, dp, dp, vp, dp, dp, dp, dp, dp, dp, dp, i32]
+        L.oracle_backward.restype = i32
+        L.oracle_backward_rows.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32,
+                                           i32, i32, i32, dp, dp, vp, dp, i32, dp, dp, i32, dp,
+                                           i32, i32]
+        L.oracle_backward_rows.restype = i32
         L.oracle_max_threads.restype = i32
         L.oracle_check_args.argtypes = [i32] * 6
         L.oracle_check_args.restype = i32
@@ -58,7 +67,9 @@ def _dt(t: torch.Tensor) -> int:
         return OR_F32
     if t.dtype == torch.bfloat16:
         return OR_BF16
-    raise TypeError(f"oracle takes float32 or bfloat16 tensors, got {t.dtype}")
+    if t.dtype == torch.float64:
+        return OR_F64
+    raise TypeError(f"oracle takes float32, bfloat16 or float64 tensors, got {t.dtype}")
 
 
 def _ptr(t: Optional[torch.Tensor]):
@@ -163,3 +174,94 @@ def forward(x: torch.Tensor, W_router: torch.Tensor, W_gate_up: torch.Tensor,
 
 def check_args(T, d, E, k, n_group, topk_group) -> bool:
     return lib().oracle_check_args(T, d, E, k, n_group, topk_group) == 0
+
+
+def _check_layer(x, W_router, W_gate_up, W_down, W_shared, inter, n_shared):
+    E = W_router.shape[0]
+    d = x.shape[1]
+    for t in (W_router, W_gate_up, W_down) + ((W_shared,) if W_shared is not None else ()):
+        assert t.dtype == x.dtype and t.is_contiguous()
+    assert W_gate_up.numel() == E * 2 * inter * d and W_down.numel() == E * d * inter
+    if n_shared:
+        assert W_shared is not None and W_shared.numel() == 3 * n_shared * inter * d
+    return E, d
+
+
+def _forced(forced_idx, T, k):
+    if forced_idx is None:
+        return None
+    fi = np.ascontiguousarray(np.asarray(forced_idx, dtype=np.int32))
+    assert fi.shape == (T, k)
+    return fi
+
+
+class Grads:
+    """Gradients of the layer, fp64, in the layouts of the forward's tensors:
+    dx [T,d], dW_router [E,d], dW_gate_up [E,2I,d], dW_down [E,d,I],
+    dW_shared [3*SI*d] (gate_up block then down block) or None; idx [T,k] the
+    expert sets used and dl [T,k] = dL/dlogit of the chosen experts."""
+
+    def __init__(self, **kw):
+        self.__dict__.update(kw)
+
+
+def backward(x, W_router, W_gate_up, W_down, W_shared, dy, k, n_group, topk_group, inter,
+             n_shared, forced_idx=None, nthreads: int = 0, score_func: str = "sigmoid",
+             bias=None) -> Grads:
+    """Gradients of L = sum(dy * y) with respect to x and every weight (the
+    chain rule through steps 1-7, written out in moe_oracle.c).  dy has the
+    dtype of x.  forced_idx [T,k]: expert sets used in place of the oracle's
+    own top-k."""
+    T = x.shape[0]
+    E, d = _check_layer(x, W_router, W_gate_up, W_down, W_shared, inter, n_shared)
+    assert dy.shape == x.shape and dy.dtype == x.dtype and dy.is_contiguous()
+    I, SI = inter, n_shared * inter
+    dx = np.zeros((T, d))
+    dWr = np.zeros((E, d))
+    dWgu = np.zeros((E, 2 * I, d))
+    dWd = np.zeros((E, d, I))
+    dWsh = np.zeros(3 * SI * d) if n_shared else None
+    idx = np.zeros((T, k), np.int32)
+    dl = np.zeros((T, k))
+    rc = lib().oracle_backward(_ptr(x), _ptr(W_router), _ptr(W_gate_up), _ptr(W_down),
+                               _ptr(W_shared), _dt(x), T, d, E, k, n_group, topk_group, I,
+                               n_shared, SCORE_FUNCS[score_func], _np_ptr(_bias(bias, E)),
+                               _np_ptr(_forced(forced_idx, T, k)), _ptr(dy), _np_ptr(dx),
+                               _np_ptr(dWr), _np_ptr(dWgu), _np_ptr(dWd), _np_ptr(dWsh),
+                               _np_ptr(idx), _np_ptr(dl), nthreads)
+    if rc != 0:
+        raise ValueError("oracle_backward: invalid arguments")
+    return Grads(dx=dx, dW_router=dWr, dW_gate_up=dWgu, dW_down=dWd, dW_shared=dWsh, idx=idx,
+                 dl=dl)
+
+
+# tensor ids of backward_rows
+ROW_DWR, ROW_DWGU, ROW_DWD, ROW_DWSH_GU, ROW_DWSH_DN = 0, 1, 2, 3, 4
+
+
+def backward_rows(x, W_router, W_gate_up, W_down, W_shared, dy, k, n_group, topk_group, inter,
+                  n_shared, dx_tokens=(), wsel=(), forced_idx=None, nthreads: int = 0,
+                  score_func: str = "sigmoid", bias=None):
+    """Selected entries of the backward at any size, each computed on its own:
+    dx rows of dx_tokens, and weight-gradient rows wsel = [(tensor id, row)]
+    (ROW_* ids; rows in the flattened [rows, cols] view of each gradient).
+    Returns (dx_rows [n, d], [row arrays])."""
+    T = x.shape[0]
+    E, d = _check_layer(x, W_router, W_gate_up, W_down, W_shared, inter, n_shared)
+    assert dy.shape == x.shape and dy.dtype == x.dtype and dy.is_contiguous()
+    I, SI = inter, n_shared * inter
+    toks = np.ascontiguousarray(np.asarray(dx_tokens, dtype=np.int32).reshape(-1))
+    ws = np.ascontiguousarray(np.asarray(wsel, dtype=np.int32).reshape(-1, 2))
+    ld = max(d, I, SI)
+    dxr = np.zeros((len(toks), d))
+    wr = np.zeros((len(ws), ld))
+    rc = lib().oracle_backward_rows(_ptr(x), _ptr(W_router), _ptr(W_gate_up), _ptr(W_down),
+                                    _ptr(W_shared), _dt(x), T, d, E, k, n_group, topk_group, I,
+                                    n_shared, SCORE_FUNCS[score_func], _np_ptr(_bias(bias, E)),
+                                    _np_ptr(_forced(forced_idx, T, k)), _ptr(dy),
+                                    _np_ptr(toks), len(toks), _np_ptr(dxr), _np_ptr(ws), len(ws),
+                                    _np_ptr(wr), ld, nthreads)
+    if rc != 0:
+        raise ValueError("oracle_backward_rows: invalid arguments")
+    lens = {ROW_DWR: d, ROW_DWGU: d, ROW_DWD: I, ROW_DWSH_GU: d, ROW_DWSH_DN: SI}
+    return dxr, [wr[i, :lens[int(t)]].copy() for i, (t, _) in enumerate(ws)]
