@@ -1,6 +1,6 @@
 /*
- * moe.h -- C ABI of the B200 (sm_100a) fine-grained Mixture-of-Experts layer
- * forward.
+ * moe.h -- C ABI of the B200 (sm_100a) fine-grained Mixture-of-Experts layer:
+ * forward, and (for training) forward with saved activations and backward.
  *
  * The layer (per token x of length d) is the one described on the FusionLLM
  * page "FusionLLM：融合 MLA、GDN 与 MoE 的高效混合架构大模型训练框架", section
@@ -254,6 +254,89 @@ MOE_API int moe_set_stage_events(void *const *events, int n);
  */
 MOE_API int moe_expert_counts_noalloc(const int32_t *topk_idx, int T, int k, int E,
                                       int32_t *counts, int32_t *offsets, void *stream);
+
+/*
+ * ---- Training: forward with saved activations, and the layer backward -----
+ *
+ * The layer is trained with the rest of the model (the FusionLLM page is a
+ * pretraining framework: section "训练优化技术", whose fused kernels include a
+ * grouped GEMM for the MoE layer; pretraining on 8 GPUs per its section
+ * "模型配置与规模"); its backward is the chain rule through the forward above,
+ * for an upstream gradient dy = dL/dy:
+ *   a_j  = dy . SwiGLU_{idx[j]}(x)   (dL/dw_j),   abar = sum_j w_j a_j
+ *   MOE_GATE_SIGMOID:      dL/dlogit_j = (a_j - abar) / sum_i s_i * s_j (1 - s_j)
+ *   MOE_GATE_SOFTMAX_TOPK: dL/dlogit_j = w_j (a_j - abar)
+ *   (only the chosen experts' logits get a gradient; the selection, the group
+ *    limit and a selection bias pass none)
+ *   dW_router[e] = sum_t dL/dlogit_{t,e} x_t,  dx += sum_j dL/dlogit_j W_router[idx[j]]
+ *   per chosen expert (weight w_j; shared experts weight 1): dh = w_j W_down^T dy,
+ *   dg = dh * up * silu'(gate), du = dh * silu(gate), dW_down += w_j dy h^T,
+ *   dW_gate += dg x^T, dW_up += du x^T, dx += W_gate^T dg + W_up^T du.
+ *
+ * moe_saved_bytes -- bytes of the `saved` buffer of moe_forward_train (bf16
+ * layers): the gate / up pre-activations, bf16, routed [T*k, 2*inter] (row
+ * t*k + j = token t's j-th chosen expert; gate columns [0, inter), up columns
+ * [inter, 2*inter)) followed by shared [T, 2*n_shared*inter] (gate columns of
+ * all shared experts, then their up columns).  0 for invalid sizes.
+ */
+MOE_API size_t moe_saved_bytes(int T, int k, int inter, int n_shared);
+
+/*
+ * moe_forward_train -- moe_forward_ex that also writes the pre-activations
+ * the backward needs into `saved` (device, moe_saved_bytes bytes, 16-byte
+ * aligned, owned by the caller until the matching moe_backward has run).  y,
+ * topk_idx_out and topk_w_out as moe_forward_ex; the backward needs the
+ * routing, so topk_idx_out and topk_w_out are required here.  bf16 layers only
+ * (MOE_ERR_UNSUPPORTED otherwise); other arguments and errors as
+ * moe_forward_ex.
+ */
+MOE_API int moe_forward_train(const void *x, const void *W_router, const void *W_gate_up,
+                              const void *W_down, const void *W_shared, int T, int d, int E,
+                              int k, int n_group, int topk_group, int inter, int n_shared,
+                              int in_dt, int out_dt, int gate, const float *expert_bias,
+                              void *y, int32_t *topk_idx_out, float *topk_w_out,
+                              int32_t *expert_load, void *saved, size_t saved_bytes,
+                              void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * moe_backward_workspace_bytes -- scratch bytes of moe_backward for these
+ * sizes (bf16 layers; 0 for invalid or unsupported sizes).  Regions: status
+ * words and tile counters, expert counts and padded offsets, the permutation
+ * (segments padded to 128 rows), x and dy rows in that order, the SwiGLU
+ * backward rows dg|du and w*h, the per-row parts of dL/dw, dL/dlogit, the
+ * chosen experts' dx rows, the shared experts' rows and their fp32 dx.
+ */
+MOE_API size_t moe_backward_workspace_bytes(int T, int d, int E, int k, int inter,
+                                            int n_shared);
+
+/*
+ * moe_backward -- gradients of the layer for the forward that
+ * moe_forward_train ran with the same x, weights, gate and `saved`:
+ *   x, W_router, W_gate_up, W_down, W_shared  the forward's inputs (bf16)
+ *   dy          device, bf16 [T, d]: dL/dy
+ *   topk_idx    device, int32 [T, k]: the forward's topk_idx_out
+ *   topk_w      device, f32 [T, k]: the forward's topk_w_out
+ *   saved       device: the forward's saved pre-activations
+ *   gate        the forward's gate
+ * Outputs (device, fp32, overwritten; same layouts as the forward tensors):
+ *   dx [T, d], dW_router [E, d], dW_gate_up [E, 2*inter, d], dW_down
+ *   [E, d, inter], dW_shared [2*SI*d + d*SI] (SI = n_shared*inter; NULL iff
+ *   n_shared == 0).  Experts no token chose get zero gradients.
+ * Every sum runs in a fixed order: results are bitwise reproducible.
+ * Requirements: in_dt == MOE_BF16, d and inter multiples of 256 (else
+ * MOE_ERR_UNSUPPORTED); workspace of moe_backward_workspace_bytes bytes (else
+ * MOE_ERR_WORKSPACE), 256-byte aligned.  Device faults as for the forward
+ * (status word of `workspace`).  T = 0 queues the zeroing of the weight
+ * gradients only.  Queues work on `stream`; no synchronisation, no
+ * allocation; capturable in a CUDA graph.
+ */
+MOE_API int moe_backward(const void *x, const void *W_router, const void *W_gate_up,
+                         const void *W_down, const void *W_shared, const void *dy,
+                         const int32_t *topk_idx, const float *topk_w, const void *saved,
+                         int T, int d, int E, int k, int inter, int n_shared, int in_dt,
+                         int gate, float *dx, float *dW_router, float *dW_gate_up,
+                         float *dW_down, float *dW_shared, void *workspace,
+                         size_t workspace_bytes, void *stream);
 
 /* moe_status_string -- static text for a status code. */
 MOE_API const char *moe_status_string(int status);

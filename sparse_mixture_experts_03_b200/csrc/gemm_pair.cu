@@ -74,7 +74,7 @@ struct __align__(16) Tile {
     int n_real;  // tokens in the tile (1..256)
     int n;       // MMA N: n_real rounded up to 16
     int end;     // 1: no more tiles for this pair
-    int pad;
+    int aux;     // KIND_WGRAD: N tile | k-blocks << 16 (b_row is then the first K row)
 };
 
 struct __align__(16) PairTail {
@@ -91,6 +91,7 @@ struct __align__(16) PairTail {
     int abort;
     int seg_off[2][kMaxGroupsP];   // first token row of each group
     int tile_off[2][kMaxGroupsP];  // first tile of each group
+    int cnt[2][kMaxGroupsP];       // token rows of each group
 };
 
 // Load-ring shapes.  A stage holds the weight tile (32 KiB) and up to BMAX
@@ -165,8 +166,11 @@ __device__ __forceinline__ void arrive_expect_tx_local(uint64_t* bar, uint32_t b
     mbar_arrive_expect_tx(bar, bytes);
 }
 // The 4 MMAs (K = 16 each) of one 64-deep k-block: descriptors of step kk
-// are the base descriptors + 2 kk (32 bytes further along the swizzled rows);
-// the first accumulates into D only if `accumulate`, the rest always do.
+// are the base descriptors + AS kk / BS kk (a K-major operand: 2 = 32 bytes
+// further along the swizzled rows; an MN-major one: 128 = 16 rows of 128 B
+// further); the first accumulates into D only if `accumulate`, the rest
+// always do.
+template <uint64_t AS = 2, uint64_t BS = 2>
 __device__ __forceinline__ void tc_mma4_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
                                              uint32_t idesc, uint32_t accumulate) {
     asm volatile(
@@ -177,8 +181,8 @@ __device__ __forceinline__ void tc_mma4_pair(uint32_t d_tmem, uint64_t a_desc, u
         "tcgen05.mma.cta_group::2.kind::f16 [%0], %5, %6, %3, q;\n\t"
         "tcgen05.mma.cta_group::2.kind::f16 [%0], %7, %8, %3, q;\n\t"
         "tcgen05.mma.cta_group::2.kind::f16 [%0], %9, %10, %3, q;\n\t}" ::"r"(d_tmem),
-        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "l"(a_desc + 2), "l"(b_desc + 2),
-        "l"(a_desc + 4), "l"(b_desc + 4), "l"(a_desc + 6), "l"(b_desc + 6)
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "l"(a_desc + AS), "l"(b_desc + BS),
+        "l"(a_desc + 2 * AS), "l"(b_desc + 2 * BS), "l"(a_desc + 3 * AS), "l"(b_desc + 3 * BS)
         : "memory");
 }
 // arrive (once) on the mbarrier at shared::cluster address `bar` when all
@@ -322,7 +326,8 @@ __device__ __forceinline__ void pair_epilogue(uint8_t* wb, uint32_t taddr, const
         for (int c = 0; c < kNTile / 32; ++c)
             srcs[c] = 32 * c + lane < t.n_real ? a.row_src[t.b_row + 32 * c + lane] : -1;
 #pragma unroll
-        for (int c = 0; c < kNTile / 32; ++c) wts[c] = srcs[c] >= 0 ? a.topk_w[srcs[c]] : 0.f;
+        for (int c = 0; c < kNTile / 32; ++c)
+            wts[c] = srcs[c] >= 0 ? (a.topk_w != nullptr ? a.topk_w[srcs[c]] : 1.f) : 0.f;
     }
 #pragma unroll
     for (int cc = 0; cc < kNTile / 32; ++cc) {
@@ -332,7 +337,7 @@ __device__ __forceinline__ void pair_epilogue(uint8_t* wb, uint32_t taddr, const
         tmem_ld32(taddr + (uint32_t)c0, v);  // weight row (lane) x tokens c0 .. c0+31
         tmem_ld_wait();
         const bool tok_ok = c0 + lane < t.n_real;  // after the transpose, lane = token
-        if constexpr (EPI == EPI_SWIGLU) {
+        if constexpr (EPI == EPI_SWIGLU || EPI == EPI_SWIGLU_SAVE) {
             // The CTA's weight rows are [16 gate, 16 up] per warp quarter: lane
             // i < 16 holds gate feature 16 wq + i, lane i + 16 the matching up
             // row.  fp32 transpose through the staging buffer, then lane = token:
@@ -363,6 +368,27 @@ __device__ __forceinline__ void pair_epilogue(uint8_t* wb, uint32_t taddr, const
                     t.ft * a.out_col_step + cta * 64 + wq * 16);
                 d[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
                 d[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
+                if constexpr (EPI == EPI_SWIGLU_SAVE) {
+                    // the pre-activations for the backward, in slot (or token) order:
+                    // gate at columns [0, F), up at [F, 2F)
+                    const int r = t.b_row + c0 + lane;
+                    const int srow = a.row_src != nullptr ? a.row_src[r] : r;
+                    uint32_t pg[8], pu[8];
+#pragma unroll
+                    for (int p = 0; p < 8; ++p) {
+                        pg[p] = pack_bf16x2(f[2 * p], f[2 * p + 1]);
+                        pu[p] = pack_bf16x2(f[16 + 2 * p], f[16 + 2 * p + 1]);
+                    }
+                    __nv_bfloat16* sv = static_cast<__nv_bfloat16*>(a.save) +
+                                        (size_t)srow * 2 * a.feat + t.ft * a.out_col_step +
+                                        cta * 64 + wq * 16;
+                    uint4* dg = reinterpret_cast<uint4*>(sv);
+                    uint4* du = reinterpret_cast<uint4*>(sv + a.feat);
+                    dg[0] = make_uint4(pg[0], pg[1], pg[2], pg[3]);
+                    dg[1] = make_uint4(pg[4], pg[5], pg[6], pg[7]);
+                    du[0] = make_uint4(pu[0], pu[1], pu[2], pu[3]);
+                    du[1] = make_uint4(pu[4], pu[5], pu[6], pu[7]);
+                }
             }
             __syncwarp();
         } else if constexpr (EPI == EPI_SCATTER) {
@@ -394,6 +420,106 @@ __device__ __forceinline__ void pair_epilogue(uint8_t* wb, uint32_t taddr, const
                                       packed[4 * q + 3]);
             }
             __syncwarp();
+        } else if constexpr (EPI == EPI_DSWIGLU) {
+            // SwiGLU backward.  fp32 transpose (token row i: its 32 features),
+            // then lane = token row r: dh_raw of features f0 .. f0 + 31 (the
+            // warp's TMEM lanes), the saved gate / up pre-activations of the
+            // row's slot, and per feature
+            //   h = silu(g) u,  dh = w dh_raw,
+            //   dg = dh u silu'(g),  du = dh silu(g),  hw = w h,
+            // with silu'(g) = sigmoid(g) (1 + g (1 - sigmoid(g))); the sum of
+            // dh_raw h over the 32 features is this warp's part of dL/dw.
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+                float* row = reinterpret_cast<float*>(stage_chunk(wb, i, lane >> 2));
+                row[lane & 3] = __uint_as_float(v[i]);
+            }
+            __syncwarp();
+            if (tok_ok) {
+                const int r = t.b_row + c0 + lane;
+                const int src = a.row_src != nullptr ? a.row_src[r] : r;
+                const float wv = a.row_src != nullptr ? a.topk_w[src] : 1.f;
+                const int F = a.feat;
+                const int f0 = t.ft * 256 + (int)cta * 128 + wq * 32;
+                const __nv_bfloat16* gp =
+                    static_cast<const __nv_bfloat16*>(a.gu_in) + (size_t)src * 2 * F + f0;
+                uint4 gq[4], uq[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    gq[q] = reinterpret_cast<const uint4*>(gp)[q];
+                    uq[q] = reinterpret_cast<const uint4*>(gp + F)[q];
+                }
+                const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(gq);
+                const __nv_bfloat162* u2 = reinterpret_cast<const __nv_bfloat162*>(uq);
+                uint32_t pdg[16], pdu[16], phw[16];
+                float part = 0.f;
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    const float4 c4 = *reinterpret_cast<const float4*>(stage_chunk(wb, lane, q));
+                    const float dr[4] = {c4.x, c4.y, c4.z, c4.w};
+                    float odg[4], odu[4], ohw[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 gg = __bfloat1622float2(g2[(4 * q + e) >> 1]);
+                        const float2 uu = __bfloat1622float2(u2[(4 * q + e) >> 1]);
+                        const float g = (e & 1) ? gg.y : gg.x;
+                        const float u = (e & 1) ? uu.y : uu.x;
+                        const float sg = 1.0f / (1.0f + __expf(-g));
+                        const float silu = g * sg;
+                        const float h = silu * u;
+                        part = fmaf(dr[e], h, part);
+                        const float dh = wv * dr[e];
+                        odg[e] = dh * u * (sg * (1.0f + g * (1.0f - sg)));
+                        odu[e] = dh * silu;
+                        ohw[e] = wv * h;
+                    }
+                    pdg[2 * q] = pack_bf16x2(odg[0], odg[1]);
+                    pdg[2 * q + 1] = pack_bf16x2(odg[2], odg[3]);
+                    pdu[2 * q] = pack_bf16x2(odu[0], odu[1]);
+                    pdu[2 * q + 1] = pack_bf16x2(odu[2], odu[3]);
+                    phw[2 * q] = pack_bf16x2(ohw[0], ohw[1]);
+                    phw[2 * q + 1] = pack_bf16x2(ohw[2], ohw[3]);
+                }
+                __nv_bfloat16* dgr =
+                    static_cast<__nv_bfloat16*>(a.dgu_out) + (size_t)r * 2 * F + f0;
+                uint4* dgq = reinterpret_cast<uint4*>(dgr);
+                uint4* duq = reinterpret_cast<uint4*>(dgr + F);
+                uint4* hwq = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.hw_out) +
+                                                      (size_t)r * F + f0);
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    dgq[q] = make_uint4(pdg[4 * q], pdg[4 * q + 1], pdg[4 * q + 2], pdg[4 * q + 3]);
+                    duq[q] = make_uint4(pdu[4 * q], pdu[4 * q + 1], pdu[4 * q + 2], pdu[4 * q + 3]);
+                    hwq[q] = make_uint4(phw[4 * q], phw[4 * q + 1], phw[4 * q + 2], phw[4 * q + 3]);
+                }
+                if (a.dw_part != nullptr) a.dw_part[(size_t)r * (F >> 5) + (f0 >> 5)] = part;
+            }
+            __syncwarp();
+        } else if constexpr (EPI == EPI_STORE_ROWS) {
+            // weight-gradient tile: lane = output row (TMEM lane), 32 columns per
+            // chunk.  Rows go through the staging buffer so that each store
+            // instruction writes 4 whole 128-byte row segments.  A tile of an
+            // empty group (no k-blocks) stores zeros.
+            const bool zero = (t.aux >> 16) == 0;
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                float4 c4 = make_float4(__uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1]),
+                                        __uint_as_float(v[4 * q + 2]),
+                                        __uint_as_float(v[4 * q + 3]));
+                if (zero) c4 = make_float4(0.f, 0.f, 0.f, 0.f);
+                *reinterpret_cast<float4*>(stage_chunk(wb, lane, q)) = c4;
+            }
+            __syncwarp();
+            float* ob = static_cast<float*>(a.out) +
+                        ((size_t)t.g * a.m_total + t.ft * 256 + cta * 128 + wq * 32) * a.out_ld +
+                        (size_t)(t.aux & 0xFFFF) * 256 + c0;
+#pragma unroll
+            for (int it = 0; it < 8; ++it) {
+                const int row = it * 4 + (lane >> 3), q = lane & 7;
+                *reinterpret_cast<float4*>(ob + (size_t)row * a.out_ld + q * 4) =
+                    *reinterpret_cast<const float4*>(stage_chunk(wb, row, q));
+            }
+            __syncwarp();
         } else {  // EPI_STORE_F32: out[b_row + token][col] = acc, fp32
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
@@ -415,7 +541,7 @@ __device__ __forceinline__ void pair_epilogue(uint8_t* wb, uint32_t taddr, const
     }
 }
 
-template <int EPI0, int EPI1, class RING>
+template <int EPI0, int EPI1, class RING, int KIND>
 __global__ void __launch_bounds__(kThreads, 1)
     pair_gemm_kernel(const __grid_constant__ PairMaps maps, const PairArgs args0,
                      const PairArgs args1, int n_problems) {
@@ -457,12 +583,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int p = 0; p < n_problems; ++p) {
             const PairArgs& a = p == 0 ? args0 : args1;
             const int ng = a.counts != nullptr ? a.n_groups : 1;
+            const int al = a.seg_align > 1 ? a.seg_align : 1;
             int carry_r = 0, carry_t = 0;
             for (int g0 = 0; g0 < ng; g0 += 32) {
                 const int g = g0 + lane;
                 const int c = g < ng ? (a.counts != nullptr ? a.counts[g] : a.static_rows) : 0;
-                const int tl = ((c + kNTile - 1) / kNTile) * a.n_ftiles;
-                int ir = c, it = tl;
+                // rows the group occupies in B (segments padded to `al` rows)
+                const int cr = (c + al - 1) / al * al;
+                const int tl = KIND == KIND_WGRAD ? (g < ng ? a.n_ftiles * a.n_ntiles : 0)
+                                                  : ((c + kNTile - 1) / kNTile) * a.n_ftiles;
+                int ir = cr, it = tl;
 #pragma unroll
                 for (int o = 1; o < 32; o <<= 1) {
                     const int nr = __shfl_up_sync(0xffffffffu, ir, o);
@@ -473,8 +603,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 }
                 if (g < ng) {
-                    tail->seg_off[p][g] = carry_r + ir - c;
+                    tail->seg_off[p][g] = carry_r + ir - cr;
                     tail->tile_off[p][g] = carry_t + it - tl;
+                    tail->cnt[p][g] = c;
                 }
                 carry_r += __shfl_sync(0xffffffffu, ir, 31);
                 carry_t += __shfl_sync(0xffffffffu, it, 31);
@@ -514,9 +645,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int lt = t.p == 0 ? tile : tile - tiles0;
         const int ng = t.p == 0 ? ng0 : ng1;
         t.g = upper_group(tail->tile_off[t.p], ng, lt);
-        const int cnt = tail->seg_off[t.p][t.g + 1] - tail->seg_off[t.p][t.g];
-        const int nch = (cnt + kNTile - 1) / kNTile;
+        const int cnt = tail->cnt[t.p][t.g];
         const int local = lt - tail->tile_off[t.p][t.g];
+        t.end = 0;
+        if (KIND == KIND_WGRAD) {
+            // M tile slow, N tile fast; K runs over the group's rows (padded
+            // to whole k-blocks with zero rows, or past the end of a dense
+            // problem's rows, which the tensor map fills with zeros)
+            t.ft = local / a.n_ntiles;
+            t.b_row = a.b_row_base + tail->seg_off[t.p][t.g];
+            t.n_real = kNTile;
+            t.n = kNTile;
+            t.aux = (local % a.n_ntiles) | (((cnt + kBK - 1) / kBK) << 16);
+            return t;
+        }
+        const int nch = (cnt + kNTile - 1) / kNTile;
         // routed experts: feature tile slow, token chunk fast (a weight tile's
         // chunks are neighbours); dense problems: token chunk slow, feature tile
         // fast (pairs running together cover whole token rows)
@@ -530,8 +673,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         t.b_row = a.b_row_base + tail->seg_off[t.p][t.g] + r0;
         t.n_real = r1 - r0;
         t.n = (t.n_real + 15) & ~15;
-        t.end = 0;
-        t.pad = 0;
+        t.aux = 0;
         return t;
     };
 
@@ -581,14 +723,21 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 if (t.end) break;
                 const PairArgs& a = t.p == 0 ? args0 : args1;
-                // token rows per CTA: N/2, loaded with the box of 16 rb rows
-                const int rb = ((t.n >> 1) + 15) >> 4;
+                // token rows per CTA: N/2, loaded with the box of 16 rb rows (an
+                // MN-major token operand: 128 K rows x 2 blocks of 64 columns)
+                const int rb = KIND == KIND_WGRAD ? 8 : ((t.n >> 1) + 15) >> 4;
                 const CUtensorMap* m = is_a ? &maps.a[t.p] : &maps.b[t.p][rb - 1];
                 const uint32_t op_bytes = is_a ? (uint32_t)kABytes : (uint32_t)rb * 4096u;
                 const int a_row0 = (int)(t.g * a.a_group_stride) + t.ft * a.a_tile_step +
                                    (int)cta * a.a_cta_step;
                 const int b_row0 = t.b_row + (int)cta * (t.n >> 1);
-                const int kb_count = a.K / kBK;
+                // MN-major weights (KIND_DGRAD): rows = K of group g, 64-column
+                // blocks = this CTA's 128 M rows; MN-major activations
+                // (KIND_WGRAD): rows = K from the group's first row
+                const int a_mn_row = KIND == KIND_WGRAD ? t.b_row : (int)(t.g * a.a_group_stride);
+                const int a_mn_blk = (t.ft * a.a_tile_step + (int)cta * a.a_cta_step) >> 6;
+                const int b_mn_blk = ((t.aux & 0xFFFF) * kNTile + (int)cta * (kNTile / 2)) >> 6;
+                const int kb_count = KIND == KIND_WGRAD ? (t.aux >> 16) : a.K / kBK;
                 for (int kb = 0; kb < kb_count; ++kb) {
                     if (!mbar_wait_bounded(&tail->empty[s], ph ^ 1u, abort_flag, status,
                                            SITE_GEMM_PRODUCER, limit)) {
@@ -601,8 +750,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const uint32_t fb = map_to_rank(&tail->full[s], 0);
                     const int atom = kb * kAtoms;
                     if (!is_a) {
-                        // 16 rb token rows x 2 k-atoms (rows past the tile's N/2 unused)
-                        tma_load_3d_pair(sa + kABytes, m, fb, 0, b_row0, atom);
+                        if (KIND == KIND_WGRAD)  // 128 K rows x this CTA's 128 N columns
+                            tma_load_3d_pair(sa + kABytes, m, fb, 0, t.b_row + kb * kBK, b_mn_blk);
+                        else  // 16 rb token rows x 2 k-atoms (rows past the tile's N/2 unused)
+                            tma_load_3d_pair(sa + kABytes, m, fb, 0, b_row0, atom);
+                    } else if (KIND != KIND_FWD) {
+                        // 128 K rows x this CTA's 128 M columns
+                        tma_load_3d_pair(sa, m, fb, 0, a_mn_row + kb * kBK, a_mn_blk);
                     } else if (a.a_mode == 0) {
                         // 128 consecutive weight rows x 2 k-atoms
                         tma_load_3d_pair(sa, m, fb, 0, a_row0, atom);
@@ -632,9 +786,19 @@ __global__ void __launch_bounds__(kThreads, 1)
             // one barrier poll, one block of 4 MMAs and two commits (a single
             // thread issues them, so its instruction count per MMA bounds the rate)
             const uint32_t empty_loc0 = smem_u32(&tail->empty[0]);
-            const uint64_t desc0 = sw128_kmajor_desc(smem_u32(smem));
+            // operand layouts: K-major (k16 steps of 32 B inside 128-byte rows,
+            // 64-deep atoms 16 KiB apart for A) or MN-major (k16 steps of 16
+            // rows x 128 B; 64-column blocks 16 KiB apart)
+            constexpr bool kAMn = KIND != KIND_FWD;
+            constexpr bool kBMn = KIND == KIND_WGRAD;
+            const uint64_t adesc0 = kAMn ? sw128_mnmajor_desc(smem_u32(smem), 16384u)
+                                         : sw128_kmajor_desc(smem_u32(smem));
+            const uint64_t bdesc0 = kBMn ? sw128_mnmajor_desc(smem_u32(smem) + kABytes, 16384u)
+                                         : sw128_kmajor_desc(smem_u32(smem) + kABytes);
+            constexpr uint64_t kAStep = kAMn ? 128 : 2;
+            constexpr uint64_t kBStep = kBMn ? 128 : 2;
+            constexpr uint64_t kAHalf = kAMn ? 4 * 128 : (kAtomBytesA >> 4);
             constexpr uint64_t kStageDesc = kStageBytes >> 4;  // descriptor step per stage
-            constexpr uint64_t kBDesc = kABytes >> 4;          // B tile after A tile
             for (;; ++it) {
                 Tile t;
                 if (!sched_get(tail, it, t, abort_flag, status, SITE_GEMM_MMA, limit)) {
@@ -652,10 +816,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + (uint32_t)(acc * kNTile);
-                const uint32_t idesc = idesc_bf16_f32(2 * kARows, t.n);
-                // the token tile's second k-atom starts 16 rb rows x 128 B after its first
-                const uint64_t b_atom_desc = (uint64_t)(((t.n >> 1) + 15) >> 4) * (2048 >> 4);
-                const int kb_count = a.K / kBK;
+                const uint32_t idesc = idesc_bf16_f32(2 * kARows, t.n, kAMn, kBMn);
+                // the token tile's second k-atom starts 16 rb rows x 128 B after its
+                // first (K-major); MN-major: 4 k16 steps further
+                const uint64_t b_atom_desc =
+                    kBMn ? 4 * 128 : (uint64_t)(((t.n >> 1) + 15) >> 4) * (2048 >> 4);
+                const int kb_count = KIND == KIND_WGRAD ? (t.aux >> 16) : a.K / kBK;
                 uint32_t accum = 0;
                 for (int kb = 0; kb < kb_count; ++kb) {
                     if (!mbar_try_wait(&tail->full[s], ph) &&
@@ -665,11 +831,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                         break;
                     }
                     tc_fence_after();
-                    const uint64_t ad = desc0 + (uint64_t)s * kStageDesc;
+                    const uint64_t ad = adesc0 + (uint64_t)s * kStageDesc;
+                    const uint64_t bd = bdesc0 + (uint64_t)s * kStageDesc;
 #pragma unroll
                     for (int at = 0; at < kAtoms; ++at) {
-                        tc_mma4_pair(d_tmem, ad + (uint64_t)at * (kAtomBytesA >> 4),
-                                     ad + kBDesc + (uint64_t)at * b_atom_desc, idesc, accum);
+                        tc_mma4_pair<kAStep, kBStep>(d_tmem, ad + (uint64_t)at * kAHalf,
+                                                     bd + (uint64_t)at * b_atom_desc, idesc,
+                                                     accum);
                         accum = 1;
                     }
                     // stage s free in both CTAs once these MMAs have read it
@@ -766,19 +934,32 @@ cudaError_t launch_selftest_timeout(int* status, unsigned long long limit_ns, cu
 }
 
 namespace {
-template <class RING>
+template <class RING, int KIND>
 cudaError_t launch_pair_ring(int epi0, int epi1, const PairMaps& maps, const PairArgs& a0,
                              const PairArgs* a1, int n_pairs, cudaStream_t s) {
     using Kern = void (*)(const PairMaps, const PairArgs, const PairArgs, int);
     Kern kern = nullptr;
-    if (epi0 == EPI_SWIGLU && epi1 == EPI_SWIGLU)
-        kern = pair_gemm_kernel<EPI_SWIGLU, EPI_SWIGLU, RING>;
-    else if (epi0 == EPI_STORE_F32 && epi1 == EPI_SCATTER)
-        kern = pair_gemm_kernel<EPI_STORE_F32, EPI_SCATTER, RING>;
-    else if (epi0 == EPI_SCATTER && epi1 == EPI_SCATTER)
-        kern = pair_gemm_kernel<EPI_SCATTER, EPI_SCATTER, RING>;
-    else
-        return cudaErrorInvalidValue;
+    if constexpr (KIND == KIND_FWD) {
+        if (epi0 == EPI_SWIGLU && epi1 == EPI_SWIGLU)
+            kern = pair_gemm_kernel<EPI_SWIGLU, EPI_SWIGLU, RING, KIND>;
+        else if (epi0 == EPI_SWIGLU_SAVE && epi1 == EPI_SWIGLU_SAVE)
+            kern = pair_gemm_kernel<EPI_SWIGLU_SAVE, EPI_SWIGLU_SAVE, RING, KIND>;
+        else if (epi0 == EPI_STORE_F32 && epi1 == EPI_SCATTER)
+            kern = pair_gemm_kernel<EPI_STORE_F32, EPI_SCATTER, RING, KIND>;
+        else if (epi0 == EPI_SCATTER && epi1 == EPI_SCATTER)
+            kern = pair_gemm_kernel<EPI_SCATTER, EPI_SCATTER, RING, KIND>;
+    } else if constexpr (KIND == KIND_DGRAD) {
+        if (epi0 == EPI_DSWIGLU && epi1 == EPI_DSWIGLU)
+            kern = pair_gemm_kernel<EPI_DSWIGLU, EPI_DSWIGLU, RING, KIND>;
+        else if (epi0 == EPI_STORE_F32 && epi1 == EPI_SCATTER)
+            kern = pair_gemm_kernel<EPI_STORE_F32, EPI_SCATTER, RING, KIND>;
+        else if (epi0 == EPI_SCATTER && epi1 == EPI_SCATTER)
+            kern = pair_gemm_kernel<EPI_SCATTER, EPI_SCATTER, RING, KIND>;
+    } else {
+        if (epi0 == EPI_STORE_ROWS && epi1 == EPI_STORE_ROWS)
+            kern = pair_gemm_kernel<EPI_STORE_ROWS, EPI_STORE_ROWS, RING, KIND>;
+    }
+    if (kern == nullptr) return cudaErrorInvalidValue;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)RING::kSmemBytes);
     if (e != cudaSuccess) return e;
@@ -786,17 +967,35 @@ cudaError_t launch_pair_ring(int epi0, int epi1, const PairMaps& maps, const Pai
     return launch_pdl(kern, dim3(2 * n_pairs), dim3(kThreads), RING::kSmemBytes, s, 2, maps, a0,
                       np > 1 ? *a1 : a0, np);
 }
+
+template <int KIND>
+cudaError_t launch_pair_kind(int epi0, int epi1, const PairMaps& maps, const PairArgs& a0,
+                             const PairArgs* a1, int n_pairs, int max_tile_tokens,
+                             cudaStream_t s) {
+    if (max_tile_tokens <= 2 * NarrowRing::kBMaxRows)
+        return launch_pair_ring<NarrowRing, KIND>(epi0, epi1, maps, a0, a1, n_pairs, s);
+    if (max_tile_tokens <= 2 * MidRing::kBMaxRows)
+        return launch_pair_ring<MidRing, KIND>(epi0, epi1, maps, a0, a1, n_pairs, s);
+    return launch_pair_ring<WideRing, KIND>(epi0, epi1, maps, a0, a1, n_pairs, s);
+}
 }  // namespace
 
 cudaError_t launch_pair_gemm(int epi0, int epi1, const PairMaps& maps, const PairArgs& a0,
                              const PairArgs* a1, int n_pairs, int max_tile_tokens,
-                             cudaStream_t s) {
+                             cudaStream_t s, int kind) {
     if (a0.sched_counter == nullptr) return cudaErrorInvalidValue;
-    if (max_tile_tokens <= 2 * NarrowRing::kBMaxRows)
-        return launch_pair_ring<NarrowRing>(epi0, epi1, maps, a0, a1, n_pairs, s);
-    if (max_tile_tokens <= 2 * MidRing::kBMaxRows)
-        return launch_pair_ring<MidRing>(epi0, epi1, maps, a0, a1, n_pairs, s);
-    return launch_pair_ring<WideRing>(epi0, epi1, maps, a0, a1, n_pairs, s);
+    switch (kind) {
+        case KIND_FWD:
+            return launch_pair_kind<KIND_FWD>(epi0, epi1, maps, a0, a1, n_pairs, max_tile_tokens,
+                                              s);
+        case KIND_DGRAD:
+            return launch_pair_kind<KIND_DGRAD>(epi0, epi1, maps, a0, a1, n_pairs,
+                                                max_tile_tokens, s);
+        case KIND_WGRAD:  // tiles are always 256 columns wide
+            return launch_pair_ring<WideRing, KIND_WGRAD>(epi0, epi1, maps, a0, a1, n_pairs, s);
+        default:
+            return cudaErrorInvalidValue;
+    }
 }
 
 }  // namespace moe

@@ -261,12 +261,17 @@ MOE_API int moe_forward(const void* x, const void* W_router, const void* W_gate_
                           stream);
 }
 
-MOE_API int moe_forward_ex(const void* x, const void* W_router, const void* W_gate_up,
-                           const void* W_down, const void* W_shared, int T, int d, int E, int k,
-                           int n_group, int topk_group, int inter, int n_shared, int in_dt,
-                           int out_dt, int gate, const float* expert_bias, void* y,
-                           int32_t* topk_idx_out, float* topk_w_out, int32_t* expert_load,
-                           void* workspace, size_t workspace_bytes, void* stream) {
+}  // extern "C"
+
+namespace {
+// The forward; with `saved` (bf16 layers) the gate/up epilogue also writes the
+// pre-activations the backward reads.
+int forward_impl(const void* x, const void* W_router, const void* W_gate_up, const void* W_down,
+                 const void* W_shared, int T, int d, int E, int k, int n_group, int topk_group,
+                 int inter, int n_shared, int in_dt, int out_dt, int gate,
+                 const float* expert_bias, void* y, int32_t* topk_idx_out, float* topk_w_out,
+                 int32_t* expert_load, void* saved, void* workspace, size_t workspace_bytes,
+                 void* stream) {
     int st = check_sizes(T, d, E, k, inter, n_shared, in_dt);
     if (st != MOE_OK) return st;
     st = check_routing(E, k, n_group, topk_group);
@@ -355,6 +360,13 @@ MOE_API int moe_forward_ex(const void* x, const void* W_router, const void* W_ga
         pr.status = status;
         pr.sched_counter = status + kSchedWordGateUp;
         pr.wait_limit_ns = kWaitLimitNs;
+        const bool train = saved != nullptr;
+        if (train) {  // pre-activations of routed row r go to saved row row_src[r]
+            pr.save = saved;
+            pr.row_src = row_src;
+            pr.feat = inter;
+        }
+        const int epi_gu = train ? EPI_SWIGLU_SAVE : EPI_SWIGLU;
         // problem 1 (routed) goes in slot 1 when there are shared experts, else slot 0
         const int pr_slot = n_shared > 0 ? 1 : 0;
         if (!make_map_gate_up(&mp.a[pr_slot], W_gate_up, (uint64_t)E, inter, d) ||
@@ -369,12 +381,15 @@ MOE_API int moe_forward_ex(const void* x, const void* W_router, const void* W_ga
             ps.out = h_sh;
             ps.out_ld = SI;
             ps.a_blocks_per_group = 2 * SI / 16;
+            ps.row_src = nullptr;  // shared rows are tokens
+            ps.feat = SI;
+            ps.save = train ? static_cast<char*>(saved) + (size_t)T * k * 2 * inter * 2 : nullptr;
             if (!make_map_gate_up(&mp.a[0], Wsh_gu, 1, SI, d) ||
                 !make_token_maps(mp.b[0], x, (uint64_t)T, d))
                 return MOE_ERR_CUDA;
-            e = launch_pair_gemm(EPI_SWIGLU, EPI_SWIGLU, mp, ps, &pr, n_pairs, T, s);
+            e = launch_pair_gemm(epi_gu, epi_gu, mp, ps, &pr, n_pairs, T, s);
         } else {
-            e = launch_pair_gemm(EPI_SWIGLU, EPI_SWIGLU, mp, pr, nullptr, n_pairs, T, s);
+            e = launch_pair_gemm(epi_gu, epi_gu, mp, pr, nullptr, n_pairs, T, s);
         }
         if (e != cudaSuccess) return MOE_ERR_CUDA;
         stage_mark(3, s);
@@ -517,6 +532,48 @@ MOE_API int moe_forward_ex(const void* x, const void* W_router, const void* W_ga
     stage_mark(5, s);
     return MOE_OK;
 }
+}  // namespace
+
+extern "C" {
+
+MOE_API int moe_forward_ex(const void* x, const void* W_router, const void* W_gate_up,
+                           const void* W_down, const void* W_shared, int T, int d, int E, int k,
+                           int n_group, int topk_group, int inter, int n_shared, int in_dt,
+                           int out_dt, int gate, const float* expert_bias, void* y,
+                           int32_t* topk_idx_out, float* topk_w_out, int32_t* expert_load,
+                           void* workspace, size_t workspace_bytes, void* stream) {
+    return forward_impl(x, W_router, W_gate_up, W_down, W_shared, T, d, E, k, n_group,
+                        topk_group, inter, n_shared, in_dt, out_dt, gate, expert_bias, y,
+                        topk_idx_out, topk_w_out, expert_load, nullptr, workspace,
+                        workspace_bytes, stream);
+}
+
+MOE_API size_t moe_saved_bytes(int T, int k, int inter, int n_shared) {
+    if (T < 0 || k < 1 || k > kMaxK || inter <= 0 || n_shared < 0) return 0;
+    return (size_t)2 * 2 * inter * ((size_t)T * k + (size_t)T * n_shared);
+}
+
+MOE_API int moe_forward_train(const void* x, const void* W_router, const void* W_gate_up,
+                              const void* W_down, const void* W_shared, int T, int d, int E,
+                              int k, int n_group, int topk_group, int inter, int n_shared,
+                              int in_dt, int out_dt, int gate, const float* expert_bias,
+                              void* y, int32_t* topk_idx_out, float* topk_w_out,
+                              int32_t* expert_load, void* saved, size_t saved_bytes,
+                              void* workspace, size_t workspace_bytes, void* stream) {
+    int st = check_sizes(T, d, E, k, inter, n_shared, in_dt);
+    if (st != MOE_OK) return st;
+    if (in_dt != MOE_BF16) return MOE_ERR_UNSUPPORTED;
+    if (T > 0) {
+        if (topk_idx_out == nullptr || topk_w_out == nullptr) return MOE_ERR_INVALID_ARG;
+        if (saved == nullptr || !is_device_ptr(saved) || !aligned(saved, 16))
+            return MOE_ERR_INVALID_ARG;
+        if (saved_bytes < moe_saved_bytes(T, k, inter, n_shared)) return MOE_ERR_INVALID_ARG;
+    }
+    return forward_impl(x, W_router, W_gate_up, W_down, W_shared, T, d, E, k, n_group,
+                        topk_group, inter, n_shared, in_dt, out_dt, gate, expert_bias, y,
+                        topk_idx_out, topk_w_out, expert_load, T > 0 ? saved : nullptr,
+                        workspace, workspace_bytes, stream);
+}
 
 MOE_API int moe_set_stage_events(void* const* events, int n) {
     if (events == nullptr) {
@@ -553,6 +610,306 @@ MOE_API int moe_selftest_timeout(void* workspace, int limit_us, void* stream) {
     return ret(launch_selftest_timeout(static_cast<int*>(workspace),
                                        (unsigned long long)limit_us * 1000ull,
                                        static_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"
+
+namespace {
+
+// Workspace of the backward (bf16 layers): regions in this order.
+enum BwdRegion : int {
+    BW_STATUS, BW_COUNTS, BW_OFFSETS, BW_BLOCK_COUNTS, BW_ROW_SRC, BW_SLOT_ROW, BW_X_PERM,
+    BW_DY_PERM, BW_DGU, BW_HW, BW_DW_PART, BW_DL, BW_DX_SLOTS, BW_DGU_SH, BW_HW_SH, BW_DX_SH,
+    BW_TOTAL
+};
+struct BwdLayout {
+    size_t off[BW_TOTAL + 1];
+    int rows_cap;
+};
+
+bool make_bwd_layout(int T, int d, int E, int k, int inter, int n_shared, BwdLayout& L) {
+    if (check_sizes(T, d, E, k, inter, n_shared, MOE_BF16) != MOE_OK) return false;
+    if (d % 256 != 0 || inter % 256 != 0) return false;
+    const size_t Tk = (size_t)T * k, SI = (size_t)n_shared * inter;
+    L.rows_cap = (int)(Tk + (size_t)kRowAlign * E);
+    const size_t rc = (size_t)L.rows_cap;
+    const int nb = (T + kPermBlockTokens - 1) / kPermBlockTokens;
+    const size_t sizes[BW_TOTAL] = {
+        sizeof(int) * kStatusWords,             // STATUS (+ tile counters)
+        sizeof(int) * E,                        // COUNTS
+        sizeof(int) * (E + 1),                  // OFFSETS (segments padded to 128 rows)
+        sizeof(int) * (size_t)(nb > 0 ? nb : 1) * E,  // BLOCK_COUNTS
+        sizeof(int) * rc,                       // ROW_SRC
+        sizeof(int) * Tk,                       // SLOT_ROW: slot -> permuted row
+        2 * rc * d,                             // X_PERM
+        2 * rc * d,                             // DY_PERM
+        2 * rc * 2 * inter,                     // DGU: dg | du per permuted row
+        2 * rc * inter,                         // HW: w * h per permuted row
+        sizeof(float) * rc * (inter / 32),      // DW_PART
+        sizeof(float) * Tk,                     // DL
+        2 * Tk * d,                             // DX_SLOTS (bf16, slot order)
+        2 * (size_t)T * 2 * SI,                 // DGU_SH
+        2 * (size_t)T * SI,                     // HW_SH
+        n_shared > 0 ? sizeof(float) * (size_t)T * d : 0,  // DX_SH
+    };
+    size_t o = 0;
+    for (int i = 0; i < BW_TOTAL; ++i) {
+        L.off[i] = o;
+        o = align_up(o + sizes[i], kRegionAlign);
+    }
+    L.off[BW_TOTAL] = o;
+    return true;
+}
+
+template <typename T>
+T* bat(void* ws, const BwdLayout& L, int region) {
+    return reinterpret_cast<T*>(static_cast<char*>(ws) + L.off[region]);
+}
+
+}  // namespace
+
+extern "C" {
+
+MOE_API size_t moe_backward_workspace_bytes(int T, int d, int E, int k, int inter,
+                                            int n_shared) {
+    BwdLayout L;
+    if (!make_bwd_layout(T, d, E, k, inter, n_shared, L)) return 0;
+    return L.off[BW_TOTAL];
+}
+
+MOE_API int moe_backward(const void* x, const void* W_router, const void* W_gate_up,
+                         const void* W_down, const void* W_shared, const void* dy,
+                         const int32_t* topk_idx, const float* topk_w, const void* saved,
+                         int T, int d, int E, int k, int inter, int n_shared, int in_dt,
+                         int gate, float* dx, float* dW_router, float* dW_gate_up,
+                         float* dW_down, float* dW_shared, void* workspace,
+                         size_t workspace_bytes, void* stream) {
+    int st = check_sizes(T, d, E, k, inter, n_shared, in_dt);
+    if (st != MOE_OK) return st;
+    if (in_dt != MOE_BF16 || d % 256 != 0 || inter % 256 != 0) return MOE_ERR_UNSUPPORTED;
+    if (gate != MOE_GATE_SIGMOID && gate != MOE_GATE_SOFTMAX_TOPK) return MOE_ERR_INVALID_ARG;
+    if ((n_shared > 0) != (W_shared != nullptr) || (n_shared > 0) != (dW_shared != nullptr))
+        return MOE_ERR_INVALID_ARG;
+    BwdLayout L;
+    make_bwd_layout(T, d, E, k, inter, n_shared, L);
+    if (workspace == nullptr || workspace_bytes < L.off[BW_TOTAL]) return MOE_ERR_WORKSPACE;
+    const void* wptrs[] = {W_router, W_gate_up, W_down, dW_router, dW_gate_up, dW_down, workspace};
+    for (const void* p : wptrs)
+        if (!is_device_ptr(p) || !aligned(p, 16)) return MOE_ERR_INVALID_ARG;
+    if (n_shared > 0 && (!is_device_ptr(W_shared) || !aligned(W_shared, 16) ||
+                         !is_device_ptr(dW_shared) || !aligned(dW_shared, 16)))
+        return MOE_ERR_INVALID_ARG;
+    if (!aligned(workspace, 256)) return MOE_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const int SI = n_shared * inter;
+    if (T == 0) {  // no tokens: every weight gradient is zero
+        cudaError_t e = cudaMemsetAsync(dW_router, 0, sizeof(float) * (size_t)E * d, s);
+        if (e == cudaSuccess)
+            e = cudaMemsetAsync(dW_gate_up, 0, sizeof(float) * (size_t)E * 2 * inter * d, s);
+        if (e == cudaSuccess)
+            e = cudaMemsetAsync(dW_down, 0, sizeof(float) * (size_t)E * d * inter, s);
+        if (e == cudaSuccess && n_shared > 0)
+            e = cudaMemsetAsync(dW_shared, 0, sizeof(float) * (size_t)3 * SI * d, s);
+        return ret(e);
+    }
+    const void* tptrs[] = {x, dy, topk_idx, topk_w, saved, dx};
+    for (const void* p : tptrs)
+        if (!is_device_ptr(p) || !aligned(p, 16)) return MOE_ERR_INVALID_ARG;
+
+    int* status = bat<int>(workspace, L, BW_STATUS);
+    int32_t* counts = bat<int32_t>(workspace, L, BW_COUNTS);
+    int32_t* offsets = bat<int32_t>(workspace, L, BW_OFFSETS);
+    int32_t* block_counts = bat<int32_t>(workspace, L, BW_BLOCK_COUNTS);
+    int32_t* row_src = bat<int32_t>(workspace, L, BW_ROW_SRC);
+    int32_t* slot_row = bat<int32_t>(workspace, L, BW_SLOT_ROW);
+    void* x_perm = bat<char>(workspace, L, BW_X_PERM);
+    void* dy_perm = bat<char>(workspace, L, BW_DY_PERM);
+    void* dgu = bat<char>(workspace, L, BW_DGU);
+    void* hw = bat<char>(workspace, L, BW_HW);
+    float* dw_part = bat<float>(workspace, L, BW_DW_PART);
+    float* dl = bat<float>(workspace, L, BW_DL);
+    void* dx_slots = bat<char>(workspace, L, BW_DX_SLOTS);
+    void* dgu_sh = bat<char>(workspace, L, BW_DGU_SH);
+    void* hw_sh = bat<char>(workspace, L, BW_HW_SH);
+    float* dx_sh = n_shared > 0 ? bat<float>(workspace, L, BW_DX_SH) : nullptr;
+    const char* Wsh_gu = static_cast<const char*>(W_shared);
+    const char* Wsh_dn = Wsh_gu != nullptr ? Wsh_gu + (size_t)2 * SI * d * 2 : nullptr;
+    const char* gu_routed = static_cast<const char*>(saved);
+    const char* gu_shared = gu_routed + (size_t)T * k * 2 * inter * 2;
+    const uint64_t rows_cap = (uint64_t)L.rows_cap;
+    const int n_pairs = num_sms() / 2;
+    const int rs = n_shared > 0 ? 1 : 0;  // slot of the routed problem in each launch
+
+    // status word and the four launches' tile counters start at zero
+    cudaError_t e = cudaMemsetAsync(status, 0, sizeof(int) * kStatusWords, s);
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
+    // 1. the forward's permutation again, with segments padded to 128 rows
+    //    (whole k-blocks of the weight-gradient GEMMs), then x / dy rows
+    e = launch_permute(topk_idx, T, k, E, block_counts, counts, offsets, row_src, kRowAlign,
+                       nullptr, status, s);
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
+    e = launch_bwd_gather(x, dy, d, inter, k, offsets + E, row_src, L.rows_cap, x_perm, dy_perm,
+                          dgu, hw, slot_row, num_sms(), s);
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
+
+    PairArgs base{};
+    base.n_groups = E;
+    base.counts = counts;
+    base.seg_align = kRowAlign;
+    base.a_tile_step = 256;
+    base.a_cta_step = 128;
+    base.k = k;
+    base.status = status;
+    base.wait_limit_ns = kWaitLimitNs;
+    auto dense = [&](PairArgs a) {  // the shared experts: one group of T token rows
+        a.counts = nullptr;
+        a.static_rows = T;
+        a.seg_align = 1;
+        a.a_group_stride = 0;
+        a.row_src = nullptr;
+        a.topk_w = nullptr;
+        return a;
+    };
+
+    // 2. dh = W_down^T dy per chosen expert (weights MN-major), SwiGLU backward
+    //    in the epilogue: dg|du, w*h and the parts of dL/dw
+    {
+        PairMaps mp{};
+        PairArgs r = base;
+        r.K = d;
+        r.n_ftiles = inter / 256;
+        r.a_group_stride = d;
+        r.row_src = row_src;
+        r.topk_w = topk_w;
+        r.feat = inter;
+        r.gu_in = gu_routed;
+        r.dgu_out = dgu;
+        r.hw_out = hw;
+        r.dw_part = dw_part;
+        r.sched_counter = status + kSchedWordBwd0;
+        if (!make_map_rows_atoms(&mp.a[rs], W_down, (uint64_t)E * d, inter) ||
+            !make_token_maps(mp.b[rs], dy_perm, rows_cap, d))
+            return MOE_ERR_CUDA;
+        if (n_shared > 0) {
+            PairArgs sh = dense(r);
+            sh.n_ftiles = SI / 256;
+            sh.feat = SI;
+            sh.gu_in = gu_shared;
+            sh.dgu_out = dgu_sh;
+            sh.hw_out = hw_sh;
+            sh.dw_part = nullptr;
+            if (!make_map_rows_atoms(&mp.a[0], Wsh_dn, (uint64_t)d, SI) ||
+                !make_token_maps(mp.b[0], dy, (uint64_t)T, d))
+                return MOE_ERR_CUDA;
+            e = launch_pair_gemm(EPI_DSWIGLU, EPI_DSWIGLU, mp, sh, &r, n_pairs, T, s, KIND_DGRAD);
+        } else {
+            e = launch_pair_gemm(EPI_DSWIGLU, EPI_DSWIGLU, mp, r, nullptr, n_pairs, T, s,
+                                 KIND_DGRAD);
+        }
+        if (e != cudaSuccess) return MOE_ERR_CUDA;
+    }
+    // 3. dL/dlogit of the chosen experts
+    e = launch_router_dlogit(x, W_router, T, d, k, topk_idx, topk_w, dw_part, inter / 32,
+                             slot_row, gate, dl, s);
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
+    // 4. dx parts = W_gate_up^T [dg|du] (weights MN-major): chosen experts into
+    //    token-order slots, shared experts into fp32 rows
+    {
+        PairMaps mp{};
+        PairArgs r = base;
+        r.K = 2 * inter;
+        r.n_ftiles = d / 256;
+        r.a_group_stride = 2LL * inter;
+        r.out = dx_slots;
+        r.out_ld = d;
+        r.out_col_step = 256;
+        r.row_src = row_src;
+        r.topk_w = nullptr;  // weight 1: dg|du already carry w
+        r.sched_counter = status + kSchedWordBwd0 + 1;
+        if (!make_map_rows_atoms(&mp.a[rs], W_gate_up, (uint64_t)E * 2 * inter, d) ||
+            !make_token_maps(mp.b[rs], dgu, rows_cap, 2 * inter))
+            return MOE_ERR_CUDA;
+        if (n_shared > 0) {
+            PairArgs sh = dense(r);
+            sh.K = 2 * SI;
+            sh.out = dx_sh;
+            if (!make_map_rows_atoms(&mp.a[0], Wsh_gu, (uint64_t)2 * SI, d) ||
+                !make_token_maps(mp.b[0], dgu_sh, (uint64_t)T, 2 * SI))
+                return MOE_ERR_CUDA;
+            e = launch_pair_gemm(EPI_STORE_F32, EPI_SCATTER, mp, sh, &r, n_pairs, T, s,
+                                 KIND_DGRAD);
+        } else {
+            e = launch_pair_gemm(EPI_SCATTER, EPI_SCATTER, mp, r, nullptr, n_pairs, T, s,
+                                 KIND_DGRAD);
+        }
+        if (e != cudaSuccess) return MOE_ERR_CUDA;
+    }
+    // 5. dx = shared part + chosen experts' parts + router part (fixed order)
+    e = launch_bwd_combine(dx_sh, dx_slots, dl, topk_idx, W_router, T, d, k, dx, s);
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
+    // 6. dW_down = (w dy)^T h per expert: both operands MN-major, K = the
+    //    expert's rows
+    {
+        PairMaps mp{};
+        PairArgs r = base;
+        r.n_ftiles = d / 256;
+        r.n_ntiles = inter / 256;
+        r.m_total = d;
+        r.out = dW_down;
+        r.out_ld = inter;
+        r.sched_counter = status + kSchedWordBwd0 + 2;
+        if (!make_map_rows_atoms(&mp.a[rs], dy_perm, rows_cap, d) ||
+            !make_map_rows_atoms(&mp.b[rs][kTokenBoxes - 1], hw, rows_cap, inter))
+            return MOE_ERR_CUDA;
+        if (n_shared > 0) {
+            PairArgs sh = dense(r);
+            sh.n_ntiles = SI / 256;
+            sh.out = const_cast<char*>(reinterpret_cast<const char*>(dW_shared)) +
+                     sizeof(float) * (size_t)2 * SI * d;
+            sh.out_ld = SI;
+            if (!make_map_rows_atoms(&mp.a[0], dy, (uint64_t)T, d) ||
+                !make_map_rows_atoms(&mp.b[0][kTokenBoxes - 1], hw_sh, (uint64_t)T, SI))
+                return MOE_ERR_CUDA;
+            e = launch_pair_gemm(EPI_STORE_ROWS, EPI_STORE_ROWS, mp, sh, &r, n_pairs, 256, s,
+                                 KIND_WGRAD);
+        } else {
+            e = launch_pair_gemm(EPI_STORE_ROWS, EPI_STORE_ROWS, mp, r, nullptr, n_pairs, 256, s,
+                                 KIND_WGRAD);
+        }
+        if (e != cudaSuccess) return MOE_ERR_CUDA;
+    }
+    // 7. dW_gate_up = [dg|du]^T x per expert
+    {
+        PairMaps mp{};
+        PairArgs r = base;
+        r.n_ftiles = 2 * inter / 256;
+        r.n_ntiles = d / 256;
+        r.m_total = 2 * inter;
+        r.out = dW_gate_up;
+        r.out_ld = d;
+        r.sched_counter = status + kSchedWordBwd0 + 3;
+        if (!make_map_rows_atoms(&mp.a[rs], dgu, rows_cap, 2 * inter) ||
+            !make_map_rows_atoms(&mp.b[rs][kTokenBoxes - 1], x_perm, rows_cap, d))
+            return MOE_ERR_CUDA;
+        if (n_shared > 0) {
+            PairArgs sh = dense(r);
+            sh.n_ftiles = 2 * SI / 256;
+            sh.m_total = 2 * SI;
+            sh.out = dW_shared;
+            if (!make_map_rows_atoms(&mp.a[0], dgu_sh, (uint64_t)T, 2 * SI) ||
+                !make_map_rows_atoms(&mp.b[0][kTokenBoxes - 1], x, (uint64_t)T, d))
+                return MOE_ERR_CUDA;
+            e = launch_pair_gemm(EPI_STORE_ROWS, EPI_STORE_ROWS, mp, sh, &r, n_pairs, 256, s,
+                                 KIND_WGRAD);
+        } else {
+            e = launch_pair_gemm(EPI_STORE_ROWS, EPI_STORE_ROWS, mp, r, nullptr, n_pairs, 256, s,
+                                 KIND_WGRAD);
+        }
+        if (e != cudaSuccess) return MOE_ERR_CUDA;
+    }
+    // 8. dW_router[e] = sum of dl * x over expert e's rows
+    e = launch_router_dweight(dl, row_src, offsets, x_perm, E, d, dW_router, s);
+    return ret(e);
 }
 
 }  // extern "C"

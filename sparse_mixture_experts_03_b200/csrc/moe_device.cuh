@@ -169,12 +169,27 @@ __device__ __forceinline__ uint64_t sw128_kmajor_desc(uint32_t smem_addr) {
            ((uint64_t)(1024u >> 4) << 32) | ((uint64_t)1u << 46) | ((uint64_t)2u << 61);
 }
 
-// Instruction descriptor for kind::f16: fp32 accumulator, bf16 A and B, both
-// K-major, M x N.  Fields: D format [4,6) = 1 (F32), A format [7,10) = 1
-// (BF16), B format [10,13) = 1 (BF16), N >> 3 in [17,23), M >> 4 in [24,29).
-__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
-    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) |
-           ((uint32_t)(M >> 4) << 24);
+// Shared-memory matrix descriptor of an MN-major tile written by TMA with
+// 128-byte swizzle as [mn block of 64][k row][64 elements]: 64 consecutive
+// M (or N) elements per 128-byte row, k rows 128 B apart, 8-row swizzle atoms.
+// Leading byte offset = the distance between the 64-element MN blocks
+// (mn_block_bytes), stride byte offset = the distance between 8-row k groups
+// (1024 B); same version and layout fields as the K-major descriptor.
+__device__ __forceinline__ uint64_t sw128_mnmajor_desc(uint32_t smem_addr,
+                                                       uint32_t mn_block_bytes) {
+    return (uint64_t)((smem_addr >> 4) & 0x3FFFu) |
+           ((uint64_t)((mn_block_bytes >> 4) & 0x3FFFu) << 16) |
+           ((uint64_t)(1024u >> 4) << 32) | ((uint64_t)1u << 46) | ((uint64_t)2u << 61);
+}
+
+// Instruction descriptor for kind::f16: fp32 accumulator, bf16 A and B, M x N.
+// Fields: D format [4,6) = 1 (F32), A format [7,10) = 1 (BF16), B format
+// [10,13) = 1 (BF16), A major [15] and B major [16] (0 K-major, 1 MN-major),
+// N >> 3 in [17,23), M >> 4 in [24,29).
+__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn = false,
+                                                      bool b_mn = false) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((a_mn ? 1u : 0u) << 15) |
+           ((b_mn ? 1u : 0u) << 16) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
 }  // namespace moe

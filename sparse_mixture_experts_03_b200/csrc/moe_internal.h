@@ -52,6 +52,9 @@ constexpr int kStatusWords = 64;       // int32 words of the status region of th
 // (reset to 0, with words 0..15, by the routing kernel at the start of a forward)
 constexpr int kSchedWordGateUp = 12;
 constexpr int kSchedWordDown = 13;
+// the backward's four CTA-pair launches (the backward clears the whole status
+// region first)
+constexpr int kSchedWordBwd0 = 20;
 
 // Epilogue variants of the grouped GEMMs.
 enum Epi : int {
@@ -60,6 +63,18 @@ enum Epi : int {
                         // skipped (bf16 slots on the CTA-pair kernel, f32 on CUDA cores)
     EPI_COMBINE = 2,    // y[t] = acc + slots[t*k + 0] + ... + slots[t*k + k-1] (CUDA cores)
     EPI_STORE_F32 = 3,  // out[row] = acc, fp32 (CTA-pair kernel)
+    // training (CTA-pair kernel)
+    EPI_SWIGLU_SAVE = 4,   // SWIGLU, and the pre-activations gate|up (bf16) to save rows
+    EPI_DSWIGLU = 5,       // SwiGLU backward of dh = acc (see PairArgs)
+    EPI_STORE_ROWS = 6,    // weight-gradient tile: out[weight row][col] = acc, fp32
+};
+
+// Operand layouts and tile shapes of a CTA-pair launch.
+enum PairKind : int {
+    KIND_FWD = 0,    // A (weights) K-major, B (tokens) K-major; tiles: feature tile x token chunk
+    KIND_DGRAD = 1,  // A (weights) MN-major (their transpose is the operand), B K-major
+    KIND_WGRAD = 2,  // A and B MN-major (activation rows are K); tiles: M tile x N tile,
+                     // K = the group's rows (0 rows: a tile of zeros)
 };
 
 // CUDA-core (fp32 layers) grouped GEMM  out[r, n] = sum_c A[r, c] * B[b_row(r, n), c]  over row
@@ -152,6 +167,22 @@ struct PairArgs {
     int* status;
     int* sched_counter;      // problem 0's: tile tickets of the launch, 0 at launch
     unsigned long long wait_limit_ns;
+    // ---- training
+    int seg_align;           // group segments of B start at multiples of this (0 or 1: packed)
+    int n_ntiles;            // KIND_WGRAD: 256-wide tiles along N
+    int m_total;             // STORE_ROWS: output rows per group (n_ftiles * 256)
+    void* save;              // SWIGLU_SAVE: gate|up pre-activations, bf16 rows of 2F, row =
+                             // row_src[r] (routed) or the token (row_src == nullptr)
+    int feat;                // F: SwiGLU features of the problem (inter, or n_shared * inter)
+    // DSWIGLU: acc = dh_raw [feature, row] = (W_down^T dy)[row]; w = topk_w[row_src[r]] (1 when
+    // row_src == nullptr); reads gate|up of row_src[r] (or r) from gu_in [*, 2F] bf16, writes
+    // dgu_out[r] = (dh * u * silu'(g) | dh * silu(g)) [2F] bf16, hw_out[r] = w * silu(g) * u [F]
+    // bf16 and, with dw_part, dw_part[r * (F / 32) + part] = sum over the warp's 32 features of
+    // dh_raw * silu(g) * u.
+    const void* gu_in;
+    void* dgu_out;
+    void* hw_out;
+    float* dw_part;
 };
 // Tensor maps of one launch.  Each stage covers 128 of K (two 64-column
 // swizzle atoms).  a[p]: weights of problem p, a_mode 0: box {64, 128, 2};
@@ -164,13 +195,40 @@ struct PairMaps {
     CUtensorMap b[2][kTokenBoxes];
 };
 // Epilogue pairs (epi0 for problem 0, epi1 for problem 1): SWIGLU/SWIGLU,
-// STORE_F32/SCATTER, SCATTER/SCATTER.  a1 == nullptr: one problem.
+// STORE_F32/SCATTER, SCATTER/SCATTER, SWIGLU_SAVE/SWIGLU_SAVE (KIND_FWD);
+// DSWIGLU/DSWIGLU, STORE_F32/SCATTER, SCATTER/SCATTER (KIND_DGRAD);
+// STORE_ROWS/STORE_ROWS (KIND_WGRAD).  a1 == nullptr: one problem.
 // max_tile_tokens: an upper bound on the tokens of any tile (the batch size,
 // capped at 256); up to 128 (and again up to 64) the launch uses a deeper ring
 // of smaller stages.
 cudaError_t launch_pair_gemm(int epi0, int epi1, const PairMaps& maps, const PairArgs& a0,
                              const PairArgs* a1, int n_pairs, int max_tile_tokens,
-                             cudaStream_t s);
+                             cudaStream_t s, int kind = KIND_FWD);
+
+// ---- backward helpers (backward.cu)
+// For every row r of the padded permuted layout (rows [0, offsets_total)):
+// row_src[r] >= 0: x_perm[r] = x[t], dy_perm[r] = dy[t] (t = row_src[r] / k)
+// and slot_row[row_src[r]] = r; padding rows: x_perm, dy_perm, dgu [2F] and
+// hw [F] rows set to zero.  bf16.
+cudaError_t launch_bwd_gather(const void* x, const void* dy, int d, int F, int k,
+                              const int32_t* offsets_total, const int32_t* row_src, int rows_cap,
+                              void* x_perm, void* dy_perm, void* dgu, void* hw,
+                              int32_t* slot_row, int num_sms, cudaStream_t s);
+// dl[t*k + j] = dL/dlogit of token t's chosen expert j (gate MOE_GATE_*), from
+// dw = sum of the dw_part row of its slot, topk_w and the recomputed logits.
+cudaError_t launch_router_dlogit(const void* x, const void* Wr, int T, int d, int k,
+                                 const int32_t* idx, const float* topk_w, const float* dw_part,
+                                 int n_parts, const int32_t* slot_row, int gate, float* dl,
+                                 cudaStream_t s);
+// dx[t] = base[t] (fp32, nullable) + slots[t*k+0..k-1] (bf16) + sum_j dl[t*k+j] Wr[idx[t*k+j]],
+// in that order, fp32.
+cudaError_t launch_bwd_combine(const float* base, const void* slots, const float* dl,
+                               const int32_t* idx, const void* Wr, int T, int d, int k, float* dx,
+                               cudaStream_t s);
+// dWr[e] = sum over rows r of expert e's padded segment with row_src[r] >= 0 of
+// dl[row_src[r]] * x_perm[r], in row order, fp32.
+cudaError_t launch_router_dweight(const float* dl, const int32_t* row_src, const int32_t* offsets,
+                                  const void* x_perm, int E, int d, float* dWr, cudaStream_t s);
 
 cudaError_t launch_selftest_timeout(int* status, unsigned long long limit_ns, cudaStream_t s);
 

@@ -13,7 +13,8 @@ that projection (d for gate/up, inter for down; each shared expert is its own
 expert of inter I, so its down projection uses 1/I).
 
 Random streams: each tensor has a fixed stream id (x 0, W_router 1, W_gate_up
-2, W_down 3, shared gate_up 4, shared down 5, skew direction u 6) and is filled
+2, W_down 3, shared gate_up 4, shared down 5, skew direction u 6, upstream
+gradient dy of the backward 7) and is filled
 in chunks of 2**24 elements; chunk c of stream i is drawn by torch.randn from a
 CPU torch.Generator seeded with the 32-bit value (seed << 24) | (i << 16) | c
 (the CPU generator keeps only 32 bits of a seed, so the fields are packed into
@@ -163,3 +164,9 @@ def shared_views(W_shared: torch.Tensor, d: int, inter: int, n_shared: int):
     gu = W_shared[: 2 * SI * d].view(2 * SI, d)
     dn = W_shared[2 * SI * d: 2 * SI * d + d * SI].view(d, SI)
     return gu, dn
+
+
+def make_dy(w: Workload) -> torch.Tensor:
+    """Upstream gradient dL/dy [T, d] for the backward: N(0, 1), in the
+    workload's dtype (stream 7 of the workload's seed)."""
+    return _randn((w.T, w.d), w.seed, 7).to(torch_dtype(w.dtype)).contiguous()

@@ -35,7 +35,8 @@ ROW_ALIGN = 128
 SYMBOLS = ["moe_workspace_bytes", "moe_workspace_layout", "moe_route", "moe_forward",
            "moe_get_device_status", "moe_clear_device_status", "moe_selftest_timeout",
            "moe_set_stage_events", "moe_status_string", "moe_version",
-           "moe_expert_counts_noalloc", "moe_route_ex", "moe_forward_ex"]
+           "moe_expert_counts_noalloc", "moe_route_ex", "moe_forward_ex", "moe_saved_bytes",
+           "moe_forward_train", "moe_backward_workspace_bytes", "moe_backward"]
 GATES = {"sigmoid": 0, "softmax": 1}  # MOE_GATE_SIGMOID, MOE_GATE_SOFTMAX_TOPK
 N_STAGE_EVENTS = 6
 STAGES = ["route", "permute", "gate_up", "down", "combine"]
@@ -83,6 +84,15 @@ def lib() -> ctypes.CDLL:
         L.moe_route_ex.restype = i
         L.moe_forward_ex.argtypes = [vp] * 5 + [i] * 11 + [vp, vp, vp, vp, vp, vp, sz, vp]
         L.moe_forward_ex.restype = i
+        L.moe_saved_bytes.argtypes = [i] * 4
+        L.moe_saved_bytes.restype = sz
+        L.moe_forward_train.argtypes = ([vp] * 5 + [i] * 11 + [vp, vp, vp, vp, vp, vp, sz, vp, sz,
+                                                               vp])
+        L.moe_forward_train.restype = i
+        L.moe_backward_workspace_bytes.argtypes = [i] * 6
+        L.moe_backward_workspace_bytes.restype = sz
+        L.moe_backward.argtypes = [vp] * 9 + [i] * 8 + [vp] * 6 + [sz, vp]
+        L.moe_backward.restype = i
         _lib = L
     return _lib
 
@@ -191,6 +201,92 @@ def forward(x: torch.Tensor, W_router: torch.Tensor, W_gate_up: torch.Tensor,
                               _ptr(workspace), workspace.numel(), _stream(stream))
     _check(st, "moe_forward_ex")
     return y
+
+
+def saved_bytes(T, k, inter, n_shared) -> int:
+    """Bytes of the pre-activations moe_forward_train saves for the backward."""
+    return int(lib().moe_saved_bytes(T, k, inter, n_shared))
+
+
+def forward_train(x: torch.Tensor, W_router: torch.Tensor, W_gate_up: torch.Tensor,
+                  W_down: torch.Tensor, W_shared: Optional[torch.Tensor], k: int, n_group: int,
+                  topk_group: int, inter: int, n_shared: int,
+                  out_dtype: torch.dtype = torch.float32, y: Optional[torch.Tensor] = None,
+                  topk_idx: Optional[torch.Tensor] = None, topk_w: Optional[torch.Tensor] = None,
+                  saved: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                  stream=None, gate: str = "sigmoid", expert_bias: Optional[torch.Tensor] = None,
+                  expert_load: Optional[torch.Tensor] = None):
+    """moe_forward_train: (y, topk_idx, topk_w, saved) -- the forward plus the
+    routing and pre-activations that backward() takes."""
+    T, d = x.shape
+    E = W_router.shape[0]
+    dev = x.device
+    if y is None:
+        y = torch.empty(T, d, dtype=out_dtype, device=dev)
+    if topk_idx is None:
+        topk_idx = torch.empty(T, k, dtype=torch.int32, device=dev)
+    if topk_w is None:
+        topk_w = torch.empty(T, k, dtype=torch.float32, device=dev)
+    if saved is None:
+        saved = torch.empty(max(saved_bytes(T, k, inter, n_shared), 16), dtype=torch.uint8,
+                            device=dev)
+    if workspace is None:
+        workspace = alloc_workspace(T, d, E, k, inter, n_shared, x.dtype, dev)
+    st = lib().moe_forward_train(_ptr(x), _ptr(W_router), _ptr(W_gate_up), _ptr(W_down),
+                                 _ptr(W_shared), T, d, E, k, n_group, topk_group, inter, n_shared,
+                                 _dt(x), _dt(y), GATES[gate], _ptr(expert_bias), _ptr(y),
+                                 _ptr(topk_idx), _ptr(topk_w), _ptr(expert_load), _ptr(saved),
+                                 saved.numel(), _ptr(workspace), workspace.numel(),
+                                 _stream(stream))
+    _check(st, "moe_forward_train")
+    return y, topk_idx, topk_w, saved
+
+
+def backward_workspace_bytes(T, d, E, k, inter, n_shared) -> int:
+    n = lib().moe_backward_workspace_bytes(T, d, E, k, inter, n_shared)
+    if n == 0:
+        raise MoeError(MOE_ERR_UNSUPPORTED, "moe_backward_workspace_bytes")
+    return int(n)
+
+
+class Grads:
+    """fp32 gradients of the layer: dx [T,d], dW_router [E,d], dW_gate_up
+    [E,2I,d], dW_down [E,d,I], dW_shared [3*SI*d] or None."""
+
+    def __init__(self, dx, dW_router, dW_gate_up, dW_down, dW_shared):
+        self.dx, self.dW_router, self.dW_gate_up = dx, dW_router, dW_gate_up
+        self.dW_down, self.dW_shared = dW_down, dW_shared
+
+
+def alloc_grads(T, d, E, inter, n_shared, device="cuda") -> Grads:
+    f = dict(dtype=torch.float32, device=device)
+    SI = n_shared * inter
+    return Grads(torch.empty(T, d, **f), torch.empty(E, d, **f), torch.empty(E, 2 * inter, d, **f),
+                 torch.empty(E, d, inter, **f), torch.empty(3 * SI * d, **f) if n_shared else None)
+
+
+def backward(x: torch.Tensor, W_router: torch.Tensor, W_gate_up: torch.Tensor,
+             W_down: torch.Tensor, W_shared: Optional[torch.Tensor], dy: torch.Tensor,
+             topk_idx: torch.Tensor, topk_w: torch.Tensor, saved: torch.Tensor, k: int,
+             inter: int, n_shared: int, gate: str = "sigmoid", grads: Optional[Grads] = None,
+             workspace: Optional[torch.Tensor] = None, stream=None) -> Grads:
+    """moe_backward: gradients of the layer for the forward_train call that
+    returned topk_idx, topk_w and saved; dy = dL/dy in the dtype of x."""
+    T, d = x.shape
+    E = W_router.shape[0]
+    if grads is None:
+        grads = alloc_grads(T, d, E, inter, n_shared, x.device)
+    if workspace is None:
+        workspace = torch.empty(backward_workspace_bytes(T, d, E, k, inter, n_shared),
+                                dtype=torch.uint8, device=x.device)
+    st = lib().moe_backward(_ptr(x), _ptr(W_router), _ptr(W_gate_up), _ptr(W_down),
+                            _ptr(W_shared), _ptr(dy), _ptr(topk_idx), _ptr(topk_w), _ptr(saved),
+                            T, d, E, k, inter, n_shared, _dt(x), GATES[gate], _ptr(grads.dx),
+                            _ptr(grads.dW_router), _ptr(grads.dW_gate_up), _ptr(grads.dW_down),
+                            _ptr(grads.dW_shared), _ptr(workspace), workspace.numel(),
+                            _stream(stream))
+    _check(st, "moe_backward")
+    return grads
 
 
 def device_status(workspace: torch.Tensor, stream=None) -> Tuple[int, int]:
