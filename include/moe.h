@@ -338,6 +338,19 @@ MOE_API int moe_backward(const void *x, const void *W_router, const void *W_gate
                          float *dW_down, float *dW_shared, void *workspace,
                          size_t workspace_bytes, void *stream);
 
+/*
+ * moe_set_backward_stage_events -- the instrumentation of moe_set_stage_events
+ * for moe_backward: with n == MOE_N_BWD_STAGE_EVENTS cudaEvent_t handles,
+ * every following moe_backward records events[i]: [0] start, [1] after the
+ * permutation and row gather, [2] after dh = W_down^T dy with the SwiGLU
+ * backward, [3] after dL/dlogit, [4] after the dx parts W_gate_up^T [dg|du],
+ * [5] after the dx sum, [6] after dW_down, [7] after dW_gate_up, [8] at the end
+ * (after dW_router).  NULL entries are skipped; events == NULL turns it off.
+ * Process-wide, not thread-safe.  Returns MOE_OK or MOE_ERR_INVALID_ARG.
+ */
+#define MOE_N_BWD_STAGE_EVENTS 9
+MOE_API int moe_set_backward_stage_events(void *const *events, int n);
+
 /* moe_status_string -- static text for a status code. */
 MOE_API const char *moe_status_string(int status);
 

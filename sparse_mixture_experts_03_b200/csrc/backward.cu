@@ -194,7 +194,8 @@ __global__ void __launch_bounds__(256)
 }
 
 // Block (e, column chunk of 512): 2 columns per thread, rows of expert e's
-// segment in order.
+// segment in order; 8 rows' loads are in flight at a time (the sum still runs
+// row by row).
 __global__ void __launch_bounds__(256)
     router_dweight_kernel(const float* __restrict__ dl, const int32_t* __restrict__ row_src,
                           const int32_t* __restrict__ offsets, const __nv_bfloat162* __restrict__ xp,
@@ -206,13 +207,22 @@ __global__ void __launch_bounds__(256)
     if (c2 < d2) {
         const int r0 = offsets[e], r1 = offsets[e + 1];
         float a0 = 0.f, a1 = 0.f;
-        for (int r = r0; r < r1; ++r) {
-            const int src = row_src[r];
-            if (src < 0) continue;
-            const float g = dl[src];
-            const float2 v = __bfloat1622float2(xp[(size_t)r * d2 + c2]);
-            a0 = fmaf(g, v.x, a0);
-            a1 = fmaf(g, v.y, a1);
+        for (int rb = r0; rb < r1; rb += 8) {
+            float g[8];
+            __nv_bfloat162 v[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int r = rb + u;
+                const int src = r < r1 ? __ldg(row_src + r) : -1;
+                g[u] = src >= 0 ? __ldg(dl + src) : 0.f;
+                v[u] = src >= 0 ? xp[(size_t)r * d2 + c2] : __floats2bfloat162_rn(0.f, 0.f);
+            }
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const float2 f = __bfloat1622float2(v[u]);
+                a0 = fmaf(g[u], f.x, a0);
+                a1 = fmaf(g[u], f.y, a1);
+            }
         }
         reinterpret_cast<float2*>(dWr + (size_t)e * d)[c2] = make_float2(a0, a1);
     }

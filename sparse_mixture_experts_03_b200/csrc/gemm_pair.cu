@@ -298,6 +298,14 @@ __device__ __forceinline__ int upper_group(const int* off, int n, int v) {
     return lo;
 }
 
+// tanh by the hardware approximation (relative error about 2^-11, below the
+// bf16 rounding of the values it feeds)
+__device__ __forceinline__ float tanh_approx(float x) {
+    float y;
+    asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 __device__ __forceinline__ float silu_mul(float g, float u) {
     return __fdividef(g, 1.0f + __expf(-g)) * u;
 }
@@ -310,6 +318,166 @@ __device__ __forceinline__ uint8_t* stage_chunk(uint8_t* wb, int row, int chunk)
     return wb + row * 128 + ((chunk ^ (row & 7)) << 4);
 }
 
+// SwiGLU backward epilogue (EPI_DSWIGLU) of one tile for warp quarter wq.
+// fp32 transpose (token row i: its 32 features), then lane = token row r:
+// dh_raw of features f0 .. f0 + 31 (the warp's TMEM lanes), the saved gate /
+// up pre-activations of the row's slot, and per feature
+//   h = silu(g) u,  dh = w dh_raw,  dg = dh u silu'(g),  du = dh silu(g),
+//   hw = w h,  with silu'(g) = sigmoid(g) (1 + g (1 - sigmoid(g)));
+// the sum of dh_raw h over the 32 features is this warp's part of dL/dw.
+// The chunk loop stays rolled (its body is large: unrolled it would crowd
+// the instruction cache that the producer and MMA warps share), and the
+// global reads run ahead of it: the slot of each row two chunks ahead, its
+// gate weight and pre-activations one chunk ahead.
+struct DswigluRow {
+    int src;
+    float w;
+    uint4 g[4], u[4];
+};
+
+__device__ __forceinline__ int dswiglu_src(const Tile& t, const PairArgs& a, int c0, int lane) {
+    const int r = t.b_row + c0 + lane;
+    if (c0 + lane >= t.n_real) return -1;
+    return a.row_src != nullptr ? a.row_src[r] : r;
+}
+
+__device__ __forceinline__ void dswiglu_fetch(const PairArgs& a, int src, int f0,
+                                              DswigluRow& row) {
+    row.src = src;
+    row.w = 1.f;
+    if (src < 0) return;
+    if (a.row_src != nullptr) row.w = a.topk_w[src];
+    const uint4* gp = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.gu_in) +
+                                                     (size_t)src * 2 * a.feat + f0);
+    const uint4* up = gp + (a.feat >> 3);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        row.g[q] = __ldg(gp + q);
+        row.u[q] = __ldg(up + q);
+    }
+}
+
+__device__ __forceinline__ void dswiglu_epilogue(uint8_t* wb, uint32_t taddr, const Tile& t,
+                                                 const PairArgs& a, uint32_t cta, int wq,
+                                                 int lane) {
+    const int F = a.feat;
+    const int f0 = t.ft * 256 + (int)cta * 128 + wq * 32;
+    DswigluRow cur;
+    dswiglu_fetch(a, dswiglu_src(t, a, 0, lane), f0, cur);
+    int src_next = dswiglu_src(t, a, 32, lane);
+#pragma unroll 1
+    for (int cc = 0; cc < kNTile / 32; ++cc) {
+        const int c0 = 32 * cc;
+        if (c0 >= t.n) break;
+        uint32_t v[32];
+        tmem_ld32(taddr + (uint32_t)c0, v);
+        // the next chunk's reads go out before this chunk's work
+        DswigluRow nxt;
+        dswiglu_fetch(a, c0 + 32 < t.n ? src_next : -1, f0, nxt);
+        src_next = c0 + 64 < t.n ? dswiglu_src(t, a, c0 + 64, lane) : -1;
+        tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+            float* rowp = reinterpret_cast<float*>(stage_chunk(wb, i, lane >> 2));
+            rowp[lane & 3] = __uint_as_float(v[i]);
+        }
+        __syncwarp();
+        // per lane (= its staged row): dg, du and w h of 32 features.  dg of
+        // features 8 qq .. 8 qq + 7 goes back into the lane's own staged row at
+        // chunk qq (dh_raw chunks 2 qq, 2 qq + 1 already read), du and w h stay
+        // in registers; the rows then leave through the buffer, 4 rows x 128 B
+        // (dg | du) and 8 rows x 64 B (w h) per store instruction.
+        uint32_t pdu[16], phw[16];
+        float part = 0.f;
+        if (cur.src >= 0) {
+            const float wv = cur.w;
+            const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(cur.g);
+            const __nv_bfloat162* u2 = reinterpret_cast<const __nv_bfloat162*>(cur.u);
+#pragma unroll
+            for (int qq = 0; qq < 4; ++qq) {
+                uint32_t pdg[4];
+#pragma unroll
+                for (int hq = 0; hq < 2; ++hq) {
+                    const int q = 2 * qq + hq;
+                    const float4 c4 = *reinterpret_cast<const float4*>(stage_chunk(wb, lane, q));
+                    const float dr[4] = {c4.x, c4.y, c4.z, c4.w};
+                    float odg[4], odu[4], ohw[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 gg = __bfloat1622float2(g2[(4 * q + e) >> 1]);
+                        const float2 uu = __bfloat1622float2(u2[(4 * q + e) >> 1]);
+                        const float g = (e & 1) ? gg.y : gg.x;
+                        const float u = (e & 1) ? uu.y : uu.x;
+                        // sigmoid(g) = (1 + tanh(g / 2)) / 2: one hardware tanh
+                        const float sg = fmaf(0.5f, tanh_approx(0.5f * g), 0.5f);
+                        const float silu = g * sg;
+                        const float h = silu * u;
+                        part = fmaf(dr[e], h, part);
+                        const float dh = wv * dr[e];
+                        // silu'(g) = sigmoid(g) (1 + g (1 - sigmoid(g)))
+                        odg[e] = dh * u * fmaf(silu, 1.0f - sg, sg);
+                        odu[e] = dh * silu;
+                        ohw[e] = wv * h;
+                    }
+                    pdg[2 * hq] = pack_bf16x2(odg[0], odg[1]);
+                    pdg[2 * hq + 1] = pack_bf16x2(odg[2], odg[3]);
+                    pdu[4 * qq + 2 * hq] = pack_bf16x2(odu[0], odu[1]);
+                    pdu[4 * qq + 2 * hq + 1] = pack_bf16x2(odu[2], odu[3]);
+                    phw[4 * qq + 2 * hq] = pack_bf16x2(ohw[0], ohw[1]);
+                    phw[4 * qq + 2 * hq + 1] = pack_bf16x2(ohw[2], ohw[3]);
+                }
+                *reinterpret_cast<uint4*>(stage_chunk(wb, lane, qq)) =
+                    make_uint4(pdg[0], pdg[1], pdg[2], pdg[3]);
+            }
+#pragma unroll
+            for (int qq = 0; qq < 4; ++qq)
+                *reinterpret_cast<uint4*>(stage_chunk(wb, lane, 4 + qq)) =
+                    make_uint4(pdu[4 * qq], pdu[4 * qq + 1], pdu[4 * qq + 2], pdu[4 * qq + 3]);
+            if (a.dw_part != nullptr)
+                a.dw_part[(size_t)(t.b_row + c0 + lane) * (F >> 5) + (f0 >> 5)] = part;
+        }
+        __syncwarp();
+        {
+            // dg | du: row i = 4 it + lane / 8, 16-byte piece lane % 8
+            const int q = lane & 7;
+#pragma unroll
+            for (int it = 0; it < 8; ++it) {
+                const int i = 4 * it + (lane >> 3);
+                if (c0 + i < t.n_real) {
+                    const uint4 v4 = *reinterpret_cast<const uint4*>(stage_chunk(wb, i, q));
+                    __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(a.dgu_out) +
+                                         (size_t)(t.b_row + c0 + i) * 2 * F + f0 +
+                                         (q < 4 ? q * 8 : F + (q - 4) * 8);
+                    *reinterpret_cast<uint4*>(dst) = v4;
+                }
+            }
+        }
+        __syncwarp();
+        if (cur.src >= 0) {
+#pragma unroll
+            for (int qq = 0; qq < 4; ++qq)
+                *reinterpret_cast<uint4*>(stage_chunk(wb, lane, qq)) =
+                    make_uint4(phw[4 * qq], phw[4 * qq + 1], phw[4 * qq + 2], phw[4 * qq + 3]);
+        }
+        __syncwarp();
+        {
+            // w h: row i = 8 it + lane / 4, 16-byte piece lane % 4
+            const int q = lane & 3;
+#pragma unroll
+            for (int it = 0; it < 4; ++it) {
+                const int i = 8 * it + (lane >> 2);
+                if (c0 + i < t.n_real) {
+                    const uint4 v4 = *reinterpret_cast<const uint4*>(stage_chunk(wb, i, q));
+                    *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.hw_out) +
+                                              (size_t)(t.b_row + c0 + i) * F + f0 + q * 8) = v4;
+                }
+            }
+        }
+        __syncwarp();
+        cur = nxt;
+    }
+}
+
 // Epilogue of one tile for warp quarter wq of this CTA: TMEM lanes 32 wq ..
 // 32 wq + 31 (weight rows) x the tile's N token columns.  Each warp works on
 // its own: tcgen05.ld of 32 columns (thread = weight row, registers = tokens),
@@ -317,6 +485,10 @@ __device__ __forceinline__ uint8_t* stage_chunk(uint8_t* wb, int row, int chunk)
 template <int EPI>
 __device__ __forceinline__ void pair_epilogue(uint8_t* wb, uint32_t taddr, const Tile& t,
                                               const PairArgs& a, uint32_t cta, int wq, int lane) {
+    if constexpr (EPI == EPI_DSWIGLU) {
+        dswiglu_epilogue(wb, taddr, t, a, cta, wq, lane);
+        return;
+    }
     // SCATTER: slot index and gate weight of every token column of the tile,
     // loaded once per tile (lane l holds columns 32 c + l)
     int srcs[kNTile / 32];
@@ -418,81 +590,6 @@ __device__ __forceinline__ void pair_epilogue(uint8_t* wb, uint32_t taddr, const
                 for (int q = 0; q < 4; ++q)
                     d[q] = make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2],
                                       packed[4 * q + 3]);
-            }
-            __syncwarp();
-        } else if constexpr (EPI == EPI_DSWIGLU) {
-            // SwiGLU backward.  fp32 transpose (token row i: its 32 features),
-            // then lane = token row r: dh_raw of features f0 .. f0 + 31 (the
-            // warp's TMEM lanes), the saved gate / up pre-activations of the
-            // row's slot, and per feature
-            //   h = silu(g) u,  dh = w dh_raw,
-            //   dg = dh u silu'(g),  du = dh silu(g),  hw = w h,
-            // with silu'(g) = sigmoid(g) (1 + g (1 - sigmoid(g))); the sum of
-            // dh_raw h over the 32 features is this warp's part of dL/dw.
-#pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                float* row = reinterpret_cast<float*>(stage_chunk(wb, i, lane >> 2));
-                row[lane & 3] = __uint_as_float(v[i]);
-            }
-            __syncwarp();
-            if (tok_ok) {
-                const int r = t.b_row + c0 + lane;
-                const int src = a.row_src != nullptr ? a.row_src[r] : r;
-                const float wv = a.row_src != nullptr ? a.topk_w[src] : 1.f;
-                const int F = a.feat;
-                const int f0 = t.ft * 256 + (int)cta * 128 + wq * 32;
-                const __nv_bfloat16* gp =
-                    static_cast<const __nv_bfloat16*>(a.gu_in) + (size_t)src * 2 * F + f0;
-                uint4 gq[4], uq[4];
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    gq[q] = reinterpret_cast<const uint4*>(gp)[q];
-                    uq[q] = reinterpret_cast<const uint4*>(gp + F)[q];
-                }
-                const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(gq);
-                const __nv_bfloat162* u2 = reinterpret_cast<const __nv_bfloat162*>(uq);
-                uint32_t pdg[16], pdu[16], phw[16];
-                float part = 0.f;
-#pragma unroll
-                for (int q = 0; q < 8; ++q) {
-                    const float4 c4 = *reinterpret_cast<const float4*>(stage_chunk(wb, lane, q));
-                    const float dr[4] = {c4.x, c4.y, c4.z, c4.w};
-                    float odg[4], odu[4], ohw[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float2 gg = __bfloat1622float2(g2[(4 * q + e) >> 1]);
-                        const float2 uu = __bfloat1622float2(u2[(4 * q + e) >> 1]);
-                        const float g = (e & 1) ? gg.y : gg.x;
-                        const float u = (e & 1) ? uu.y : uu.x;
-                        const float sg = 1.0f / (1.0f + __expf(-g));
-                        const float silu = g * sg;
-                        const float h = silu * u;
-                        part = fmaf(dr[e], h, part);
-                        const float dh = wv * dr[e];
-                        odg[e] = dh * u * (sg * (1.0f + g * (1.0f - sg)));
-                        odu[e] = dh * silu;
-                        ohw[e] = wv * h;
-                    }
-                    pdg[2 * q] = pack_bf16x2(odg[0], odg[1]);
-                    pdg[2 * q + 1] = pack_bf16x2(odg[2], odg[3]);
-                    pdu[2 * q] = pack_bf16x2(odu[0], odu[1]);
-                    pdu[2 * q + 1] = pack_bf16x2(odu[2], odu[3]);
-                    phw[2 * q] = pack_bf16x2(ohw[0], ohw[1]);
-                    phw[2 * q + 1] = pack_bf16x2(ohw[2], ohw[3]);
-                }
-                __nv_bfloat16* dgr =
-                    static_cast<__nv_bfloat16*>(a.dgu_out) + (size_t)r * 2 * F + f0;
-                uint4* dgq = reinterpret_cast<uint4*>(dgr);
-                uint4* duq = reinterpret_cast<uint4*>(dgr + F);
-                uint4* hwq = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.hw_out) +
-                                                      (size_t)r * F + f0);
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    dgq[q] = make_uint4(pdg[4 * q], pdg[4 * q + 1], pdg[4 * q + 2], pdg[4 * q + 3]);
-                    duq[q] = make_uint4(pdu[4 * q], pdu[4 * q + 1], pdu[4 * q + 2], pdu[4 * q + 3]);
-                    hwq[q] = make_uint4(phw[4 * q], phw[4 * q + 1], phw[4 * q + 2], phw[4 * q + 3]);
-                }
-                if (a.dw_part != nullptr) a.dw_part[(size_t)r * (F >> 5) + (f0 >> 5)] = part;
             }
             __syncwarp();
         } else if constexpr (EPI == EPI_STORE_ROWS) {

@@ -175,6 +175,13 @@ void stage_mark(int i, cudaStream_t s) {
     if (g_stage_events_on && g_stage_events[i] != nullptr) cudaEventRecord(g_stage_events[i], s);
 }
 
+cudaEvent_t g_bwd_events[MOE_N_BWD_STAGE_EVENTS];
+bool g_bwd_events_on = false;
+
+void bwd_mark(int i, cudaStream_t s) {
+    if (g_bwd_events_on && g_bwd_events[i] != nullptr) cudaEventRecord(g_bwd_events[i], s);
+}
+
 }  // namespace
 
 extern "C" {
@@ -741,6 +748,7 @@ MOE_API int moe_backward(const void* x, const void* W_router, const void* W_gate
     const int rs = n_shared > 0 ? 1 : 0;  // slot of the routed problem in each launch
 
     // status word and the four launches' tile counters start at zero
+    bwd_mark(0, s);
     cudaError_t e = cudaMemsetAsync(status, 0, sizeof(int) * kStatusWords, s);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
     // 1. the forward's permutation again, with segments padded to 128 rows
@@ -751,6 +759,7 @@ MOE_API int moe_backward(const void* x, const void* W_router, const void* W_gate
     e = launch_bwd_gather(x, dy, d, inter, k, offsets + E, row_src, L.rows_cap, x_perm, dy_perm,
                           dgu, hw, slot_row, num_sms(), s);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
+    bwd_mark(1, s);
 
     PairArgs base{};
     base.n_groups = E;
@@ -807,11 +816,13 @@ MOE_API int moe_backward(const void* x, const void* W_router, const void* W_gate
                                  KIND_DGRAD);
         }
         if (e != cudaSuccess) return MOE_ERR_CUDA;
+        bwd_mark(2, s);
     }
     // 3. dL/dlogit of the chosen experts
     e = launch_router_dlogit(x, W_router, T, d, k, topk_idx, topk_w, dw_part, inter / 32,
                              slot_row, gate, dl, s);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
+    bwd_mark(3, s);
     // 4. dx parts = W_gate_up^T [dg|du] (weights MN-major): chosen experts into
     //    token-order slots, shared experts into fp32 rows
     {
@@ -843,10 +854,12 @@ MOE_API int moe_backward(const void* x, const void* W_router, const void* W_gate
                                  KIND_DGRAD);
         }
         if (e != cudaSuccess) return MOE_ERR_CUDA;
+        bwd_mark(4, s);
     }
     // 5. dx = shared part + chosen experts' parts + router part (fixed order)
     e = launch_bwd_combine(dx_sh, dx_slots, dl, topk_idx, W_router, T, d, k, dx, s);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
+    bwd_mark(5, s);
     // 6. dW_down = (w dy)^T h per expert: both operands MN-major, K = the
     //    expert's rows
     {
@@ -877,6 +890,7 @@ MOE_API int moe_backward(const void* x, const void* W_router, const void* W_gate
                                  KIND_WGRAD);
         }
         if (e != cudaSuccess) return MOE_ERR_CUDA;
+        bwd_mark(6, s);
     }
     // 7. dW_gate_up = [dg|du]^T x per expert
     {
@@ -906,10 +920,24 @@ MOE_API int moe_backward(const void* x, const void* W_router, const void* W_gate
                                  KIND_WGRAD);
         }
         if (e != cudaSuccess) return MOE_ERR_CUDA;
+        bwd_mark(7, s);
     }
     // 8. dW_router[e] = sum of dl * x over expert e's rows
     e = launch_router_dweight(dl, row_src, offsets, x_perm, E, d, dW_router, s);
-    return ret(e);
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
+    bwd_mark(8, s);
+    return MOE_OK;
+}
+
+MOE_API int moe_set_backward_stage_events(void* const* events, int n) {
+    if (events == nullptr) {
+        g_bwd_events_on = false;
+        return MOE_OK;
+    }
+    if (n != MOE_N_BWD_STAGE_EVENTS) return MOE_ERR_INVALID_ARG;
+    for (int i = 0; i < n; ++i) g_bwd_events[i] = static_cast<cudaEvent_t>(events[i]);
+    g_bwd_events_on = true;
+    return MOE_OK;
 }
 
 }  // extern "C"

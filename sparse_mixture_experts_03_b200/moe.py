@@ -36,7 +36,8 @@ SYMBOLS = ["moe_workspace_bytes", "moe_workspace_layout", "moe_route", "moe_forw
            "moe_get_device_status", "moe_clear_device_status", "moe_selftest_timeout",
            "moe_set_stage_events", "moe_status_string", "moe_version",
            "moe_expert_counts_noalloc", "moe_route_ex", "moe_forward_ex", "moe_saved_bytes",
-           "moe_forward_train", "moe_backward_workspace_bytes", "moe_backward"]
+           "moe_forward_train", "moe_backward_workspace_bytes", "moe_backward",
+           "moe_set_backward_stage_events"]
 GATES = {"sigmoid": 0, "softmax": 1}  # MOE_GATE_SIGMOID, MOE_GATE_SOFTMAX_TOPK
 N_STAGE_EVENTS = 6
 STAGES = ["route", "permute", "gate_up", "down", "combine"]
@@ -93,6 +94,8 @@ def lib() -> ctypes.CDLL:
         L.moe_backward_workspace_bytes.restype = sz
         L.moe_backward.argtypes = [vp] * 9 + [i] * 8 + [vp] * 6 + [sz, vp]
         L.moe_backward.restype = i
+        L.moe_set_backward_stage_events.argtypes = [ctypes.POINTER(vp), i]
+        L.moe_set_backward_stage_events.restype = i
         _lib = L
     return _lib
 
@@ -317,6 +320,23 @@ def set_stage_events(events) -> None:
     arr = (ctypes.c_void_p * len(events))(
         *[ctypes.c_void_p(e.cuda_event if e is not None else None) for e in events])
     _check(lib().moe_set_stage_events(arr, len(events)), "moe_set_stage_events")
+
+
+BWD_STAGES = ["gather", "dgrad_down", "dlogit", "dgrad_gate_up", "dx_sum", "wgrad_down",
+              "wgrad_gate_up", "dweight_router"]
+N_BWD_STAGE_EVENTS = len(BWD_STAGES) + 1
+
+
+def set_backward_stage_events(events) -> None:
+    """Record torch.cuda.Event objects at the stage boundaries of every
+    following backward (None turns it off); see set_stage_events."""
+    if events is None:
+        _check(lib().moe_set_backward_stage_events(None, 0), "moe_set_backward_stage_events")
+        return
+    arr = (ctypes.c_void_p * len(events))(
+        *[ctypes.c_void_p(e.cuda_event if e is not None else None) for e in events])
+    _check(lib().moe_set_backward_stage_events(arr, len(events)),
+           "moe_set_backward_stage_events")
 
 
 class MoELayer:
