@@ -1,10 +1,13 @@
-"""Benchmark of the MoE layer forward on B200 (one process per GPU).
+"""Benchmark of the MoE layer on B200 (one process per GPU).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload prefill]
+    python bench.py --step train --workload train ...   # forward + backward
     python bench.py --impl reference ...        # the CPU oracle, timed on host cores
 
 One step = one full layer forward (routing, permutation, routed and shared
-expert GEMMs, combine) over one batch of T tokens already resident in HBM.
+expert GEMMs, combine) over one batch of T tokens already resident in HBM;
+with --step train, one forward with saved pre-activations plus the layer
+backward (all gradients) over that batch.
 Under torchrun every rank runs its own batch with a full weight replica
 (token-parallel, no collective on the data path): weak scaling, value = all
 ranks' tokens / max-over-ranks time.  Prints one JSON line on rank 0.
@@ -268,6 +271,284 @@ def run_reference(args, w):
     print(json.dumps(out), flush=True)
 
 
+TRAIN_METRIC = ("MoE layer training step (forward + backward) tokens/sec and TFLOP/s at 1 B200; "
+                "% of roofline (TC or HBM)")
+
+
+def dy_batch(w, rank: int) -> torch.Tensor:
+    """Upstream gradient of rank `rank` (stream 7, seed offset by the rank)."""
+    return _randn((w.T, w.d), w.seed + rank, 7).to(torch.bfloat16)
+
+
+def oracle_train_sample(w, inp, dy, toks, nthreads, args):
+    """The oracle's forward + backward of the sub-batch `toks` (its own batch)."""
+    import oracle
+    xs, dys = inp.x[toks].contiguous(), dy[toks].contiguous()
+    kw = oracle_gating(args, w)
+    oracle.forward(xs, inp.W_router, inp.W_gate_up, inp.W_down, inp.W_shared, w.k, w.n_group,
+                   w.topk_group, w.inter, w.n_shared, nthreads=nthreads, **kw)
+    oracle.backward(xs, inp.W_router, inp.W_gate_up, inp.W_down, inp.W_shared, dys, w.k,
+                    w.n_group, w.topk_group, w.inter, w.n_shared, nthreads=nthreads, **kw)
+
+
+def train_sample_size(w, inp, dy, args, budget_s: float, nthreads: int) -> int:
+    probe = np.arange(min(w.T, max(8, nthreads)), dtype=np.int64)
+    t0 = time.perf_counter()
+    oracle_train_sample(w, inp, dy, probe, nthreads, args)
+    per_tok = (time.perf_counter() - t0) / len(probe)
+    return int(max(1, min(w.T, budget_s / max(per_tok, 1e-9))))
+
+
+def cpu_baseline_train(w, inp, dy, args, budget_s: float = 15.0):
+    """The oracle's forward + backward (as it stands) on a sub-batch of the
+    workload's tokens, sized to about budget_s of host time."""
+    nthreads = os.cpu_count() or 1
+    n = train_sample_size(w, inp, dy, args, budget_s, nthreads)
+    toks = np.linspace(0, w.T - 1, n).astype(np.int64)
+    t0 = time.perf_counter()
+    oracle_train_sample(w, inp, dy, toks, nthreads, args)
+    dt = time.perf_counter() - t0
+    return {"value": n / dt, "unit": "tokens/s", "cores": nthreads, "kind": "oracle",
+            "sample": f"forward + backward of a sub-batch of {n} of the {w.T} tokens of the "
+                      f"{w.name} workload (fp64, all gradients of that sub-batch), {dt:.1f} s wall"}
+
+
+def run_reference_train(args, w):
+    """--impl reference --step train: the oracle's forward + backward on a
+    bounded sub-batch per step, rank 0 only."""
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if int(os.environ.get("RANK", "0")) != 0:
+        return
+    inp = make_inputs(w)
+    dy = dy_batch(w, 0)
+    nthreads = os.cpu_count() or 1
+    total_steps = args.steps + args.warmup
+    n = train_sample_size(w, inp, dy, args, 150.0 / max(total_steps, 1), nthreads)
+    rng = np.random.default_rng(0)
+    times = []
+    for s_ in range(total_steps):
+        toks = np.sort(rng.choice(w.T, size=n, replace=False)).astype(np.int64)
+        t0 = time.perf_counter()
+        oracle_train_sample(w, inp, dy, toks, nthreads, args)
+        if s_ >= args.warmup:
+            times.append(time.perf_counter() - t0)
+    sec = sum(times) / len(times)
+    value = n / sec
+    flops = accounting.train_step_flops(n, w.d, w.E, w.k, w.inter, w.n_shared)
+    cfg = run_config(w, world, args)
+    cfg["step"] = "forward + backward"
+    out = {
+        "impl": "reference", "metric": TRAIN_METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": cfg, "tflops": flops / sec / 1e12,
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": nthreads, "kind": "oracle",
+                         "sample": f"forward + backward of {n} random tokens of {w.T} per step"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(out), flush=True)
+
+
+def run_train(args, w):
+    """--step train: one step = moe_forward_train + moe_backward over one batch
+    resident in HBM (all gradients: dx, dW_router, dW_gate_up, dW_down,
+    dW_shared)."""
+    world, rank, local = dist_setup()
+    dev = torch.device("cuda", local)
+    inp = make_inputs(w)
+    inp.x = rank_batch(w, inp, rank)
+    dy_host = dy_batch(w, rank)
+    x, dy = inp.x.to(dev), dy_host.to(dev)
+    Wr, Wgu, Wd = inp.W_router.to(dev), inp.W_gate_up.to(dev), inp.W_down.to(dev)
+    Wsh = inp.W_shared.to(dev) if inp.W_shared is not None else None
+    f32 = dict(dtype=torch.float32, device=dev)
+    y = torch.empty(w.T, w.d, **f32)
+    idx = torch.empty(w.T, w.k, dtype=torch.int32, device=dev)
+    wt = torch.empty(w.T, w.k, **f32)
+    saved = torch.empty(moe.saved_bytes(w.T, w.k, w.inter, w.n_shared), dtype=torch.uint8,
+                        device=dev)
+    ws = moe.alloc_workspace(w.T, w.d, w.E, w.k, w.inter, w.n_shared, x.dtype, dev)
+    bws = torch.empty(moe.backward_workspace_bytes(w.T, w.d, w.E, w.k, w.inter, w.n_shared),
+                      dtype=torch.uint8, device=dev)
+    grads = moe.alloc_grads(w.T, w.d, w.E, w.inter, w.n_shared, dev)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, **f32)
+    stream = torch.cuda.current_stream()
+    bias = torch.from_numpy(bias_ramp(w, args.gate)).to(dev) if args.expert_bias else None
+    load = torch.empty(w.E, dtype=torch.int32, device=dev) if args.expert_bias else None
+
+    def step(xin=x, dyin=dy, yout=y, dxout=None):
+        moe.forward_train(xin, Wr, Wgu, Wd, Wsh, w.k, w.n_group, w.topk_group, w.inter,
+                          w.n_shared, y=yout, topk_idx=idx, topk_w=wt, saved=saved,
+                          workspace=ws, gate=args.gate, expert_bias=bias, expert_load=load)
+        g = grads if dxout is None else moe.Grads(dxout, grads.dW_router, grads.dW_gate_up,
+                                                  grads.dW_down, grads.dW_shared)
+        moe.backward(xin, Wr, Wgu, Wd, Wsh, dyin, idx, wt, saved, w.k, w.inter, w.n_shared,
+                     gate=args.gate, grads=g, workspace=bws)
+
+    def check(where):
+        for buf in (ws, bws):
+            st, site = moe.device_status(buf)
+            if st != moe.MOE_OK:
+                raise SystemExit(f"device status {where}: {moe.status_string(st)} (site {site})")
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    check("after warm-up")
+
+    # ---- timed region (as for the forward): per-step events, L2 flushed
+    # between steps; the dominant launch (dh = W_down^T dy with the SwiGLU
+    # backward) is bracketed by backward stage events on every 8th step only.
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    dom_steps = [i for i in range(args.steps) if i % 8 == 0] or [0]
+    dom_ev = {i: [torch.cuda.Event(enable_timing=True) for _ in range(2)] for i in dom_steps}
+    n_stage = min(args.steps, 20)
+    f_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(moe.N_STAGE_EVENTS)]
+            for _ in range(n_stage)]
+    b_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(moe.N_BWD_STAGE_EVENTS)]
+            for _ in range(n_stage)]
+    for evs in f_ev + b_ev + list(dom_ev.values()):
+        for e in evs:
+            e.record(stream)
+    torch.cuda.synchronize()
+    nb = moe.N_BWD_STAGE_EVENTS
+    barrier(world)
+    with ClockSampler(local) as clocks:
+        for i in range(args.steps):
+            if args.l2 == "flush":
+                flush.fill_(float(i))
+            if i in dom_ev:
+                moe.set_backward_stage_events([None, dom_ev[i][0], dom_ev[i][1]] +
+                                              [None] * (nb - 3))
+            else:
+                moe.set_backward_stage_events(None)
+            starts[i].record(stream)
+            step()
+            ends[i].record(stream)
+        moe.set_backward_stage_events(None)
+        torch.cuda.synchronize()
+    barrier(world)
+    ms = max_over_ranks(sum(s_.elapsed_time(e) for s_, e in zip(starts, ends)) / args.steps, world)
+    dom_ms = sum(a.elapsed_time(b) for a, b in dom_ev.values()) / len(dom_ev)
+    # ---- per-stage breakdown of forward and backward (instrumented pass)
+    for i in range(n_stage):
+        if args.l2 == "flush":
+            flush.fill_(float(i))
+        moe.set_stage_events(f_ev[i])
+        moe.set_backward_stage_events(b_ev[i])
+        step()
+    moe.set_stage_events(None)
+    moe.set_backward_stage_events(None)
+    torch.cuda.synchronize()
+    check("after timing")
+    fst = np.mean([[e[j].elapsed_time(e[j + 1]) for j in range(len(e) - 1)] for e in f_ev], 0)
+    bst = np.mean([[e[j].elapsed_time(e[j + 1]) for j in range(len(e) - 1)] for e in b_ev], 0)
+
+    # ---- end to end through the public calls: every step copies x and dy
+    # from pinned host memory and reads y and dx back (what the layer hands
+    # the rest of the model); copies on two streams, double-buffered.
+    x_host, dy_host = inp.x.pin_memory(), dy_host.pin_memory()
+    y_host = [torch.empty(w.T, w.d).pin_memory() for _ in range(2)]
+    dx_host = [torch.empty(w.T, w.d).pin_memory() for _ in range(2)]
+    x_dev = [torch.empty_like(x) for _ in range(2)]
+    dy_dev = [torch.empty_like(dy) for _ in range(2)]
+    y_dev = [torch.empty_like(y) for _ in range(2)]
+    dx_dev = [torch.empty_like(grads.dx) for _ in range(2)]
+    s_h2d, s_d2h = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+
+    def e2e_run(n_steps, e_start=None, e_stop=None):
+        h2d_done = [torch.cuda.Event() for _ in range(n_steps)]
+        comp_done = [torch.cuda.Event() for _ in range(n_steps)]
+        d2h_done = [torch.cuda.Event() for _ in range(n_steps)]
+        if e_start is not None:
+            e_start.record(s_h2d)
+        for i in range(n_steps):
+            b = i & 1
+            with torch.cuda.stream(s_h2d):
+                if i >= 2:
+                    s_h2d.wait_event(comp_done[i - 2])
+                x_dev[b].copy_(x_host, non_blocking=True)
+                dy_dev[b].copy_(dy_host, non_blocking=True)
+                h2d_done[i].record(s_h2d)
+            stream.wait_event(h2d_done[i])
+            if i >= 2:
+                stream.wait_event(d2h_done[i - 2])
+            step(x_dev[b], dy_dev[b], y_dev[b], dx_dev[b])
+            comp_done[i].record(stream)
+            with torch.cuda.stream(s_d2h):
+                s_d2h.wait_event(comp_done[i])
+                y_host[b].copy_(y_dev[b], non_blocking=True)
+                dx_host[b].copy_(dx_dev[b], non_blocking=True)
+                d2h_done[i].record(s_d2h)
+        if e_stop is not None:
+            e_stop.record(s_d2h)
+        torch.cuda.synchronize()
+
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e2e_run(3)
+    barrier(world)
+    e2e_steps = max(5, args.steps // 4)
+    e2e_run(e2e_steps, e0, e1)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, world)
+
+    # ---- accounting
+    n_touched = accounting.touched_experts(idx.cpu().numpy(), w.E)
+    flops = accounting.train_step_flops(w.T, w.d, w.E, w.k, w.inter, w.n_shared)
+    bytes_alg = accounting.train_step_bytes(w.T, w.d, w.E, w.k, w.inter, w.n_shared, n_touched)
+    pk = peaks()
+    t_tensor = flops / (pk["bf16_tflops"] * 1e12)
+    t_hbm = bytes_alg / (pk["hbm_gbs"] * 1e9)
+    roof_ms = max(t_tensor, t_hbm) * 1e3
+    dom_flops = accounting.dgrad_down_flops(w.T, w.d, w.k, w.inter, w.n_shared)
+    dom_ach = dom_flops / (dom_ms * 1e-3) / 1e12
+    launches = (1 + (1 if w.T <= 1024 else 3) + 1 + 2 + 1) + ((1 if w.T <= 1024 else 3) + 8)
+    cfg = run_config(w, world, args)
+    cfg["step"] = "forward (saving pre-activations) + backward (dx and all weight gradients, fp32)"
+    out = {
+        "metric": TRAIN_METRIC, "value": world * w.T / (ms * 1e-3), "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) activations and upstream gradient, N(0,1/fan_in) "
+                "weights; no dataset)",
+        "config": cfg, "tflops": flops / (ms * 1e-3) / 1e12,
+        "roofline_layer": {"bound": "tensor" if t_tensor >= t_hbm else "hbm",
+                           "roofline_ms": roof_ms, "frac": roof_ms / ms,
+                           "peak_tflops": pk["bf16_tflops"], "hbm_gbs": pk["hbm_gbs"],
+                           "alg_flops": flops, "alg_bytes": bytes_alg,
+                           "touched_experts": n_touched, "peak_source": pk["source"]},
+        "roofline": {"bound": "tensor",
+                     "kernel": "pair_gemm_kernel<DSWIGLU,DSWIGLU,KIND_DGRAD> (dh = W_down^T dy, "
+                               "shared and routed experts, SwiGLU backward in the epilogue)",
+                     "achieved": dom_ach, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                     "frac": dom_ach / pk["bf16_tflops"], "traffic": None,
+                     "flops_per_launch": dom_flops, "avg_launch_ms": dom_ms,
+                     "timed_launches": len(dom_ev),
+                     "peak_kind": f"bf16 burst ({pk['source']})",
+                     **({"frac_of_sustained_peak": dom_ach / pk["bf16_tflops_sustained"]}
+                        if pk.get("bf16_tflops_sustained") else {})},
+        "stage_ms": {"forward": {n: float(v) for n, v in zip(moe.STAGES, fst)},
+                     "backward": {n: float(v) for n, v in zip(moe.BWD_STAGES, bst)}},
+        "stage_ms_note": f"separate pass of {n_stage} steps with an event at every stage "
+                         "boundary",
+        "gpu_launches": launches * args.steps,
+        "e2e": {"value": world * w.T / (e2e_ms * 1e-3), "unit": "tokens/s",
+                "h2d_bytes_per_step": 2 * x.numel() * x.element_size(),
+                "d2h_bytes_per_step": 2 * y.numel() * y.element_size(), "ms_per_step": e2e_ms,
+                "copies": "x and dy in, y and dx out; pinned host buffers, two copy streams, "
+                          "double-buffered, overlapping neighbouring steps"},
+        "clocks": clocks.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline_train(w, inp, dy_host, args)
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -283,12 +564,21 @@ def main():
                     help="routing gate (the FusionLLM sigmoid gate is the headline)")
     ap.add_argument("--expert-bias", action="store_true",
                     help="add a selection-only expert bias (and read back the expert loads)")
+    ap.add_argument("--step", default="forward", choices=["forward", "train"],
+                    help="forward: the layer forward (headline); train: forward with saved "
+                         "pre-activations + backward")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
     w = WORKLOADS[args.workload]
     if args.impl == "reference":
-        run_reference(args, w)
+        if args.step == "train":
+            run_reference_train(args, w)
+        else:
+            run_reference(args, w)
+        return
+    if args.step == "train":
+        run_train(args, w)
         return
 
     world, rank, local = dist_setup()

@@ -49,3 +49,36 @@ def layer_bytes(T: int, d: int, E: int, inter: int, n_shared: int, n_touched: in
     are implementation traffic and are not counted."""
     w = (n_touched + n_shared) * ffn_params(d, inter) + E * d
     return w * in_bytes + T * d * in_bytes + T * d * out_bytes
+
+
+# ---- training step (forward + backward of the layer)
+
+def backward_flops_per_token(d: int, k: int, inter: int, n_shared: int) -> int:
+    """FLOPs of the chain rule per token: for every chosen and shared expert
+    the input-gradient GEMMs (W_down^T dy, W_gate_up^T [dg|du]) and the
+    weight-gradient GEMMs, each with the FLOPs of the forward GEMM it mirrors
+    (2x the expert's forward); the router gets gradients on the k chosen
+    logits only: 2*d*k for dx and 2*d*k for dW_router."""
+    return 2 * (k + n_shared) * ffn_flops_per_token(d, inter) + 4 * d * k
+
+
+def train_step_flops(T: int, d: int, E: int, k: int, inter: int, n_shared: int) -> int:
+    return T * (flops_per_token(d, E, k, inter, n_shared)
+                + backward_flops_per_token(d, k, inter, n_shared))
+
+
+def train_step_bytes(T: int, d: int, E: int, k: int, inter: int, n_shared: int,
+                     n_touched: int) -> int:
+    """Algorithmic HBM bytes of forward + backward: the touched experts',
+    shared and router weights read twice (bf16), their gradients written once
+    (fp32), x and dy read (bf16), y and dx written (fp32), and the saved gate /
+    up pre-activations written and read back (bf16)."""
+    w = (n_touched + n_shared) * ffn_params(d, inter) + E * d
+    saved = 2 * inter * (T * k + T * n_shared) * 2
+    return 2 * w * 2 + w * 4 + 2 * T * d * 2 + 2 * T * d * 4 + 2 * saved
+
+
+def dgrad_down_flops(T: int, d: int, k: int, inter: int, n_shared: int) -> int:
+    """W_down^T dy for every chosen and shared expert row (the launch that
+    carries the SwiGLU backward)."""
+    return 2 * T * k * d * inter + 2 * T * d * n_shared * inter
