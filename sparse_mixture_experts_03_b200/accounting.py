@@ -76,9 +76,3 @@ def train_step_bytes(T: int, d: int, E: int, k: int, inter: int, n_shared: int,
     w = (n_touched + n_shared) * ffn_params(d, inter) + E * d
     saved = 2 * inter * (T * k + T * n_shared) * 2
     return 2 * w * 2 + w * 4 + 2 * T * d * 2 + 2 * T * d * 4 + 2 * saved
-
-
-def dgrad_down_flops(T: int, d: int, k: int, inter: int, n_shared: int) -> int:
-    """W_down^T dy for every chosen and shared expert row (the launch that
-    carries the SwiGLU backward)."""
-    return 2 * T * k * d * inter + 2 * T * d * n_shared * inter
