@@ -7,8 +7,8 @@
 //                    backward epilogue, then dL/dlogit of the chosen experts
 //   bwd_combine      dx = shared part + chosen experts' parts + router part,
 //                    in a fixed order
-//   router_dweight   dW_router[e] = sum of dl * x over expert e's rows, in row
-//                    order
+//   router_dweight   dW_router[e] = sum of dl * x over expert e's rows: fixed
+//                    row slices, then the slices in order
 // The gate derivatives follow the chain rule through the gates of
 // "FusionLLM：融合 MLA、GDN 与 MoE 的高效混合架构大模型训练框架", section
 // "混合专家（MoE）" (sigmoid scores, weights normalised over the chosen
@@ -193,19 +193,26 @@ __global__ void __launch_bounds__(256)
     pdl_trigger();
 }
 
-// Block (e, column chunk of 512): 2 columns per thread, rows of expert e's
-// segment in order; 8 rows' loads are in flight at a time (the sum still runs
-// row by row).
+// dW_router in two passes with a fixed summation order.  Pass 1: block (e,
+// column chunk of 512, slice z) sums the rows of slice z of expert e's
+// segment (the segment cut into kDwSlices nearly equal row ranges), 2 columns
+// per thread, 8 rows' loads in flight, into part[z][e][:].  Pass 2 adds the
+// slices in order z = 0, 1, ...
+constexpr int kDwSlices = kDwParts;
+
 __global__ void __launch_bounds__(256)
-    router_dweight_kernel(const float* __restrict__ dl, const int32_t* __restrict__ row_src,
-                          const int32_t* __restrict__ offsets, const __nv_bfloat162* __restrict__ xp,
-                          int d, float* __restrict__ dWr) {
-    const int e = blockIdx.x;
+    router_dweight_part_kernel(const float* __restrict__ dl, const int32_t* __restrict__ row_src,
+                               const int32_t* __restrict__ offsets,
+                               const __nv_bfloat162* __restrict__ xp, int E, int d,
+                               float* __restrict__ part) {
+    const int e = blockIdx.x, z = blockIdx.z;
     const int c2 = blockIdx.y * blockDim.x + threadIdx.x;  // column pair
     pdl_wait();
     const int d2 = d >> 1;
     if (c2 < d2) {
-        const int r0 = offsets[e], r1 = offsets[e + 1];
+        const int s0 = offsets[e], n = offsets[e + 1] - s0;
+        const int r0 = s0 + (int)((long long)z * n / kDwSlices);
+        const int r1 = s0 + (int)((long long)(z + 1) * n / kDwSlices);
         float a0 = 0.f, a1 = 0.f;
         for (int rb = r0; rb < r1; rb += 8) {
             float g[8];
@@ -224,7 +231,26 @@ __global__ void __launch_bounds__(256)
                 a1 = fmaf(g[u], f.y, a1);
             }
         }
-        reinterpret_cast<float2*>(dWr + (size_t)e * d)[c2] = make_float2(a0, a1);
+        reinterpret_cast<float2*>(part + ((size_t)z * E + e) * d)[c2] = make_float2(a0, a1);
+    }
+    pdl_trigger();
+}
+
+__global__ void __launch_bounds__(256)
+    router_dweight_sum_kernel(const float4* __restrict__ part, int n4, float4* __restrict__ dWr) {
+    const int i = blockIdx.x * blockDim.x + threadIdx.x;
+    pdl_wait();
+    if (i < n4) {
+        float4 a = part[i];
+#pragma unroll
+        for (int z = 1; z < kDwSlices; ++z) {
+            const float4 b = part[(size_t)z * n4 + i];
+            a.x += b.x;
+            a.y += b.y;
+            a.z += b.z;
+            a.w += b.w;
+        }
+        dWr[i] = a;
     }
     pdl_trigger();
 }
@@ -280,10 +306,17 @@ cudaError_t launch_bwd_combine(const float* base, const void* slots, const float
 }
 
 cudaError_t launch_router_dweight(const float* dl, const int32_t* row_src, const int32_t* offsets,
-                                  const void* x_perm, int E, int d, float* dWr, cudaStream_t s) {
+                                  const void* x_perm, int E, int d, float* part, float* dWr,
+                                  cudaStream_t s) {
     const unsigned cy = (unsigned)((d / 2 + 255) / 256);
-    return launch_pdl(router_dweight_kernel, dim3((unsigned)E, cy), dim3(256), 0, s, 1, dl,
-                      row_src, offsets, static_cast<const __nv_bfloat162*>(x_perm), d, dWr);
+    cudaError_t e = launch_pdl(router_dweight_part_kernel, dim3((unsigned)E, cy, kDwSlices),
+                               dim3(256), 0, s, 1, dl, row_src, offsets,
+                               static_cast<const __nv_bfloat162*>(x_perm), E, d, part);
+    if (e != cudaSuccess) return e;
+    const int n4 = E * d / 4;
+    return launch_pdl(router_dweight_sum_kernel, dim3((unsigned)((n4 + 255) / 256)), dim3(256), 0,
+                      s, 1, reinterpret_cast<const float4*>(part), n4,
+                      reinterpret_cast<float4*>(dWr));
 }
 
 }  // namespace moe

@@ -306,6 +306,29 @@ __device__ __forceinline__ float tanh_approx(float x) {
     return y;
 }
 
+// Packed pairs of fp32 values (one 64-bit register pair) for the two-wide
+// fp32 arithmetic of sm_100 (fma / mul .rn.f32x2): half the instructions.
+__device__ __forceinline__ uint64_t pk2(float a, float b) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+    return r;
+}
+__device__ __forceinline__ float2 up2(uint64_t v) {
+    float2 r;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(v));
+    return r;
+}
+__device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t r;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+    return r;
+}
+
 __device__ __forceinline__ float silu_mul(float g, float u) {
     return __fdividef(g, 1.0f + __expf(-g)) * u;
 }
@@ -390,7 +413,10 @@ __device__ __forceinline__ void dswiglu_epilogue(uint8_t* wb, uint32_t taddr, co
         uint32_t pdu[16], phw[16];
         float part = 0.f;
         if (cur.src >= 0) {
-            const float wv = cur.w;
+            const uint64_t W2 = pk2(cur.w, cur.w);
+            const uint64_t kHalf2 = pk2(0.5f, 0.5f), kOne2 = pk2(1.f, 1.f),
+                           kNeg12 = pk2(-1.f, -1.f);
+            uint64_t PART = pk2(0.f, 0.f);
             const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(cur.g);
             const __nv_bfloat162* u2 = reinterpret_cast<const __nv_bfloat162*>(cur.u);
 #pragma unroll
@@ -400,31 +426,34 @@ __device__ __forceinline__ void dswiglu_epilogue(uint8_t* wb, uint32_t taddr, co
                 for (int hq = 0; hq < 2; ++hq) {
                     const int q = 2 * qq + hq;
                     const float4 c4 = *reinterpret_cast<const float4*>(stage_chunk(wb, lane, q));
-                    const float dr[4] = {c4.x, c4.y, c4.z, c4.w};
-                    float odg[4], odu[4], ohw[4];
+                    const uint64_t dr2[2] = {pk2(c4.x, c4.y), pk2(c4.z, c4.w)};
+                    float2 odg[2], odu[2], ohw[2];
+                    // features 4 q + 2 pp, 4 q + 2 pp + 1 as one pair
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float2 gg = __bfloat1622float2(g2[(4 * q + e) >> 1]);
-                        const float2 uu = __bfloat1622float2(u2[(4 * q + e) >> 1]);
-                        const float g = (e & 1) ? gg.y : gg.x;
-                        const float u = (e & 1) ? uu.y : uu.x;
-                        // sigmoid(g) = (1 + tanh(g / 2)) / 2: one hardware tanh
-                        const float sg = fmaf(0.5f, tanh_approx(0.5f * g), 0.5f);
-                        const float silu = g * sg;
-                        const float h = silu * u;
-                        part = fmaf(dr[e], h, part);
-                        const float dh = wv * dr[e];
-                        // silu'(g) = sigmoid(g) (1 + g (1 - sigmoid(g)))
-                        odg[e] = dh * u * fmaf(silu, 1.0f - sg, sg);
-                        odu[e] = dh * silu;
-                        ohw[e] = wv * h;
+                    for (int pp = 0; pp < 2; ++pp) {
+                        const float2 gg = __bfloat1622float2(g2[2 * q + pp]);
+                        const float2 uu = __bfloat1622float2(u2[2 * q + pp]);
+                        const uint64_t G = pk2(gg.x, gg.y), U = pk2(uu.x, uu.y);
+                        // sigmoid(g) = (1 + tanh(g / 2)) / 2: one hardware tanh each
+                        const float2 hg = up2(mul2(G, kHalf2));
+                        const uint64_t SG =
+                            fma2(pk2(tanh_approx(hg.x), tanh_approx(hg.y)), kHalf2, kHalf2);
+                        const uint64_t SILU = mul2(G, SG);
+                        const uint64_t H = mul2(SILU, U);
+                        PART = fma2(dr2[pp], H, PART);
+                        const uint64_t DH = mul2(dr2[pp], W2);
+                        // silu'(g) = sigmoid(g) (1 + g (1 - sigmoid(g))) = silu (1 - sg) + sg
+                        const uint64_t DS = fma2(SILU, fma2(SG, kNeg12, kOne2), SG);
+                        odg[pp] = up2(mul2(mul2(DH, U), DS));
+                        odu[pp] = up2(mul2(DH, SILU));
+                        ohw[pp] = up2(mul2(H, W2));
                     }
-                    pdg[2 * hq] = pack_bf16x2(odg[0], odg[1]);
-                    pdg[2 * hq + 1] = pack_bf16x2(odg[2], odg[3]);
-                    pdu[4 * qq + 2 * hq] = pack_bf16x2(odu[0], odu[1]);
-                    pdu[4 * qq + 2 * hq + 1] = pack_bf16x2(odu[2], odu[3]);
-                    phw[4 * qq + 2 * hq] = pack_bf16x2(ohw[0], ohw[1]);
-                    phw[4 * qq + 2 * hq + 1] = pack_bf16x2(ohw[2], ohw[3]);
+                    pdg[2 * hq] = pack_bf16x2(odg[0].x, odg[0].y);
+                    pdg[2 * hq + 1] = pack_bf16x2(odg[1].x, odg[1].y);
+                    pdu[4 * qq + 2 * hq] = pack_bf16x2(odu[0].x, odu[0].y);
+                    pdu[4 * qq + 2 * hq + 1] = pack_bf16x2(odu[1].x, odu[1].y);
+                    phw[4 * qq + 2 * hq] = pack_bf16x2(ohw[0].x, ohw[0].y);
+                    phw[4 * qq + 2 * hq + 1] = pack_bf16x2(ohw[1].x, ohw[1].y);
                 }
                 *reinterpret_cast<uint4*>(stage_chunk(wb, lane, qq)) =
                     make_uint4(pdg[0], pdg[1], pdg[2], pdg[3]);
@@ -433,6 +462,8 @@ __device__ __forceinline__ void dswiglu_epilogue(uint8_t* wb, uint32_t taddr, co
             for (int qq = 0; qq < 4; ++qq)
                 *reinterpret_cast<uint4*>(stage_chunk(wb, lane, 4 + qq)) =
                     make_uint4(pdu[4 * qq], pdu[4 * qq + 1], pdu[4 * qq + 2], pdu[4 * qq + 3]);
+            const float2 part2 = up2(PART);  // even and odd features' sums
+            part = part2.x + part2.y;
             if (a.dw_part != nullptr)
                 a.dw_part[(size_t)(t.b_row + c0 + lane) * (F >> 5) + (f0 >> 5)] = part;
         }

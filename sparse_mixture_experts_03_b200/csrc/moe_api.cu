@@ -627,7 +627,7 @@ namespace {
 enum BwdRegion : int {
     BW_STATUS, BW_COUNTS, BW_OFFSETS, BW_BLOCK_COUNTS, BW_ROW_SRC, BW_SLOT_ROW, BW_X_PERM,
     BW_DY_PERM, BW_DGU, BW_HW, BW_DW_PART, BW_DL, BW_DX_SLOTS, BW_DGU_SH, BW_HW_SH, BW_DX_SH,
-    BW_TOTAL
+    BW_DWR_PART, BW_TOTAL
 };
 struct BwdLayout {
     size_t off[BW_TOTAL + 1];
@@ -658,6 +658,7 @@ bool make_bwd_layout(int T, int d, int E, int k, int inter, int n_shared, BwdLay
         2 * (size_t)T * 2 * SI,                 // DGU_SH
         2 * (size_t)T * SI,                     // HW_SH
         n_shared > 0 ? sizeof(float) * (size_t)T * d : 0,  // DX_SH
+        sizeof(float) * (size_t)kDwParts * E * d,  // DWR_PART: row-slice sums of dW_router
     };
     size_t o = 0;
     for (int i = 0; i < BW_TOTAL; ++i) {
@@ -923,7 +924,8 @@ MOE_API int moe_backward(const void* x, const void* W_router, const void* W_gate
         bwd_mark(7, s);
     }
     // 8. dW_router[e] = sum of dl * x over expert e's rows
-    e = launch_router_dweight(dl, row_src, offsets, x_perm, E, d, dW_router, s);
+    e = launch_router_dweight(dl, row_src, offsets, x_perm, E, d,
+                              bat<float>(workspace, L, BW_DWR_PART), dW_router, s);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
     bwd_mark(8, s);
     return MOE_OK;

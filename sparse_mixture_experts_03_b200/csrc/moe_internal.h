@@ -226,9 +226,12 @@ cudaError_t launch_bwd_combine(const float* base, const void* slots, const float
                                const int32_t* idx, const void* Wr, int T, int d, int k, float* dx,
                                cudaStream_t s);
 // dWr[e] = sum over rows r of expert e's padded segment with row_src[r] >= 0 of
-// dl[row_src[r]] * x_perm[r], in row order, fp32.
+// dl[row_src[r]] * x_perm[r], fp32: kDwParts fixed row slices of the segment
+// summed in row order into part [kDwParts, E, d], then the slices in order.
+constexpr int kDwParts = 8;
 cudaError_t launch_router_dweight(const float* dl, const int32_t* row_src, const int32_t* offsets,
-                                  const void* x_perm, int E, int d, float* dWr, cudaStream_t s);
+                                  const void* x_perm, int E, int d, float* part, float* dWr,
+                                  cudaStream_t s);
 
 cudaError_t launch_selftest_timeout(int* status, unsigned long long limit_ns, cudaStream_t s);
 
