@@ -1,8 +1,8 @@
 // Memory-bound helper kernels of the layer backward (the GEMMs are the
 // CTA-pair kernels of gemm_pair.cu):
-//   bwd_gather       x and dy rows into the padded permuted layout; zero
-//                    padding rows of every row-indexed GEMM operand; the
-//                    inverse of row_src (slot -> permuted row)
+//   bwd_gather       x and dy rows into the padded permuted layout (each
+//                    token's rows read once); zero padding rows of every
+//                    row-indexed GEMM operand
 //   router_dlogit    dL/dw from the per-warp partial sums of the SwiGLU
 //                    backward epilogue, then dL/dlogit of the chosen experts
 //   bwd_combine      dx = shared part + chosen experts' parts + router part,
@@ -22,44 +22,62 @@ namespace moe {
 
 namespace {
 
-// One warp per row of the padded permuted layout.
+// Part 1: one warp per token, its x and dy rows read once (16-byte vectors,
+// all of a lane's loads before its stores) and written to the token's k rows.
+// Part 2: one warp per row, zeroing padding rows.
 __global__ void __launch_bounds__(256)
-    bwd_gather_kernel(const uint4* __restrict__ x, const uint4* __restrict__ dy, int vd, int vf,
-                      int k, const int32_t* __restrict__ total_rows,
-                      const int32_t* __restrict__ row_src, uint4* __restrict__ x_perm,
-                      uint4* __restrict__ dy_perm, uint4* __restrict__ dgu,
-                      uint4* __restrict__ hw, int32_t* __restrict__ slot_row) {
+    bwd_gather_kernel(const uint4* __restrict__ x, const uint4* __restrict__ dy, int T, int vd,
+                      int vf, int k, const int32_t* __restrict__ total_rows,
+                      const int32_t* __restrict__ row_src, const int32_t* __restrict__ slot_row,
+                      uint4* __restrict__ x_perm, uint4* __restrict__ dy_perm,
+                      uint4* __restrict__ dgu, uint4* __restrict__ hw) {
     const int lane = threadIdx.x & 31;
     const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int nw = (gridDim.x * blockDim.x) >> 5;
     pdl_wait();
+    for (int t = gw; t < T; t += nw) {
+        const uint4* xs = x + (size_t)t * vd;
+        const uint4* ys = dy + (size_t)t * vd;
+        for (int i0 = 0; i0 < vd; i0 += 4 * 32) {
+            uint4 a[4], b[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int i = i0 + u * 32 + lane;
+                if (i < vd) {
+                    a[u] = __ldcs(xs + i);
+                    b[u] = __ldcs(ys + i);
+                }
+            }
+            for (int j = 0; j < k; ++j) {
+                const size_t r = (size_t)slot_row[(size_t)t * k + j];
+                uint4* xo = x_perm + r * vd;
+                uint4* yo = dy_perm + r * vd;
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int i = i0 + u * 32 + lane;
+                    if (i < vd) {
+                        xo[i] = a[u];
+                        yo[i] = b[u];
+                    }
+                }
+            }
+        }
+    }
+    // padding rows are K rows of the weight-gradient GEMMs: all zero
     const int total = *total_rows;
     const uint4 z = make_uint4(0u, 0u, 0u, 0u);
     for (int r = gw; r < total; r += nw) {
-        const int src = row_src[r];
+        if (row_src[r] >= 0) continue;
         uint4* xo = x_perm + (size_t)r * vd;
         uint4* yo = dy_perm + (size_t)r * vd;
-        if (src >= 0) {
-            const int t = src / k;
-            const uint4* xs = x + (size_t)t * vd;
-            const uint4* ys = dy + (size_t)t * vd;
-            for (int i = lane; i < vd; i += 32) {
-                const uint4 a = __ldg(xs + i), b = __ldg(ys + i);
-                xo[i] = a;
-                yo[i] = b;
-            }
-            if (lane == 0) slot_row[src] = r;
-        } else {
-            // padding rows are K rows of the weight-gradient GEMMs: all zero
-            for (int i = lane; i < vd; i += 32) {
-                xo[i] = z;
-                yo[i] = z;
-            }
-            uint4* go = dgu + (size_t)r * 2 * vf;
-            for (int i = lane; i < 2 * vf; i += 32) go[i] = z;
-            uint4* ho = hw + (size_t)r * vf;
-            for (int i = lane; i < vf; i += 32) ho[i] = z;
+        for (int i = lane; i < vd; i += 32) {
+            xo[i] = z;
+            yo[i] = z;
         }
+        uint4* go = dgu + (size_t)r * 2 * vf;
+        for (int i = lane; i < 2 * vf; i += 32) go[i] = z;
+        uint4* ho = hw + (size_t)r * vf;
+        for (int i = lane; i < vf; i += 32) ho[i] = z;
     }
     pdl_trigger();
 }
@@ -96,11 +114,12 @@ __global__ void __launch_bounds__(256)
         w[j] = 0.f;
         sc[j] = 0.f;
         if (j < k) {
-            // every lane sums the same parts in the same order
+            // lane l sums parts l, l + 32, ...; then a fixed xor tree (every
+            // lane ends with the same sum, in the same order)
             const float* pp = dw_part + (size_t)slot_row[(size_t)t * k + j] * n_parts;
             float acc = 0.f;
-            for (int p = 0; p < n_parts; ++p) acc += pp[p];
-            dw[j] = acc;
+            for (int p = lane; p < n_parts; p += 32) acc += pp[p];
+            dw[j] = warp_sum(acc);
             w[j] = topk_w[(size_t)t * k + j];
             abar = fmaf(w[j], dw[j], abar);
         }
@@ -257,18 +276,18 @@ __global__ void __launch_bounds__(256)
 
 }  // namespace
 
-cudaError_t launch_bwd_gather(const void* x, const void* dy, int d, int F, int k,
-                              const int32_t* offsets_total, const int32_t* row_src, int rows_cap,
-                              void* x_perm, void* dy_perm, void* dgu, void* hw,
-                              int32_t* slot_row, int num_sms, cudaStream_t s) {
+cudaError_t launch_bwd_gather(const void* x, const void* dy, int T, int d, int F, int k,
+                              const int32_t* offsets_total, const int32_t* row_src,
+                              const int32_t* slot_row, int rows_cap, void* x_perm, void* dy_perm,
+                              void* dgu, void* hw, int num_sms, cudaStream_t s) {
     int blocks = (rows_cap + 7) / 8;
     if (blocks > num_sms * 8) blocks = num_sms * 8;
     if (blocks < 1) blocks = 1;
     return launch_pdl(bwd_gather_kernel, dim3(blocks), dim3(256), 0, s, 1,
-                      static_cast<const uint4*>(x), static_cast<const uint4*>(dy), d / 8, F / 8, k,
-                      offsets_total, row_src, static_cast<uint4*>(x_perm),
+                      static_cast<const uint4*>(x), static_cast<const uint4*>(dy), T, d / 8, F / 8,
+                      k, offsets_total, row_src, slot_row, static_cast<uint4*>(x_perm),
                       static_cast<uint4*>(dy_perm), static_cast<uint4*>(dgu),
-                      static_cast<uint4*>(hw), slot_row);
+                      static_cast<uint4*>(hw));
 }
 
 cudaError_t launch_router_dlogit(const void* x, const void* Wr, int T, int d, int k,

@@ -755,10 +755,10 @@ MOE_API int moe_backward(const void* x, const void* W_router, const void* W_gate
     // 1. the forward's permutation again, with segments padded to 128 rows
     //    (whole k-blocks of the weight-gradient GEMMs), then x / dy rows
     e = launch_permute(topk_idx, T, k, E, block_counts, counts, offsets, row_src, kRowAlign,
-                       nullptr, status, s);
+                       nullptr, status, s, slot_row);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
-    e = launch_bwd_gather(x, dy, d, inter, k, offsets + E, row_src, L.rows_cap, x_perm, dy_perm,
-                          dgu, hw, slot_row, num_sms(), s);
+    e = launch_bwd_gather(x, dy, T, d, inter, k, offsets + E, row_src, slot_row, L.rows_cap,
+                          x_perm, dy_perm, dgu, hw, num_sms(), s);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
     bwd_mark(1, s);
 

@@ -113,10 +113,12 @@ cudaError_t launch_route_f32(const void* x, const void* Wr, int T, int d, int E,
                              int* status, cudaStream_t s);
 
 // Segments of the permuted layout are padded to a multiple of `align` rows
-// (1: unpadded) with row_src = -1 on padding rows.
+// (1: unpadded) with row_src = -1 on padding rows; slot_row (nullable) gets
+// the inverse: slot t*k + j -> its row.
 cudaError_t launch_permute(const int32_t* idx, int T, int k, int E, int32_t* block_counts,
                            int32_t* counts, int32_t* offsets, int32_t* row_src, int align,
-                           int32_t* load_out, int* status, cudaStream_t s);
+                           int32_t* load_out, int* status, cudaStream_t s,
+                           int32_t* slot_row = nullptr);
 cudaError_t launch_gather_rows(const void* x, int d, int elem_bytes, int k,
                                const int32_t* offsets_total, const int32_t* row_src,
                                int rows_cap, void* x_perm, int num_sms, cudaStream_t s);
@@ -206,14 +208,14 @@ cudaError_t launch_pair_gemm(int epi0, int epi1, const PairMaps& maps, const Pai
                              cudaStream_t s, int kind = KIND_FWD);
 
 // ---- backward helpers (backward.cu)
-// For every row r of the padded permuted layout (rows [0, offsets_total)):
-// row_src[r] >= 0: x_perm[r] = x[t], dy_perm[r] = dy[t] (t = row_src[r] / k)
-// and slot_row[row_src[r]] = r; padding rows: x_perm, dy_perm, dgu [2F] and
-// hw [F] rows set to zero.  bf16.
-cudaError_t launch_bwd_gather(const void* x, const void* dy, int d, int F, int k,
-                              const int32_t* offsets_total, const int32_t* row_src, int rows_cap,
-                              void* x_perm, void* dy_perm, void* dgu, void* hw,
-                              int32_t* slot_row, int num_sms, cudaStream_t s);
+// Rows of the padded permuted layout (rows [0, offsets_total)): each token's
+// x and dy rows are read once and written to its k rows slot_row[t*k + j];
+// padding rows (row_src < 0) of x_perm, dy_perm, dgu [2F] and hw [F] are set
+// to zero.  bf16.
+cudaError_t launch_bwd_gather(const void* x, const void* dy, int T, int d, int F, int k,
+                              const int32_t* offsets_total, const int32_t* row_src,
+                              const int32_t* slot_row, int rows_cap, void* x_perm, void* dy_perm,
+                              void* dgu, void* hw, int num_sms, cudaStream_t s);
 // dl[t*k + j] = dL/dlogit of token t's chosen expert j (gate MOE_GATE_*), from
 // dw = sum of the dw_part row of its slot, topk_w and the recomputed logits.
 cudaError_t launch_router_dlogit(const void* x, const void* Wr, int T, int d, int k,

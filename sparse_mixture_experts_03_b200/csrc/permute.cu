@@ -141,7 +141,7 @@ __global__ void __launch_bounds__(1024) perm_scan_kernel(int32_t* __restrict__ b
 __global__ void __launch_bounds__(kPermBlockTokens) perm_rank_kernel(
     const int32_t* __restrict__ idx, int T, int k, int E,
     const int32_t* __restrict__ block_base, const int32_t* __restrict__ offsets,
-    int32_t* __restrict__ row_src, int* status) {
+    int32_t* __restrict__ row_src, int32_t* __restrict__ slot_row, int* status) {
     __shared__ int wbase[kWarps][kMaxE];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int t = blockIdx.x * kPermBlockTokens + tid;
@@ -173,9 +173,10 @@ __global__ void __launch_bounds__(kPermBlockTokens) perm_rank_kernel(
     for (int j = 0; j < kMaxK; ++j) {
         if (my[j] >= 0) {
             int pos = wbase[warp][my[j]] + rank[j];
-            if (pos < offsets[my[j] + 1])
+            if (pos < offsets[my[j] + 1]) {
                 row_src[pos] = t * k + j;
-            else
+                if (slot_row != nullptr) slot_row[t * k + j] = pos;
+            } else
                 set_status(status, MOE_ERR_DEVICE, SITE_PERMUTE, pos);
         }
     }
@@ -192,7 +193,7 @@ constexpr int kSmallWarps = kSmallTokens / 32;
 __global__ void __launch_bounds__(kSmallTokens) perm_small_kernel(
     const int32_t* __restrict__ idx, int T, int k, int E, int align, int32_t* __restrict__ counts,
     int32_t* __restrict__ offsets, int32_t* __restrict__ row_src, int32_t* __restrict__ load_out,
-    int* status) {
+    int32_t* __restrict__ slot_row, int* status) {
     __shared__ int wcnt[kSmallWarps][kMaxE];  // per-warp counts, then per-warp bases
     __shared__ int s_cnt[kMaxE];
     __shared__ int s_off[kMaxE + 1];
@@ -254,7 +255,11 @@ __global__ void __launch_bounds__(kSmallTokens) perm_small_kernel(
     __syncthreads();
 #pragma unroll
     for (int j = 0; j < kMaxK; ++j)
-        if (my[j] >= 0) row_src[wcnt[warp][my[j]] + rank[j]] = tid * k + j;
+        if (my[j] >= 0) {
+            const int pos = wcnt[warp][my[j]] + rank[j];
+            row_src[pos] = tid * k + j;
+            if (slot_row != nullptr) slot_row[tid * k + j] = pos;
+        }
     pdl_trigger();
 }
 
@@ -404,10 +409,11 @@ __global__ void __launch_bounds__(256) combine_slots_bf16_kernel(
 
 cudaError_t launch_permute(const int32_t* idx, int T, int k, int E, int32_t* block_counts,
                            int32_t* counts, int32_t* offsets, int32_t* row_src, int align,
-                           int32_t* load_out, int* status, cudaStream_t s) {
+                           int32_t* load_out, int* status, cudaStream_t s, int32_t* slot_row) {
     if (T <= kSmallTokens)
         return launch_pdl(perm_small_kernel, dim3(1), dim3((unsigned)((T + 31) / 32 * 32)), 0, s,
-                          1, idx, T, k, E, align, counts, offsets, row_src, load_out, status);
+                          1, idx, T, k, E, align, counts, offsets, row_src, load_out, slot_row,
+                          status);
     const int nb = (T + kPermBlockTokens - 1) / kPermBlockTokens;
     cudaError_t e = launch_pdl(perm_count_kernel, dim3(nb), dim3(kPermBlockTokens), 0, s, 1, idx,
                                T, k, E, block_counts, status);
@@ -417,7 +423,7 @@ cudaError_t launch_permute(const int32_t* idx, int T, int k, int E, int32_t* blo
     if (e != cudaSuccess) return e;
     return launch_pdl(perm_rank_kernel, dim3(nb), dim3(kPermBlockTokens), 0, s, 1, idx, T, k, E,
                       static_cast<const int32_t*>(block_counts),
-                      static_cast<const int32_t*>(offsets), row_src, status);
+                      static_cast<const int32_t*>(offsets), row_src, slot_row, status);
 }
 
 cudaError_t launch_expert_counts(const int32_t* idx, int T, int k, int E,
