@@ -84,3 +84,45 @@ def test_forward_rejects_bad_workspace_and_shared_mismatch():
     # bf16 path needs d % 256
     assert L.moe_forward(None, None, None, None, None, 8, 192, 8, 2, 1, 1, 128, 0, moe.MOE_BF16,
                          moe.MOE_F32, None, None, None, None, 0, None) == moe.MOE_ERR_UNSUPPORTED
+
+
+def _backward(T=8, d=256, E=8, k=2, I=256, S=0, dt=moe.MOE_BF16, gate=0, W_sh=None, dW_sh=None,
+              ws=None, wsb=0):
+    return moe.lib().moe_backward(None, None, None, None, W_sh, None, None, None, None, T, d, E,
+                                  k, I, S, dt, gate, None, None, None, None, dW_sh, ws, wsb, None)
+
+
+def test_training_entry_points_reject_invalid_arguments_on_host():
+    assert _backward(dt=moe.MOE_F32) == moe.MOE_ERR_UNSUPPORTED      # bf16 layers only
+    assert _backward(I=128) == moe.MOE_ERR_UNSUPPORTED               # inter % 256
+    assert _backward(d=100) == moe.MOE_ERR_UNSUPPORTED               # d % 64 (size check)
+    assert _backward(d=320) == moe.MOE_ERR_UNSUPPORTED               # d % 256 (bf16 GEMMs)
+    assert _backward(gate=5) == moe.MOE_ERR_INVALID_ARG              # unknown gate
+    assert _backward(S=1) == moe.MOE_ERR_INVALID_ARG                 # shared count without weights
+    assert _backward(S=0, W_sh=ctypes.c_void_p(256)) == moe.MOE_ERR_INVALID_ARG
+    assert _backward() == moe.MOE_ERR_WORKSPACE                      # no workspace
+    assert _backward(ws=ctypes.c_void_p(256), wsb=16) == moe.MOE_ERR_WORKSPACE
+    assert _backward(k=9) == moe.MOE_ERR_INVALID_ARG                 # k > 8
+    # forward_train: bf16 only; T > 0 needs routing outputs and a saved buffer
+    L = moe.lib()
+    ft = lambda dt, saved, sb, idx=None, w=None: L.moe_forward_train(
+        None, None, None, None, None, 8, 256, 8, 2, 1, 1, 256, 0, dt, moe.MOE_F32, 0, None, None,
+        idx, w, None, saved, sb, None, 0, None)
+    assert ft(moe.MOE_F32, None, 0) == moe.MOE_ERR_UNSUPPORTED
+    assert ft(moe.MOE_BF16, None, 0) == moe.MOE_ERR_INVALID_ARG       # no topk outputs
+    assert ft(moe.MOE_BF16, None, 0, ctypes.c_void_p(256), ctypes.c_void_p(512)) == \
+        moe.MOE_ERR_INVALID_ARG                                       # no saved buffer
+
+
+def test_training_buffer_sizes():
+    T, d, E, k, I, S = 4096, 2048, 64, 6, 1536, 4
+    # saved: routed [T*k, 2I] then shared [T, 2*S*I], bf16
+    assert moe.saved_bytes(T, k, I, S) == 2 * (T * k * 2 * I + T * 2 * S * I)
+    assert moe.saved_bytes(T, k, I, 0) == 2 * T * k * 2 * I
+    n = moe.backward_workspace_bytes(T, d, E, k, I, S)
+    rows_cap = T * k + moe.ROW_ALIGN * E
+    # at least: x and dy rows, dg|du and w*h per padded row, dx slots, shared rows
+    assert n >= 2 * rows_cap * (2 * d + 3 * I) + 2 * T * k * d + 2 * T * 3 * S * I
+    assert n % 1024 == 0
+    assert moe.lib().moe_backward_workspace_bytes(T, d, E, k, 1664, S) == 0  # inter % 256
+    assert moe.lib().moe_backward_workspace_bytes(T, 2112, E, k, I, S) == 0  # d % 256

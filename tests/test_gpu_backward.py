@@ -232,3 +232,80 @@ def test_full_size_sampled_train_batch():
             (oracle.ROW_DWD, int(rng.integers(E * d))),
             (oracle.ROW_DWSH_GU, int(rng.integers(2 * SI)))]
     sampled_check(w, [0, 16383, 32767], wsel)
+
+
+def test_training_step_in_a_cuda_graph_matches_eager():
+    """forward_train + backward captured once and replayed: the same bits as
+    the eager calls (the backward clears its status word and tile counters
+    inside every replay)."""
+    w = SMALL[1]
+    inp, dy = make_inputs(w), make_dy(w)
+    r = run_gpu(w, inp, dy)
+    c = lambda t: None if t is None else t.to(DEV)
+    y = torch.empty_like(r["y"])
+    idx, tw, saved = torch.empty_like(r["idx"]), torch.empty_like(r["tw"]), torch.empty_like(
+        r["saved"])
+    fws = moe.alloc_workspace(w.T, w.d, w.E, w.k, w.inter, w.n_shared, torch.bfloat16)
+    bws = torch.empty_like(r["ws"])
+    g = moe.alloc_grads(w.T, w.d, w.E, w.inter, w.n_shared, DEV)
+
+    def step(stream):
+        moe.forward_train(r["x"], r["Wr"], r["Wgu"], r["Wd"], r["Wsh"], w.k, w.n_group,
+                          w.topk_group, w.inter, w.n_shared, y=y, topk_idx=idx, topk_w=tw,
+                          saved=saved, workspace=fws, stream=stream)
+        moe.backward(r["x"], r["Wr"], r["Wgu"], r["Wd"], r["Wsh"], r["dy"], idx, tw, saved, w.k,
+                     w.inter, w.n_shared, grads=g, workspace=bws, stream=stream)
+
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        step(s)
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        step(torch.cuda.current_stream())
+    for _ in range(2):
+        for t in (g.dx, g.dW_router, g.dW_gate_up, g.dW_down, g.dW_shared):
+            t.zero_()
+        graph.replay()
+        torch.cuda.synchronize()
+        assert moe.device_status(bws)[0] == moe.MOE_OK
+        assert torch.equal(y, r["y"])
+        for name in ("dx", "dW_router", "dW_gate_up", "dW_down", "dW_shared"):
+            assert torch.equal(getattr(g, name), getattr(r["g"], name)), name
+    del graph
+
+
+def test_backward_with_selection_bias():
+    """A selection-only bias moves the expert sets; the gradients follow the
+    sets chosen and the unbiased weights (the oracle with the same bias)."""
+    w = SMALL[1]
+    inp, dy = make_inputs(w), make_dy(w)
+    bias = np.random.default_rng(9).permutation(np.linspace(-0.1, 0.1, w.E)).astype(np.float32)
+    c = lambda t: None if t is None else t.to(DEV)
+    x, Wr, Wgu, Wd, Wsh, dyd = (c(inp.x), c(inp.W_router), c(inp.W_gate_up), c(inp.W_down),
+                                c(inp.W_shared), c(dy))
+    b = torch.from_numpy(bias).to(DEV)
+    y, idx, tw, saved = moe.forward_train(x, Wr, Wgu, Wd, Wsh, w.k, w.n_group, w.topk_group,
+                                          w.inter, w.n_shared, expert_bias=b)
+    g = moe.backward(x, Wr, Wgu, Wd, Wsh, dyd, idx, tw, saved, w.k, w.inter, w.n_shared)
+    torch.cuda.synchronize()
+    gpu_idx, gpu_w = idx.cpu().numpy(), tw.cpu().numpy()
+    ref_r = oracle.route(inp.x, inp.W_router, w.k, w.n_group, w.topk_group, bias=bias)
+    rep = check_routing(gpu_idx, gpu_w, ref_r, w.n_group, w.topk_group, w.E)
+    forced = None
+    if rep.n_set_mismatch_near_tie:
+        forced = ref_r.idx.copy()
+        forced[rep.mismatched_tokens] = gpu_idx[rep.mismatched_tokens]
+    ref = oracle.backward(inp.x, inp.W_router, inp.W_gate_up, inp.W_down, inp.W_shared, dy, w.k,
+                          w.n_group, w.topk_group, w.inter, w.n_shared, forced_idx=forced,
+                          bias=bias)
+    # the bias changed some sets relative to the unbiased routing
+    plain = oracle.route(inp.x, inp.W_router, w.k, w.n_group, w.topk_group)
+    assert (np.sort(plain.idx, 1) != np.sort(ref.idx, 1)).any(1).sum() > 0
+    assert_close(g.dx.cpu().numpy(), ref.dx, "dx")
+    assert_close(g.dW_router.cpu().numpy(), ref.dW_router, "dW_router")
+    assert_close(g.dW_gate_up.cpu().numpy(), ref.dW_gate_up, "dW_gate_up")
+    assert_close(g.dW_down.cpu().numpy(), ref.dW_down, "dW_down")
+    assert_close(g.dW_shared.cpu().numpy(), ref.dW_shared, "dW_shared")
