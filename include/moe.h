@@ -302,9 +302,10 @@ MOE_API int moe_forward_train(const void *x, const void *W_router, const void *W
  * moe_backward_workspace_bytes -- scratch bytes of moe_backward for these
  * sizes (bf16 layers; 0 for invalid or unsupported sizes).  Regions: status
  * words and tile counters, expert counts and padded offsets, the permutation
- * (segments padded to 128 rows), x and dy rows in that order, the SwiGLU
- * backward rows dg|du and w*h, the per-row parts of dL/dw, dL/dlogit, the
- * chosen experts' dx rows, the shared experts' rows and their fp32 dx.
+ * (segments padded to 128 rows) and its inverse, x and dy rows in that order,
+ * the SwiGLU backward rows dg|du and w*h, the per-row parts of dL/dw,
+ * dL/dlogit, the chosen experts' dx rows, the shared experts' rows and their
+ * fp32 dx, and row-slice sums of dW_router.
  */
 MOE_API size_t moe_backward_workspace_bytes(int T, int d, int E, int k, int inter,
                                             int n_shared);
