@@ -403,6 +403,10 @@ def run_train(args, w):
     n_stage = min(args.steps, 20)
     f_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(nf)] for _ in range(n_stage)]
     b_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(nb)] for _ in range(n_stage)]
+    for evs in f_ev + b_ev:  # create the CUDA handles the library records into
+        for e in evs:
+            e.record(stream)
+    torch.cuda.synchronize()
     for i in range(n_stage):
         if args.l2 == "flush":
             flush.fill_(float(i))
