@@ -90,8 +90,9 @@ __device__ __forceinline__ float warp_sum(float v) {
 
 // One warp per token.  dw_j: the parts of its slot's row summed in part
 // order.  Sigmoid gate (w_j = s_j / S): dl_j = (dw_j - sum_i w_i dw_i) / S *
-// s_j (1 - s_j), with s_j recomputed from the chosen logits x . Wr[e_j] (fp32
-// sums of the bf16 products) and S their sum.  Softmax over the chosen logits:
+// s_j (1 - s_j); S and the s_j come from one recomputed logit, that of the
+// top choice (w_0 >= 1/k): S = sigmoid(x . Wr[e_0]) / w_0 (fp32 sum of the
+// bf16 products), s_j = w_j S.  Softmax over the chosen logits:
 // dl_j = w_j (dw_j - sum_i w_i dw_i).
 __global__ void __launch_bounds__(256)
     router_dlogit_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restrict__ Wr,
@@ -106,13 +107,12 @@ __global__ void __launch_bounds__(256)
         pdl_trigger();
         return;
     }
-    float dw[kMaxK], w[kMaxK], sc[kMaxK];
+    float dw[kMaxK], w[kMaxK];
     float abar = 0.f;
 #pragma unroll
     for (int j = 0; j < kMaxK; ++j) {
         dw[j] = 0.f;
         w[j] = 0.f;
-        sc[j] = 0.f;
         if (j < k) {
             // lane l sums parts l, l + 32, ...; then a fixed xor tree (every
             // lane ends with the same sum, in the same order)
@@ -124,40 +124,31 @@ __global__ void __launch_bounds__(256)
             abar = fmaf(w[j], dw[j], abar);
         }
     }
+    float v = 0.f;
     if (gate == MOE_GATE_SIGMOID) {
         const __nv_bfloat16* xr = x + (size_t)t * d;
-        float S = 0.f;
+        const __nv_bfloat16* wr = Wr + (size_t)idx[(size_t)t * k] * d;
+        float acc = 0.f;
+        for (int c = 2 * lane; c < d; c += 64) {
+            const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(xr + c));
+            const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(wr + c));
+            acc = fmaf(a.x, b.x, acc);
+            acc = fmaf(a.y, b.y, acc);
+        }
+        const float s0 = 1.0f / (1.0f + __expf(-warp_sum(acc)));
+        const float S = s0 / w[0];
 #pragma unroll
-        for (int j = 0; j < kMaxK; ++j) {
-            if (j >= k) break;
-            const __nv_bfloat16* wr = Wr + (size_t)idx[(size_t)t * k + j] * d;
-            float acc = 0.f;
-            for (int c = 2 * lane; c < d; c += 64) {
-                const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(xr + c));
-                const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(wr + c));
-                acc = fmaf(a.x, b.x, acc);
-                acc = fmaf(a.y, b.y, acc);
+        for (int j = 0; j < kMaxK; ++j)
+            if (j == lane) {
+                const float sj = w[j] * S;
+                v = (dw[j] - abar) / S * sj * (1.0f - sj);
             }
-            const float l = warp_sum(acc);
-            sc[j] = 1.0f / (1.0f + __expf(-l));
-            S += sc[j];
-        }
-        if (lane < k) {
-            float v = 0.f;
-#pragma unroll
-            for (int j = 0; j < kMaxK; ++j)
-                if (j == lane) v = (dw[j] - abar) / S * sc[j] * (1.0f - sc[j]);
-            dl[(size_t)t * k + lane] = v;
-        }
     } else {
-        if (lane < k) {
-            float v = 0.f;
 #pragma unroll
-            for (int j = 0; j < kMaxK; ++j)
-                if (j == lane) v = w[j] * (dw[j] - abar);
-            dl[(size_t)t * k + lane] = v;
-        }
+        for (int j = 0; j < kMaxK; ++j)
+            if (j == lane) v = w[j] * (dw[j] - abar);
     }
+    if (lane < k) dl[(size_t)t * k + lane] = v;
     pdl_trigger();
 }
 
