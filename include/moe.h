@@ -274,10 +274,13 @@ MOE_API int moe_expert_counts_noalloc(const int32_t *topk_idx, int T, int k, int
  *   dW_gate += dg x^T, dW_up += du x^T, dx += W_gate^T dg + W_up^T du.
  *
  * moe_saved_bytes -- bytes of the `saved` buffer of moe_forward_train (bf16
- * layers): the gate / up pre-activations, bf16, routed [T*k, 2*inter] (row
- * t*k + j = token t's j-th chosen expert; gate columns [0, inter), up columns
- * [inter, 2*inter)) followed by shared [T, 2*n_shared*inter] (gate columns of
- * all shared experts, then their up columns).  0 for invalid sizes.
+ * layers): the gate / up pre-activations, bf16, in blocks of 16 features.
+ * Routed part: [inter/16][T*k][16 gate | 16 up], rows in expert-contiguous
+ * order (expert 0's tokens in token order, then expert 1's, ...); then the
+ * shared part [n_shared*inter/16][T][16 gate | 16 up] (feature f of block b is
+ * shared feature 16 b + f, counting all shared experts' features in order).
+ * The layout lets each warp of the GEMMs write and read 32 rows x 64 B in one
+ * piece.  0 for invalid sizes.
  */
 MOE_API size_t moe_saved_bytes(int T, int k, int inter, int n_shared);
 

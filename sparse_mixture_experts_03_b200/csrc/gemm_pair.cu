@@ -92,6 +92,7 @@ struct __align__(16) PairTail {
     int seg_off[2][kMaxGroupsP];   // first token row of each group
     int tile_off[2][kMaxGroupsP];  // first tile of each group
     int cnt[2][kMaxGroupsP];       // token rows of each group
+    int useg_off[2][kMaxGroupsP];  // first row of each group with unpadded segments
 };
 
 // Load-ring shapes.  A stage holds the weight tile (32 KiB) and up to BMAX
@@ -364,29 +365,36 @@ __device__ __forceinline__ int dswiglu_src(const Tile& t, const PairArgs& a, int
     return a.row_src != nullptr ? a.row_src[r] : r;
 }
 
-__device__ __forceinline__ void dswiglu_fetch(const PairArgs& a, int src, int f0,
+// rf: the row's index in the forward's row order (the saved layout's rows);
+// features f0 .. f0 + 31 are two 16-feature blocks [16 gate | 16 up].
+__device__ __forceinline__ void dswiglu_fetch(const PairArgs& a, int src, int rf, int f0,
                                               DswigluRow& row) {
     row.src = src;
     row.w = 1.f;
     if (src < 0) return;
     if (a.row_src != nullptr) row.w = a.topk_w[src];
-    const uint4* gp = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.gu_in) +
-                                                     (size_t)src * 2 * a.feat + f0);
-    const uint4* up = gp + (a.feat >> 3);
+    const __nv_bfloat16* gu = static_cast<const __nv_bfloat16*>(a.gu_in);
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-        row.g[q] = __ldg(gp + q);
-        row.u[q] = __ldg(up + q);
+    for (int b = 0; b < 2; ++b) {
+        const uint4* p = reinterpret_cast<const uint4*>(
+            gu + ((size_t)((f0 >> 4) + b) * a.gu_rows + rf) * 32);
+        row.g[2 * b] = __ldg(p);
+        row.g[2 * b + 1] = __ldg(p + 1);
+        row.u[2 * b] = __ldg(p + 2);
+        row.u[2 * b + 1] = __ldg(p + 3);
     }
 }
 
 __device__ __forceinline__ void dswiglu_epilogue(uint8_t* wb, uint32_t taddr, const Tile& t,
                                                  const PairArgs& a, uint32_t cta, int wq,
-                                                 int lane) {
+                                                 int lane, int row_shift) {
     const int F = a.feat;
     const int f0 = t.ft * 256 + (int)cta * 128 + wq * 32;
+    // forward row of this tile's row r: r + row_shift (the forward's segments
+    // are unpadded, this launch's are padded to 128 rows)
+    const int rf0 = t.b_row + lane + row_shift;
     DswigluRow cur;
-    dswiglu_fetch(a, dswiglu_src(t, a, 0, lane), f0, cur);
+    dswiglu_fetch(a, dswiglu_src(t, a, 0, lane), rf0, f0, cur);
     int src_next = dswiglu_src(t, a, 32, lane);
 #pragma unroll 1
     for (int cc = 0; cc < kNTile / 32; ++cc) {
@@ -396,7 +404,7 @@ __device__ __forceinline__ void dswiglu_epilogue(uint8_t* wb, uint32_t taddr, co
         tmem_ld32(taddr + (uint32_t)c0, v);
         // the next chunk's reads go out before this chunk's work
         DswigluRow nxt;
-        dswiglu_fetch(a, c0 + 32 < t.n ? src_next : -1, f0, nxt);
+        dswiglu_fetch(a, c0 + 32 < t.n ? src_next : -1, rf0 + c0 + 32, f0, nxt);
         src_next = c0 + 64 < t.n ? dswiglu_src(t, a, c0 + 64, lane) : -1;
         tmem_ld_wait();
 #pragma unroll
@@ -515,11 +523,13 @@ __device__ __forceinline__ void dswiglu_epilogue(uint8_t* wb, uint32_t taddr, co
 // transpose through its staging buffer, then thread = token for the stores.
 template <int EPI>
 __device__ __forceinline__ void pair_epilogue(uint8_t* wb, uint32_t taddr, const Tile& t,
-                                              const PairArgs& a, uint32_t cta, int wq, int lane) {
+                                              const PairArgs& a, uint32_t cta, int wq, int lane,
+                                              int row_shift) {
     if constexpr (EPI == EPI_DSWIGLU) {
-        dswiglu_epilogue(wb, taddr, t, a, cta, wq, lane);
+        dswiglu_epilogue(wb, taddr, t, a, cta, wq, lane, row_shift);
         return;
     }
+    (void)row_shift;
     // SCATTER: slot index and gate weight of every token column of the tile,
     // loaded once per tile (lane l holds columns 32 c + l)
     int srcs[kNTile / 32];
@@ -572,25 +582,23 @@ __device__ __forceinline__ void pair_epilogue(uint8_t* wb, uint32_t taddr, const
                 d[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
                 d[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
                 if constexpr (EPI == EPI_SWIGLU_SAVE) {
-                    // the pre-activations for the backward, in slot (or token) order:
-                    // gate at columns [0, F), up at [F, 2F)
+                    // the pre-activations for the backward: blocks of 16 features,
+                    // [block][row][16 gate | 16 up] with this launch's row order, so
+                    // the warp's 32 consecutive rows are 2 KiB in one piece
                     const int r = t.b_row + c0 + lane;
-                    const int srow = a.row_src != nullptr ? a.row_src[r] : r;
+                    const int blk = (t.ft * a.out_col_step + (int)cta * 64 + wq * 16) >> 4;
                     uint32_t pg[8], pu[8];
 #pragma unroll
                     for (int p = 0; p < 8; ++p) {
                         pg[p] = pack_bf16x2(f[2 * p], f[2 * p + 1]);
                         pu[p] = pack_bf16x2(f[16 + 2 * p], f[16 + 2 * p + 1]);
                     }
-                    __nv_bfloat16* sv = static_cast<__nv_bfloat16*>(a.save) +
-                                        (size_t)srow * 2 * a.feat + t.ft * a.out_col_step +
-                                        cta * 64 + wq * 16;
-                    uint4* dg = reinterpret_cast<uint4*>(sv);
-                    uint4* du = reinterpret_cast<uint4*>(sv + a.feat);
-                    dg[0] = make_uint4(pg[0], pg[1], pg[2], pg[3]);
-                    dg[1] = make_uint4(pg[4], pg[5], pg[6], pg[7]);
-                    du[0] = make_uint4(pu[0], pu[1], pu[2], pu[3]);
-                    du[1] = make_uint4(pu[4], pu[5], pu[6], pu[7]);
+                    uint4* sv = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.save) +
+                                                         ((size_t)blk * a.gu_rows + r) * 32);
+                    sv[0] = make_uint4(pg[0], pg[1], pg[2], pg[3]);
+                    sv[1] = make_uint4(pg[4], pg[5], pg[6], pg[7]);
+                    sv[2] = make_uint4(pu[0], pu[1], pu[2], pu[3]);
+                    sv[3] = make_uint4(pu[4], pu[5], pu[6], pu[7]);
                 }
             }
             __syncwarp();
@@ -712,7 +720,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const PairArgs& a = p == 0 ? args0 : args1;
             const int ng = a.counts != nullptr ? a.n_groups : 1;
             const int al = a.seg_align > 1 ? a.seg_align : 1;
-            int carry_r = 0, carry_t = 0;
+            int carry_r = 0, carry_t = 0, carry_u = 0;
             for (int g0 = 0; g0 < ng; g0 += 32) {
                 const int g = g0 + lane;
                 const int c = g < ng ? (a.counts != nullptr ? a.counts[g] : a.static_rows) : 0;
@@ -720,23 +728,27 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int cr = (c + al - 1) / al * al;
                 const int tl = KIND == KIND_WGRAD ? (g < ng ? a.n_ftiles * a.n_ntiles : 0)
                                                   : ((c + kNTile - 1) / kNTile) * a.n_ftiles;
-                int ir = cr, it = tl;
+                int ir = cr, it = tl, iu = c;
 #pragma unroll
                 for (int o = 1; o < 32; o <<= 1) {
                     const int nr = __shfl_up_sync(0xffffffffu, ir, o);
                     const int nt = __shfl_up_sync(0xffffffffu, it, o);
+                    const int nu = __shfl_up_sync(0xffffffffu, iu, o);
                     if (lane >= o) {
                         ir += nr;
                         it += nt;
+                        iu += nu;
                     }
                 }
                 if (g < ng) {
                     tail->seg_off[p][g] = carry_r + ir - cr;
                     tail->tile_off[p][g] = carry_t + it - tl;
                     tail->cnt[p][g] = c;
+                    tail->useg_off[p][g] = carry_u + iu - c;
                 }
                 carry_r += __shfl_sync(0xffffffffu, ir, 31);
                 carry_t += __shfl_sync(0xffffffffu, it, 31);
+                carry_u += __shfl_sync(0xffffffffu, iu, 31);
             }
             if (lane == 0) {
                 tail->seg_off[p][ng] = carry_r;
@@ -1018,10 +1030,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t taddr =
                 tmem_base + (uint32_t)(acc * kNTile) + ((uint32_t)(wq * 32) << 16);
             // lane quarter wq = weight rows 32 wq .. 32 wq + 31 of this CTA
+            const int row_shift = tail->useg_off[t.p][t.g] - tail->seg_off[t.p][t.g];
             if (t.p == 0)
-                pair_epilogue<EPI0>(wstage, taddr, t, args0, cta, wq, lane);
+                pair_epilogue<EPI0>(wstage, taddr, t, args0, cta, wq, lane, row_shift);
             else
-                pair_epilogue<EPI1>(wstage, taddr, t, args1, cta, wq, lane);
+                pair_epilogue<EPI1>(wstage, taddr, t, args1, cta, wq, lane, row_shift);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(map_to_rank(&tail->tempty[acc], 0));

@@ -368,9 +368,9 @@ int forward_impl(const void* x, const void* W_router, const void* W_gate_up, con
         pr.sched_counter = status + kSchedWordGateUp;
         pr.wait_limit_ns = kWaitLimitNs;
         const bool train = saved != nullptr;
-        if (train) {  // pre-activations of routed row r go to saved row row_src[r]
+        if (train) {  // pre-activations in the saved layout, rows in this launch's order
             pr.save = saved;
-            pr.row_src = row_src;
+            pr.gu_rows = T * k;
             pr.feat = inter;
         }
         const int epi_gu = train ? EPI_SWIGLU_SAVE : EPI_SWIGLU;
@@ -389,6 +389,7 @@ int forward_impl(const void* x, const void* W_router, const void* W_gate_up, con
             ps.out_ld = SI;
             ps.a_blocks_per_group = 2 * SI / 16;
             ps.row_src = nullptr;  // shared rows are tokens
+            ps.gu_rows = T;
             ps.feat = SI;
             ps.save = train ? static_cast<char*>(saved) + (size_t)T * k * 2 * inter * 2 : nullptr;
             if (!make_map_gate_up(&mp.a[0], Wsh_gu, 1, SI, d) ||
@@ -792,6 +793,7 @@ MOE_API int moe_backward(const void* x, const void* W_router, const void* W_gate
         r.row_src = row_src;
         r.topk_w = topk_w;
         r.feat = inter;
+        r.gu_rows = T * k;
         r.gu_in = gu_routed;
         r.dgu_out = dgu;
         r.hw_out = hw;
@@ -804,6 +806,7 @@ MOE_API int moe_backward(const void* x, const void* W_router, const void* W_gate
             PairArgs sh = dense(r);
             sh.n_ftiles = SI / 256;
             sh.feat = SI;
+            sh.gu_rows = T;
             sh.gu_in = gu_shared;
             sh.dgu_out = dgu_sh;
             sh.hw_out = hw_sh;

@@ -173,11 +173,14 @@ struct PairArgs {
     int seg_align;           // group segments of B start at multiples of this (0 or 1: packed)
     int n_ntiles;            // KIND_WGRAD: 256-wide tiles along N
     int m_total;             // STORE_ROWS: output rows per group (n_ftiles * 256)
-    void* save;              // SWIGLU_SAVE: gate|up pre-activations, bf16 rows of 2F, row =
-                             // row_src[r] (routed) or the token (row_src == nullptr)
+    void* save;              // SWIGLU_SAVE: gate|up pre-activations, bf16, blocks of 16
+                             // features: [F/16][gu_rows][16 gate | 16 up], rows in this
+                             // launch's order (expert-contiguous, unpadded; or tokens)
+    int gu_rows;             // SWIGLU_SAVE / DSWIGLU: rows of the saved layout
     int feat;                // F: SwiGLU features of the problem (inter, or n_shared * inter)
     // DSWIGLU: acc = dh_raw [feature, row] = (W_down^T dy)[row]; w = topk_w[row_src[r]] (1 when
-    // row_src == nullptr); reads gate|up of row_src[r] (or r) from gu_in [*, 2F] bf16, writes
+    // row_src == nullptr); reads gate|up of the row's forward position (r minus the padding
+    // before its segment) from gu_in (the SWIGLU_SAVE layout), writes
     // dgu_out[r] = (dh * u * silu'(g) | dh * silu(g)) [2F] bf16, hw_out[r] = w * silu(g) * u [F]
     // bf16 and, with dw_part, dw_part[r * (F / 32) + part] = sum over the warp's 32 features of
     // dh_raw * silu(g) * u.

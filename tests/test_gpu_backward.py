@@ -126,16 +126,22 @@ def test_forward_train_output_equals_forward():
     torch.cuda.synchronize()
     assert torch.equal(y0, y1)
     # the saved pre-activations are the bf16 gate / up projections of the
-    # chosen experts' rows: spot-check against x . W in fp32
-    I = w.inter
-    sv = saved[: w.T * w.k * 2 * I * 2].view(torch.bfloat16).view(w.T * w.k, 2 * I).float().cpu()
+    # chosen experts' rows, in the documented layout: blocks of 16 features,
+    # [I/16][T*k][16 gate | 16 up], rows expert by expert in token order
+    I, Tk = w.inter, w.T * w.k
+    sv = saved[: Tk * 2 * I * 2].view(torch.bfloat16).view(I // 16, Tk, 32).float().cpu()
     x32, Wgu32 = inp.x.float(), inp.W_gate_up.float()
-    idx_c = idx.cpu()
+    idx_c = idx.cpu().numpy()
+    start = np.concatenate([[0], np.cumsum(np.bincount(idx_c.ravel(), minlength=w.E))])
     for t in (0, w.T // 2, w.T - 1):
         for j in range(w.k):
             e = int(idx_c[t, j])
-            ref = Wgu32[e] @ x32[t]
-            np.testing.assert_allclose(sv[t * w.k + j].numpy(), ref.numpy(), rtol=1e-2, atol=2e-2)
+            row = start[e] + int((idx_c[:t] == e).any(axis=1).sum())  # earlier tokens on e
+            ref = (Wgu32[e] @ x32[t]).numpy()
+            got_g = sv[:, row, :16].reshape(-1).numpy()
+            got_u = sv[:, row, 16:].reshape(-1).numpy()
+            np.testing.assert_allclose(got_g, ref[:I], rtol=1e-2, atol=2e-2)
+            np.testing.assert_allclose(got_u, ref[I:], rtol=1e-2, atol=2e-2)
 
 
 def test_backward_is_deterministic():
