@@ -345,14 +345,14 @@ __device__ __forceinline__ uint8_t* stage_chunk(uint8_t* wb, int row, int chunk)
 // SwiGLU backward epilogue (EPI_DSWIGLU) of one tile for warp quarter wq.
 // fp32 transpose (token row i: its 32 features), then lane = token row r:
 // dh_raw of features f0 .. f0 + 31 (the warp's TMEM lanes), the saved gate /
-// up pre-activations of the row's slot, and per feature
+// up pre-activations of the row (at its forward position), and per feature
 //   h = silu(g) u,  dh = w dh_raw,  dg = dh u silu'(g),  du = dh silu(g),
 //   hw = w h,  with silu'(g) = sigmoid(g) (1 + g (1 - sigmoid(g)));
 // the sum of dh_raw h over the 32 features is this warp's part of dL/dw.
 // The chunk loop stays rolled (its body is large: unrolled it would crowd
 // the instruction cache that the producer and MMA warps share), and the
-// global reads run ahead of it: the slot of each row two chunks ahead, its
-// gate weight and pre-activations one chunk ahead.
+// global reads run ahead of it: the slot of each row two chunks ahead (for its
+// gate weight), its gate weight and pre-activations one chunk ahead.
 struct DswigluRow {
     int src;
     float w;
