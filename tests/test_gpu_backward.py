@@ -315,3 +315,14 @@ def test_backward_with_selection_bias():
     assert_close(g.dW_gate_up.cpu().numpy(), ref.dW_gate_up, "dW_gate_up")
     assert_close(g.dW_down.cpu().numpy(), ref.dW_down, "dW_down")
     assert_close(g.dW_shared.cpu().numpy(), ref.dW_shared, "dW_shared")
+
+
+def test_full_size_sampled_skewed_batch():
+    """The load-skewed workload (40% of tokens on expert 0, T = 16384): rows
+    of the overloaded expert's gradients and of a light one, and dx rows."""
+    w = WORKLOADS["skewed"]
+    E, I, d, SI = w.E, w.inter, w.d, w.n_shared * w.inter
+    wsel = [(oracle.ROW_DWGU, 0 * 2 * I + 17), (oracle.ROW_DWGU, 0 * 2 * I + I + 900),
+            (oracle.ROW_DWD, 0 * d + 1234), (oracle.ROW_DWGU, 37 * 2 * I + 5),
+            (oracle.ROW_DWR, 0), (oracle.ROW_DWSH_GU, 333)]
+    sampled_check(w, [0, 8191, 16383], wsel)
