@@ -47,3 +47,34 @@ def test_flop_counter_equals_gemm_enumeration(d, E, k, I, S):
     # FusionLLM layer: 189.0 MFLOP per token
     if (d, E, k, I, S) == (2048, 64, 6, 1536, 4):
         assert abs(total / 1e6 - 189.0) < 0.1
+
+
+@pytest.mark.parametrize("d,E,k,I,S", [(2048, 64, 6, 1536, 4), (256, 8, 2, 256, 1)])
+def test_training_step_flops_equal_gemm_enumeration(d, E, k, I, S):
+    """The training step's FLOPs per token: the forward's GEMMs plus, per
+    chosen and shared expert, the input-gradient GEMMs (dh = W_down^T dy,
+    dx = W_gate^T dg + W_up^T du) and the weight-gradient GEMMs (dW_down,
+    dW_gate, dW_up), each with the shape of the forward GEMM it mirrors; and
+    for the router the gradient of the k chosen logits only (dx and
+    dW_router: 2*d*k each)."""
+    fwd = [(1, E, d)]
+    bwd = []
+    for _ in range(k + S):
+        fwd += [(1, I, d), (1, I, d), (1, d, I)]
+        bwd += [(1, I, d), (1, d, I), (1, d, I)]          # dh; dx from dg and du
+        bwd += [(d, I, 1), (I, d, 1), (I, d, 1)]          # dW_down, dW_gate, dW_up
+    bwd += [(1, d, k), (k, d, 1)]                         # router: dx, dW_router
+    per_token = sum(2 * m * n * kk for m, n, kk in fwd + bwd)
+    T = 1000
+    assert accounting.train_step_flops(T, d, E, k, I, S) == T * per_token
+    # forward + backward of the FusionLLM layer ≈ 3x the forward's expert work
+    if (d, E, k, I, S) == (2048, 64, 6, 1536, 4):
+        assert abs(per_token / accounting.flops_per_token(d, E, k, I, S) - 3.0) < 0.01
+
+
+def test_training_step_bytes():
+    T, d, E, k, I, S = 4096, 2048, 64, 6, 1536, 4
+    w = (E + S) * 3 * d * I + E * d        # every expert touched, plus shared and router
+    saved = 2 * I * (T * k + T * S) * 2    # bf16 gate | up per routed slot and shared row
+    want = 2 * w * 2 + w * 4 + 2 * T * d * 2 + 2 * T * d * 4 + 2 * saved
+    assert accounting.train_step_bytes(T, d, E, k, I, S, E) == want
