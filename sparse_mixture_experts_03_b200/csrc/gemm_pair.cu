@@ -206,6 +206,11 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar_cluster) {
     asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster)
                  : "memory");
 }
+// The same arrive without release semantics (orders no earlier memory access).
+__device__ __forceinline__ void mbar_arrive_cluster_relaxed(uint32_t bar_cluster) {
+    asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster)
+                 : "memory");
+}
 
 // Wait for phase `parity` of a local barrier whose arrivals may come from the
 // other CTA of the pair (acquire at cluster scope), bounded like
@@ -999,17 +1004,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ------------------------------------------------ epilogue (warps 2..5, both CTAs)
         const int wq = warp & 3;  // TMEM lane quarter this warp may access
         uint8_t* wstage = reinterpret_cast<uint8_t*>(tail->stage) + wq * 4096;
-        for (int it = 0;; ++it) {
-            Tile t{};
-            bool sched_ok = true;
-            if (lane == 0)
-                sched_ok = sched_get(tail, it, t, abort_flag, status, SITE_GEMM_EPILOGUE, limit);
-            sched_ok = __shfl_sync(0xffffffffu, (int)sched_ok, 0) != 0;
-            {
-                int* w = reinterpret_cast<int*>(&t);
+        // Entry `it` of the tile ring, broadcast to the warp.  The epilogue reads
+        // one entry ahead: entry it + 1 is taken once tile it's accumulator is
+        // ready and before tile it's stores, so the release that frees the
+        // ring entry does not wait for those stores to drain.
+        auto get_tile = [&](int it, Tile& t) {
+            bool ok = true;
+            if (lane == 0) ok = sched_get(tail, it, t, abort_flag, status, SITE_GEMM_EPILOGUE, limit);
+            int* w = reinterpret_cast<int*>(&t);
 #pragma unroll
-                for (int q = 0; q < 8; ++q) w[q] = __shfl_sync(0xffffffffu, w[q], 0);
-            }
+            for (int q = 0; q < 8; ++q) w[q] = __shfl_sync(0xffffffffu, w[q], 0);
+            return __shfl_sync(0xffffffffu, (int)ok, 0) != 0;
+        };
+        Tile t_next{};
+        bool ok_next = get_tile(0, t_next);
+        for (int it = 0;; ++it) {
+            const Tile t = t_next;
+            const bool sched_ok = ok_next;
             // the 4 warps read the same sequence: they vote before leaving so
             // that none is left waiting on a named barrier
             if (!epi_all(sched_ok)) {
@@ -1027,6 +1038,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 break;
             }
             tc_fence_after();
+            // the next ring entry (always published: the last tile is followed
+            // by an end entry)
+            ok_next = get_tile(it + 1, t_next);
             const uint32_t taddr =
                 tmem_base + (uint32_t)(acc * kNTile) + ((uint32_t)(wq * 32) << 16);
             // lane quarter wq = weight rows 32 wq .. 32 wq + 31 of this CTA
@@ -1035,9 +1049,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 pair_epilogue<EPI0>(wstage, taddr, t, args0, cta, wq, lane, row_shift);
             else
                 pair_epilogue<EPI1>(wstage, taddr, t, args1, cta, wq, lane, row_shift);
+            // The accumulator is free: tcgen05.wait::ld has completed this warp's
+            // TMEM reads, and the tcgen05 fence pair orders them before the MMA
+            // thread's reuse.  The arrive is relaxed: the tile's global stores
+            // need no ordering against the MMAs, and a release here would wait
+            // for all of them to drain.
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive_cluster(map_to_rank(&tail->tempty[acc], 0));
+            if (lane == 0) mbar_arrive_cluster_relaxed(map_to_rank(&tail->tempty[acc], 0));
         }
     }
 
