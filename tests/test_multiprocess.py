@@ -72,12 +72,14 @@ def test_two_gloo_ranks_replicas():
         assert r["cfg"]["parallelism"] == "token-parallel x2 (replicas)"
 
 
-def test_reference_arm_other_ranks_exit_quietly():
+@pytest.mark.parametrize("step", ["forward", "train"])
+def test_reference_arm_other_ranks_exit_quietly(step):
     """Under a launcher, the reference arm runs on rank 0 only; rank 1 prints
-    nothing and exits 0 (no GPU, no oracle work)."""
+    nothing and exits 0 (no GPU, no oracle work), for the forward and for the
+    training step."""
     env = dict(os.environ, RANK="1", WORLD_SIZE="2", LOCAL_RANK="1")
     r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
-                        "--steps", "1", "--warmup", "3"], env=env, capture_output=True,
-                       text=True, timeout=300)
+                        "--step", step, "--steps", "1", "--warmup", "3"], env=env,
+                       capture_output=True, text=True, timeout=300)
     assert r.returncode == 0, r.stderr
     assert r.stdout.strip() == ""
