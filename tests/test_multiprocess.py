@@ -1,7 +1,7 @@
 """Host-side multi-rank logic of the benchmark (token-parallel replicas), run as
 two gloo ranks on the CPU: rank setup from the launcher's environment,
-per-rank token batches with shared weights, barrier and max-over-ranks of the
-timings.  The data path has no collective, so nothing else crosses ranks."""
+per-rank token batches (and upstream gradients) with shared weights, barrier
+and max-over-ranks of the timings.  The data path has no collective, so nothing else crosses ranks."""
 import os
 import socket
 import subprocess
@@ -39,10 +39,15 @@ def _rank_main(rank: int, world: int, port: int, q):
         dist.all_gather(xs, x.float())
         ws = [torch.empty_like(inp.W_gate_up.float()) for _ in range(world)]
         dist.all_gather(ws, inp.W_gate_up.float())
+        # the training step's upstream gradient: each rank its own
+        dy = bench.dy_batch(w, got_rank).float()
+        dys = [torch.empty_like(dy) for _ in range(world)]
+        dist.all_gather(dys, dy)
         bench.barrier(got_world, cuda=False)
         mx = bench.max_over_ranks(float(10 + got_rank), got_world, device="cpu")
         q.put({"rank": got_rank, "world": got_world, "local": got_local, "max": mx,
                "x_differ": not torch.equal(xs[0], xs[1]),
+               "dy_differ": not torch.equal(dys[0], dys[1]),
                "w_same": torch.equal(ws[0], ws[1]),
                "cfg": bench.run_config(w, got_world)})
         dist.destroy_process_group()
@@ -67,7 +72,7 @@ def test_two_gloo_ranks_replicas():
         assert "error" not in r, r
         assert r["world"] == world and r["local"] == r["rank"]
         assert r["max"] == 10 + world - 1  # max over ranks, seen by every rank
-        assert r["x_differ"] and r["w_same"]
+        assert r["x_differ"] and r["w_same"] and r["dy_differ"]
         assert r["cfg"]["global_batch"] == world * 16
         assert r["cfg"]["parallelism"] == "token-parallel x2 (replicas)"
 
