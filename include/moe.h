@@ -234,12 +234,12 @@ MOE_API int moe_set_stage_events(void *const *events, int n);
  * of a routing result, for callers that must not allocate device memory or
  * pass a workspace on the call path (e.g. a serving step whose device memory
  * is planned once up front).  The pages have no counterpart of this entry
- * point: it is the histogram + scan of the permutation stage ("开源混合架构大模
- * 型技术解析", section 四: tokens grouped by the expert they go to), exposed on
- * its own with its scratch in a fixed device array of the library.
- *   topk_idx  device, int32[T, k]: expert ids (ids outside [0, E) are not
- *             counted)
- *   counts    device, int32[E]   out: tokens routed to each expert
+ * point; it computes the histogram and scan of the permutation stage on its
+ * own, with its scratch in a fixed device array of the library.
+ *   topk_idx  device, int32[T, k]: expert ids; every occurrence counts (a
+ *             row that repeats an id adds it as often as it appears); ids
+ *             outside [0, E) are skipped without an error
+ *   counts    device, int32[E]   out: occurrences of each expert id
  *   offsets   device, int32[E+1] out: exclusive prefix sum of counts
  *             (unpadded segments; offsets[E] = number of counted ids)
  * Limits: 1 <= k <= 8, k <= E <= 256, ceil(T/256) * E <= 65536 (the fixed

@@ -63,6 +63,8 @@ constexpr int kSchedDepth = 8;
 // readers of each ring entry: in CTA 0 the token producer, the MMA issuer and
 // the 4 epilogue warps; in CTA 1 both producers and the 4 epilogue warps
 constexpr int kSchedReaders = 2 * (2 + kEpiWarps);
+// bound of the producers' drain of issued copies when a launch gives up early
+constexpr uint64_t kAbortDrainNs = 1000000;  // 1 ms
 
 // One tile of a launch, decoded once by the scheduler and passed through the
 // ring as two 16-byte words.
@@ -843,6 +845,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t ph = 0;
             bool ok = true;
             int next = pair;
+            // stages this lane has issued a copy into, and the parity of the
+            // full-barrier phase of that copy (for the drain on abort)
+            uint32_t issued = 0, issued_ph = 0;
             for (int j = 0; ok; ++j) {
                 Tile t;
                 if (is_sched) {
@@ -913,9 +918,31 @@ __global__ void __launch_bounds__(kThreads, 1)
                                              ((t.ft * a.a_tile_step + (int)cta * a.a_cta_step) >> 4),
                                          atom);
                     }
+                    issued |= 1u << s;
+                    issued_ph = (issued_ph & ~(1u << s)) | (ph << s);
                     if (++s == kStages) {
                         s = 0;
                         ph ^= 1u;
+                    }
+                }
+            }
+            if (!ok) {
+                // Leaving early (a wait ran out or another role gave up): no
+                // copy this lane issued may still be writing this CTA's shared
+                // memory when the CTA exits.  In the pair's first CTA every
+                // issued stage's full barrier is waited for (it also counts
+                // the other CTA's bytes of that stage); a stage the other CTA
+                // never filled does not complete and ends the bounded wait.
+                // The second CTA cannot wait on those barriers, so it holds
+                // for a fixed settle time, far above a copy's latency.
+                if (cta == 0) {
+                    for (int st = 0; st < kStages; ++st)
+                        if (issued & (1u << st))
+                            mbar_wait_bounded(&tail->full[st], (issued_ph >> st) & 1u, nullptr,
+                                              status, SITE_GEMM_DRAIN, kAbortDrainNs);
+                } else if (issued != 0) {
+                    const uint64_t t0 = clock64();
+                    while ((uint64_t)clock64() - t0 < 2 * kAbortDrainNs) {
                     }
                 }
             }

@@ -9,6 +9,8 @@
 
 #include <utility>
 
+#include "../../include/moe.h"
+
 namespace moe {
 
 // Every kernel of the forward is launched with programmatic dependent launch:
@@ -55,6 +57,21 @@ constexpr int kSchedWordDown = 13;
 // the backward's four CTA-pair launches (the backward clears the whole status
 // region first)
 constexpr int kSchedWordBwd0 = 20;
+
+// Bound of every device-side wait of the forward and backward kernels.
+constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s per wait
+
+// ---- host helpers (host_util.cu)
+// E % n_group == 0, 1 <= topk_group <= n_group, k <= topk_group * E / n_group
+int check_routing(int E, int k, int n_group, int topk_group);
+// gate is a moe_gate; bias / load, when given, are 4-byte aligned device pointers
+int check_gating(int gate, const float* bias, const int32_t* load);
+bool aligned(const void* p, size_t a);
+// p is device or managed memory (a host pointer is caught before any launch)
+bool is_device_ptr(const void* p);
+// SM count of the current device (cached)
+int num_sms();
+inline int ret(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
 
 // Epilogue variants of the grouped GEMMs.
 enum Epi : int {
@@ -119,17 +136,21 @@ cudaError_t launch_permute(const int32_t* idx, int T, int k, int E, int32_t* blo
                            int32_t* counts, int32_t* offsets, int32_t* row_src, int align,
                            int32_t* load_out, int* status, cudaStream_t s,
                            int32_t* slot_row = nullptr);
+// x_perm[r] = x[row_src[r] / k] for the rows r < *offsets_total with row_src
+// >= 0; with w_dst also w_dst[r] = w_src[row_src[r]].
 cudaError_t launch_gather_rows(const void* x, int d, int elem_bytes, int k,
                                const int32_t* offsets_total, const int32_t* row_src,
-                               int rows_cap, void* x_perm, int num_sms, cudaStream_t s);
-// y[t] = base[t] + slots[t*k + 0] + ... + slots[t*k + k-1] in fp32, in that
-// order (base: fp32 [T, d] or nullptr for none).
-// Per-expert counts and unpadded segment offsets of a routing result
-// (histogram + scan only); block_counts holds ceil(T/256) * E int32.  Expert
-// ids outside [0, E) are not counted.
+                               int rows_cap, void* x_perm, int num_sms, cudaStream_t s,
+                               const float* w_src = nullptr, float* w_dst = nullptr);
+// Per-expert counts and unpadded segment offsets of a table of expert ids
+// (histogram + scan only); block_counts holds ceil(T/256) * E int32.  Every
+// occurrence of an id counts (a row may repeat one); ids outside [0, E) are
+// not counted.
 cudaError_t launch_expert_counts(const int32_t* idx, int T, int k, int E,
                                  int32_t* block_counts, int32_t* counts, int32_t* offsets,
                                  cudaStream_t s);
+// y[t] = base[t] + slots[t*k + 0] + ... + slots[t*k + k-1] in fp32, in that
+// order (base: fp32 [T, d] or nullptr for none).
 cudaError_t launch_combine_slots(const void* slots, int slots_bf16, const float* base, int T,
                                  int d, int k, void* y, int out_f32, cudaStream_t s);
 
@@ -199,6 +220,16 @@ struct PairMaps {
     CUtensorMap a[2];
     CUtensorMap b[2][kTokenBoxes];
 };
+// Tensor maps (bf16, 128-byte swizzle).  make_map_rows_atoms: a [rows, K]
+// matrix as {64, rows, K/64}, box {64, box_rows, 2} (box_rows rows x 128 of
+// K); make_token_maps: the kTokenBoxes maps of one token matrix (boxes of 16,
+// 32, ..., 128 rows); make_map_gate_up: a [G][2][F][K] gate/up weight as
+// {64, 16, 2, G*2F/16, K/64}, box {64, 16, 2, 4, 2} (4 x (16 gate rows, the
+// 16 matching up rows) x 128 of K).  False if the driver rejects the map.
+bool make_map_rows_atoms(CUtensorMap* m, const void* base, uint64_t rows, uint64_t K,
+                         uint32_t box_rows = 128);
+bool make_token_maps(CUtensorMap (&m)[kTokenBoxes], const void* base, uint64_t rows, uint64_t K);
+bool make_map_gate_up(CUtensorMap* m, const void* base, uint64_t G, uint64_t F, uint64_t K);
 // Epilogue pairs (epi0 for problem 0, epi1 for problem 1): SWIGLU/SWIGLU,
 // STORE_F32/SCATTER, SCATTER/SCATTER, SWIGLU_SAVE/SWIGLU_SAVE (KIND_FWD);
 // DSWIGLU/DSWIGLU, STORE_F32/SCATTER, SCATTER/SCATTER (KIND_DGRAD);

@@ -5,10 +5,10 @@
 // Who needs it: callers that must not allocate device memory (or hand over a
 // workspace) on the call path -- for instance a serving step whose device
 // memory is planned once up front, where a per-call allocation would either
-// synchronise the device or not fit the plan.  The operation is the
-// histogram + exclusive scan of the permutation stage (the dispatch step of
-// "开源混合架构大模型技术解析", section 四: tokens are grouped by the expert
-// they go to), with unpadded segments.
+// synchronise the device or not fit the plan.  The pages have no counterpart
+// of this entry point: it is the histogram + exclusive scan of the
+// permutation stage on its own, with unpadded segments.  Every occurrence of
+// an id counts, so a row that repeats an expert adds it twice.
 //
 // The scratch is the file-scope array below: nothing is allocated, no
 // allocating library is called.  Its device address is taken once per device

@@ -45,7 +45,11 @@ __device__ __forceinline__ bool holds(const int (&my)[kMaxK], int e) {
     return h;
 }
 
-// Histogram of each block of 256 tokens: block_counts[b][e].
+// Histogram of each block of 256 tokens: block_counts[b][e].  kCountIds
+// false: tokens that hold expert e (a routing result names an expert at most
+// once per token); true: occurrences of id e in the block's rows, so a row
+// that repeats an id counts it as often as it appears.
+template <bool kCountIds>
 __global__ void __launch_bounds__(kPermBlockTokens) perm_count_kernel(
     const int32_t* __restrict__ idx, int T, int k, int E, int32_t* __restrict__ block_counts,
     int* status) {
@@ -56,8 +60,16 @@ __global__ void __launch_bounds__(kPermBlockTokens) perm_count_kernel(
     int my[kMaxK];
     load_slots(idx, t, T, k, E, my, status);
     for (int e = 0; e < E; ++e) {
-        unsigned b = __ballot_sync(0xffffffffu, holds(my, e));
-        if (lane == 0) wcnt[warp][e] = __popc(b);
+        int c;
+        if constexpr (kCountIds) {
+            int m = 0;
+#pragma unroll
+            for (int j = 0; j < kMaxK; ++j) m += my[j] == e ? 1 : 0;
+            c = __reduce_add_sync(0xffffffffu, m);
+        } else {
+            c = __popc(__ballot_sync(0xffffffffu, holds(my, e)));
+        }
+        if (lane == 0) wcnt[warp][e] = c;
     }
     __syncthreads();
     for (int e = tid; e < E; e += kPermBlockTokens) {
@@ -265,12 +277,15 @@ __global__ void __launch_bounds__(kSmallTokens) perm_small_kernel(
 
 // x_perm[r] = x[row_src[r] / k] for every real row r < offsets[E]; one warp
 // per row, 16-byte vectors, up to 8 vectors per lane loaded before any store
-// so each lane keeps 8 loads in flight.
+// so each lane keeps 8 loads in flight.  With w_dst, also w_dst[r] =
+// w_src[row_src[r]] (the gate weight of the row's slot).
 __global__ void __launch_bounds__(256) gather_rows_kernel(const uint4* __restrict__ x,
                                                           int vec_per_row, int k,
                                                           const int32_t* __restrict__ total_rows,
                                                           const int32_t* __restrict__ row_src,
-                                                          uint4* __restrict__ x_perm) {
+                                                          uint4* __restrict__ x_perm,
+                                                          const float* __restrict__ w_src,
+                                                          float* __restrict__ w_dst) {
     const int lane = threadIdx.x & 31;
     const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int nw = (gridDim.x * blockDim.x) >> 5;
@@ -279,6 +294,7 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint4* __restric
     for (int r = gw; r < total; r += nw) {
         const int src = row_src[r];
         if (src < 0) continue;
+        if (w_dst != nullptr && lane == 0) w_dst[r] = w_src[src];
         const uint4* s = x + (size_t)(src / k) * vec_per_row;
         uint4* dst = x_perm + (size_t)r * vec_per_row;
         for (int i0 = 0; i0 < vec_per_row; i0 += 8 * 32) {
@@ -415,8 +431,8 @@ cudaError_t launch_permute(const int32_t* idx, int T, int k, int E, int32_t* blo
                           1, idx, T, k, E, align, counts, offsets, row_src, load_out, slot_row,
                           status);
     const int nb = (T + kPermBlockTokens - 1) / kPermBlockTokens;
-    cudaError_t e = launch_pdl(perm_count_kernel, dim3(nb), dim3(kPermBlockTokens), 0, s, 1, idx,
-                               T, k, E, block_counts, status);
+    cudaError_t e = launch_pdl(perm_count_kernel<false>, dim3(nb), dim3(kPermBlockTokens), 0, s,
+                               1, idx, T, k, E, block_counts, status);
     if (e != cudaSuccess) return e;
     e = launch_pdl(perm_scan_kernel, dim3(1), dim3(1024), 0, s, 1, block_counts, nb, E, align,
                    counts, offsets, row_src, load_out);
@@ -431,7 +447,8 @@ cudaError_t launch_expert_counts(const int32_t* idx, int T, int k, int E,
                                  cudaStream_t s) {
     const int nb = (T + kPermBlockTokens - 1) / kPermBlockTokens;
     if (nb > 0)
-        perm_count_kernel<<<nb, kPermBlockTokens, 0, s>>>(idx, T, k, E, block_counts, nullptr);
+        perm_count_kernel<true><<<nb, kPermBlockTokens, 0, s>>>(idx, T, k, E, block_counts,
+                                                                nullptr);
     // align 1: no padding rows, so the scan writes no row_src entry
     perm_scan_kernel<<<1, 1024, 0, s>>>(block_counts, nb, E, 1, counts, offsets, nullptr, nullptr);
     return cudaGetLastError();
@@ -439,14 +456,15 @@ cudaError_t launch_expert_counts(const int32_t* idx, int T, int k, int E,
 
 cudaError_t launch_gather_rows(const void* x, int d, int elem_bytes, int k,
                                const int32_t* offsets_total, const int32_t* row_src,
-                               int rows_cap, void* x_perm, int num_sms, cudaStream_t s) {
+                               int rows_cap, void* x_perm, int num_sms, cudaStream_t s,
+                               const float* w_src, float* w_dst) {
     const int vec = d * elem_bytes / 16;
     int blocks = num_sms * 8;
     const int need = (rows_cap + 7) / 8;
     if (blocks > need) blocks = need > 0 ? need : 1;
     return launch_pdl(gather_rows_kernel, dim3(blocks), dim3(256), 0, s, 1,
                       static_cast<const uint4*>(x), vec, k, offsets_total, row_src,
-                      static_cast<uint4*>(x_perm));
+                      static_cast<uint4*>(x_perm), w_src, w_dst);
 }
 
 cudaError_t launch_combine_slots(const void* slots, int slots_bf16, const float* base, int T,

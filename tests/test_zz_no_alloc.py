@@ -78,3 +78,27 @@ def test_sizes_beyond_the_fixed_scratch_are_rejected():
     ref = np.bincount(idx.cpu().numpy().ravel(), minlength=256)
     np.testing.assert_array_equal(counts.cpu().numpy(), ref)
     np.testing.assert_array_equal(offsets.cpu().numpy(), np.concatenate([[0], np.cumsum(ref)]))
+
+
+def test_repeated_and_out_of_range_ids_count_per_occurrence():
+    """Rows given by the caller may repeat an id ([3, 3] counts expert 3
+    twice) and may hold ids outside [0, E), which are skipped: the counts are
+    np.bincount of the in-range ids, on two calls in a row."""
+    E, k, T = 16, 4, 1000
+    g = torch.Generator().manual_seed(5)
+    idx = torch.randint(0, E, (T, k), generator=g, dtype=torch.int32)
+    idx[::3, 1] = idx[::3, 0]             # repeats inside a row
+    idx[7] = torch.tensor([3, 3, 3, 3])
+    idx[11, 2] = E                        # out of range: skipped
+    idx[13, 0] = -1
+    ids = idx.numpy().ravel()
+    ref = np.bincount(ids[(ids >= 0) & (ids < E)], minlength=E)
+    idx_d = idx.to(DEV)
+    for _ in range(2):
+        counts = torch.full((E,), -7, dtype=torch.int32, device=DEV)
+        offsets = torch.full((E + 1,), -7, dtype=torch.int32, device=DEV)
+        moe.expert_counts_noalloc(idx_d, E, counts, offsets)
+        torch.cuda.synchronize()
+        np.testing.assert_array_equal(counts.cpu().numpy(), ref)
+        np.testing.assert_array_equal(offsets.cpu().numpy(),
+                                      np.concatenate([[0], np.cumsum(ref)]))
