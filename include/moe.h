@@ -355,6 +355,103 @@ MOE_API int moe_backward(const void *x, const void *W_router, const void *W_gate
 #define MOE_N_BWD_STAGE_EVENTS 9
 MOE_API int moe_set_backward_stage_events(void *const *events, int n);
 
+/*
+ * ---- Expert parallelism ---------------------------------------------------
+ *
+ * The layer spread over n_ranks GPUs, rank r holding the routed experts
+ * [r E_l, (r+1) E_l) (E_l = E / n_ranks) and a copy of the router and shared
+ * experts: each rank routes its own tokens, sends each chosen (token, expert)
+ * row to the rank that owns the expert, the owners run their experts on what
+ * they received, and the weighted results come back to be summed
+ * ("大模型工程（一）：Transformer 到 MoE", section "混合专家：更多参数，相同 FLOPs":
+ * experts on different GPUs, token exchange by all-to-all over NVLink; its
+ * Mixtral / Qwen3-MoE / DeepSeek-V3 comparison: expert groups per GPU).  The
+ * two exchanges are the caller's (NCCL all-to-all); these calls are the
+ * compute around them.  bf16 layers only (else MOE_ERR_UNSUPPORTED); d a
+ * multiple of 256 and inter of 128.  Results equal moe_forward's: the same
+ * routing, the same fp32-accumulated expert GEMMs, each routed row scaled by
+ * its gate weight and rounded once to bf16, and the same fixed-order sum.
+ *
+ * moe_dispatch_workspace_bytes -- scratch bytes of moe_dispatch (0 if invalid).
+ */
+MOE_API size_t moe_dispatch_workspace_bytes(int T, int E, int k);
+
+/*
+ * moe_dispatch -- routing (as moe_route_ex) and the permutation of this
+ * rank's T tokens into expert-contiguous rows.
+ *   topk_idx, topk_w  device int32 / f32 [T, k] out: the routing
+ *   counts     device int32 [E] out: rows for each expert (destination rank
+ *              of expert e: e / E_l, so rank q's rows are the contiguous
+ *              block of experts [q E_l, (q+1) E_l))
+ *   x_perm     device bf16 [T*k, d] out: row r is x of the token of slot
+ *              t*k + j, rows ordered by expert, inside an expert by token
+ *   w_perm     device f32 [T*k] out: the gate weight w_j of row r
+ *   slot_row   device int32 [T*k] out: slot t*k + j -> its row r
+ *   workspace  device, moe_dispatch_workspace_bytes, 256-byte aligned
+ * Other arguments and errors as moe_route_ex.  T = 0 zeroes counts.
+ */
+MOE_API int moe_dispatch(const void *x, const void *W_router, int T, int d, int E, int k,
+                         int n_group, int topk_group, int in_dt, int gate,
+                         const float *expert_bias, int32_t *topk_idx, float *topk_w,
+                         int32_t *counts, void *x_perm, float *w_perm, int32_t *slot_row,
+                         void *workspace, size_t workspace_bytes, void *stream);
+
+/* moe_experts_workspace_bytes -- scratch bytes of moe_experts_forward for R
+ * received rows (0 if invalid). */
+MOE_API size_t moe_experts_workspace_bytes(int R, int d, int E_local, int inter);
+
+/*
+ * moe_experts_forward -- the local experts on the rows this rank received.
+ *   x_rows       device bf16 [R, d]: the received rows, grouped by source
+ *                rank (0, 1, ...), inside a source by local expert, in the
+ *                source's order (the concatenation of the sources' x_perm
+ *                blocks for this rank)
+ *   w_rows       device f32 [R]: the gate weight of each received row
+ *   recv_counts  device int32 [n_src, E_local]: rows from each source for
+ *                each local expert (sum = R; a sum above R computes nothing
+ *                and sets MOE_ERR_DEVICE in the status word)
+ *   W_gate_up    device bf16 [E_local, 2*inter, d], W_down [E_local, d, inter]:
+ *                this rank's experts
+ *   y_rows       device bf16 [R, d] out: row i = w_rows[i] * SwiGLU expert
+ *                of row i (fp32 accumulation, rounded once), in the receive
+ *                order, ready to be sent back
+ *   workspace    moe_experts_workspace_bytes(R, ...), 256-byte aligned; its
+ *                first 256 bytes are the status word (moe_get_device_status)
+ * Limits: n_src * E_local <= 2048.  R = 0 queues nothing.
+ */
+MOE_API int moe_experts_forward(const void *x_rows, const float *w_rows,
+                                const int32_t *recv_counts, int n_src, int R,
+                                const void *W_gate_up, const void *W_down, int d, int E_local,
+                                int inter, int in_dt, void *y_rows, void *workspace,
+                                size_t workspace_bytes, void *stream);
+
+/* moe_shared_workspace_bytes -- scratch bytes of moe_shared_forward. */
+MOE_API size_t moe_shared_workspace_bytes(int T, int d, int inter, int n_shared);
+
+/*
+ * moe_shared_forward -- the n_shared >= 1 shared experts on T tokens:
+ * y_shared = sum_s SwiGLU_shared_s(x), device f32 [T, d] out (W_shared laid
+ * out as for moe_forward).  Independent of the exchange: it can run on
+ * another stream while the rows are in flight.
+ */
+MOE_API int moe_shared_forward(const void *x, const void *W_shared, int T, int d, int inter,
+                               int n_shared, int in_dt, float *y_shared, void *workspace,
+                               size_t workspace_bytes, void *stream);
+
+/*
+ * moe_combine -- y[t] = shared[t] + rows[slot_row[t*k + 0]] + ... +
+ * rows[slot_row[t*k + k-1]] in fp32, in that order (bitwise reproducible).
+ *   rows      device bf16 [n_rows, d]: the rows sent back, in x_perm order
+ *   slot_row  device int32 [T*k]: moe_dispatch's slot_row
+ *   shared    device f32 [T, d] or NULL (no shared experts)
+ *   y         device out_dt [T, d] out
+ *   status_ws device workspace whose status word receives MOE_ERR_DEVICE
+ *             for a slot_row entry outside [0, n_rows), or NULL
+ */
+MOE_API int moe_combine(const void *rows, int n_rows, const int32_t *slot_row,
+                        const float *shared, int T, int d, int k, int out_dt, void *y,
+                        void *status_ws, void *stream);
+
 /* moe_status_string -- static text for a status code. */
 MOE_API const char *moe_status_string(int status);
 

@@ -37,7 +37,9 @@ SYMBOLS = ["moe_workspace_bytes", "moe_workspace_layout", "moe_route", "moe_forw
            "moe_set_stage_events", "moe_status_string", "moe_version",
            "moe_expert_counts_noalloc", "moe_route_ex", "moe_forward_ex", "moe_saved_bytes",
            "moe_forward_train", "moe_backward_workspace_bytes", "moe_backward",
-           "moe_set_backward_stage_events"]
+           "moe_set_backward_stage_events", "moe_dispatch_workspace_bytes", "moe_dispatch",
+           "moe_experts_workspace_bytes", "moe_experts_forward", "moe_shared_workspace_bytes",
+           "moe_shared_forward", "moe_combine"]
 GATES = {"sigmoid": 0, "softmax": 1}  # MOE_GATE_SIGMOID, MOE_GATE_SOFTMAX_TOPK
 N_STAGE_EVENTS = 6
 STAGES = ["route", "permute", "gate_up", "down", "combine"]
@@ -96,6 +98,20 @@ def lib() -> ctypes.CDLL:
         L.moe_backward.restype = i
         L.moe_set_backward_stage_events.argtypes = [ctypes.POINTER(vp), i]
         L.moe_set_backward_stage_events.restype = i
+        L.moe_dispatch_workspace_bytes.argtypes = [i] * 3
+        L.moe_dispatch_workspace_bytes.restype = sz
+        L.moe_dispatch.argtypes = [vp, vp] + [i] * 8 + [vp] * 8 + [sz, vp]
+        L.moe_dispatch.restype = i
+        L.moe_experts_workspace_bytes.argtypes = [i] * 4
+        L.moe_experts_workspace_bytes.restype = sz
+        L.moe_experts_forward.argtypes = [vp, vp, vp, i, i, vp, vp, i, i, i, i, vp, vp, sz, vp]
+        L.moe_experts_forward.restype = i
+        L.moe_shared_workspace_bytes.argtypes = [i] * 4
+        L.moe_shared_workspace_bytes.restype = sz
+        L.moe_shared_forward.argtypes = [vp, vp, i, i, i, i, i, vp, vp, sz, vp]
+        L.moe_shared_forward.restype = i
+        L.moe_combine.argtypes = [vp, i, vp, vp, i, i, i, i, vp, vp, vp]
+        L.moe_combine.restype = i
         _lib = L
     return _lib
 
@@ -337,6 +353,94 @@ def set_backward_stage_events(events) -> None:
         *[ctypes.c_void_p(e.cuda_event if e is not None else None) for e in events])
     _check(lib().moe_set_backward_stage_events(arr, len(events)),
            "moe_set_backward_stage_events")
+
+
+# ---- expert parallelism (the compute on either side of the all-to-all exchanges)
+
+class Dispatched:
+    """One rank's moe_dispatch result: topk_idx / topk_w [T,k], counts int32
+    [E] (rows per expert), x_perm bf16 [T*k,d] (rows by expert, then token),
+    w_perm f32 [T*k] (each row's gate weight), slot_row int32 [T*k] (slot
+    t*k+j -> its row)."""
+
+    def __init__(self, topk_idx, topk_w, counts, x_perm, w_perm, slot_row):
+        self.topk_idx, self.topk_w, self.counts = topk_idx, topk_w, counts
+        self.x_perm, self.w_perm, self.slot_row = x_perm, w_perm, slot_row
+
+
+def _scratch(n: int, device) -> torch.Tensor:
+    if n == 0:
+        raise MoeError(MOE_ERR_INVALID_ARG, "workspace size")
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def dispatch(x: torch.Tensor, W_router: torch.Tensor, k: int, n_group: int, topk_group: int,
+             gate: str = "sigmoid", expert_bias: Optional[torch.Tensor] = None,
+             workspace: Optional[torch.Tensor] = None, stream=None) -> Dispatched:
+    """moe_dispatch: routing and expert-contiguous rows of this rank's tokens."""
+    T, d = x.shape
+    E = W_router.shape[0]
+    dev = x.device
+    out = Dispatched(torch.empty(T, k, dtype=torch.int32, device=dev),
+                     torch.empty(T, k, dtype=torch.float32, device=dev),
+                     torch.empty(E, dtype=torch.int32, device=dev),
+                     torch.empty(T * k, d, dtype=x.dtype, device=dev),
+                     torch.empty(T * k, dtype=torch.float32, device=dev),
+                     torch.empty(T * k, dtype=torch.int32, device=dev))
+    if workspace is None:
+        workspace = _scratch(lib().moe_dispatch_workspace_bytes(T, E, k), dev)
+    _check(lib().moe_dispatch(_ptr(x), _ptr(W_router), T, d, E, k, n_group, topk_group, _dt(x),
+                              GATES[gate], _ptr(expert_bias), _ptr(out.topk_idx),
+                              _ptr(out.topk_w), _ptr(out.counts), _ptr(out.x_perm),
+                              _ptr(out.w_perm), _ptr(out.slot_row), _ptr(workspace),
+                              workspace.numel(), _stream(stream)), "moe_dispatch")
+    return out
+
+
+def experts_forward(x_rows: torch.Tensor, w_rows: torch.Tensor, recv_counts: torch.Tensor,
+                    W_gate_up: torch.Tensor, W_down: torch.Tensor, inter: int,
+                    y_rows: Optional[torch.Tensor] = None,
+                    workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """moe_experts_forward: y_rows bf16 [R,d] = w * local expert(row), in the
+    receive order; recv_counts int32 [n_src, E_local] on the device."""
+    R, d = x_rows.shape
+    n_src, E_l = recv_counts.shape
+    if y_rows is None:
+        y_rows = torch.empty(R, d, dtype=x_rows.dtype, device=x_rows.device)
+    if workspace is None:
+        workspace = _scratch(lib().moe_experts_workspace_bytes(R, d, E_l, inter), x_rows.device)
+    _check(lib().moe_experts_forward(_ptr(x_rows), _ptr(w_rows), _ptr(recv_counts), n_src, R,
+                                     _ptr(W_gate_up), _ptr(W_down), d, E_l, inter, _dt(x_rows),
+                                     _ptr(y_rows), _ptr(workspace), workspace.numel(),
+                                     _stream(stream)), "moe_experts_forward")
+    return y_rows
+
+
+def shared_forward(x: torch.Tensor, W_shared: torch.Tensor, inter: int, n_shared: int,
+                   y_shared: Optional[torch.Tensor] = None,
+                   workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """moe_shared_forward: fp32 [T,d] sum of the shared experts."""
+    T, d = x.shape
+    if y_shared is None:
+        y_shared = torch.empty(T, d, dtype=torch.float32, device=x.device)
+    if workspace is None:
+        workspace = _scratch(lib().moe_shared_workspace_bytes(T, d, inter, n_shared), x.device)
+    _check(lib().moe_shared_forward(_ptr(x), _ptr(W_shared), T, d, inter, n_shared, _dt(x),
+                                    _ptr(y_shared), _ptr(workspace), workspace.numel(),
+                                    _stream(stream)), "moe_shared_forward")
+    return y_shared
+
+
+def combine(rows: torch.Tensor, slot_row: torch.Tensor, shared: Optional[torch.Tensor], T: int,
+            k: int, out_dtype: torch.dtype = torch.float32, y: Optional[torch.Tensor] = None,
+            status_ws: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """moe_combine: y [T,d] = shared + the k rows of each token, in order."""
+    n_rows, d = rows.shape
+    if y is None:
+        y = torch.empty(T, d, dtype=out_dtype, device=rows.device)
+    _check(lib().moe_combine(_ptr(rows), n_rows, _ptr(slot_row), _ptr(shared), T, d, k, _dt(y),
+                             _ptr(y), _ptr(status_ws), _stream(stream)), "moe_combine")
+    return y
 
 
 class MoELayer:
