@@ -30,7 +30,8 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 from sparse_mixture_experts_03_b200 import accounting, moe  # noqa: E402
-from sparse_mixture_experts_03_b200.inputs import WORKLOADS, _randn, make_inputs  # noqa: E402
+from sparse_mixture_experts_03_b200.inputs import (  # noqa: E402
+    SKEW_SHIFT, WORKLOADS, _randn, make_inputs)
 
 METRIC = "MoE layer tokens/sec and TFLOP/s at 1 B200; % of roofline (TC or HBM)"
 L2_FLUSH_BYTES = 512 << 20  # > 126 MB L2
@@ -147,10 +148,15 @@ def barrier(world: int, cuda: bool = True):
 
 def rank_batch(w, inp, rank: int) -> torch.Tensor:
     """Token batch of one rank (host tensor): rank 0 takes the workload's x,
-    rank r > 0 its own draw (seed + r); the weights are the same on every rank."""
+    rank r > 0 its own draw (seed + r), shifted along the same skew direction
+    as rank 0's for the load-skewed workload; the weights are the same on
+    every rank."""
     if rank == 0:
         return inp.x
-    return _randn((w.T, w.d), w.seed + rank, 0).to(inp.x.dtype)
+    x = _randn((w.T, w.d), w.seed + rank, 0)
+    if w.skew:
+        x.add_(inp.skew_u, alpha=SKEW_SHIFT)
+    return x.to(inp.x.dtype)
 
 
 def profiled_traffic(w):

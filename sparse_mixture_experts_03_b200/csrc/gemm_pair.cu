@@ -165,6 +165,23 @@ __device__ __forceinline__ void tma_load_5d_pair(void* smem_dst, const CUtensorM
         "r"(c3), "r"(c4)
         : "memory");
 }
+// L2 prefetch of the box of a tensor map at these coordinates (no shared
+// memory written, no completion to wait for).
+__device__ __forceinline__ void tma_prefetch_l2_3d(const CUtensorMap* map, int c0, int c1,
+                                                   int c2) {
+    asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(c0), "r"(c1), "r"(c2)
+                 : "memory");
+}
+__device__ __forceinline__ void tma_prefetch_l2_5d(const CUtensorMap* map, int c0, int c1, int c2,
+                                                   int c3, int c4) {
+    asm volatile(
+        "cp.async.bulk.prefetch.tensor.5d.L2.global.tile [%0, {%1, %2, %3, %4, %5}];" ::"l"(
+            reinterpret_cast<uint64_t>(map)),
+        "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(c4)
+        : "memory");
+}
 __device__ __forceinline__ void arrive_expect_tx_local(uint64_t* bar, uint32_t bytes) {
     mbar_arrive_expect_tx(bar, bytes);
 }
@@ -717,6 +734,47 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tail->abort = 0;
         fence_barrier_init();
+    }
+    if (KIND == KIND_FWD && warp == 0 && lane == 0) {
+        // The weights are inputs no earlier kernel writes: while the previous
+        // kernels (routing, permutation) finish, bring this CTA's half of the
+        // weight tile of the pair's first tile into L2.  The first tile is
+        // the pair's index; a problem with expert counts (not yet known here)
+        // is taken to have one token chunk per expert, as at small batches
+        // (a wrong guess only prefetches a tile another pair will load).
+        int lt = pair, p = 0;
+        const int ng0_s = args0.counts != nullptr ? args0.n_groups : 1;
+        if (args0.counts == nullptr && n_problems > 1) {
+            const int tiles0_s = ((args0.static_rows + kNTile - 1) / kNTile) * args0.n_ftiles;
+            if (lt >= tiles0_s) {
+                lt -= tiles0_s;
+                p = 1;
+            }
+        }
+        const PairArgs& a = p == 0 ? args0 : args1;
+        const int ng = p == 0 ? ng0_s : (args1.counts != nullptr ? args1.n_groups : 1);
+        int g, ft;
+        if (a.counts == nullptr) {
+            g = 0;
+            ft = lt % a.n_ftiles;
+        } else {
+            g = lt / a.n_ftiles;
+            ft = lt % a.n_ftiles;
+        }
+        if (g < ng && a.n_ftiles > 0) {
+            const CUtensorMap* m = &maps.a[p];
+            const int kb_n = a.K / kBK;
+            const int a_row0 = (int)(g * a.a_group_stride) + ft * a.a_tile_step +
+                               (int)cta * a.a_cta_step;
+            const int blk = g * a.a_blocks_per_group +
+                            ((ft * a.a_tile_step + (int)cta * a.a_cta_step) >> 4);
+            for (int kb = 0; kb < kb_n; ++kb) {
+                if (a.a_mode == 0)
+                    tma_prefetch_l2_3d(m, 0, a_row0, kb * kAtoms);
+                else
+                    tma_prefetch_l2_5d(m, 0, 0, 0, blk, kb * kAtoms);
+            }
+        }
     }
     // everything below reads or writes memory of earlier kernels (counts,
     // token rows, outputs): wait until the previous kernel has completed

@@ -159,8 +159,9 @@ def test_permutation_stage_prefill():
     permutation_check(w, inp, idx, ws)
 
 
-def test_permutation_stage_small_ragged():
-    w = SMALL[2][1]
+@pytest.mark.parametrize("i", [1, 2], ids=["f32_shared", "bf16_ragged"])
+def test_permutation_stage_small_ragged(i):
+    w = SMALL[i][1]
     inp = make_inputs(w)
     y, idx, wt, ws = run_forward(w, inp)
     permutation_check(w, inp, idx, ws)
