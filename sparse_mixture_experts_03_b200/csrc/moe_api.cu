@@ -1,12 +1,15 @@
 // C ABI of the MoE layer forward: argument checks, workspace layout, TMA
 // descriptors and the launch sequence
-//   route -> permute (histogram, scan, rank) -> gather rows
+//   route -> permute (histogram, scan, stable ranks) and gather rows, in one
+//   launch
 //   -> gate/up grouped GEMM + SwiGLU (routed; shared)
 //   -> down grouped GEMM with weighted scatter to token-order slots (routed)
 //   -> down GEMM of the shared experts with the fixed-order final sum.
 // Everything runs on the caller's stream; nothing here synchronises it except
 // moe_get_device_status, and nothing here allocates device memory.
 #include <cudaTypedefs.h>
+
+#include <algorithm>
 #include <limits.h>
 #include <stdlib.h>
 #include <string.h>
@@ -49,7 +52,9 @@ bool make_layout(int T, int d, int E, int k, int inter, int n_shared, int in_dt,
         sizeof(int) * kStatusWords,                     // STATUS
         sizeof(int) * E,                                // COUNTS
         sizeof(int) * (E + 1),                          // OFFSETS
-        sizeof(int) * (size_t)(L.nb > 0 ? L.nb : 1) * E,  // BLOCK_COUNTS
+        // BLOCK_COUNTS: per 256-token block, or per CTA (<= ceil(T/32)) of the
+        // one-launch permutation
+        sizeof(int) * (size_t)std::max(std::max(L.nb, (T + 31) / 32), 1) * E,
         sizeof(int) * Tk,                               // TOPK_IDX
         sizeof(float) * Tk,                             // TOPK_W
         sizeof(int) * (size_t)L.rows_cap,               // ROW_SRC
@@ -232,11 +237,22 @@ int forward_impl(const void* x, const void* W_router, const void* W_gate_up, con
     // 2. permutation: histogram, scan, stable ranks, row gather
     // the CTA-pair GEMMs (bf16) take unpadded expert segments; the CUDA-core
     // kernels (fp32) take segments padded to their 128-row tiles
-    e = launch_permute(idx, T, k, E, block_counts, counts, offsets, row_src,
-                       bf16 ? 1 : kRowAlign, expert_load, status, s);
-    if (e != cudaSuccess) return MOE_ERR_CUDA;
-    e = launch_gather_rows(x, d, bf16 ? 2 : 4, k, offsets + E, row_src, L.rows_cap, x_perm,
-                           num_sms(), s);
+    if (T <= kSmallPermTokens) {
+        e = launch_permute_gather_small(idx, T, k, E, bf16 ? 1 : kRowAlign, counts, offsets,
+                                        row_src, expert_load, status, x, d, bf16 ? 2 : 4,
+                                        x_perm, num_sms(), s);
+    } else if (permute_gather_grid_fits(T, E, num_sms())) {
+        e = launch_permute_gather_grid(idx, T, k, E, bf16 ? 1 : kRowAlign, block_counts, counts,
+                                       offsets, row_src, expert_load, status,
+                                       status + kGridBarWordPermute, kWaitLimitNs, x, d,
+                                       bf16 ? 2 : 4, x_perm, num_sms(), s);
+    } else {
+        e = launch_permute(idx, T, k, E, block_counts, counts, offsets, row_src,
+                           bf16 ? 1 : kRowAlign, expert_load, status, s);
+        if (e != cudaSuccess) return MOE_ERR_CUDA;
+        e = launch_gather_rows(x, d, bf16 ? 2 : 4, k, offsets + E, row_src, L.rows_cap, x_perm,
+                               num_sms(), s);
+    }
     if (e != cudaSuccess) return MOE_ERR_CUDA;
     stage_mark(2, s);
 

@@ -201,6 +201,7 @@ __global__ void __launch_bounds__(kPermBlockTokens) perm_rank_kernel(
 // token order).
 constexpr int kSmallTokens = 1024;
 constexpr int kSmallWarps = kSmallTokens / 32;
+constexpr int kPermGatherThreads = 512;
 
 __global__ void __launch_bounds__(kSmallTokens) perm_small_kernel(
     const int32_t* __restrict__ idx, int T, int k, int E, int align, int32_t* __restrict__ counts,
@@ -272,6 +273,287 @@ __global__ void __launch_bounds__(kSmallTokens) perm_small_kernel(
             row_src[pos] = tid * k + j;
             if (slot_row != nullptr) slot_row[tid * k + j] = pos;
         }
+    pdl_trigger();
+}
+
+// Copy token row t of x into row `row` of x_perm: one warp, 16-byte vectors,
+// up to 8 per lane in flight.
+__device__ __forceinline__ void copy_row_warp(const uint4* __restrict__ x, int vec_per_row, int t,
+                                              uint4* __restrict__ x_perm, int row, int lane) {
+    const uint4* src = x + (size_t)t * vec_per_row;
+    uint4* dst = x_perm + (size_t)row * vec_per_row;
+    for (int i0 = 0; i0 < vec_per_row; i0 += 8 * 32) {
+        uint4 v[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int i = i0 + u * 32 + lane;
+            if (i < vec_per_row) v[u] = __ldg(src + i);
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int i = i0 + u * 32 + lane;
+            if (i < vec_per_row) dst[i] = v[u];
+        }
+    }
+}
+
+// Small batches (T <= 1024) in one launch of several CTAs: every CTA derives
+// the whole permutation from the routing result on chip, CTA 0 writes it out
+// (counts, offsets, row_src, padding rows, slot_row), and all CTAs copy token
+// rows into x_perm, one warp per (token, slot).  Same layout and order as the
+// kernels above; a routing result names an expert at most once per token.
+//
+// Stable ranks come from a bitmap per expert over the tokens: bit t of
+// bits[e] is set when token t chose e, so the rank of token t inside
+// segment e is the number of set bits below t -- a per-word prefix count plus
+// one masked popcount, independent of E.
+__global__ void __launch_bounds__(kPermGatherThreads) perm_gather_small_kernel(
+    const int32_t* __restrict__ idx, int T, int k, int E, int align,
+    int32_t* __restrict__ counts, int32_t* __restrict__ offsets, int32_t* __restrict__ row_src,
+    int32_t* __restrict__ load_out, int32_t* __restrict__ slot_row, int* status,
+    const uint4* __restrict__ x, int vec_per_row, uint4* __restrict__ x_perm) {
+    extern __shared__ __align__(16) uint32_t pg_sm[];
+    const int W = (T + 31) >> 5;  // bitmap words per expert
+    uint32_t* bits = pg_sm;                                     // [E][W]
+    int* pre = reinterpret_cast<int*>(bits + (size_t)E * W);    // [E][W] bits below word w
+    int* s_cnt = pre + (size_t)E * W;                           // [E]
+    int* s_off = s_cnt + E;                                     // [E + 1]
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int nwarps = blockDim.x >> 5;
+    const int n_slots = T * k;
+    const bool writer = blockIdx.x == 0;
+    for (int i = tid; i < E * W; i += blockDim.x) bits[i] = 0u;
+    pdl_wait();
+    __syncthreads();
+    for (int s = tid; s < n_slots; s += blockDim.x) {
+        const int e = idx[s];
+        if (e < 0 || e >= E) {
+            if (writer) set_status(status, MOE_ERR_DEVICE, SITE_PERMUTE, e);
+            continue;
+        }
+        const int t = s / k;
+        atomicOr(&bits[e * W + (t >> 5)], 1u << (t & 31));
+    }
+    __syncthreads();
+    // per expert (one warp each): exclusive prefix of the word popcounts
+    for (int e = warp; e < E; e += nwarps) {
+        const int v = lane < W ? __popc(bits[e * W + lane]) : 0;
+        int incl = v;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int n = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += n;
+        }
+        if (lane < W) pre[e * W + lane] = incl - v;
+        if (lane == 31) s_cnt[e] = incl;
+    }
+    __syncthreads();
+    if (warp == 0) {  // segment offsets: exclusive scan of the padded sizes
+        int carry = 0;
+        for (int e0 = 0; e0 < E; e0 += 32) {
+            const int e = e0 + lane;
+            const int v = e < E ? (s_cnt[e] + align - 1) / align * align : 0;
+            int incl = v;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int n = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += n;
+            }
+            if (e < E) s_off[e] = carry + incl - v;
+            carry += __shfl_sync(0xffffffffu, incl, 31);
+        }
+        if (lane == 0) s_off[E] = carry;
+    }
+    __syncthreads();
+    // row of slot s (token t, expert e): segment start + stable rank
+    auto row_of = [&](int e, int t) {
+        const int w = t >> 5;
+        return s_off[e] + pre[e * W + w] + __popc(bits[e * W + w] & ((1u << (t & 31)) - 1u));
+    };
+    if (writer) {
+        for (int e = tid; e < E; e += blockDim.x) {
+            counts[e] = s_cnt[e];
+            if (load_out != nullptr) load_out[e] = s_cnt[e];
+        }
+        for (int e = tid; e <= E; e += blockDim.x) offsets[e] = s_off[e];
+        if (align > 1)
+            for (int i = tid; i < E * align; i += blockDim.x) {
+                const int e = i / align, r = i % align;
+                const int row = s_off[e] + s_cnt[e] + r;
+                if (row < s_off[e + 1]) row_src[row] = -1;
+            }
+        for (int s = tid; s < n_slots; s += blockDim.x) {
+            const int e = idx[s];
+            if (e < 0 || e >= E) continue;
+            const int pos = row_of(e, s / k);
+            row_src[pos] = s;
+            if (slot_row != nullptr) slot_row[s] = pos;
+        }
+    }
+    // the row copies: one warp per slot
+    const int gw = blockIdx.x * nwarps + warp, nw = gridDim.x * nwarps;
+    for (int s = gw; s < n_slots; s += nw) {
+        const int e = idx[s];
+        if (e < 0 || e >= E) continue;
+        const int t = s / k;
+        copy_row_warp(x, vec_per_row, t, x_perm, row_of(e, t), lane);
+    }
+    pdl_trigger();
+}
+
+// Larger batches in one launch: CTA b owns tokens [b TB, (b+1) TB) (TB a
+// multiple of 32, one CTA per SM at most, all resident together).
+//   1. per-expert bitmaps of its tokens, the per-word prefix counts and its
+//      per-expert counts, published in block_counts[b][e];
+//   2. a grid-wide barrier (an arrival counter in the status region, reset
+//      by the routing kernel; the wait is bounded and reports
+//      MOE_ERR_TIMEOUT);
+//   3. every CTA sums the published counts: totals (-> segment offsets) and
+//      the counts of the CTAs before it (-> its base inside each segment);
+//      CTA 0 writes counts, offsets, padding rows; each CTA writes row_src
+//      of its slots and copies its tokens' rows into x_perm.
+// Same layout and stable order as the histogram / scan / rank kernels; the k
+// ids of a token are distinct.
+__global__ void __launch_bounds__(kPermGatherThreads) perm_gather_grid_kernel(
+    const int32_t* __restrict__ idx, int T, int k, int E, int align, int TB,
+    int32_t* __restrict__ block_counts, int32_t* __restrict__ counts,
+    int32_t* __restrict__ offsets, int32_t* __restrict__ row_src, int32_t* __restrict__ load_out,
+    int* status, int* grid_bar, unsigned long long wait_limit_ns, const uint4* __restrict__ x,
+    int vec_per_row, uint4* __restrict__ x_perm) {
+    extern __shared__ __align__(16) uint32_t pg_sm[];
+    const int W = TB >> 5;
+    uint32_t* bits = pg_sm;                                   // [E][W]
+    int* pre = reinterpret_cast<int*>(bits + (size_t)E * W);  // [E][W]
+    int* s_cnt = pre + (size_t)E * W;                         // [E] this CTA's counts
+    int* s_tot = s_cnt + E;                                   // [E] all CTAs
+    int* s_base = s_tot + E;                                  // [E] CTAs before this one
+    int* s_off = s_base + E;                                  // [E + 1]
+    __shared__ int s_abort;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int nwarps = blockDim.x >> 5;
+    const int P = gridDim.x, b = blockIdx.x;
+    const int t0 = b * TB, t1 = min(T, t0 + TB);
+    const int s0 = t0 * k, s1 = t1 * k;
+    const bool writer = b == 0;
+    for (int i = tid; i < E * W; i += blockDim.x) bits[i] = 0u;
+    for (int e = tid; e < E; e += blockDim.x) {
+        s_tot[e] = 0;
+        s_base[e] = 0;
+    }
+    if (tid == 0) s_abort = 0;
+    pdl_wait();
+    __syncthreads();
+    for (int s = s0 + tid; s < s1; s += blockDim.x) {
+        const int e = idx[s];
+        if (e < 0 || e >= E) {
+            set_status(status, MOE_ERR_DEVICE, SITE_PERMUTE, e);
+            continue;
+        }
+        const int t = s / k - t0;
+        atomicOr(&bits[e * W + (t >> 5)], 1u << (t & 31));
+    }
+    __syncthreads();
+    for (int e = warp; e < E; e += nwarps) {
+        int carry = 0;
+        for (int w0 = 0; w0 < W; w0 += 32) {
+            const int w = w0 + lane;
+            const int v = w < W ? __popc(bits[e * W + w]) : 0;
+            int incl = v;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int n = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += n;
+            }
+            if (w < W) pre[e * W + w] = carry + incl - v;
+            carry += __shfl_sync(0xffffffffu, incl, 31);
+        }
+        if (lane == 0) {
+            s_cnt[e] = carry;
+            block_counts[(size_t)b * E + e] = carry;
+        }
+    }
+    // grid-wide barrier: every CTA's counts are published
+    __syncthreads();
+    if (tid == 0) {
+        __threadfence();
+        atomicAdd(grid_bar, 1);
+        const unsigned long long c0 = clock64();
+        while (*reinterpret_cast<volatile int*>(grid_bar) < P) {
+            if ((unsigned long long)(clock64() - c0) > 2ull * wait_limit_ns) {
+                set_status(status, MOE_ERR_TIMEOUT, SITE_PERMUTE, b);
+                s_abort = 1;
+                break;
+            }
+            __nanosleep(64);
+        }
+        __threadfence();
+    }
+    __syncthreads();
+    if (s_abort) return;
+    // totals and this CTA's base: column sums of block_counts, split over
+    // the threads (parts of the CTA list per expert), combined with integer
+    // atomics (order-independent)
+    {
+        const int parts = max(1, (int)blockDim.x / E);
+        const int e = tid % E, part = tid / E;
+        if (part < parts) {
+            int tot = 0, base = 0;
+            for (int q = part; q < P; q += parts) {
+                const int c = __ldcg(block_counts + (size_t)q * E + e);
+                tot += c;
+                if (q < b) base += c;
+            }
+            atomicAdd(&s_tot[e], tot);
+            atomicAdd(&s_base[e], base);
+        }
+    }
+    __syncthreads();
+    if (warp == 0) {  // segment offsets: exclusive scan of the padded totals
+        int carry = 0;
+        for (int e0 = 0; e0 < E; e0 += 32) {
+            const int e = e0 + lane;
+            const int v = e < E ? (s_tot[e] + align - 1) / align * align : 0;
+            int incl = v;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int n = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += n;
+            }
+            if (e < E) s_off[e] = carry + incl - v;
+            carry += __shfl_sync(0xffffffffu, incl, 31);
+        }
+        if (lane == 0) s_off[E] = carry;
+    }
+    __syncthreads();
+    auto row_of = [&](int e, int t) {  // t relative to t0
+        const int w = t >> 5;
+        return s_off[e] + s_base[e] + pre[e * W + w] +
+               __popc(bits[e * W + w] & ((1u << (t & 31)) - 1u));
+    };
+    if (writer) {
+        for (int e = tid; e < E; e += blockDim.x) {
+            counts[e] = s_tot[e];
+            if (load_out != nullptr) load_out[e] = s_tot[e];
+        }
+        for (int e = tid; e <= E; e += blockDim.x) offsets[e] = s_off[e];
+        if (align > 1)
+            for (int i = tid; i < E * align; i += blockDim.x) {
+                const int e = i / align, r = i % align;
+                const int row = s_off[e] + s_tot[e] + r;
+                if (row < s_off[e + 1]) row_src[row] = -1;
+            }
+    }
+    for (int s = s0 + tid; s < s1; s += blockDim.x) {
+        const int e = idx[s];
+        if (e < 0 || e >= E) continue;
+        row_src[row_of(e, s / k - t0)] = s;
+    }
+    for (int s = s0 + warp; s < s1; s += nwarps) {
+        const int e = idx[s];
+        if (e < 0 || e >= E) continue;
+        const int t = s / k;
+        copy_row_warp(x, vec_per_row, t, x_perm, row_of(e, t - t0), lane);
+    }
     pdl_trigger();
 }
 
@@ -440,6 +722,57 @@ cudaError_t launch_permute(const int32_t* idx, int T, int k, int E, int32_t* blo
     return launch_pdl(perm_rank_kernel, dim3(nb), dim3(kPermBlockTokens), 0, s, 1, idx, T, k, E,
                       static_cast<const int32_t*>(block_counts),
                       static_cast<const int32_t*>(offsets), row_src, slot_row, status);
+}
+
+cudaError_t launch_permute_gather_small(const int32_t* idx, int T, int k, int E, int align,
+                                       int32_t* counts, int32_t* offsets, int32_t* row_src,
+                                       int32_t* load_out, int* status, const void* x, int d,
+                                       int elem_bytes, void* x_perm, int num_sms,
+                                       cudaStream_t s) {
+    if (T > kSmallTokens || T < 1) return cudaErrorInvalidValue;
+    const int W = (T + 31) / 32;
+    const size_t smem = (size_t)E * W * 8 + (size_t)(2 * E + 1) * 4;
+    cudaError_t e = cudaFuncSetAttribute(perm_gather_small_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    const int warps_per_cta = kPermGatherThreads / 32;
+    int blocks = (T * k + warps_per_cta - 1) / warps_per_cta;
+    if (blocks > num_sms) blocks = num_sms;
+    if (blocks < 1) blocks = 1;
+    return launch_pdl(perm_gather_small_kernel, dim3((unsigned)blocks), dim3(kPermGatherThreads),
+                      smem, s, 1, idx, T, k, E, align, counts, offsets, row_src, load_out,
+                      static_cast<int32_t*>(nullptr), status, static_cast<const uint4*>(x),
+                      d * elem_bytes / 16, static_cast<uint4*>(x_perm));
+}
+
+bool permute_gather_grid_fits(int T, int E, int num_sms) {
+    if (T < 1 || num_sms < 1) return false;
+    int P = (T + 31) / 32;
+    if (P > num_sms) P = num_sms;
+    const int TB = ((T + P - 1) / P + 31) / 32 * 32;
+    const size_t smem = (size_t)E * (TB / 32) * 8 + (size_t)(4 * E + 1) * 4;
+    return smem <= kPermGatherGridMaxSmem;
+}
+
+cudaError_t launch_permute_gather_grid(const int32_t* idx, int T, int k, int E, int align,
+                                      int32_t* block_counts, int32_t* counts, int32_t* offsets,
+                                      int32_t* row_src, int32_t* load_out, int* status,
+                                      int* grid_bar, unsigned long long wait_limit_ns,
+                                      const void* x, int d, int elem_bytes, void* x_perm,
+                                      int num_sms, cudaStream_t s) {
+    if (!permute_gather_grid_fits(T, E, num_sms)) return cudaErrorInvalidValue;
+    int P = (T + 31) / 32;
+    if (P > num_sms) P = num_sms;
+    const int TB = ((T + P - 1) / P + 31) / 32 * 32;
+    P = (T + TB - 1) / TB;
+    const size_t smem = (size_t)E * (TB / 32) * 8 + (size_t)(4 * E + 1) * 4;
+    cudaError_t e = cudaFuncSetAttribute(perm_gather_grid_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    return launch_pdl(perm_gather_grid_kernel, dim3((unsigned)P), dim3(kPermGatherThreads), smem,
+                      s, 1, idx, T, k, E, align, TB, block_counts, counts, offsets, row_src,
+                      load_out, status, grid_bar, wait_limit_ns, static_cast<const uint4*>(x),
+                      d * elem_bytes / 16, static_cast<uint4*>(x_perm));
 }
 
 cudaError_t launch_expert_counts(const int32_t* idx, int T, int k, int E,

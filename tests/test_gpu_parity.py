@@ -73,6 +73,10 @@ SMALL = [
     # T > 1024 with d = 512: the whole-d router
     ("bf16_T1500", Workload("bf16_T1500", T=1500, d=512, E=32, k=4, n_group=4, topk_group=2,
                             inter=128, n_shared=1, dtype="bf16")),
+    # fp32 above 1024 tokens: the one-launch permutation with 128-row padded
+    # segments, token blocks of 32 over 41 CTAs, E = 256 bitmaps
+    ("f32_T1300_E256", Workload("f32_T1300_E256", T=1300, d=128, E=256, k=5, n_group=16,
+                                topk_group=8, inter=128, n_shared=1, dtype="f32")),
 ]
 
 
@@ -152,16 +156,24 @@ def permutation_check(w, inp, idx, ws):
             assert torch.equal(xp[offsets[e]:offsets[e] + cnt_ref[e]], inp.x[torch.from_numpy(t)])
 
 
-def test_permutation_stage_prefill():
-    w = WORKLOADS["prefill"]
+@pytest.mark.parametrize("name", ["prefill", "decode", "skewed", "train"])
+def test_permutation_stage_full_size(name):
+    w = WORKLOADS[name]
     inp = make_inputs(w)
     y, idx, wt, ws = run_forward(w, inp)
     permutation_check(w, inp, idx, ws)
 
 
-@pytest.mark.parametrize("i", [1, 2], ids=["f32_shared", "bf16_ragged"])
-def test_permutation_stage_small_ragged(i):
-    w = SMALL[i][1]
+# T <= 1024 runs the one-CTA-derives-all permutation + row gather, larger T
+# the grid-wide one (token blocks per CTA, one grid barrier); both rank by
+# per-expert token bitmaps
+PERM_CASES = ["f32_shared", "bf16_ragged", "bf16_one_token", "bf16_multi_tile", "bf16_E256",
+              "bf16_E128_T1100", "bf16_T1500", "f32_T1300_E256"]
+
+
+@pytest.mark.parametrize("name", PERM_CASES)
+def test_permutation_stage_small_ragged(name):
+    w = dict(SMALL)[name]
     inp = make_inputs(w)
     y, idx, wt, ws = run_forward(w, inp)
     permutation_check(w, inp, idx, ws)
