@@ -537,10 +537,10 @@ def run_train(args, w):
     roof_ms = max(t_tensor, t_hbm) * 1e3
     dom_flops = dom[2]
     dom_ach = dom_flops / (dom_ms * 1e-3) / 1e12
-    # forward: route, permutation (1 or 3), gather, 2 GEMMs, final sum; backward:
+    # forward: route, permutation with the row gather, 2 GEMMs, final sum; backward:
     # permutation (1 or 3), gather, dgrad GEMM, dL/dlogit, dgrad GEMM, dx sum,
     # 2 weight-gradient GEMMs, dW_router (2)
-    launches = (1 + (1 if w.T <= 1024 else 3) + 1 + 2 + 1) + ((1 if w.T <= 1024 else 3) + 9)
+    launches = (1 + 1 + 2 + 1) + ((1 if w.T <= 1024 else 3) + 9)
     cfg = run_config(w, world, args)
     cfg["step"] = "forward (saving pre-activations) + backward (dx and all weight gradients, fp32)"
     out = {
@@ -781,9 +781,9 @@ def main():
                "peak": pk["hbm_gbs"], "unit": "GB/s", "bytes_per_launch": g1_bytes,
                "peak_kind": f"HBM copy ({pk['source']})"}
     dom["frac"] = dom["achieved"] / dom["peak"]
-    # route, permutation (one kernel up to 1024 tokens, else count + scan +
-    # rank), row gather, the two GEMM launches, final sum
-    launches_per_step = (1 + (1 if w.T <= 1024 else 3) + 1 + 2 + 1) if w.dtype == "bf16" else None
+    # route, permutation with the row gather (one launch), the two GEMM
+    # launches, final sum
+    launches_per_step = (1 + 1 + 2 + 1) if w.dtype == "bf16" else None
     value = world * w.T / (ms * 1e-3)
     out = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
