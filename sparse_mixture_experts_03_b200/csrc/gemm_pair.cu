@@ -585,6 +585,7 @@ __device__ __forceinline__ void pair_epilogue(uint8_t* wb, uint32_t taddr, const
                 row[lane & 3] = __uint_as_float(v[i]);
             }
             __syncwarp();
+            uint4 h_row[2];  // lane = token: h of its 16 features, bf16
             if (tok_ok) {
                 float f[32];
 #pragma unroll
@@ -600,11 +601,8 @@ __device__ __forceinline__ void pair_epilogue(uint8_t* wb, uint32_t taddr, const
                 for (int p = 0; p < 8; ++p)
                     packed[p] = pack_bf16x2(silu_mul(f[2 * p], f[16 + 2 * p]),
                                             silu_mul(f[2 * p + 1], f[16 + 2 * p + 1]));
-                uint4* d = reinterpret_cast<uint4*>(
-                    static_cast<__nv_bfloat16*>(a.out) + (size_t)(t.b_row + c0 + lane) * a.out_ld +
-                    t.ft * a.out_col_step + cta * 64 + wq * 16);
-                d[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
-                d[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
+                h_row[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+                h_row[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
                 if constexpr (EPI == EPI_SWIGLU_SAVE) {
                     // the pre-activations for the backward: blocks of 16 features,
                     // [block][row][16 gate | 16 up] with this launch's row order, so
@@ -626,6 +624,28 @@ __device__ __forceinline__ void pair_epilogue(uint8_t* wb, uint32_t taddr, const
                 }
             }
             __syncwarp();
+            // h rows (32 B each) through the staged rows, 2 lanes per row: each
+            // store instruction writes 16 whole 32-byte row pieces (lanes 8 g ..
+            // 8 g + 7 take 4 rows 2 apart: disjoint chunk positions)
+            if (tok_ok) {
+                *reinterpret_cast<uint4*>(stage_chunk(wb, lane, 0)) = h_row[0];
+                *reinterpret_cast<uint4*>(stage_chunk(wb, lane, 1)) = h_row[1];
+            }
+            __syncwarp();
+            {
+                const int q = lane & 1, g = lane >> 3;
+#pragma unroll
+                for (int it = 0; it < 2; ++it) {
+                    const int i = 16 * it + 2 * ((lane >> 1) & 3) + (g & 1) + 8 * (g >> 1);
+                    if (c0 + i < t.n_real)
+                        *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.out) +
+                                                  (size_t)(t.b_row + c0 + i) * a.out_ld +
+                                                  t.ft * a.out_col_step + cta * 64 + wq * 16 +
+                                                  q * 8) =
+                            *reinterpret_cast<const uint4*>(stage_chunk(wb, i, q));
+                }
+            }
+            __syncwarp();
         } else if constexpr (EPI == EPI_SCATTER) {
             // fp32 transpose through the staging buffer (token row i: 32 features x
             // 4 B), then lane = token: its 32 features times its own gate weight,
@@ -638,21 +658,38 @@ __device__ __forceinline__ void pair_epilogue(uint8_t* wb, uint32_t taddr, const
                 row[lane & 3] = __uint_as_float(v[i]);
             }
             __syncwarp();
-            if (src >= 0) {
-                uint32_t packed[16];
+            uint32_t packed[16];
 #pragma unroll
-                for (int q = 0; q < 8; ++q) {
-                    const float4 f = *reinterpret_cast<const float4*>(stage_chunk(wb, lane, q));
-                    packed[2 * q] = pack_bf16x2(wv * f.x, wv * f.y);
-                    packed[2 * q + 1] = pack_bf16x2(wv * f.z, wv * f.w);
+            for (int q = 0; q < 8; ++q) {
+                const float4 f = *reinterpret_cast<const float4*>(stage_chunk(wb, lane, q));
+                packed[2 * q] = pack_bf16x2(wv * f.x, wv * f.y);
+                packed[2 * q + 1] = pack_bf16x2(wv * f.z, wv * f.w);
+            }
+            __syncwarp();
+            // the bf16 row (64 B) back into the lane's staged row, then 4 lanes
+            // per row: each store instruction writes 8 whole 64-byte row pieces
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+                *reinterpret_cast<uint4*>(stage_chunk(wb, lane, q)) =
+                    make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2],
+                               packed[4 * q + 3]);
+            __syncwarp();
+            {
+                // lanes 8 g .. 8 g + 7 take rows r and r + 4 (disjoint chunk
+                // positions of the swizzle: no bank conflict)
+                const int q = lane & 3;
+                const int sub = (lane >> 2) & 1, g = lane >> 3;
+#pragma unroll
+                for (int it = 0; it < 4; ++it) {
+                    const int i = 8 * it + g + 4 * sub;
+                    const int si = __shfl_sync(0xffffffffu, src, i);
+                    if (si >= 0) {
+                        const uint4 v4 = *reinterpret_cast<const uint4*>(stage_chunk(wb, i, q));
+                        *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.out) +
+                                                  (size_t)si * a.out_ld + t.ft * a.out_col_step +
+                                                  cta * 128 + wq * 32 + q * 8) = v4;
+                    }
                 }
-                uint4* d = reinterpret_cast<uint4*>(
-                    static_cast<__nv_bfloat16*>(a.out) + (size_t)src * a.out_ld +
-                    t.ft * a.out_col_step + cta * 128 + wq * 32);
-#pragma unroll
-                for (int q = 0; q < 4; ++q)
-                    d[q] = make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2],
-                                      packed[4 * q + 3]);
             }
             __syncwarp();
         } else if constexpr (EPI == EPI_STORE_ROWS) {
@@ -688,13 +725,20 @@ __device__ __forceinline__ void pair_epilogue(uint8_t* wb, uint32_t taddr, const
                 row[lane & 3] = __uint_as_float(v[i]);
             }
             __syncwarp();
-            if (tok_ok) {
-                float4* d = reinterpret_cast<float4*>(
-                    static_cast<float*>(a.out) + (size_t)(t.b_row + c0 + lane) * a.out_ld +
-                    t.ft * a.out_col_step + cta * 128 + wq * 32);
+            {
+                // 8 lanes per token row: each store instruction writes 4 whole
+                // 128-byte row pieces
+                const int q = lane & 7;
 #pragma unroll
-                for (int q = 0; q < 8; ++q)
-                    d[q] = *reinterpret_cast<const float4*>(stage_chunk(wb, lane, q));
+                for (int it = 0; it < 8; ++it) {
+                    const int i = 4 * it + (lane >> 3);
+                    if (c0 + i < t.n_real)
+                        *reinterpret_cast<float4*>(static_cast<float*>(a.out) +
+                                                   (size_t)(t.b_row + c0 + i) * a.out_ld +
+                                                   t.ft * a.out_col_step + cta * 128 + wq * 32 +
+                                                   q * 4) =
+                            *reinterpret_cast<const float4*>(stage_chunk(wb, i, q));
+                }
             }
             __syncwarp();
         }
