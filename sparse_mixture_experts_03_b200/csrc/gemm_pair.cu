@@ -51,6 +51,10 @@ constexpr int kABytes = kARows * kBK * 2;        // 32 KiB: 2 atoms x 128 weight
 constexpr int kMaxStages = 6;
 constexpr int kAtomBytesA = kARows * 128;        // 16 KiB between the atoms of a tile
 constexpr int kNTile = 256;                      // tokens per tile
+// The weight producer of the gate/up launch brings the k-block this many
+// steps ahead of its current load into L2 (a tile's first touch of a weight
+// tile comes from HBM; the ring holds too few bytes to cover that latency)
+constexpr int kPrefetchAhead = 2;
 constexpr int kTmemCols = 512;                   // 2 accumulators x 256 fp32 columns
 constexpr int kThreads = 224;                    // 7 warps: producers 0 and 6, MMA 1, epilogue 2..5
 constexpr int kBProducerWarp = 6;
@@ -1015,10 +1019,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                     } else {
                         // 4 blocks x (16 gate rows, 16 up rows) of features
                         // ft * a_tile_step + cta * a_cta_step ... + 63 of group g, x 2 k-atoms
-                        tma_load_5d_pair(sa, m, fb, 0, 0, 0,
-                                         t.g * a.a_blocks_per_group +
-                                             ((t.ft * a.a_tile_step + (int)cta * a.a_cta_step) >> 4),
-                                         atom);
+                        const int blk = t.g * a.a_blocks_per_group +
+                                        ((t.ft * a.a_tile_step + (int)cta * a.a_cta_step) >> 4);
+                        tma_load_5d_pair(sa, m, fb, 0, 0, 0, blk, atom);
+                        // the same rows kPrefetchAhead k-blocks further on towards L2
+                        if (kb + kPrefetchAhead < kb_count)
+                            tma_prefetch_l2_5d(m, 0, 0, 0, blk, atom + kPrefetchAhead * kAtoms);
                     }
                     issued |= 1u << s;
                     issued_ph = (issued_ph & ~(1u << s)) | (ph << s);
