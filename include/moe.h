@@ -98,7 +98,8 @@ enum {
     MOE_WS_COUNTS = 1,       /* int32[E]   tokens routed to each expert                */
     MOE_WS_OFFSETS = 2,      /* int32[E+1] first row of each expert in the permuted
                                 layout (bf16: unpadded; f32: padded to 128 rows)     */
-    MOE_WS_BLOCK_COUNTS = 3, /* int32[ceil(T/256) * E] per-block histogram / bases     */
+    MOE_WS_BLOCK_COUNTS = 3, /* int32[max(ceil(T/256), ceil(T/32)) * E] per-block
+                                histogram (the permutation's token blocks)          */
     MOE_WS_TOPK_IDX = 4,     /* int32[T*k] chosen experts (used when no output given)  */
     MOE_WS_TOPK_W = 5,       /* f32[T*k]   gate weights                               */
     MOE_WS_ROW_SRC = 6,      /* int32[rows_cap] permuted row -> t*k + j, or -1 (pad)    */

@@ -22,6 +22,8 @@
 //                         in top-k order (fixed order: bitwise reproducible)
 #include <limits.h>
 
+#include <algorithm>
+
 #include "moe_device.cuh"
 #include "moe_internal.h"
 
@@ -199,7 +201,9 @@ size_t layout(const size_t (&sizes)[N], size_t (&off)[N + 1]) {
 bool dispatch_layout(int T, int E, int k, size_t (&off)[DP_TOTAL + 1]) {
     if (T < 0 || E < 1 || E > kMaxE || k < 1 || k > kMaxK || k > E) return false;
     if ((long long)T * k >= (long long)INT_MAX / 2) return false;
-    const size_t nb = (size_t)(T + kPermBlockTokens - 1) / kPermBlockTokens;
+    // block counts: per 256-token block, or per CTA of the one-launch permutation
+    const size_t nb = std::max((size_t)(T + kPermBlockTokens - 1) / kPermBlockTokens,
+                               (size_t)(T + 31) / 32);
     const size_t sizes[DP_TOTAL] = {sizeof(int) * kStatusWords, sizeof(int) * (E + 1),
                                     sizeof(int) * (nb > 0 ? nb : 1) * E,
                                     sizeof(int) * ((size_t)T * k + 1)};
@@ -274,8 +278,20 @@ MOE_API int moe_dispatch(const void* x, const void* W_router, int T, int d, int 
     cudaError_t e = launch_route_bf16(x, W_router, T, d, E, k, n_group, topk_group, gate,
                                       expert_bias, topk_idx, topk_w, status, s);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
-    e = launch_permute(topk_idx, T, k, E, region<int32_t>(workspace, off, DP_BLOCK_COUNTS), counts,
-                       offsets, row_src, 1, nullptr, status, s, slot_row);
+    // permutation, rows and their gate weights in one launch (the routing
+    // kernel has reset the grid-barrier word of the status region)
+    int32_t* block_counts = region<int32_t>(workspace, off, DP_BLOCK_COUNTS);
+    if (T <= kSmallPermTokens)
+        return ret(launch_permute_gather_small(topk_idx, T, k, E, 1, counts, offsets, row_src,
+                                               nullptr, status, x, d, 2, x_perm, num_sms(), s,
+                                               slot_row, topk_w, w_perm));
+    if (permute_gather_grid_fits(T, E, num_sms()))
+        return ret(launch_permute_gather_grid(topk_idx, T, k, E, 1, block_counts, counts, offsets,
+                                              row_src, nullptr, status,
+                                              status + kGridBarWordPermute, kWaitLimitNs, x, d, 2,
+                                              x_perm, num_sms(), s, slot_row, topk_w, w_perm));
+    e = launch_permute(topk_idx, T, k, E, block_counts, counts, offsets, row_src, 1, nullptr,
+                       status, s, slot_row);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
     return ret(launch_gather_rows(x, d, 2, k, offsets + E, row_src, T * k, x_perm, num_sms(), s,
                                   topk_w, w_perm));

@@ -589,7 +589,8 @@ __device__ __forceinline__ void pair_epilogue(uint8_t* wb, uint32_t taddr, const
                 row[lane & 3] = __uint_as_float(v[i]);
             }
             __syncwarp();
-            uint4 h_row[2];  // lane = token: h of its 16 features, bf16
+            uint4 h_row[2];   // lane = token: h of its 16 features, bf16
+            uint4 sv_row[4];  // SWIGLU_SAVE: its [16 gate | 16 up] pre-activations, bf16
             if (tok_ok) {
                 float f[32];
 #pragma unroll
@@ -611,20 +612,17 @@ __device__ __forceinline__ void pair_epilogue(uint8_t* wb, uint32_t taddr, const
                     // the pre-activations for the backward: blocks of 16 features,
                     // [block][row][16 gate | 16 up] with this launch's row order, so
                     // the warp's 32 consecutive rows are 2 KiB in one piece
-                    const int r = t.b_row + c0 + lane;
-                    const int blk = (t.ft * a.out_col_step + (int)cta * 64 + wq * 16) >> 4;
+                    // (stored below, through the staged rows)
                     uint32_t pg[8], pu[8];
 #pragma unroll
                     for (int p = 0; p < 8; ++p) {
                         pg[p] = pack_bf16x2(f[2 * p], f[2 * p + 1]);
                         pu[p] = pack_bf16x2(f[16 + 2 * p], f[16 + 2 * p + 1]);
                     }
-                    uint4* sv = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.save) +
-                                                         ((size_t)blk * a.gu_rows + r) * 32);
-                    sv[0] = make_uint4(pg[0], pg[1], pg[2], pg[3]);
-                    sv[1] = make_uint4(pg[4], pg[5], pg[6], pg[7]);
-                    sv[2] = make_uint4(pu[0], pu[1], pu[2], pu[3]);
-                    sv[3] = make_uint4(pu[4], pu[5], pu[6], pu[7]);
+                    sv_row[0] = make_uint4(pg[0], pg[1], pg[2], pg[3]);
+                    sv_row[1] = make_uint4(pg[4], pg[5], pg[6], pg[7]);
+                    sv_row[2] = make_uint4(pu[0], pu[1], pu[2], pu[3]);
+                    sv_row[3] = make_uint4(pu[4], pu[5], pu[6], pu[7]);
                 }
             }
             __syncwarp();
@@ -650,6 +648,31 @@ __device__ __forceinline__ void pair_epilogue(uint8_t* wb, uint32_t taddr, const
                 }
             }
             __syncwarp();
+            if constexpr (EPI == EPI_SWIGLU_SAVE) {
+                // the pre-activations for the backward: blocks of 16 features,
+                // [block][row][16 gate | 16 up] with this launch's row order, so
+                // the warp's 32 consecutive rows are 2 KiB in one piece; each
+                // store instruction writes 512 contiguous bytes (8 rows)
+                if (tok_ok) {
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)
+                        *reinterpret_cast<uint4*>(stage_chunk(wb, lane, q)) = sv_row[q];
+                }
+                __syncwarp();
+                const int blk = (t.ft * a.out_col_step + (int)cta * 64 + wq * 16) >> 4;
+                const int q = lane & 3;
+                const int sub = (lane >> 2) & 1, g = lane >> 3;
+#pragma unroll
+                for (int it = 0; it < 4; ++it) {
+                    const int i = 8 * it + g + 4 * sub;
+                    if (c0 + i < t.n_real)
+                        *reinterpret_cast<uint4*>(
+                            static_cast<__nv_bfloat16*>(a.save) +
+                            ((size_t)blk * a.gu_rows + t.b_row + c0 + i) * 32 + q * 8) =
+                            *reinterpret_cast<const uint4*>(stage_chunk(wb, i, q));
+                }
+                __syncwarp();
+            }
         } else if constexpr (EPI == EPI_SCATTER) {
             // fp32 transpose through the staging buffer (token row i: 32 features x
             // 4 B), then lane = token: its 32 features times its own gate weight,

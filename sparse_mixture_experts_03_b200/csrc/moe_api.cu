@@ -560,7 +560,8 @@ bool make_bwd_layout(int T, int d, int E, int k, int inter, int n_shared, BwdLay
         sizeof(int) * kStatusWords,             // STATUS (+ tile counters)
         sizeof(int) * E,                        // COUNTS
         sizeof(int) * (E + 1),                  // OFFSETS (segments padded to 128 rows)
-        sizeof(int) * (size_t)(nb > 0 ? nb : 1) * E,  // BLOCK_COUNTS
+        // BLOCK_COUNTS: per 256-token block, or per CTA of the one-launch permutation
+        sizeof(int) * (size_t)std::max(std::max(nb, (T + 31) / 32), 1) * E,
         sizeof(int) * rc,                       // ROW_SRC
         sizeof(int) * Tk,                       // SLOT_ROW: slot -> permuted row
         2 * rc * d,                             // X_PERM
@@ -669,8 +670,18 @@ MOE_API int moe_backward(const void* x, const void* W_router, const void* W_gate
     if (e != cudaSuccess) return MOE_ERR_CUDA;
     // 1. the forward's permutation again, with segments padded to 128 rows
     //    (whole k-blocks of the weight-gradient GEMMs), then x / dy rows
-    e = launch_permute(topk_idx, T, k, E, block_counts, counts, offsets, row_src, kRowAlign,
-                       nullptr, status, s, slot_row);
+    if (T <= kSmallPermTokens)
+        e = launch_permute_gather_small(topk_idx, T, k, E, kRowAlign, counts, offsets, row_src,
+                                        nullptr, status, nullptr, d, 2, nullptr, num_sms(), s,
+                                        slot_row);
+    else if (permute_gather_grid_fits(T, E, num_sms()))
+        e = launch_permute_gather_grid(topk_idx, T, k, E, kRowAlign, block_counts, counts, offsets,
+                                       row_src, nullptr, status, status + kGridBarWordPermute,
+                                       kWaitLimitNs, nullptr, d, 2, nullptr, num_sms(), s,
+                                       slot_row);
+    else
+        e = launch_permute(topk_idx, T, k, E, block_counts, counts, offsets, row_src, kRowAlign,
+                           nullptr, status, s, slot_row);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
     e = launch_bwd_gather(x, dy, T, d, inter, k, offsets + E, row_src, slot_row, L.rows_cap,
                           x_perm, dy_perm, dgu, hw, num_sms(), s);

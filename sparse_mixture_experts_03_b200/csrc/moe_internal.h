@@ -54,7 +54,8 @@ constexpr int kStatusWords = 64;       // int32 words of the status region of th
 // (reset to 0, with words 0..15, by the routing kernel at the start of a forward)
 constexpr int kSchedWordGateUp = 12;
 constexpr int kSchedWordDown = 13;
-// arrival counter of the permutation's grid-wide barrier (same reset)
+// arrival counter of the permutation's grid-wide barrier (same reset; the
+// backward and the expert-parallel dispatch reset it the same way)
 constexpr int kGridBarWordPermute = 14;
 // the backward's four CTA-pair launches (the backward clears the whole status
 // region first)
@@ -144,20 +145,24 @@ cudaError_t launch_gather_rows(const void* x, int d, int elem_bytes, int k,
                                const int32_t* offsets_total, const int32_t* row_src,
                                int rows_cap, void* x_perm, int num_sms, cudaStream_t s,
                                const float* w_src = nullptr, float* w_dst = nullptr);
-// T <= 1024: launch_permute followed by launch_gather_rows, in one launch of
-// several CTAs (each derives the permutation; CTA 0 writes it out).  The k
-// ids of a token are distinct.
+// launch_permute followed by launch_gather_rows in one launch.  T <= 1024:
+// several CTAs, each derives the permutation, CTA 0 writes it out.  The k ids
+// of a token are distinct.  x == nullptr: no row copies (the permutation
+// alone); slot_row (nullable): slot -> row; w_dst (nullable): w_dst[row] =
+// w_src[slot].
 constexpr int kSmallPermTokens = 1024;
 cudaError_t launch_permute_gather_small(const int32_t* idx, int T, int k, int E, int align,
                                        int32_t* counts, int32_t* offsets, int32_t* row_src,
                                        int32_t* load_out, int* status, const void* x, int d,
                                        int elem_bytes, void* x_perm, int num_sms,
-                                       cudaStream_t s);
+                                       cudaStream_t s, int32_t* slot_row = nullptr,
+                                       const float* w_src = nullptr, float* w_dst = nullptr);
 // T > 1024: the same in one launch of at most num_sms CTAs (token blocks of
 // a multiple of 32), which meet at one grid-wide barrier: *grid_bar must be 0
-// at launch (a status word the routing kernel resets).  block_counts holds
-// min(num_sms, ceil(T/32)) * E int32.  False from _fits when the per-CTA
-// bitmaps would not fit in shared memory (use the separate kernels then).
+// at launch (a status word the routing kernel, or the backward's status
+// reset, zeroes).  block_counts holds min(num_sms, ceil(T/32)) * E int32.
+// False from _fits when the per-CTA bitmaps would not fit in shared memory
+// (use the separate kernels then).
 constexpr size_t kPermGatherGridMaxSmem = 160 * 1024;
 bool permute_gather_grid_fits(int T, int E, int num_sms);
 cudaError_t launch_permute_gather_grid(const int32_t* idx, int T, int k, int E, int align,
@@ -165,7 +170,8 @@ cudaError_t launch_permute_gather_grid(const int32_t* idx, int T, int k, int E, 
                                       int32_t* row_src, int32_t* load_out, int* status,
                                       int* grid_bar, unsigned long long wait_limit_ns,
                                       const void* x, int d, int elem_bytes, void* x_perm,
-                                      int num_sms, cudaStream_t s);
+                                      int num_sms, cudaStream_t s, int32_t* slot_row = nullptr,
+                                      const float* w_src = nullptr, float* w_dst = nullptr);
 // Per-expert counts and unpadded segment offsets of a table of expert ids
 // (histogram + scan only); block_counts holds ceil(T/256) * E int32.  Every
 // occurrence of an id counts (a row may repeat one); ids outside [0, E) are

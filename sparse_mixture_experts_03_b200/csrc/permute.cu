@@ -307,11 +307,13 @@ __device__ __forceinline__ void copy_row_warp(const uint4* __restrict__ x, int v
 // bits[e] is set when token t chose e, so the rank of token t inside
 // segment e is the number of set bits below t -- a per-word prefix count plus
 // one masked popcount, independent of E.
+template <bool kRows, bool kWeights>
 __global__ void __launch_bounds__(kPermGatherThreads) perm_gather_small_kernel(
     const int32_t* __restrict__ idx, int T, int k, int E, int align,
     int32_t* __restrict__ counts, int32_t* __restrict__ offsets, int32_t* __restrict__ row_src,
     int32_t* __restrict__ load_out, int32_t* __restrict__ slot_row, int* status,
-    const uint4* __restrict__ x, int vec_per_row, uint4* __restrict__ x_perm) {
+    const uint4* __restrict__ x, int vec_per_row, uint4* __restrict__ x_perm,
+    const float* __restrict__ w_src, float* __restrict__ w_dst) {
     extern __shared__ __align__(16) uint32_t pg_sm[];
     const int W = (T + 31) >> 5;  // bitmap words per expert
     uint32_t* bits = pg_sm;                                     // [E][W]
@@ -390,13 +392,19 @@ __global__ void __launch_bounds__(kPermGatherThreads) perm_gather_small_kernel(
             if (slot_row != nullptr) slot_row[s] = pos;
         }
     }
-    // the row copies: one warp per slot
-    const int gw = blockIdx.x * nwarps + warp, nw = gridDim.x * nwarps;
-    for (int s = gw; s < n_slots; s += nw) {
-        const int e = idx[s];
-        if (e < 0 || e >= E) continue;
-        const int t = s / k;
-        copy_row_warp(x, vec_per_row, t, x_perm, row_of(e, t), lane);
+    // the row copies (kRows) and gate weights (kWeights): one warp per slot
+    if constexpr (kRows || kWeights) {
+        const int gw = blockIdx.x * nwarps + warp, nw = gridDim.x * nwarps;
+        for (int s = gw; s < n_slots; s += nw) {
+            const int e = idx[s];
+            if (e < 0 || e >= E) continue;
+            const int t = s / k;
+            const int row = row_of(e, t);
+            if constexpr (kWeights) {
+                if (lane == 0) w_dst[row] = w_src[s];
+            }
+            if constexpr (kRows) copy_row_warp(x, vec_per_row, t, x_perm, row, lane);
+        }
     }
     pdl_trigger();
 }
@@ -414,12 +422,14 @@ __global__ void __launch_bounds__(kPermGatherThreads) perm_gather_small_kernel(
 //      of its slots and copies its tokens' rows into x_perm.
 // Same layout and stable order as the histogram / scan / rank kernels; the k
 // ids of a token are distinct.
+template <bool kRows, bool kWeights>
 __global__ void __launch_bounds__(kPermGatherThreads) perm_gather_grid_kernel(
     const int32_t* __restrict__ idx, int T, int k, int E, int align, int TB,
     int32_t* __restrict__ block_counts, int32_t* __restrict__ counts,
     int32_t* __restrict__ offsets, int32_t* __restrict__ row_src, int32_t* __restrict__ load_out,
-    int* status, int* grid_bar, unsigned long long wait_limit_ns, const uint4* __restrict__ x,
-    int vec_per_row, uint4* __restrict__ x_perm) {
+    int32_t* __restrict__ slot_row, int* status, int* grid_bar, unsigned long long wait_limit_ns,
+    const uint4* __restrict__ x, int vec_per_row, uint4* __restrict__ x_perm,
+    const float* __restrict__ w_src, float* __restrict__ w_dst) {
     extern __shared__ __align__(16) uint32_t pg_sm[];
     const int W = TB >> 5;
     uint32_t* bits = pg_sm;                                   // [E][W]
@@ -546,13 +556,21 @@ __global__ void __launch_bounds__(kPermGatherThreads) perm_gather_grid_kernel(
     for (int s = s0 + tid; s < s1; s += blockDim.x) {
         const int e = idx[s];
         if (e < 0 || e >= E) continue;
-        row_src[row_of(e, s / k - t0)] = s;
+        const int pos = row_of(e, s / k - t0);
+        row_src[pos] = s;
+        if (slot_row != nullptr) slot_row[s] = pos;
     }
-    for (int s = s0 + warp; s < s1; s += nwarps) {
-        const int e = idx[s];
-        if (e < 0 || e >= E) continue;
-        const int t = s / k;
-        copy_row_warp(x, vec_per_row, t, x_perm, row_of(e, t - t0), lane);
+    if constexpr (kRows || kWeights) {
+        for (int s = s0 + warp; s < s1; s += nwarps) {
+            const int e = idx[s];
+            if (e < 0 || e >= E) continue;
+            const int t = s / k;
+            const int row = row_of(e, t - t0);
+            if constexpr (kWeights) {
+                if (lane == 0) w_dst[row] = w_src[s];
+            }
+            if constexpr (kRows) copy_row_warp(x, vec_per_row, t, x_perm, row, lane);
+        }
     }
     pdl_trigger();
 }
@@ -728,21 +746,26 @@ cudaError_t launch_permute_gather_small(const int32_t* idx, int T, int k, int E,
                                        int32_t* counts, int32_t* offsets, int32_t* row_src,
                                        int32_t* load_out, int* status, const void* x, int d,
                                        int elem_bytes, void* x_perm, int num_sms,
-                                       cudaStream_t s) {
+                                       cudaStream_t s, int32_t* slot_row, const float* w_src,
+                                       float* w_dst) {
     if (T > kSmallTokens || T < 1) return cudaErrorInvalidValue;
     const int W = (T + 31) / 32;
     const size_t smem = (size_t)E * W * 8 + (size_t)(2 * E + 1) * 4;
-    cudaError_t e = cudaFuncSetAttribute(perm_gather_small_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    auto kern = x != nullptr ? (w_dst != nullptr ? perm_gather_small_kernel<true, true>
+                                                 : perm_gather_small_kernel<true, false>)
+                             : (w_dst != nullptr ? perm_gather_small_kernel<false, true>
+                                                 : perm_gather_small_kernel<false, false>);
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
     if (e != cudaSuccess) return e;
     const int warps_per_cta = kPermGatherThreads / 32;
     int blocks = (T * k + warps_per_cta - 1) / warps_per_cta;
     if (blocks > num_sms) blocks = num_sms;
-    if (blocks < 1) blocks = 1;
-    return launch_pdl(perm_gather_small_kernel, dim3((unsigned)blocks), dim3(kPermGatherThreads),
-                      smem, s, 1, idx, T, k, E, align, counts, offsets, row_src, load_out,
-                      static_cast<int32_t*>(nullptr), status, static_cast<const uint4*>(x),
-                      d * elem_bytes / 16, static_cast<uint4*>(x_perm));
+    if (blocks < 1 || (x == nullptr && w_dst == nullptr)) blocks = 1;
+    return launch_pdl(kern, dim3((unsigned)blocks), dim3(kPermGatherThreads), smem, s, 1, idx, T,
+                      k, E, align, counts, offsets, row_src, load_out, slot_row, status,
+                      static_cast<const uint4*>(x), x != nullptr ? d * elem_bytes / 16 : 0,
+                      static_cast<uint4*>(x_perm), w_src, w_dst);
 }
 
 bool permute_gather_grid_fits(int T, int E, int num_sms) {
@@ -759,20 +782,26 @@ cudaError_t launch_permute_gather_grid(const int32_t* idx, int T, int k, int E, 
                                       int32_t* row_src, int32_t* load_out, int* status,
                                       int* grid_bar, unsigned long long wait_limit_ns,
                                       const void* x, int d, int elem_bytes, void* x_perm,
-                                      int num_sms, cudaStream_t s) {
+                                      int num_sms, cudaStream_t s, int32_t* slot_row,
+                                      const float* w_src, float* w_dst) {
     if (!permute_gather_grid_fits(T, E, num_sms)) return cudaErrorInvalidValue;
     int P = (T + 31) / 32;
     if (P > num_sms) P = num_sms;
     const int TB = ((T + P - 1) / P + 31) / 32 * 32;
     P = (T + TB - 1) / TB;
     const size_t smem = (size_t)E * (TB / 32) * 8 + (size_t)(4 * E + 1) * 4;
-    cudaError_t e = cudaFuncSetAttribute(perm_gather_grid_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    auto kern = x != nullptr ? (w_dst != nullptr ? perm_gather_grid_kernel<true, true>
+                                                 : perm_gather_grid_kernel<true, false>)
+                             : (w_dst != nullptr ? perm_gather_grid_kernel<false, true>
+                                                 : perm_gather_grid_kernel<false, false>);
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
     if (e != cudaSuccess) return e;
-    return launch_pdl(perm_gather_grid_kernel, dim3((unsigned)P), dim3(kPermGatherThreads), smem,
+    return launch_pdl(kern, dim3((unsigned)P), dim3(kPermGatherThreads), smem,
                       s, 1, idx, T, k, E, align, TB, block_counts, counts, offsets, row_src,
-                      load_out, status, grid_bar, wait_limit_ns, static_cast<const uint4*>(x),
-                      d * elem_bytes / 16, static_cast<uint4*>(x_perm));
+                      load_out, slot_row, status, grid_bar, wait_limit_ns,
+                      static_cast<const uint4*>(x), x != nullptr ? d * elem_bytes / 16 : 0,
+                      static_cast<uint4*>(x_perm), w_src, w_dst);
 }
 
 cudaError_t launch_expert_counts(const int32_t* idx, int T, int k, int E,

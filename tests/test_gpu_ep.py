@@ -75,6 +75,8 @@ def emulate(w: Workload, inp, T_per_rank):
 CASES = [
     # the FusionLLM layer at prefill over 8 ranks of 512 tokens (8 experts each)
     ("prefill_8_ranks", WORKLOADS["prefill"], [512] * 8),
+    # 2 ranks of 2048 tokens: the dispatch's grid-wide permutation (T > 1024)
+    ("prefill_2_ranks", WORKLOADS["prefill"], [2048, 2048]),
     # decode over 4 ranks, ragged
     ("decode_4_ranks", WORKLOADS["decode"], [20, 1, 31, 12]),
     # small layer, 2 ranks, one rank with a single token, no shared experts
