@@ -538,9 +538,9 @@ def run_train(args, w):
     dom_flops = dom[2]
     dom_ach = dom_flops / (dom_ms * 1e-3) / 1e12
     # forward: route, permutation with the row gather, 2 GEMMs, final sum; backward:
-    # permutation (1 or 3), gather, dgrad GEMM, dL/dlogit, dgrad GEMM, dx sum,
-    # 2 weight-gradient GEMMs, dW_router (2)
-    launches = (1 + 1 + 2 + 1) + ((1 if w.T <= 1024 else 3) + 9)
+    # permutation, gather, dgrad GEMM, dL/dlogit, dgrad GEMM, dx sum, 2
+    # weight-gradient GEMMs, dW_router (2)
+    launches = (1 + 1 + 2 + 1) + (1 + 9)
     cfg = run_config(w, world, args)
     cfg["step"] = "forward (saving pre-activations) + backward (dx and all weight gradients, fp32)"
     out = {
