@@ -11,6 +11,13 @@
 // the real rows come first, in increasing token order (stable), then padding
 // rows whose row_src is -1.  row_src[r] = t*k + j for the row holding slot j
 // of token t.
+//
+// Two implementations give the same layout: the forward, the backward and
+// the expert-parallel dispatch use one launch that derives the permutation
+// from per-expert token bitmaps and copies the rows in the same kernel
+// (perm_gather_small_kernel up to 1024 tokens, perm_gather_grid_kernel
+// above); the histogram / scan / rank kernels serve the allocation-free
+// counts and the sizes whose bitmaps would not fit in shared memory.
 #include "moe_device.cuh"
 #include "moe_internal.h"
 
@@ -300,8 +307,9 @@ __device__ __forceinline__ void copy_row_warp(const uint4* __restrict__ x, int v
 // Small batches (T <= 1024) in one launch of several CTAs: every CTA derives
 // the whole permutation from the routing result on chip, CTA 0 writes it out
 // (counts, offsets, row_src, padding rows, slot_row), and all CTAs copy token
-// rows into x_perm, one warp per (token, slot).  Same layout and order as the
-// kernels above; a routing result names an expert at most once per token.
+// rows into x_perm (kRows) and gate weights into w_dst (kWeights), one warp
+// per (token, slot).  Same layout and order as the kernels above; a routing
+// result names an expert at most once per token.
 //
 // Stable ranks come from a bitmap per expert over the tokens: bit t of
 // bits[e] is set when token t chose e, so the rank of token t inside
@@ -419,7 +427,8 @@ __global__ void __launch_bounds__(kPermGatherThreads) perm_gather_small_kernel(
 //   3. every CTA sums the published counts: totals (-> segment offsets) and
 //      the counts of the CTAs before it (-> its base inside each segment);
 //      CTA 0 writes counts, offsets, padding rows; each CTA writes row_src
-//      of its slots and copies its tokens' rows into x_perm.
+//      (and slot_row) of its slots and copies its tokens' rows into x_perm
+//      (kRows) and their gate weights into w_dst (kWeights).
 // Same layout and stable order as the histogram / scan / rank kernels; the k
 // ids of a token are distinct.
 template <bool kRows, bool kWeights>
