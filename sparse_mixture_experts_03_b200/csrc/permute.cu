@@ -423,7 +423,8 @@ __global__ void __launch_bounds__(kPermGatherThreads) perm_gather_small_kernel(
 //      per-expert counts, published in block_counts[b][e];
 //   2. a grid-wide barrier (an arrival counter in the status region, reset
 //      by the routing kernel; the wait is bounded and reports
-//      MOE_ERR_TIMEOUT);
+//      MOE_ERR_TIMEOUT, after which every CTA that gives up, or sees that
+//      another gave up, leaves zero counts and offsets behind);
 //   3. every CTA sums the published counts: totals (-> segment offsets) and
 //      the counts of the CTAs before it (-> its base inside each segment);
 //      CTA 0 writes counts, offsets, padding rows; each CTA writes row_src
@@ -506,9 +507,20 @@ __global__ void __launch_bounds__(kPermGatherThreads) perm_gather_grid_kernel(
             __nanosleep(64);
         }
         __threadfence();
+        // a CTA that gave up has recorded MOE_ERR_TIMEOUT before the last
+        // arrival could let the others pass: they see it here and give up too
+        if (*reinterpret_cast<volatile int*>(status) == MOE_ERR_TIMEOUT) s_abort = 1;
     }
     __syncthreads();
-    if (s_abort) return;
+    if (s_abort) {
+        // no segment then: the GEMMs see zero routed rows (never a row_src
+        // entry this launch did not write)
+        for (int e = tid; e <= E; e += blockDim.x) {
+            if (e < E) counts[e] = 0;
+            offsets[e] = 0;
+        }
+        return;
+    }
     // totals and this CTA's base: column sums of block_counts, split over
     // the threads (parts of the CTA list per expert), combined with integer
     // atomics (order-independent)

@@ -118,22 +118,33 @@ class ExpertParallelMoE:
                 y_shared = self.shared(x)
         else:
             y_shared = self.shared(x)
-        recv_counts = torch.empty(N * E_l, dtype=disp.counts.dtype, device=x.device)
-        dist.all_to_all_single(recv_counts, disp.counts, group=self.group)
-        send = rank_rows(disp.counts.tolist(), N)
+        counts = disp.counts
+        send = rank_rows(counts.tolist(), N)
+        bad = sum(send) != T * self.k
+        if bad:
+            # a device error in the dispatch (its status word says which): this
+            # rank announces no rows, takes the same exchange steps as every
+            # other rank, and raises at the end
+            counts = torch.zeros_like(counts)
+            send = [0] * N
+        recv_counts = torch.empty(N * E_l, dtype=counts.dtype, device=x.device)
+        dist.all_to_all_single(recv_counts, counts, group=self.group)
         recv = rank_rows(recv_counts.tolist(), N)  # [src][e] blocks sum to rows per source
         recv_counts = recv_counts.view(N, E_l)
-        R = sum(recv)
+        R, n_send = sum(recv), sum(send)
         x_recv = torch.empty(R, d, dtype=disp.x_perm.dtype, device=x.device)
         w_recv = torch.empty(R, dtype=disp.w_perm.dtype, device=x.device)
-        dist.all_to_all_single(x_recv, disp.x_perm, recv, send, group=self.group)
-        dist.all_to_all_single(w_recv, disp.w_perm, recv, send, group=self.group)
+        dist.all_to_all_single(x_recv, disp.x_perm[:n_send], recv, send, group=self.group)
+        dist.all_to_all_single(w_recv, disp.w_perm[:n_send], recv, send, group=self.group)
         y_recv = self.experts(x_recv, w_recv, recv_counts.contiguous())
-        rows_back = torch.empty(T * self.k, d, dtype=y_recv.dtype, device=x.device)
+        rows_back = torch.empty(n_send, d, dtype=y_recv.dtype, device=x.device)
         dist.all_to_all_single(rows_back, y_recv, send, recv, group=self.group)
         if side is not None:
             torch.cuda.current_stream(x.device).wait_stream(side)
             y_shared.record_stream(torch.cuda.current_stream(x.device))
+        if bad:
+            raise RuntimeError("dispatch: the expert counts do not add up to T*k (a device "
+                               "error; see moe.device_status of the dispatch workspace)")
         return self.combine(rows_back, disp, y_shared, T)
 
     __call__ = forward

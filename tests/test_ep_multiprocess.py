@@ -91,6 +91,17 @@ class CpuOps:
         return y
 
 
+class BadCountsOps(CpuOps):
+    """CpuOps whose dispatch reports counts that do not add up to T*k, as a
+    device error in moe_dispatch would leave them (fault injected on the host)."""
+
+    @staticmethod
+    def dispatch(*args, **kw):
+        d = CpuOps.dispatch(*args, **kw)
+        d.counts[0] += 5
+        return d
+
+
 def layer_for_rank(w, inp, rank, world, ops):
     from sparse_mixture_experts_03_b200.ep import ExpertParallelMoE
     E_l = w.E // world
@@ -105,7 +116,7 @@ def rank_tokens(T_per_rank, rank):
     return lo, lo + T_per_rank[rank]
 
 
-def _rank_main(rank, world, port, case, q):
+def _rank_main(rank, world, port, case, q, bad_ranks=()):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     sys.path.insert(0, ROOT)
     sys.path.insert(0, os.path.join(ROOT, "tests"))
@@ -126,8 +137,14 @@ def _rank_main(rank, world, port, case, q):
             inp.x = inp.x.float().abs().add(0.1).to(inp.x.dtype)
         lo, hi = rank_tokens(T_per_rank, rank)
         x = inp.x[lo:hi].contiguous()
-        layer = layer_for_rank(w, inp, rank, world, CpuOps())
-        y = layer(x)
+        ops = BadCountsOps() if rank in bad_ranks else CpuOps()
+        layer = layer_for_rank(w, inp, rank, world, ops)
+        try:
+            y = layer(x)
+        except RuntimeError as err:  # the injected device error, raised after the exchanges
+            q.put({"rank": rank, "raised": str(err)})
+            dist.destroy_process_group()
+            return
         y_ref, _, _ = oracle.forward(x, inp.W_router, inp.W_gate_up, inp.W_down, inp.W_shared,
                                      w.k, w.n_group, w.topk_group, w.inter, w.n_shared)
         err = float(np.abs(y.numpy() - y_ref).max()) if y.numel() else 0.0
@@ -174,6 +191,29 @@ def test_expert_parallel_exchange_on_gloo_ranks(name):
     for r in sorted(res, key=lambda r: r["rank"]):
         assert "error" not in r, r["error"]
         assert r["err"] <= 1e-9 * max(1.0, r["scale"]), r
+
+
+def test_dispatch_error_on_one_rank_raises_there_and_others_finish():
+    """Rank 1's dispatch reports inconsistent counts: it announces no rows,
+    takes every exchange step the other rank takes (no collective is left
+    waiting) and raises at the end; rank 0's tokens, computed on both ranks'
+    experts, still match the oracle."""
+    sys.path.insert(0, ROOT)
+    world, case = _cases()["two_ranks"]
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank_main, args=(r, world, port, case, q, (1,)))
+             for r in range(world)]
+    for p in procs:
+        p.start()
+    res = {r["rank"]: r for r in (q.get(timeout=240) for _ in range(world))}
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    assert "error" not in res[0], res[0].get("error")
+    assert res[0]["err"] <= 1e-9 * max(1.0, res[0]["scale"]), res[0]
+    assert "do not add up" in res[1].get("raised", ""), res[1]
 
 
 def test_rank_rows_splits_expert_blocks():
