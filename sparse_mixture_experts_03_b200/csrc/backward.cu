@@ -204,44 +204,66 @@ __global__ void __launch_bounds__(256)
 }
 
 // dW_router in two passes with a fixed summation order.  Pass 1: block (e,
-// column chunk of 512, slice z) sums the rows of slice z of expert e's
-// segment (the segment cut into kDwSlices nearly equal row ranges), 2 columns
-// per thread, 8 rows' loads in flight, into part[z][e][:].  Pass 2 adds the
-// slices in order z = 0, 1, ...
+// column chunk of 2048, slice z) sums the rows of slice z of expert e's
+// segment (the segment cut into kDwSlices nearly equal row ranges), in row
+// order, into part[z][e][:]: 8 columns per thread (16-byte loads), 8 rows'
+// loads in flight.  The rows' gate gradients go through shared memory 256 at
+// a time, so the row loads depend on nothing but the row index (padding rows
+// of the segment are zero rows of x_perm and take a zero gradient).  Pass 2
+// adds the slices in order z = 0, 1, ...
 constexpr int kDwSlices = kDwParts;
+constexpr int kDwChunk = 256;
 
 __global__ void __launch_bounds__(256)
     router_dweight_part_kernel(const float* __restrict__ dl, const int32_t* __restrict__ row_src,
-                               const int32_t* __restrict__ offsets,
-                               const __nv_bfloat162* __restrict__ xp, int E, int d,
-                               float* __restrict__ part) {
+                               const int32_t* __restrict__ offsets, const uint4* __restrict__ xp,
+                               int E, int d, float* __restrict__ part) {
+    __shared__ float s_g[kDwChunk];    // dl of the chunk's rows (0 on padding rows)
+    __shared__ int s_ok[kDwChunk];     // the row is a real one
     const int e = blockIdx.x, z = blockIdx.z;
-    const int c2 = blockIdx.y * blockDim.x + threadIdx.x;  // column pair
+    const int c8 = blockIdx.y * blockDim.x + threadIdx.x;  // group of 8 columns
+    const int d8 = d >> 3;
     pdl_wait();
-    const int d2 = d >> 1;
-    if (c2 < d2) {
-        const int s0 = offsets[e], n = offsets[e + 1] - s0;
-        const int r0 = s0 + (int)((long long)z * n / kDwSlices);
-        const int r1 = s0 + (int)((long long)(z + 1) * n / kDwSlices);
-        float a0 = 0.f, a1 = 0.f;
-        for (int rb = r0; rb < r1; rb += 8) {
-            float g[8];
-            __nv_bfloat162 v[8];
+    const int s0 = offsets[e], n = offsets[e + 1] - s0;
+    const int r0 = s0 + (int)((long long)z * n / kDwSlices);
+    const int r1 = s0 + (int)((long long)(z + 1) * n / kDwSlices);
+    float a[8];
 #pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                const int r = rb + u;
-                const int src = r < r1 ? __ldg(row_src + r) : -1;
-                g[u] = src >= 0 ? __ldg(dl + src) : 0.f;
-                v[u] = src >= 0 ? xp[(size_t)r * d2 + c2] : __floats2bfloat162_rn(0.f, 0.f);
-            }
+    for (int q = 0; q < 8; ++q) a[q] = 0.f;
+    for (int cb = r0; cb < r1; cb += kDwChunk) {
+        const int nr = min(kDwChunk, r1 - cb);
+        __syncthreads();  // the previous chunk's gradients are no longer read
+        for (int i = threadIdx.x; i < nr; i += blockDim.x) {
+            const int src = __ldg(row_src + cb + i);
+            s_g[i] = src >= 0 ? __ldg(dl + src) : 0.f;
+            s_ok[i] = src >= 0;
+        }
+        __syncthreads();
+        if (c8 < d8) {
+            for (int rb = 0; rb < nr; rb += 8) {
+                uint4 v[8];
 #pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                const float2 f = __bfloat1622float2(v[u]);
-                a0 = fmaf(g[u], f.x, a0);
-                a1 = fmaf(g[u], f.y, a1);
+                for (int u = 0; u < 8; ++u)
+                    if (rb + u < nr) v[u] = __ldg(xp + (size_t)(cb + rb + u) * d8 + c8);
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    if (rb + u >= nr) break;
+                    const float g = s_g[rb + u];
+                    const uint4 w = s_ok[rb + u] ? v[u] : make_uint4(0u, 0u, 0u, 0u);
+                    const uint32_t w4[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                    for (int h = 0; h < 4; ++h) {
+                        a[2 * h] = fmaf(g, __uint_as_float(w4[h] << 16), a[2 * h]);
+                        a[2 * h + 1] = fmaf(g, __uint_as_float(w4[h] & 0xffff0000u), a[2 * h + 1]);
+                    }
+                }
             }
         }
-        reinterpret_cast<float2*>(part + ((size_t)z * E + e) * d)[c2] = make_float2(a0, a1);
+    }
+    if (c8 < d8) {
+        float4* o = reinterpret_cast<float4*>(part + ((size_t)z * E + e) * d) + 2 * c8;
+        o[0] = make_float4(a[0], a[1], a[2], a[3]);
+        o[1] = make_float4(a[4], a[5], a[6], a[7]);
     }
     pdl_trigger();
 }
@@ -318,10 +340,10 @@ cudaError_t launch_bwd_combine(const float* base, const void* slots, const float
 cudaError_t launch_router_dweight(const float* dl, const int32_t* row_src, const int32_t* offsets,
                                   const void* x_perm, int E, int d, float* part, float* dWr,
                                   cudaStream_t s) {
-    const unsigned cy = (unsigned)((d / 2 + 255) / 256);
+    const unsigned cy = (unsigned)((d / 8 + 255) / 256);
     cudaError_t e = launch_pdl(router_dweight_part_kernel, dim3((unsigned)E, cy, kDwSlices),
                                dim3(256), 0, s, 1, dl, row_src, offsets,
-                               static_cast<const __nv_bfloat162*>(x_perm), E, d, part);
+                               static_cast<const uint4*>(x_perm), E, d, part);
     if (e != cudaSuccess) return e;
     const int n4 = E * d / 4;
     return launch_pdl(router_dweight_sum_kernel, dim3((unsigned)((n4 + 255) / 256)), dim3(256), 0,
