@@ -202,86 +202,10 @@ __global__ void __launch_bounds__(kPermBlockTokens) perm_rank_kernel(
     pdl_trigger();
 }
 
-// Small batches (T <= 1024): histogram, scan and stable ranks in one CTA of
-// T threads rounded up to a warp, thread t holding token t -- the three
-// kernels above in one launch, same results (row order inside an expert =
-// token order).
+// Largest batch of the one-launch permutation in which every CTA derives
+// the whole permutation.
 constexpr int kSmallTokens = 1024;
-constexpr int kSmallWarps = kSmallTokens / 32;
 constexpr int kPermGatherThreads = 512;
-
-__global__ void __launch_bounds__(kSmallTokens) perm_small_kernel(
-    const int32_t* __restrict__ idx, int T, int k, int E, int align, int32_t* __restrict__ counts,
-    int32_t* __restrict__ offsets, int32_t* __restrict__ row_src, int32_t* __restrict__ load_out,
-    int32_t* __restrict__ slot_row, int* status) {
-    __shared__ int wcnt[kSmallWarps][kMaxE];  // per-warp counts, then per-warp bases
-    __shared__ int s_cnt[kMaxE];
-    __shared__ int s_off[kMaxE + 1];
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int nthr = blockDim.x, nwarps = nthr >> 5;
-    pdl_wait();
-    int my[kMaxK], rank[kMaxK];
-    load_slots(idx, tid, T, k, E, my, status);
-#pragma unroll
-    for (int j = 0; j < kMaxK; ++j) rank[j] = 0;
-    const unsigned lt = (1u << lane) - 1u;
-    for (int e = 0; e < E; ++e) {
-        const unsigned b = __ballot_sync(0xffffffffu, holds(my, e));
-        if (lane == 0) wcnt[warp][e] = __popc(b);
-#pragma unroll
-        for (int j = 0; j < kMaxK; ++j)
-            if (my[j] == e) rank[j] = __popc(b & lt);
-    }
-    __syncthreads();
-    for (int e = tid; e < E; e += nthr) {
-        int c = 0;
-        for (int w = 0; w < nwarps; ++w) c += wcnt[w][e];
-        s_cnt[e] = c;
-    }
-    __syncthreads();
-    if (tid < 32) {  // warp scan of the padded segment sizes
-        int carry = 0;
-        for (int e0 = 0; e0 < E; e0 += 32) {
-            const int e = e0 + tid;
-            const int v = e < E ? (s_cnt[e] + align - 1) / align * align : 0;
-            int incl = v;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const int n = __shfl_up_sync(0xffffffffu, incl, o);
-                if (tid >= o) incl += n;
-            }
-            if (e < E) s_off[e] = carry + incl - v;
-            carry += __shfl_sync(0xffffffffu, incl, 31);
-        }
-        if (tid == 0) s_off[E] = carry;
-    }
-    __syncthreads();
-    for (int e = tid; e < E; e += nthr) {
-        int run = s_off[e];
-        for (int w = 0; w < nwarps; ++w) {
-            const int c = wcnt[w][e];
-            wcnt[w][e] = run;
-            run += c;
-        }
-        counts[e] = s_cnt[e];
-        if (load_out != nullptr) load_out[e] = s_cnt[e];
-    }
-    for (int e = tid; e <= E; e += nthr) offsets[e] = s_off[e];
-    for (int i = tid; i < E * align; i += nthr) {
-        const int e = i / align, r = i % align;
-        const int row = s_off[e] + s_cnt[e] + r;
-        if (row < s_off[e + 1]) row_src[row] = -1;
-    }
-    __syncthreads();
-#pragma unroll
-    for (int j = 0; j < kMaxK; ++j)
-        if (my[j] >= 0) {
-            const int pos = wcnt[warp][my[j]] + rank[j];
-            row_src[pos] = tid * k + j;
-            if (slot_row != nullptr) slot_row[tid * k + j] = pos;
-        }
-    pdl_trigger();
-}
 
 // Copy token row t of x into row `row` of x_perm: one warp, 16-byte vectors,
 // up to 8 per lane in flight.
@@ -747,10 +671,6 @@ __global__ void __launch_bounds__(256) combine_slots_bf16_kernel(
 cudaError_t launch_permute(const int32_t* idx, int T, int k, int E, int32_t* block_counts,
                            int32_t* counts, int32_t* offsets, int32_t* row_src, int align,
                            int32_t* load_out, int* status, cudaStream_t s, int32_t* slot_row) {
-    if (T <= kSmallTokens)
-        return launch_pdl(perm_small_kernel, dim3(1), dim3((unsigned)((T + 31) / 32 * 32)), 0, s,
-                          1, idx, T, k, E, align, counts, offsets, row_src, load_out, slot_row,
-                          status);
     const int nb = (T + kPermBlockTokens - 1) / kPermBlockTokens;
     cudaError_t e = launch_pdl(perm_count_kernel<false>, dim3(nb), dim3(kPermBlockTokens), 0, s,
                                1, idx, T, k, E, block_counts, status);
